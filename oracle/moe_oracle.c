@@ -1,0 +1,498 @@
+/*
+ * moe_oracle.c -- plain, slow, fp64 CPU oracle for the forward pass of a sparse
+ * Mixture-of-Experts SwiGLU FFN layer (noisy Top-K routing, capacity dispatch,
+ * gate-weighted combine, gate statistics).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call
+ * this file: only the tests, the package smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant with the
+ * CUDA library; the only thing both sides consume is the seeded input data.
+ *
+ * Every floating-point input is widened exactly to double (bf16 -> f32 -> f64 is
+ * exact) and all arithmetic is done in double.  There is no blocking, fusion or
+ * reordering beyond what the formulas state: each function is the definition
+ * written out as index loops, so it can be checked against the pages by eye.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [UPCYCLE]  "Llama 3 Meets MoE: Efficient Upcycling" (paper review), section 3
+ *             "核心公式": MoE output y = sum_i G(x)_i E_i(x); noisy Top-k routing
+ *             G = Softmax(KeepTopK(H, k)), H_i = (x W_g)_i + StandardNormal() *
+ *             Softplus((x W_noise)_i); KeepTopK; expert capacity =
+ *             tokens per batch / N * CF with overflow tokens excluded; section 5
+ *             "路由器算法消融实验": Mixtral type (KeepTopK then Softmax) vs ST type
+ *             (Softmax then KeepTopK); section 2 "解决方案概述": experts made by
+ *             copying the dense FFN.
+ *  [V2]       "LLaMA-MoE v2: 基于后训练混合专家模型的稀疏性探索与技术突破",
+ *             section "专家构建方法" (independent neuron partition: split the
+ *             intermediate-neuron index set U into M equal disjoint subsets),
+ *             section "门控机制设计" (noisy gate, L_balance = lambda sum f_i P_i),
+ *             section "重新缩放机制与负载均衡" (y = N/k sum G_i E_i), and the code
+ *             sample in "代码实现示例" (SwiGLU expert down(silu(gate(x)) * up(x))).
+ *  [HUB]      "从大炼到巧炼：LLaMA-MoE 如何用 MoE 架构让 LLM 变快变省", section
+ *             "持续预训练" (Gate Load and Gate Importance are monitored).
+ *
+ * Readings where the pages are silent or ambiguous (each is also listed in the
+ * design notes of the repository):
+ *  - the partition permutation is supplied by the caller;
+ *  - the noise draw StandardNormal() is a supplied [T,E] tensor;
+ *  - the per-expert bias (when given) is added to the clean logits;
+ *  - Top-k ties go to the lower expert index; slots are ordered by descending H;
+ *  - capacity drops are per (token, expert) assignment, lower token index wins;
+ *  - a dropped assignment contributes nothing (the residual outside the layer
+ *    carries x); the remaining weights are not renormalised;
+ *  - f_i = routed count_i / (T k), P_i = mean over tokens of the full softmax of
+ *    the routing logits H (pre-drop);
+ *  - gate importance_i = sum over tokens of the final gate weight of expert i;
+ *  - softplus is the plain function log(1 + e^z).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* element types of the inputs the oracle reads (its own constants) */
+#define ORC_F32 0
+#define ORC_BF16 1
+
+#define ORC_MIXTRAL 0
+#define ORC_ST 1
+
+#define ORC_DISJOINT 0
+#define ORC_COPY 1
+
+#define ORC_EINVAL (-1)
+
+/* Exact widening of one stored element to double. */
+static double orc_load(const void *p, int dt, size_t i)
+{
+    if (dt == ORC_F32)
+        return (double)((const float *)p)[i];
+    uint32_t u = ((uint32_t)((const uint16_t *)p)[i]) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static size_t orc_esize(int dt) { return dt == ORC_F32 ? 4 : 2; }
+
+int oracle_version(void) { return 1; }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------- */
+/* a0. Expert construction [V2 "专家构建方法"; UPCYCLE section 2].
+ * DISJOINT: expert e owns intermediate neurons perm[e*m .. (e+1)*m), m = d_ff/E;
+ *   W1_e = W1[idx_e, :], W3_e = W3[idx_e, :], W2_e = W2[:, idx_e].
+ * COPY: every expert is the whole FFN (m = d_ff).
+ * W1, W3 are [d_ff][d] (out x in), W2 is [d][d_ff].  Outputs, in the input's
+ * element type: W1e, W3e [E][m][d], W2e [E][d][m].  A pure element gather. */
+int oracle_partition(const void *W1, const void *W3, const void *W2, int dt,
+                     int d, int d_ff, int E, int mode, const int32_t *perm,
+                     void *W1e, void *W3e, void *W2e)
+{
+    if (d <= 0 || d_ff <= 0 || E <= 0)
+        return ORC_EINVAL;
+    if (mode == ORC_DISJOINT && (d_ff % E != 0 || perm == NULL))
+        return ORC_EINVAL;
+    const size_t es = orc_esize(dt);
+    const int m = (mode == ORC_DISJOINT) ? d_ff / E : d_ff;
+    for (int e = 0; e < E; ++e) {
+        for (int i = 0; i < m; ++i) {
+            int src = (mode == ORC_DISJOINT) ? perm[(size_t)e * m + i] : i;
+            if (src < 0 || src >= d_ff)
+                return ORC_EINVAL;
+            for (int c = 0; c < d; ++c) {
+                size_t s = (size_t)src * d + c;
+                size_t o = ((size_t)e * m + i) * d + c;
+                memcpy((char *)W1e + o * es, (const char *)W1 + s * es, es);
+                memcpy((char *)W3e + o * es, (const char *)W3 + s * es, es);
+            }
+            for (int r = 0; r < d; ++r) {
+                size_t s = (size_t)r * d_ff + src;
+                size_t o = ((size_t)e * d + r) * m + i;
+                memcpy((char *)W2e + o * es, (const char *)W2 + s * es, es);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Softplus(z) = log(1 + e^z), written in the overflow-free form
+ * max(z, 0) + log1p(exp(-|z|)), which is the same function. */
+double oracle_softplus(double z) { return (z > 0 ? z : 0.0) + log1p(exp(-fabs(z))); }
+
+/* SiLU (Swish) of the SwiGLU expert [V2 code sample, Expert.act_fn]: z * sigmoid(z). */
+double oracle_silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* Ordering used by KeepTopK: larger value first, then lower expert index. */
+typedef struct {
+    double v;
+    int e;
+} orc_key;
+
+static int orc_key_cmp(const void *a, const void *b)
+{
+    const orc_key *x = (const orc_key *)a, *y = (const orc_key *)b;
+    if (x->v > y->v)
+        return -1;
+    if (x->v < y->v)
+        return 1;
+    return (x->e < y->e) ? -1 : (x->e > y->e);
+}
+
+/* KeepTopK [UPCYCLE section 3]: the indices of the k largest entries of h[0..E),
+ * found by a full sort of (value desc, index asc).  idx[j] is the j-th largest.
+ * Returns ORC_EINVAL if any entry is NaN. */
+int oracle_topk(int E, int k, const double *h, int32_t *idx)
+{
+    if (E <= 0 || k <= 0 || k > E)
+        return ORC_EINVAL;
+    orc_key *keys = (orc_key *)malloc(sizeof(orc_key) * (size_t)E);
+    if (!keys)
+        return ORC_EINVAL;
+    for (int e = 0; e < E; ++e) {
+        if (isnan(h[e])) {
+            free(keys);
+            return ORC_EINVAL;
+        }
+        keys[e].v = h[e];
+        keys[e].e = e;
+    }
+    qsort(keys, (size_t)E, sizeof(orc_key), orc_key_cmp);
+    for (int j = 0; j < k; ++j)
+        idx[j] = keys[j].e;
+    free(keys);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* a1. Router [UPCYCLE section 3 and section 5; V2 "门控机制设计"].
+ *   L_t = x_t . W_g (+ b)            (W_g stored [d][E])
+ *   H_t = L_t + eps_t * Softplus(x_t . W_noise)   if W_noise is given
+ *   idx_t = KeepTopK(H_t, k)
+ *   Mixtral: G_tj = exp(H_t,idx_j) / sum_{j'<k} exp(H_t,idx_j')
+ *   ST:      G_tj = exp(H_t,idx_j) / sum_{e<E} exp(H_t,e)
+ * Also (all optional, may be NULL):
+ *   H_out [T][E]            the routing logits H,
+ *   probs_sum [E]           sum over tokens of softmax(H_t) over all E,
+ *   clean_probs_sum [E]     sum over tokens of softmax(L_t) (page-2 sketch variant),
+ *   importance [E]          sum over tokens of the gate weight given to expert e.
+ * x, W_g, W_noise share element type dt; eps [T][E] and b [E] are f32. */
+int oracle_router(int T, int d, int E, int k, int router_type,
+                  const void *x, int dt, const void *Wg, const void *Wnoise,
+                  const float *eps, const float *bias,
+                  double *H_out, int32_t *idx, double *G,
+                  double *probs_sum, double *clean_probs_sum, double *importance)
+{
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
+        return ORC_EINVAL;
+    if (Wnoise != NULL && eps == NULL)
+        return ORC_EINVAL;
+    int bad = 0;
+    double *P = (double *)calloc((size_t)T * E + 1, sizeof(double));
+    double *PC = (double *)calloc((size_t)T * E + 1, sizeof(double));
+    if (!P || !PC) {
+        free(P);
+        free(PC);
+        return ORC_EINVAL;
+    }
+#pragma omp parallel for schedule(static) reduction(| : bad)
+    for (int t = 0; t < T; ++t) {
+        double *L = (double *)malloc(sizeof(double) * (size_t)E * 2);
+        double *H = L + E;
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0, accn = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double xv = orc_load(x, dt, (size_t)t * d + c);
+                acc += xv * orc_load(Wg, dt, (size_t)c * E + e);
+                if (Wnoise)
+                    accn += xv * orc_load(Wnoise, dt, (size_t)c * E + e);
+            }
+            if (bias)
+                acc += (double)bias[e];
+            L[e] = acc;
+            H[e] = Wnoise ? acc + (double)eps[(size_t)t * E + e] * oracle_softplus(accn) : acc;
+        }
+        if (H_out)
+            for (int e = 0; e < E; ++e)
+                H_out[(size_t)t * E + e] = H[e];
+        int32_t *it = idx + (size_t)t * k;
+        if (oracle_topk(E, k, H, it) != 0) {
+            bad = 1;
+            for (int j = 0; j < k; ++j) {
+                it[j] = -1;
+                G[(size_t)t * k + j] = 0.0;
+            }
+            free(L);
+            continue;
+        }
+        /* full softmax of H (used by ST weights and by P) */
+        double hmax = H[it[0]];
+        double zall = 0.0;
+        for (int e = 0; e < E; ++e)
+            zall += exp(H[e] - hmax);
+        for (int e = 0; e < E; ++e)
+            P[(size_t)t * E + e] = exp(H[e] - hmax) / zall;
+        /* softmax of the clean logits L (page-2 sketch's P) */
+        double lmax = L[0];
+        for (int e = 1; e < E; ++e)
+            if (L[e] > lmax)
+                lmax = L[e];
+        double zl = 0.0;
+        for (int e = 0; e < E; ++e)
+            zl += exp(L[e] - lmax);
+        for (int e = 0; e < E; ++e)
+            PC[(size_t)t * E + e] = exp(L[e] - lmax) / zl;
+        if (router_type == ORC_MIXTRAL) {
+            double zsel = 0.0;
+            for (int j = 0; j < k; ++j)
+                zsel += exp(H[it[j]] - hmax);
+            for (int j = 0; j < k; ++j)
+                G[(size_t)t * k + j] = exp(H[it[j]] - hmax) / zsel;
+        } else {
+            for (int j = 0; j < k; ++j)
+                G[(size_t)t * k + j] = P[(size_t)t * E + it[j]];
+        }
+        free(L);
+    }
+    /* token-ordered sums */
+    for (int e = 0; e < E; ++e) {
+        double s = 0.0, sc = 0.0, si = 0.0;
+        for (int t = 0; t < T; ++t) {
+            s += P[(size_t)t * E + e];
+            sc += PC[(size_t)t * E + e];
+            for (int j = 0; j < k; ++j)
+                if (idx[(size_t)t * k + j] == e)
+                    si += G[(size_t)t * k + j];
+        }
+        if (probs_sum)
+            probs_sum[e] = s;
+        if (clean_probs_sum)
+            clean_probs_sum[e] = sc;
+        if (importance)
+            importance[e] = si;
+    }
+    free(P);
+    free(PC);
+    return bad ? ORC_EINVAL : 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Expert capacity [UPCYCLE section 3 "容量因子"]: tokens per batch / N * CF,
+ * read with tokens = T (not T*k) and rounded up to a whole token.
+ * cf < 0 means no limit (returns -1). */
+int oracle_capacity(int T, int E, double cf)
+{
+    if (cf < 0)
+        return -1;
+    return (int)ceil((double)T / (double)E * cf);
+}
+
+/* a2. Dispatch with capacity [UPCYCLE section 3 "容量因子"].
+ * Assignments (t, j) are visited in token order (t outer, slot j inner).  Each
+ * expert keeps a running count; an assignment whose rank within its expert is
+ * >= C is dropped (C < 0: no limit), so the lower token index wins.
+ *   counts[e]   routed (pre-drop) assignments of expert e
+ *   kept[e]     min(counts[e], C)
+ *   offsets[e]  exclusive prefix sum of kept (offsets[E] = R)
+ *   row_token[r] token of kept row r; rows are grouped by expert, token-ascending
+ *   slot_row[t*k+j] row of assignment (t, j), or -1 if dropped
+ * Entries of idx outside [0, E) are treated as dropped.  Returns R. */
+int oracle_dispatch(int T, int E, int k, const int32_t *idx, int C,
+                    int32_t *counts, int32_t *kept, int32_t *offsets,
+                    int32_t *row_token, int32_t *slot_row)
+{
+    if (T < 0 || E <= 0 || k <= 0)
+        return ORC_EINVAL;
+    int32_t *rank = (int32_t *)malloc(sizeof(int32_t) * ((size_t)T * k + 1));
+    if (!rank)
+        return ORC_EINVAL;
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E) {
+                rank[(size_t)t * k + j] = -1;
+                continue;
+            }
+            rank[(size_t)t * k + j] = counts[e]++;
+        }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        kept[e] = (C < 0 || counts[e] < C) ? counts[e] : C;
+        offsets[e + 1] = offsets[e] + kept[e];
+    }
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            size_t a = (size_t)t * k + j;
+            int e = idx[a];
+            int r = rank[a];
+            if (r < 0 || r >= kept[e]) {
+                slot_row[a] = -1;
+                continue;
+            }
+            int row = offsets[e] + r;
+            slot_row[a] = row;
+            row_token[row] = t;
+        }
+    free(rank);
+    return offsets[E];
+}
+
+/* ------------------------------------------------------------------------- */
+/* a3 + a4. One SwiGLU expert applied to n input rows [V2 code sample, Expert]:
+ *   out_r = W2_e ( silu(W1_e x_r) * (W3_e x_r) ),  e = expert_of_row[r]
+ * Expert weights in the standard layout W1e, W3e [E][m][d], W2e [E][d][m]
+ * (element type dt, as produced by oracle_partition).  x_rows [n][d] has type
+ * xdt.  out [n][d] double.  If h is not NULL it receives the [n][m] activations. */
+int oracle_expert_ffn(int d, int m, int E, const void *W1e, const void *W3e,
+                      const void *W2e, int dt, const void *x_rows, int xdt,
+                      const int32_t *expert_of_row, int n, double *out, double *h)
+{
+    if (d <= 0 || m <= 0 || E <= 0 || n < 0)
+        return ORC_EINVAL;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int r = 0; r < n; ++r) {
+        int e = expert_of_row[r];
+        if (e < 0 || e >= E) {
+            bad = 1;
+            continue;
+        }
+        double *xr = (double *)malloc(sizeof(double) * ((size_t)d + m));
+        double *hr = xr + d;
+        for (int c = 0; c < d; ++c)
+            xr[c] = orc_load(x_rows, xdt, (size_t)r * d + c);
+        for (int i = 0; i < m; ++i) {
+            double g = 0.0, u = 0.0;
+            size_t base = ((size_t)e * m + i) * d;
+            for (int c = 0; c < d; ++c) {
+                g += orc_load(W1e, dt, base + c) * xr[c];
+                u += orc_load(W3e, dt, base + c) * xr[c];
+            }
+            hr[i] = oracle_silu(g) * u;
+            if (h)
+                h[(size_t)r * m + i] = hr[i];
+        }
+        for (int o = 0; o < d; ++o) {
+            double acc = 0.0;
+            size_t base = ((size_t)e * d + o) * m;
+            for (int i = 0; i < m; ++i)
+                acc += orc_load(W2e, dt, base + i) * hr[i];
+            out[(size_t)r * d + o] = acc;
+        }
+        free(xr);
+    }
+    return bad ? ORC_EINVAL : 0;
+}
+
+/* The dense SwiGLU FFN the experts were cut from: y = W2 (silu(W1 x) * (W3 x)),
+ * W1, W3 [d_ff][d], W2 [d][d_ff].  x [n][d] (type xdt), y [n][d] double. */
+int oracle_dense_ffn(int d, int d_ff, const void *W1, const void *W3, const void *W2,
+                     int dt, const void *x, int xdt, int n, double *y)
+{
+    if (d <= 0 || d_ff <= 0 || n < 0)
+        return ORC_EINVAL;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n; ++r) {
+        double *xr = (double *)malloc(sizeof(double) * ((size_t)d + d_ff));
+        double *hr = xr + d;
+        for (int c = 0; c < d; ++c)
+            xr[c] = orc_load(x, xdt, (size_t)r * d + c);
+        for (int i = 0; i < d_ff; ++i) {
+            double g = 0.0, u = 0.0;
+            for (int c = 0; c < d; ++c) {
+                g += orc_load(W1, dt, (size_t)i * d + c) * xr[c];
+                u += orc_load(W3, dt, (size_t)i * d + c) * xr[c];
+            }
+            hr[i] = oracle_silu(g) * u;
+        }
+        for (int o = 0; o < d; ++o) {
+            double acc = 0.0;
+            for (int i = 0; i < d_ff; ++i)
+                acc += orc_load(W2, dt, (size_t)o * d_ff + i) * hr[i];
+            y[(size_t)r * d + o] = acc;
+        }
+        free(xr);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* a5. Gate-weighted combine [UPCYCLE section 3, y = sum_i G(x)_i E_i(x); V2
+ * "重新缩放机制", y = N/k sum_i G(x)_i E_i(x)]:
+ *   y_t = scale * sum_{j<k, slot kept} G_tj * out_{slot_row[t,j]}
+ * out_rows [R][d] double, G [T][k] double, y [T][d] double.  A token whose
+ * slots are all dropped gets y_t = 0. */
+int oracle_combine(int T, int d, int k, const double *out_rows, const int32_t *slot_row,
+                   const double *G, double scale, double *y)
+{
+    if (T < 0 || d <= 0 || k <= 0)
+        return ORC_EINVAL;
+    for (int t = 0; t < T; ++t)
+        for (int o = 0; o < d; ++o) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int r = slot_row[(size_t)t * k + j];
+                if (r >= 0)
+                    acc += G[(size_t)t * k + j] * out_rows[(size_t)r * d + o];
+            }
+            y[(size_t)t * d + o] = scale * acc;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* a6. Gate statistics [V2 "门控机制设计", L_balance = lambda sum_i f_i P_i;
+ * HUB "持续预训练": Gate Load, Gate Importance].
+ *   f_e = counts_e / (T k),  P_e = probs_sum_e / T,  L = lambda sum_e f_e P_e.
+ * T = 0 gives f = P = 0 and L = 0. */
+int oracle_gate_stats(int T, int E, int k, const int32_t *counts, const double *probs_sum,
+                      double lambda, double *f, double *P, double *L)
+{
+    if (T < 0 || E <= 0 || k <= 0)
+        return ORC_EINVAL;
+    double s = 0.0;
+    for (int e = 0; e < E; ++e) {
+        f[e] = T > 0 ? (double)counts[e] / ((double)T * k) : 0.0;
+        P[e] = T > 0 ? probs_sum[e] / (double)T : 0.0;
+        s += f[e] * P[e];
+    }
+    *L = lambda * s;
+    return 0;
+}
+
+/* The load-balance loss as the V2 code sample computes it (information only):
+ * frequency = per-expert sum of gate weights normalised to sum 1 (with the
+ * sample's 1e-6 guard), P = mean softmax of the clean logits, times E. */
+int oracle_balance_sketch(int T, int E, int k, const int32_t *idx, const double *G,
+                          const double *clean_probs_sum, double *L)
+{
+    if (T <= 0 || E <= 0 || k <= 0)
+        return ORC_EINVAL;
+    double *w = (double *)calloc((size_t)E, sizeof(double));
+    double tot = 0.0, s = 0.0;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(size_t)t * k + j];
+            if (e >= 0 && e < E)
+                w[e] += G[(size_t)t * k + j];
+        }
+    for (int e = 0; e < E; ++e)
+        tot += w[e];
+    for (int e = 0; e < E; ++e)
+        s += (w[e] / (tot + 1e-6)) * (clean_probs_sum[e] / (double)T);
+    *L = s * (double)E;
+    free(w);
+    return 0;
+}
