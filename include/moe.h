@@ -1,0 +1,253 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of a sparse Mixture-of-Experts
+ * SwiGLU FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (notation: T tokens, model width d, dense FFN width d_ff, E experts,
+ * k experts per token, m neurons per expert, R kept (token, expert) rows):
+ *
+ *   a0  experts are equal disjoint random subsets of the dense FFN's
+ *       intermediate neurons, or whole copies of it
+ *         ["LLaMA-MoE v2: 基于后训练混合专家模型的稀疏性探索与技术突破",
+ *          section "专家构建方法"; "Llama 3 Meets MoE: Efficient Upcycling",
+ *          section 2 "解决方案概述"]
+ *   a1  H = x W_g (+ b) + eps * Softplus(x W_noise);  idx = KeepTopK(H, k);
+ *       Mixtral type G = Softmax over the k kept logits, ST type G = the full
+ *       softmax at the kept experts
+ *         ["Llama 3 Meets MoE", section 3 "核心公式" (Noisy Top-k routing) and
+ *          section 5 "路由器算法消融实验"]
+ *   a2  expert capacity C = tokens per batch / E * CF; assignments past an
+ *       expert's capacity are dropped (lower token index wins)
+ *         ["Llama 3 Meets MoE", section 3 "容量因子"]
+ *   a3  h = silu(x W1_e^T) * (x W3_e^T)        (SwiGLU expert, first half)
+ *   a4  out = h W2_e^T                           (second half)
+ *         ["LLaMA-MoE v2", code sample "代码实现示例", class Expert]
+ *   a5  y_t = s * sum_j G_tj out_{row(t,j)},  s = E/k with rescale, else 1
+ *         ["Llama 3 Meets MoE", section 3, y = sum_i G(x)_i E_i(x);
+ *          "LLaMA-MoE v2", section "重新缩放机制与负载均衡"]
+ *   a6  gate load, gate importance, f_e, P_e, L_balance = lambda sum f_e P_e
+ *         ["LLaMA-MoE v2", section "门控机制设计"; "从大炼到巧炼：LLaMA-MoE 如何用
+ *          MoE 架构让 LLM 变快变省", section "持续预训练" (monitored metrics)]
+ *
+ * Conventions
+ *  - Every entry point returns MOE_OK (0) or a negative moe_status_t.  On error
+ *    nothing was launched and moe_last_error_string() describes the problem.
+ *  - Pointers named as device pointers must be CUDA device memory of the
+ *    current device; the caller owns every buffer.  The library allocates no
+ *    device memory: internal scratch lives in the caller's workspace, sized by
+ *    moe_workspace_size() and zeroed once by moe_workspace_init().
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
+ *    void*; NULL is the legacy default stream).  Calls never synchronise the
+ *    host with the device, except moe_get_device_status().
+ *  - Errors found by kernels (an expert index outside [0,E), a NaN routing
+ *    logit, a wait that ran out) are recorded in a status word inside the
+ *    workspace; the first one sticks until read with clear=1.
+ *  - Device pointers must be 16-byte aligned (MOE_ERR_ALIGN otherwise).
+ *  - Row-major everywhere; "[A][B]" means B is the contiguous dimension.
+ *  - Element type of activations and expert/router weights is `dtype`
+ *    (MOE_BF16 or MOE_F32); gate weights, noise, bias and statistics are f32;
+ *    indices are int32.  bf16 paths accumulate in f32.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,    /* null pointer, k < 1, k > E, E > 64, T < 0, ... */
+    MOE_ERR_SHAPE = -2,          /* d % 8 != 0, d_ff % E != 0 (disjoint), too large */
+    MOE_ERR_ALIGN = -3,          /* device pointer not 16-byte aligned */
+    MOE_ERR_DTYPE = -4,          /* dtype not MOE_BF16 / MOE_F32, or unsupported mix */
+    MOE_ERR_CUDA = -5,           /* a CUDA runtime/driver call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = -6, /* a kernel wait ran past its limit (device status) */
+    MOE_ERR_DEVICE_BADINDEX = -7,/* expert index out of range or NaN logit (device status) */
+    MOE_ERR_WORKSPACE = -8,      /* workspace smaller than moe_workspace_size() */
+    MOE_ERR_UNSUPPORTED = -9     /* no kernel for this device or configuration */
+} moe_status_t;
+
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+enum { MOE_ROUTER_MIXTRAL = 0, MOE_ROUTER_ST = 1 };
+enum { MOE_PARTITION_DISJOINT = 0, MOE_PARTITION_COPY = 1, MOE_PARTITION_STACKED = 2 };
+
+#define MOE_MAX_EXPERTS 64
+#define MOE_MAX_TOPK 8
+
+/* Layer description, passed by pointer, read only during the call. */
+typedef struct {
+    int32_t T;             /* tokens in the batch (>= 0) */
+    int32_t d;             /* model width (multiple of 8) */
+    int32_t E;             /* experts, 1..64 */
+    int32_t k;             /* experts per token, 1..min(E, 8) */
+    int32_t m;             /* neurons per expert (d_ff/E disjoint, d_ff copies) */
+    int32_t dtype;         /* MOE_BF16 or MOE_F32 */
+    int32_t router_type;   /* MOE_ROUTER_MIXTRAL or MOE_ROUTER_ST */
+    int32_t capacity;      /* rows kept per expert; < 0 means no limit */
+    int32_t rescale;       /* nonzero: combine scales by E/k */
+    float balance_lambda;  /* lambda of L_balance */
+} moe_params_t;
+
+/* Library version string (static storage). */
+const char *moe_version(void);
+
+/* Message of the last error returned on the calling thread (thread-local storage). */
+const char *moe_last_error_string(void);
+
+/* Number of kernels this process has launched through the library so far. */
+uint64_t moe_launch_count(void);
+
+/* Expert capacity ["Llama 3 Meets MoE", section 3 "容量因子"]: tokens per batch
+ * divided by the number of experts times the capacity factor, rounded up to a
+ * whole token: ceil(T * cf / E).  cf < 0 returns -1 (no limit).  Host-only. */
+int32_t moe_capacity(int32_t T, int32_t E, double cf);
+
+/* ---- packed expert weight layout (a0 output, a3/a4 input) ----------------
+ * W13_e [E][2*m16][d], m16 = m rounded up to a multiple of 16.  Rows come in
+ *   groups of 32: rows 32b..32b+15 are the W1 (gate, inside silu) rows of
+ *   expert neurons 16b..16b+15, rows 32b+16..32b+31 their W3 (up) rows.  Rows
+ *   of neurons >= m are zero.
+ * W2_e  [E][d][m8], m8 = m rounded up to a multiple of 8; columns >= m are zero.
+ * h     [rows][m8] (the SwiGLU activations; columns >= m are never read). */
+int64_t moe_packed_w13_elems(int32_t E, int32_t m, int32_t d);
+int64_t moe_packed_w2_elems(int32_t E, int32_t m, int32_t d);
+int32_t moe_h_ld(int32_t m);
+
+/* a0. Builds the packed expert weights from a dense SwiGLU FFN
+ * ["LLaMA-MoE v2", section "专家构建方法" (IndependentRandom: the index set of
+ * intermediate neurons split into E equal disjoint subsets);
+ * "Llama 3 Meets MoE", section 2 (upcycling: E copies of the FFN)].
+ *   mode DISJOINT: W1, W3 [d_ff][d], W2 [d][d_ff] (nn.Linear out x in);
+ *                  m = d_ff / E; expert e owns neurons perm[e*m .. e*m+m);
+ *                  perm [d_ff] int32 device, a permutation of 0..d_ff-1.
+ *   mode COPY:     same inputs, m = d_ff, every expert is the whole FFN; perm unused.
+ *   mode STACKED:  already-built experts (e.g. perturbed copies): W1, W3 [E][d_ff][d],
+ *                  W2 [E][d][d_ff]; m = d_ff; perm unused.
+ * Outputs W13_e, W2_e in the packed layout above (device, caller-allocated with
+ * moe_packed_*_elems elements of dtype).  A perm entry outside [0, d_ff) writes
+ * a zero neuron and sets MOE_ERR_DEVICE_BADINDEX in the status word of `ws`
+ * (ws may be NULL, then such entries are only zeroed).
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE (d % 8, d_ff % E in DISJOINT),
+ * MOE_ERR_DTYPE, MOE_ERR_ALIGN, MOE_ERR_CUDA. */
+int moe_partition_experts(const void *W1, const void *W3, const void *W2,
+                          int32_t d, int32_t d_ff, int32_t E, int32_t mode,
+                          const int32_t *perm, int32_t dtype,
+                          void *W13_e, void *W2_e, void *ws, void *stream);
+
+/* Bytes of workspace the calls below need for `p` (covers every call with the
+ * same or smaller T, E, d).  Host-only, never fails (returns 0 on bad params). */
+size_t moe_workspace_size(const moe_params_t *p);
+
+/* Zeroes a freshly allocated workspace (status word and counters).  Call once
+ * after allocation; the library keeps it consistent afterwards. */
+int moe_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* a1. Router ["Llama 3 Meets MoE", section 3 "Noisy Top-k 路由", section 5].
+ *   x [T][d] (dtype), Wg [d][E] (dtype), Wnoise [d][E] (dtype, NULL: no noise),
+ *   noise [T][E] f32 (the StandardNormal() draws; required iff Wnoise given),
+ *   bias [E] f32 (NULL: none; added to the clean logits).
+ * Outputs (device): topk_idx [T][k] int32 (slot j holds the j-th largest H;
+ *   ties go to the lower expert index), topk_w [T][k] f32 (gate weights),
+ *   probs_sum [E] f32 (sum over tokens of the full softmax of H),
+ *   importance [E] f32 (sum over tokens of the gate weight of each expert).
+ * A NaN logit sets MOE_ERR_DEVICE_BADINDEX and writes idx -1, weight 0. */
+int moe_route(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
+              const float *noise, const float *bias, int32_t *topk_idx, float *topk_w,
+              float *probs_sum, float *importance, void *ws, size_t ws_bytes, void *stream);
+
+/* a2. Dispatch with capacity ["Llama 3 Meets MoE", section 3 "容量因子"].
+ * Stable counting sort of the T*k assignments by expert, token-ascending inside
+ * an expert; assignment (t,j) is dropped iff its rank inside its expert is
+ * >= p->capacity (no limit when < 0).  Outputs (device):
+ *   counts [E] (routed, pre-drop = gate load), kept [E] = min(counts, C),
+ *   offsets [E+1] exclusive prefix sum of kept (offsets[E] = R),
+ *   row_token [T*k] (first R entries: token of each kept row),
+ *   slot_row [T][k] (row of each assignment, -1 if dropped),
+ *   x_perm [T*k][d] (dtype; first R rows: x of row_token, grouped by expert).
+ * topk_idx entries outside [0,E) are dropped and set MOE_ERR_DEVICE_BADINDEX. */
+int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx,
+                 void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
+                 int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
+
+/* a3. First half of every expert's SwiGLU FFN on its kept rows
+ * ["LLaMA-MoE v2", code sample, class Expert: down(silu(gate(x)) * up(x))]:
+ *   h[r] = silu(x_perm[r] W1_e^T) * (x_perm[r] W3_e^T) for rows r in
+ *   [offsets[e], offsets[e+1]).  x_perm [T*k][d], W13_e packed, h [T*k][m8].
+ * bf16: tcgen05 tensor cores, f32 accumulate, h rounded to bf16.
+ * f32: CUDA-core FMA in f32 (no TF32).  Row tables stay on the device. */
+int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
+                  const void *W13_e, void *h, void *ws, size_t ws_bytes, void *stream);
+
+/* a4. Second half: out[r] = h[r] W2_e^T.  h [T*k][m8], W2_e packed, out [T*k][d]. */
+int moe_expert_down(const moe_params_t *p, const void *h, const int32_t *offsets,
+                    const void *W2_e, void *out, void *ws, size_t ws_bytes, void *stream);
+
+/* a3 then a4. */
+int moe_expert_ffn(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
+                   const void *W13_e, const void *W2_e, void *h, void *out, void *ws,
+                   size_t ws_bytes, void *stream);
+
+/* a5. Combine ["Llama 3 Meets MoE", section 3; "LLaMA-MoE v2", rescale]:
+ *   y[t] = s * sum_{j<k, slot_row[t][j] >= 0} topk_w[t][j] * out[slot_row[t][j]],
+ * summed in slot order in f32; s = E/k if p->rescale else 1.  A token whose
+ * slots were all dropped gets y = 0.  out [T*k][d], y [T][d] (dtype). */
+int moe_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
+                const float *topk_w, void *y, void *stream);
+
+/* a6. Gate statistics ["LLaMA-MoE v2", section "门控机制设计"]:
+ *   f[e] = counts[e] / (T k),  P[e] = probs_sum[e] / T,
+ *   loss[0] = lambda * sum_e f[e] P[e]   (all f32 device outputs; T = 0 gives 0). */
+int moe_gate_stats(const moe_params_t *p, const int32_t *counts, const float *probs_sum,
+                   float *f, float *P, float *loss, void *stream);
+
+/* Every buffer moe_forward touches (device pointers, caller-owned). */
+typedef struct {
+    /* inputs */
+    const void *x;          /* [T][d] */
+    const void *Wg;         /* [d][E] */
+    const void *Wnoise;     /* [d][E] or NULL */
+    const float *noise;     /* [T][E] or NULL */
+    const float *bias;      /* [E] or NULL */
+    const void *W13_e;      /* packed */
+    const void *W2_e;       /* packed */
+    /* outputs */
+    void *y;                /* [T][d] */
+    float *loss;            /* [1] L_balance */
+    int32_t *counts;        /* [E] gate load (pre-drop) */
+    float *importance;      /* [E] gate importance */
+    float *f;               /* [E] */
+    float *P;               /* [E] */
+    /* intermediates (kept for inspection) */
+    int32_t *topk_idx;      /* [T][k] */
+    float *topk_w;          /* [T][k] */
+    float *probs_sum;       /* [E] */
+    void *x_perm;           /* [T*k][d] */
+    int32_t *row_token;     /* [T*k] */
+    int32_t *slot_row;      /* [T][k] */
+    int32_t *kept;          /* [E] */
+    int32_t *offsets;       /* [E+1] */
+    void *h;                /* [T*k][m8] */
+    void *out;              /* [T*k][d] */
+} moe_buffers_t;
+
+/* a1 -> a2 -> a3 -> a4 -> a5 -> a6 on one stream, no host synchronisation. */
+int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t ws_bytes,
+                void *stream);
+
+/* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
+ * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards. */
+int moe_get_device_status(void *ws, int32_t *status, int32_t clear, void *stream);
+
+/* Time limit, in nanoseconds, of every bounded wait inside the kernels that
+ * launch after this call (default 2e9).  0 makes every such wait give up at its
+ * first check, which exercises the timeout path; tests use it.  Host-only. */
+void moe_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,132 @@
+"""The C ABI without a GPU: libmoe.so loads, exports every function include/moe.h
+declares, its host-only helpers agree with the oracle, and argument validation
+rejects bad calls before anything reaches the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import oracle
+import top_routing_grouped_noisy_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    return moe.lib()
+
+
+def test_library_exports_every_declared_function(L):
+    names = _declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(L, n), "libmoe.so does not export %s" % n
+    assert len(L.moe_version()) > 0
+
+
+def test_binding_wraps_every_declared_function():
+    src = open(os.path.join(ROOT, "top_routing_grouped_noisy_b200", "__init__.py")).read()
+    for n in _declared_functions():
+        assert '"%s"' % n in src, "binding has no signature for %s" % n
+
+
+@pytest.mark.parametrize("T,E,cf", [(32768, 8, 1.0), (32768, 8, 4.0), (10, 3, 1.0),
+                                    (16384, 16, 1.25), (7, 8, 0.5), (100, 8, -1.0), (0, 4, 2.0)])
+def test_capacity_matches_oracle(T, E, cf):
+    assert moe.moe_capacity(T, E, cf) == oracle.capacity(T, E, cf)
+
+
+def test_layout_helpers():
+    assert moe.packed_w13_elems(8, 1376, 4096) == 8 * 2 * 1376 * 4096
+    assert moe.packed_w13_elems(8, 100, 64) == 8 * 2 * 112 * 64
+    assert moe.packed_w2_elems(8, 100, 64) == 8 * 64 * 104
+    assert moe.h_ld(1376) == 1376 and moe.h_ld(172) == 176
+    assert moe.packed_w13_elems(0, 1, 1) == 0
+
+
+def test_workspace_size_and_invalid_params():
+    p = moe.params(16384, 4096, 8, 2, 1376)
+    assert moe.moe_workspace_size(p) > 0
+    bigger = moe.params(32768, 4096, 8, 2, 1376)
+    assert moe.moe_workspace_size(bigger) >= moe.moe_workspace_size(p)
+    for bad in (moe.params(16, 4096, 8, 9, 1376), moe.params(16, 4096, 65, 2, 1376),
+                moe.params(16, 100, 8, 2, 1376), moe.params(-1, 64, 8, 2, 16),
+                moe.params(16, 64, 8, 0, 16), moe.params(16, 64, 8, 2, 0)):
+        assert moe.moe_workspace_size(bad) == 0
+
+
+def _fake(addr=1 << 20):
+    return C.c_void_p(addr)
+
+
+def test_validation_codes_without_touching_the_device(L):
+    """Every one of these returns before any CUDA call is made."""
+    P = moe.params(64, 64, 8, 2, 16)
+    f = [_fake(0x100000 + 256 * i) for i in range(12)]
+    ws_bytes = moe.moe_workspace_size(P)
+    # NULL params
+    assert L.moe_route(None, *f[:10], ws_bytes, None) == moe.MOE_ERR_INVALID_ARG
+    # k > E
+    bad = moe.params(64, 64, 4, 5, 16)
+    assert L.moe_route(C.byref(bad), *f[:10], ws_bytes, None) == moe.MOE_ERR_INVALID_ARG
+    assert b"k=5" in L.moe_last_error_string()
+    # d not a multiple of 8
+    bad = moe.params(64, 60, 8, 2, 16)
+    assert L.moe_dispatch(C.byref(bad), *f[:9], ws_bytes, None) == moe.MOE_ERR_SHAPE
+    # bad dtype
+    bad = moe.params(64, 64, 8, 2, 16, dtype=7)
+    assert L.moe_combine(C.byref(bad), *f[:4], None) == moe.MOE_ERR_DTYPE
+    # misaligned pointer
+    mis = list(f[:10])
+    mis[0] = _fake(0x100008)
+    assert L.moe_route(C.byref(P), *mis, ws_bytes, None) == moe.MOE_ERR_ALIGN
+    assert b"'x'" in L.moe_last_error_string()
+    # NULL required output
+    nul = list(f[:10])
+    nul[8] = None
+    assert L.moe_route(C.byref(P), *nul, ws_bytes, None) == moe.MOE_ERR_INVALID_ARG
+    # noise projection without the noise draws
+    nn = list(f[:10])
+    nn[3] = None
+    assert L.moe_route(C.byref(P), *nn, ws_bytes, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_route(C.byref(P), *f[:10], ws_bytes - 1, None) == moe.MOE_ERR_WORKSPACE
+    # partition: d_ff not divisible by E, missing perm, bad mode
+    assert L.moe_partition_experts(*f[:3], 64, 100, 8, moe.DISJOINT, f[3], moe.MOE_BF16,
+                                   f[4], f[5], None, None) == moe.MOE_ERR_SHAPE
+    assert L.moe_partition_experts(*f[:3], 64, 128, 8, moe.DISJOINT, None, moe.MOE_BF16,
+                                   f[4], f[5], None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_partition_experts(*f[:3], 64, 128, 8, 9, None, moe.MOE_BF16,
+                                   f[4], f[5], None, None) == moe.MOE_ERR_INVALID_ARG
+    # status readback with NULL output
+    assert L.moe_get_device_status(f[0], None, 0, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_needs_no_token_buffers(L):
+    """T = 0: token-sized buffers may be NULL; the expert GEMMs and the combine return
+    at once without launching anything."""
+    P = moe.params(0, 64, 8, 2, 16)
+    ws_bytes = moe.moe_workspace_size(P)
+    off, w, ws = _fake(0x200000), _fake(0x300000), _fake(0x400000)
+    before = moe.moe_launch_count()
+    assert L.moe_expert_up(C.byref(P), None, off, w, None, ws, ws_bytes, None) == moe.MOE_OK
+    assert L.moe_expert_down(C.byref(P), None, off, w, None, ws, ws_bytes, None) == moe.MOE_OK
+    assert L.moe_combine(C.byref(P), None, None, None, None, None) == moe.MOE_OK
+    assert moe.moe_launch_count() == before
+
+
+def test_wait_limit_setter_is_host_only(L):
+    moe.moe_set_wait_limit_ns(123)
+    moe.moe_set_wait_limit_ns(2_000_000_000)

@@ -1,0 +1,217 @@
+"""GPU parity of every step of the layer against the fp64 oracle, through the C ABI.
+
+Small cases span several 128x256 tensor-core tiles with ragged row, column and K
+tails; the full-size cases run the workloads the benchmark times, in the same
+launch configuration, and compare routing and dispatch on every token and the
+layer output on a seeded sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import harness as H
+import oracle
+import top_routing_grouped_noisy_b200 as moe
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+W = wl.Workload
+SMALL = {
+    "mid_mixtral_noisy": W("mid_mixtral_noisy", T=1000, d=512, d_ff=2752, E=8, k=2, noisy=True,
+                           rescale=True, seed=11),
+    "mid_st_bias_cap": W("mid_st_bias_cap", T=700, d=256, d_ff=1024, E=16, k=4, router=wl.ST,
+                         noisy=True, bias=True, rescale=True, cf=1.0, seed=12),
+    "e64_k8": W("e64_k8", T=300, d=128, d_ff=1024, E=64, k=8, noisy=True, seed=13),
+    "e32_st": W("e32_st", T=500, d=256, d_ff=768, E=32, k=3, router=wl.ST, noisy=True, seed=14),
+    "odd_m_d": W("odd_m_d", T=333, d=200, d_ff=800, E=8, k=2, seed=15),
+    "copy_perturbed_cf1": W("copy_perturbed_cf1", T=600, d=256, d_ff=384, E=4, k=2, cf=1.0,
+                            partition=wl.COPY, perturb=1e-3, seed=16),
+    "copy_exact": W("copy_exact", T=256, d=128, d_ff=256, E=4, k=2, partition=wl.COPY,
+                    seed=17),
+    "single_expert": W("single_expert", T=100, d=64, d_ff=64, E=1, k=1, rescale=True, seed=18),
+    "k_eq_E": W("k_eq_E", T=128, d=64, d_ff=128, E=4, k=4, seed=19),
+    "one_token": W("one_token", T=1, d=256, d_ff=512, E=8, k=2, noisy=True, seed=20),
+    "tiny_cap": W("tiny_cap", T=200, d=64, d_ff=256, E=8, k=2, cf=0.25, seed=21),
+    "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
+                          router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
+    "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",
+                    noisy=True, rescale=True, seed=23),
+}
+
+
+def _G_atol(w):
+    return 1e-5 if w.dtype == "f32" else 5e-5
+
+
+def _full_check(w, inp, rows_sample=None, tok_sample=None, capacity=None):
+    p, bufs, ws, status, weights = H.run_forward(w, inp, capacity=capacity)
+    assert status == 0, "device status %d" % status
+    r, ties = H.check_routing(w, inp, bufs, _G_atol(w))
+    dsp = H.check_dispatch(w, inp, p, bufs)
+    OW = H.oracle_weights(w, inp)
+    rows = None
+    if rows_sample is not None and dsp["R"] > rows_sample:
+        rows = np.sort(np.random.default_rng(w.seed).choice(dsp["R"], rows_sample, replace=False))
+    H.check_expert_rows(w, bufs, dsp, OW, rows)
+    good = np.nonzero(~ties)[0]
+    if tok_sample is not None and len(good) > tok_sample:
+        good = np.sort(np.random.default_rng(w.seed + 1).choice(good, tok_sample, replace=False))
+    e = H.check_y(w, bufs, r, dsp, OW, good)
+    H.check_loss(w, bufs, r)
+    return dict(p=p, bufs=bufs, ws=ws, r=r, ties=ties, dsp=dsp, y_err=e, weights=weights)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_parity_small(name):
+    w = SMALL[name]
+    inp = wl.make_inputs(w)
+    _full_check(w, inp)
+
+
+def test_tiny_fp32_workload_full():
+    w = wl.WORKLOADS["tiny_fp32"]
+    inp = wl.make_inputs(w)
+    res = _full_check(w, inp)
+    assert res["y_err"] <= 1e-5
+
+
+@pytest.mark.parametrize("mode", ["disjoint_bf16", "copy_f32", "stacked_bf16", "odd_m"])
+def test_partition_parity(mode):
+    if mode == "disjoint_bf16":
+        w = W("p", T=1, d=128, d_ff=1024, E=8, k=2, seed=31)
+    elif mode == "copy_f32":
+        w = W("p", T=1, d=64, d_ff=96, E=4, k=2, dtype="f32", partition=wl.COPY, seed=32)
+    elif mode == "stacked_bf16":
+        w = W("p", T=1, d=64, d_ff=80, E=3, k=2, partition=wl.COPY, perturb=1e-2, seed=33)
+    else:
+        w = W("p", T=1, d=40, d_ff=8 * 13, E=8, k=2, seed=34)  # m = 13
+    inp = wl.make_inputs(w)
+    W13_e, W2_e = H.gpu_weights(w, inp)
+    torch.cuda.synchronize()
+    W1e, W3e, W2e = H.oracle_weights(w, inp)
+    g1, g3 = H.unpack_w13(W13_e, w.E, w.m, w.d)
+    g2 = H.unpack_w2(W2_e, w.E, w.m, w.d)
+    np.testing.assert_array_equal(H.raw(g1.contiguous()), W1e)
+    np.testing.assert_array_equal(H.raw(g3.contiguous()), W3e)
+    np.testing.assert_array_equal(H.raw(g2.contiguous()), W2e)
+    # padding rows/columns are zero
+    m16, m8 = (w.m + 15) // 16 * 16, (w.m + 7) // 8 * 8
+    full = W13_e.view(w.E, m16 // 16, 2, 16, w.d)
+    gate_all = full[:, :, 0].reshape(w.E, m16, w.d)
+    assert not gate_all[:, w.m:].float().abs().sum()
+    assert not W2_e.view(w.E, w.d, m8)[:, :, w.m:].float().abs().sum()
+
+
+def test_steps_reproduce_forward_bit_exactly():
+    """The six step calls give the same bytes as moe_forward, and reruns are identical."""
+    w = SMALL["mid_st_bias_cap"]
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, (W13_e, W2_e) = H.run_forward(w, inp)
+    dev = "cuda"
+    b2 = moe.ForwardBuffers(p)
+    x, Wg, Wn, eps, bias = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps", "bias"))
+    moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b2.topk_idx, b2.topk_w, b2.probs_sum,
+                  b2.importance)
+    moe.moe_dispatch(p, x, b2.topk_idx, ws, b2.x_perm, b2.row_token, b2.slot_row, b2.counts,
+                     b2.kept, b2.offsets)
+    moe.moe_expert_up(p, b2.x_perm, b2.offsets, W13_e, b2.h, ws)
+    moe.moe_expert_down(p, b2.h, b2.offsets, W2_e, b2.out, ws)
+    moe.moe_combine(p, b2.out, b2.slot_row, b2.topk_w, b2.y)
+    moe.moe_gate_stats(p, b2.counts, b2.probs_sum, b2.f, b2.P, b2.loss)
+    torch.cuda.synchronize()
+    R = int(bufs.offsets[-1])
+    for n in ("y", "topk_idx", "topk_w", "probs_sum", "importance", "counts", "kept",
+              "offsets", "slot_row", "loss", "f", "P"):
+        assert torch.equal(getattr(bufs, n), getattr(b2, n)), n
+    assert torch.equal(bufs.out[:R], b2.out[:R])
+    assert torch.equal(bufs.row_token[:R], b2.row_token[:R])
+
+
+def test_empty_batch():
+    w = W("empty", T=0, d=64, d_ff=128, E=4, k=2, noisy=True, seed=40)
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, _ = H.run_forward(w, inp)
+    assert status == 0
+    assert bufs.counts.tolist() == [0] * 4 and bufs.offsets.tolist() == [0] * 5
+    assert bufs.probs_sum.abs().sum().item() == 0 and float(bufs.loss[0]) == 0.0
+
+
+def test_capacity_zero_drops_everything():
+    w = W("cap0", T=77, d=64, d_ff=128, E=4, k=2, seed=41)
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, _ = H.run_forward(w, inp, capacity=0)
+    assert status == 0
+    assert bufs.kept.tolist() == [0] * 4 and int(bufs.offsets[-1]) == 0
+    assert (bufs.slot_row == -1).all()
+    assert bufs.y.float().abs().sum().item() == 0.0
+    assert bufs.counts.sum().item() == 77 * 2
+
+
+def test_nan_input_sets_badindex_status():
+    w = W("nan", T=64, d=64, d_ff=128, E=4, k=2, seed=42)
+    inp = wl.make_inputs(w)
+    inp["x"][5, 3] = float("nan")
+    p, bufs, ws, status, _ = H.run_forward(w, inp)
+    assert status == moe.MOE_ERR_DEVICE_BADINDEX
+    assert (bufs.topk_idx[5] == -1).all() and (bufs.slot_row[5] == -1).all()
+    assert moe.moe_get_device_status(ws) == 0  # cleared by the previous read
+
+
+def test_out_of_range_index_is_dropped_and_reported():
+    w = W("badidx", T=40, d=64, d_ff=128, E=4, k=2, seed=43)
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    b = moe.ForwardBuffers(p)
+    idx = torch.tensor([[0, 1]] * 40, dtype=torch.int32, device="cuda")
+    idx[3, 1] = 7
+    idx[9, 0] = -2
+    x = inp["x"].cuda()
+    moe.moe_dispatch(p, x, idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts, b.kept,
+                     b.offsets)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_DEVICE_BADINDEX
+    d = oracle.dispatch(idx.cpu().numpy(), 4, -1)
+    np.testing.assert_array_equal(b.slot_row.cpu().numpy(), d["slot_row"])
+    assert b.counts.tolist() == d["counts"].tolist()
+
+
+def test_dense_equivalence_on_gpu():
+    """All E disjoint experts at gate weight 1 (k = E fed through dispatch and the
+    expert GEMMs, combine weights 1, no rescale) reproduce the dense FFN."""
+    w = W("dense", T=200, d=256, d_ff=1024, E=8, k=8, seed=44)
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    W13_e, W2_e = H.gpu_weights(w, inp, ws)
+    b = moe.ForwardBuffers(p)
+    x = inp["x"].cuda()
+    idx = torch.arange(8, dtype=torch.int32, device="cuda").repeat(w.T, 1).contiguous()
+    ones = torch.ones(w.T, 8, dtype=torch.float32, device="cuda")
+    moe.moe_dispatch(p, x, idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts, b.kept,
+                     b.offsets)
+    moe.moe_expert_ffn(p, b.x_perm, b.offsets, W13_e, W2_e, b.h, b.out, ws)
+    moe.moe_combine(p, b.out, b.slot_row, ones, b.y)
+    torch.cuda.synchronize()
+    dense = oracle.dense_ffn(H.raw(inp["W1"]), H.raw(inp["W3"]), H.raw(inp["W2"]),
+                             H.raw(inp["x"]))
+    assert H.rel_err(H.f64(b.y), dense) <= 1e-2
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+FULL = ["tiny_fp32", "moe_2of8", "moe_4of16", "e8t2_cf1", "e8t2_cf4"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(name):
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w, device="cuda")
+    big = w.name.startswith("e8t2")
+    res = _full_check(w, inp, rows_sample=64 if big else 256, tok_sample=32 if big else 128)
+    if w.cf >= 0:
+        C = moe.moe_capacity(w.T, w.E, w.cf)
+        assert C == oracle.capacity(w.T, w.E, w.cf)
+        assert (res["bufs"].kept.cpu() <= C).all()

@@ -1,0 +1,295 @@
+"""Python binding of libmoe.so, the B200 (sm_100a) forward pass of a sparse
+Mixture-of-Experts SwiGLU FFN layer (noisy Top-K routing, capacity dispatch,
+grouped expert GEMMs on tcgen05 tensor cores, gate-weighted combine).
+
+The functions mirror the C ABI in ``include/moe.h`` one to one and only marshal
+arguments: torch tensors are passed as device pointers together with torch's
+current CUDA stream; every step of the layer runs in the library's kernels.
+PyTorch provides device memory and streams only.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+import ctypes as C
+import os
+
+import torch
+
+__all__ = [
+    "MoeError", "Params", "lib", "params", "moe_capacity", "moe_version", "moe_launch_count",
+    "moe_partition_experts", "moe_workspace_size", "Workspace", "moe_route", "moe_dispatch",
+    "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
+    "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
+    "packed_w13_elems", "packed_w2_elems", "h_ld",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_SHAPE = -2
+MOE_ERR_ALIGN = -3
+MOE_ERR_DTYPE = -4
+MOE_ERR_CUDA = -5
+MOE_ERR_DEVICE_TIMEOUT = -6
+MOE_ERR_DEVICE_BADINDEX = -7
+MOE_ERR_WORKSPACE = -8
+MOE_ERR_UNSUPPORTED = -9
+
+MOE_F32 = 0
+MOE_BF16 = 1
+MIXTRAL = 0
+ST = 1
+DISJOINT = 0
+COPY = 1
+STACKED = 2
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("libmoe error %d: %s" % (code, msg))
+        self.code = code
+
+
+class Params(C.Structure):
+    _fields_ = [("T", C.c_int32), ("d", C.c_int32), ("E", C.c_int32), ("k", C.c_int32),
+                ("m", C.c_int32), ("dtype", C.c_int32), ("router_type", C.c_int32),
+                ("capacity", C.c_int32), ("rescale", C.c_int32), ("balance_lambda", C.c_float)]
+
+
+_BUF_FIELDS = ["x", "Wg", "Wnoise", "noise", "bias", "W13_e", "W2_e", "y", "loss", "counts",
+               "importance", "f", "P", "topk_idx", "topk_w", "probs_sum", "x_perm", "row_token",
+               "slot_row", "kept", "offsets", "h", "out"]
+
+
+class _Buffers(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in _BUF_FIELDS]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmoe.so (raises ImportError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libmoe.so not found at %s; build it with "
+                              "`python -m top_routing_grouped_noisy_b200.build`" % LIB_PATH)
+        L = C.CDLL(LIB_PATH)
+        v, i32, i64, sz, f64 = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_double
+        P = C.POINTER(Params)
+        sig = {
+            "moe_version": (C.c_char_p, []),
+            "moe_last_error_string": (C.c_char_p, []),
+            "moe_launch_count": (C.c_uint64, []),
+            "moe_set_wait_limit_ns": (None, [C.c_uint64]),
+            "moe_capacity": (i32, [i32, i32, f64]),
+            "moe_packed_w13_elems": (i64, [i32, i32, i32]),
+            "moe_packed_w2_elems": (i64, [i32, i32, i32]),
+            "moe_h_ld": (i32, [i32]),
+            "moe_partition_experts": (C.c_int, [v, v, v, i32, i32, i32, i32, v, i32, v, v, v, v]),
+            "moe_workspace_size": (sz, [P]),
+            "moe_workspace_init": (C.c_int, [v, sz, v]),
+            "moe_route": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v, sz, v]),
+            "moe_dispatch": (C.c_int, [P, v, v, v, v, v, v, v, v, v, sz, v]),
+            "moe_expert_up": (C.c_int, [P, v, v, v, v, v, sz, v]),
+            "moe_expert_down": (C.c_int, [P, v, v, v, v, v, sz, v]),
+            "moe_expert_ffn": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
+            "moe_combine": (C.c_int, [P, v, v, v, v, v]),
+            "moe_gate_stats": (C.c_int, [P, v, v, v, v, v, v]),
+            "moe_forward": (C.c_int, [P, C.POINTER(_Buffers), v, sz, v]),
+            "moe_get_device_status": (C.c_int, [v, C.POINTER(i32), i32, v]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != MOE_OK:
+        raise MoeError(rc, lib().moe_last_error_string().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor, got %r" % type(t))
+    if not t.is_cuda:
+        raise ValueError("libmoe takes CUDA tensors (got a %s tensor)" % t.device)
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return t.data_ptr() or None
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(dt):
+    if dt == torch.bfloat16:
+        return MOE_BF16
+    if dt == torch.float32:
+        return MOE_F32
+    raise TypeError("libmoe computes in bf16 or f32, not %s" % dt)
+
+
+def moe_version() -> str:
+    return lib().moe_version().decode()
+
+
+def moe_launch_count() -> int:
+    return int(lib().moe_launch_count())
+
+
+def moe_set_wait_limit_ns(ns: int) -> None:
+    lib().moe_set_wait_limit_ns(int(ns))
+
+
+def moe_capacity(T: int, E: int, cf: float) -> int:
+    return int(lib().moe_capacity(T, E, float(cf)))
+
+
+def packed_w13_elems(E, m, d):
+    return int(lib().moe_packed_w13_elems(E, m, d))
+
+
+def packed_w2_elems(E, m, d):
+    return int(lib().moe_packed_w2_elems(E, m, d))
+
+
+def h_ld(m):
+    return int(lib().moe_h_ld(m))
+
+
+def params(T, d, E, k, m, dtype=torch.bfloat16, router_type=MIXTRAL, capacity=-1,
+           rescale=False, balance_lambda=0.0) -> Params:
+    return Params(T, d, E, k, m, _dtype_code(dtype) if isinstance(dtype, torch.dtype) else dtype,
+                  router_type, capacity, 1 if rescale else 0, balance_lambda)
+
+
+def moe_workspace_size(p: Params) -> int:
+    return int(lib().moe_workspace_size(C.byref(p)))
+
+
+class Workspace:
+    """Caller-owned scratch for the library (a zeroed torch uint8 buffer)."""
+
+    def __init__(self, p: Params, device=None, nbytes=None):
+        n = nbytes if nbytes is not None else moe_workspace_size(p)
+        if n <= 0:
+            raise MoeError(MOE_ERR_INVALID_ARG, "invalid parameters for the workspace")
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        self.nbytes = n
+        _check(lib().moe_workspace_init(_p(self.buf), n, _stream()))
+
+    @property
+    def ptr(self):
+        return self.buf.data_ptr()
+
+
+def moe_get_device_status(ws: Workspace, clear=True, stream=None) -> int:
+    st = C.c_int32(0)
+    _check(lib().moe_get_device_status(ws.ptr, C.byref(st), 1 if clear else 0, _stream(stream)))
+    return st.value
+
+
+def moe_partition_experts(W1, W3, W2, E, mode=DISJOINT, perm=None, ws=None, out=None,
+                          stream=None):
+    """a0: packed expert weights (W13_e, W2_e) from a dense FFN (or stacked experts)."""
+    dt = _dtype_code(W1.dtype)
+    if mode == STACKED:
+        d_ff, d = W1.shape[1], W1.shape[2]
+    else:
+        d_ff, d = W1.shape
+    m = d_ff // E if mode == DISJOINT else d_ff
+    if out is None:
+        W13_e = torch.empty(packed_w13_elems(E, m, d), dtype=W1.dtype, device=W1.device)
+        W2_e = torch.empty(packed_w2_elems(E, m, d), dtype=W1.dtype, device=W1.device)
+    else:
+        W13_e, W2_e = out
+    _check(lib().moe_partition_experts(_p(W1), _p(W3), _p(W2), d, d_ff, E, mode, _p(perm), dt,
+                                       _p(W13_e), _p(W2_e), ws.ptr if ws is not None else None,
+                                       _stream(stream)))
+    return W13_e, W2_e
+
+
+def moe_route(p, x, Wg, Wnoise, noise, bias, ws, topk_idx, topk_w, probs_sum, importance,
+              stream=None):
+    _check(lib().moe_route(C.byref(p), _p(x), _p(Wg), _p(Wnoise), _p(noise), _p(bias),
+                           _p(topk_idx), _p(topk_w), _p(probs_sum), _p(importance), ws.ptr,
+                           ws.nbytes, _stream(stream)))
+
+
+def moe_dispatch(p, x, topk_idx, ws, x_perm, row_token, slot_row, counts, kept, offsets,
+                 stream=None):
+    _check(lib().moe_dispatch(C.byref(p), _p(x), _p(topk_idx), _p(x_perm), _p(row_token),
+                              _p(slot_row), _p(counts), _p(kept), _p(offsets), ws.ptr,
+                              ws.nbytes, _stream(stream)))
+
+
+def moe_expert_up(p, x_perm, offsets, W13_e, h, ws, stream=None):
+    _check(lib().moe_expert_up(C.byref(p), _p(x_perm), _p(offsets), _p(W13_e), _p(h), ws.ptr,
+                               ws.nbytes, _stream(stream)))
+
+
+def moe_expert_down(p, h, offsets, W2_e, out, ws, stream=None):
+    _check(lib().moe_expert_down(C.byref(p), _p(h), _p(offsets), _p(W2_e), _p(out), ws.ptr,
+                                 ws.nbytes, _stream(stream)))
+
+
+def moe_expert_ffn(p, x_perm, offsets, W13_e, W2_e, h, out, ws, stream=None):
+    _check(lib().moe_expert_ffn(C.byref(p), _p(x_perm), _p(offsets), _p(W13_e), _p(W2_e), _p(h),
+                                _p(out), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def moe_combine(p, out, slot_row, topk_w, y, stream=None):
+    _check(lib().moe_combine(C.byref(p), _p(out), _p(slot_row), _p(topk_w), _p(y),
+                             _stream(stream)))
+
+
+def moe_gate_stats(p, counts, probs_sum, f, P, loss, stream=None):
+    _check(lib().moe_gate_stats(C.byref(p), _p(counts), _p(probs_sum), _p(f), _p(P), _p(loss),
+                                _stream(stream)))
+
+
+class ForwardBuffers:
+    """Every intermediate and output tensor of one layer forward, allocated with torch."""
+
+    def __init__(self, p: Params, device="cuda"):
+        dt = torch.bfloat16 if p.dtype == MOE_BF16 else torch.float32
+        T, d, E, k = p.T, p.d, p.E, p.k
+        rows = max(T * k, 1)
+        i32 = dict(dtype=torch.int32, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.y = torch.empty(max(T, 1), d, dtype=dt, device=device)[:T]
+        self.loss = torch.empty(1, **f32)
+        self.counts = torch.empty(E, **i32)
+        self.importance = torch.empty(E, **f32)
+        self.f = torch.empty(E, **f32)
+        self.P = torch.empty(E, **f32)
+        self.topk_idx = torch.empty(max(T, 1), k, **i32)[:T]
+        self.topk_w = torch.empty(max(T, 1), k, **f32)[:T]
+        self.probs_sum = torch.empty(E, **f32)
+        self.x_perm = torch.empty(rows, d, dtype=dt, device=device)
+        self.row_token = torch.empty(rows, **i32)
+        self.slot_row = torch.empty(max(T, 1), k, **i32)[:T]
+        self.kept = torch.empty(E, **i32)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.h = torch.empty(rows, h_ld(p.m), dtype=dt, device=device)
+        self.out = torch.empty(rows, d, dtype=dt, device=device)
+
+
+def moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs: ForwardBuffers, Wnoise=None, noise=None,
+                bias=None, stream=None):
+    b = _Buffers()
+    vals = dict(x=x, Wg=Wg, Wnoise=Wnoise, noise=noise, bias=bias, W13_e=W13_e, W2_e=W2_e)
+    for n in _BUF_FIELDS:
+        t = vals[n] if n in vals else getattr(bufs, n)
+        setattr(b, n, _p(t))
+    _check(lib().moe_forward(C.byref(p), C.byref(b), ws.ptr, ws.nbytes, _stream(stream)))
+    return bufs

@@ -1,0 +1,117 @@
+// combine.cu -- a5: gate-weighted combine and a6: gate statistics.
+//
+// a5 ("Llama 3 Meets MoE: Efficient Upcycling", section 3: y = sum_i G(x)_i E_i(x);
+// "LLaMA-MoE v2", section "重新缩放机制与负载均衡": y = N/k sum_i G(x)_i E_i(x)):
+//   y[t] = s * sum_{j<k, kept} G[t][j] * out[slot_row[t][j]]
+// in the gather form (one writer per output element, slot order, f32 accumulate),
+// so it needs no atomics and is bit-reproducible.  16-byte loads and stores.
+//
+// a6 ("LLaMA-MoE v2", section "门控机制设计": L_balance = lambda sum_i f_i P_i):
+//   f[e] = counts[e] / (T k), P[e] = probs_sum[e] / T.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+template <typename E_T>
+__global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ out,
+                                                      const int32_t *__restrict__ slot_row,
+                                                      const float *__restrict__ w, int T, int d,
+                                                      int k, float scale, E_T *__restrict__ y)
+{
+    constexpr int VN = Vec<E_T>::N;
+    const int nv = d / VN;
+    const int64_t items = (int64_t)T * nv;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / nv;
+        const int v = (int)(i - t * nv);
+        float acc[VN];
+#pragma unroll
+        for (int q = 0; q < VN; ++q)
+            acc[q] = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int32_t row = slot_row[t * k + j];
+            if (row < 0)
+                continue;
+            const float g = w[t * k + j];
+            const uint4 raw = ld_nc_na(out + (int64_t)row * d + (int64_t)v * VN);
+            float f[VN];
+            if constexpr (sizeof(E_T) == 2) {
+                bf16x8_to_f32(raw, f);
+            } else {
+                f[0] = __uint_as_float(raw.x);
+                f[1] = __uint_as_float(raw.y);
+                f[2] = __uint_as_float(raw.z);
+                f[3] = __uint_as_float(raw.w);
+            }
+#pragma unroll
+            for (int q = 0; q < VN; ++q)
+                acc[q] = fmaf(g, f[q], acc[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < VN; ++q)
+            acc[q] *= scale;
+        uint4 o;
+        if constexpr (sizeof(E_T) == 2) {
+            o = f32x8_to_bf16(acc);
+        } else {
+            o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
+                           __float_as_uint(acc[2]), __float_as_uint(acc[3]));
+        }
+        st_v4(y + t * d + (int64_t)v * VN, o);
+    }
+}
+
+__global__ void gate_stats_kernel(const int32_t *__restrict__ counts,
+                                  const float *__restrict__ probs_sum, int T, int E, int k,
+                                  float lambda, float *__restrict__ f, float *__restrict__ P,
+                                  float *__restrict__ loss)
+{
+    __shared__ double s_fp[MOE_MAX_EXPERTS];
+    const int e = threadIdx.x;
+    if (e < E) {
+        const double fe = T > 0 ? (double)counts[e] / ((double)T * k) : 0.0;
+        const double pe = T > 0 ? (double)probs_sum[e] / (double)T : 0.0;
+        f[e] = (float)fe;
+        P[e] = (float)pe;
+        s_fp[e] = fe * pe;
+    }
+    __syncthreads();
+    if (e == 0) {
+        double s = 0.0;
+        for (int i = 0; i < E; ++i)
+            s += s_fp[i];
+        loss[0] = (float)(lambda * s);
+    }
+}
+
+cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
+                           const float *w, void *y, cudaStream_t s)
+{
+    const float scale = p->rescale ? (float)p->E / (float)p->k : 1.0f;
+    const int VN = p->dtype == MOE_BF16 ? 8 : 4;
+    const int64_t items = (int64_t)p->T * (p->d / VN);
+    const int64_t blocks = (items + 255) / 256;
+    const unsigned grid = (unsigned)(blocks < (1 << 30) ? blocks : (1 << 30));
+    if (p->dtype == MOE_BF16)
+        combine_kernel<bf16><<<grid, 256, 0, s>>>((const bf16 *)out, slot_row, w, p->T, p->d,
+                                                  p->k, scale, (bf16 *)y);
+    else
+        combine_kernel<float><<<grid, 256, 0, s>>>((const float *)out, slot_row, w, p->T, p->d,
+                                                   p->k, scale, (float *)y);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_stats(const moe_params_t *p, const int32_t *counts,
+                              const float *probs_sum, float *f, float *P, float *loss,
+                              cudaStream_t s)
+{
+    gate_stats_kernel<<<1, MOE_MAX_EXPERTS, 0, s>>>(counts, probs_sum, p->T, p->E, p->k,
+                                                    p->balance_lambda, f, P, loss);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,94 @@
+// common.cuh -- helpers shared by the kernels of libmoe.so (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libmoe targets sm_100a (B200) only"
+#endif
+
+namespace moe {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- workspace
+// The first 256 bytes of the caller's workspace are a header; word 0 is the
+// device status word (0 or a MOE_ERR_DEVICE_* code; the first error sticks).
+constexpr size_t kWsHeader = 256;
+
+__device__ __forceinline__ void set_status(int32_t *status, int32_t code)
+{
+    if (status != nullptr)
+        atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- element I/O
+template <typename T> struct Vec;  // 16-byte vector of T
+template <> struct Vec<float> {
+    static constexpr int N = 4;
+};
+template <> struct Vec<bf16> {
+    static constexpr int N = 8;
+};
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// 16-byte global loads.  nc: read-only path, no L1 allocation (streamed once).
+__device__ __forceinline__ uint4 ld_nc_na(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ uint4 ld_nc(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void st_v4(void *p, uint4 v)
+{
+    *reinterpret_cast<uint4 *>(p) = v;
+}
+
+// unpack 8 bf16 held in a uint4 to f32 / pack back
+__device__ __forceinline__ void bf16x8_to_f32(uint4 v, float *f)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float *f)
+{
+    uint4 v;
+    v.x = pack_bf16x2(f[0], f[1]);
+    v.y = pack_bf16x2(f[2], f[3]);
+    v.z = pack_bf16x2(f[4], f[5]);
+    v.w = pack_bf16x2(f[6], f[7]);
+    return v;
+}
+
+}  // namespace moe

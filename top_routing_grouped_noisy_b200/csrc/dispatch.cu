@@ -1,0 +1,178 @@
+// dispatch.cu -- a2: capacity-factor dispatch ("Llama 3 Meets MoE: Efficient
+// Upcycling", section 3 "容量因子": expert capacity = tokens per batch / N x CF;
+// overflow tokens are left out of the expert computation).
+//
+// A deterministic stable counting sort of the T*k (token, expert) assignments
+// by expert, token-ascending inside an expert.  An assignment is kept iff its
+// rank inside its expert is < C, so the lower token index wins.
+//
+//   scan kernel (one CTA): per 32-token chunk and expert, the number of tokens
+//     of the chunk routed to the expert (one warp ballot per expert), then an
+//     exclusive scan over chunks per expert -> the rank base of each chunk;
+//     counts, kept = min(counts, C), offsets = exclusive scan of kept.
+//   scatter kernel (one CTA per chunk): each assignment's rank = chunk base +
+//     ballot prefix inside the chunk; slot_row / row_token; then the chunk's x
+//     rows are read once (16-byte loads) and written to each kept row.
+// No atomics decide any output, so every output is bit-reproducible.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(
+    const int32_t *__restrict__ idx, int T, int k, int E, int C, int32_t *__restrict__ hist,
+    int32_t *__restrict__ counts, int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
+    int32_t *status)
+{
+    __shared__ int32_t s_count[MOE_MAX_EXPERTS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarp = blockDim.x >> 5;
+    const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
+    // phase 1: per-chunk histograms, hist[e][chunk]
+    for (int c = warp; c < nch; c += nwarp) {
+        const int64_t t = (int64_t)c * kDispatchChunk + lane;
+        int ej[MOE_MAX_TOPK];
+        for (int j = 0; j < k; ++j) {
+            int e = -1;
+            if (t < T) {
+                e = idx[t * k + j];
+                if (e < 0 || e >= E) {
+                    set_status(status, MOE_ERR_DEVICE_BADINDEX);
+                    e = -1;
+                }
+            }
+            ej[j] = e;
+        }
+        for (int e = 0; e < E; ++e) {
+            bool has = false;
+            for (int j = 0; j < k; ++j)
+                has |= ej[j] == e;
+            const unsigned b = __ballot_sync(0xffffffffu, has);
+            if (lane == 0)
+                hist[(int64_t)e * nch + c] = __popc(b);
+        }
+    }
+    __syncthreads();
+    // phase 2: exclusive scan over chunks, one warp per expert
+    for (int e = warp; e < E; e += nwarp) {
+        int32_t run = 0;
+        int32_t *h = hist + (int64_t)e * nch;
+        for (int base = 0; base < nch; base += 32) {
+            const int c = base + lane;
+            const int32_t v = c < nch ? h[c] : 0;
+            int32_t incl = v;
+#pragma unroll
+            for (int s = 1; s < 32; s <<= 1) {
+                const int32_t u = __shfl_up_sync(0xffffffffu, incl, s);
+                if (lane >= s)
+                    incl += u;
+            }
+            if (c < nch)
+                h[c] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0)
+            s_count[e] = run;
+    }
+    __syncthreads();
+    // phase 3: capacity clip and expert offsets
+    if (threadIdx.x == 0) {
+        int32_t off = 0;
+        offsets[0] = 0;
+        for (int e = 0; e < E; ++e) {
+            const int32_t cnt = s_count[e];
+            const int32_t kp = (C < 0 || cnt < C) ? cnt : C;
+            counts[e] = cnt;
+            kept[e] = kp;
+            off += kp;
+            offsets[e + 1] = off;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) dispatch_scatter_kernel(
+    const char *__restrict__ x, int64_t row_bytes, const int32_t *__restrict__ idx, int T, int k,
+    int E, const int32_t *__restrict__ hist, const int32_t *__restrict__ kept,
+    const int32_t *__restrict__ offsets, char *__restrict__ x_perm,
+    int32_t *__restrict__ row_token, int32_t *__restrict__ slot_row)
+{
+    __shared__ int32_t s_row[kDispatchChunk][MOE_MAX_TOPK];
+    const int c = blockIdx.x;
+    const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
+    const int64_t t0 = (int64_t)c * kDispatchChunk;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int64_t t = t0 + lane;
+        const unsigned lt = (1u << lane) - 1u;
+        int ej[MOE_MAX_TOPK], rowj[MOE_MAX_TOPK];
+        for (int j = 0; j < k; ++j) {
+            int e = -1;
+            if (t < T) {
+                e = idx[t * k + j];
+                if (e < 0 || e >= E)
+                    e = -1;  // reported by the scan kernel
+            }
+            ej[j] = e;
+            rowj[j] = -1;
+        }
+        for (int e = 0; e < E; ++e) {
+            bool has = false;
+            for (int j = 0; j < k; ++j)
+                has |= ej[j] == e;
+            const unsigned b = __ballot_sync(0xffffffffu, has);
+            if (has) {
+                const int32_t rank = hist[(int64_t)e * nch + c] + __popc(b & lt);
+                const int32_t row = rank < kept[e] ? offsets[e] + rank : -1;
+                for (int j = 0; j < k; ++j)
+                    if (ej[j] == e)
+                        rowj[j] = row;
+            }
+        }
+        for (int j = 0; j < k; ++j) {
+            s_row[lane][j] = rowj[j];
+            if (t < T) {
+                slot_row[t * k + j] = rowj[j];
+                if (rowj[j] >= 0)
+                    row_token[rowj[j]] = (int32_t)t;
+            }
+        }
+    }
+    __syncthreads();
+    const int ntok = (int)((int64_t)T - t0 < kDispatchChunk ? (int64_t)T - t0 : kDispatchChunk);
+    const int nv = (int)(row_bytes / 16);
+    const int items = ntok * nv;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < items; i += blockDim.x) {
+        const int l = i / nv, v = i - l * nv;
+        const uint4 val = ld_nc_na(x + (t0 + l) * row_bytes + (int64_t)v * 16);
+        for (int j = 0; j < k; ++j) {
+            const int32_t row = s_row[l][j];
+            if (row >= 0)
+                st_v4(x_perm + (int64_t)row * row_bytes + (int64_t)v * 16, val);
+        }
+    }
+}
+
+cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
+                            void *x_perm, int32_t *row_token, int32_t *slot_row,
+                            int32_t *counts, int32_t *kept, int32_t *offsets, char *ws,
+                            int32_t *status, cudaStream_t s)
+{
+    const WsLayout L = ws_layout(p);
+    int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
+    dispatch_scan_kernel<<<1, 1024, 0, s>>>(idx, p->T, p->k, p->E, p->capacity, hist, counts,
+                                            kept, offsets, status);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || p->T == 0)
+        return e;
+    const int nch = ceil_div(p->T, kDispatchChunk);
+    const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
+    dispatch_scatter_kernel<<<nch, 256, 0, s>>>((const char *)x, row_bytes, idx, p->T, p->k,
+                                                p->E, hist, kept, offsets, (char *)x_perm,
+                                                row_token, slot_row);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,73 @@
+// kernels.h -- internal interface between the C-ABI layer (api.cu) and the
+// kernel translation units of libmoe.so.  Not installed, not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Tokens handled by one dispatch CTA (one warp ballot per expert).
+constexpr int kDispatchChunk = 32;
+// Smallest number of tokens one router CTA handles (sizes the partial sums).
+constexpr int kRouterMinTokens = 8;
+// Warps of a router CTA (bf16: split-K over the warps; f32: one token per warp).
+constexpr int kRouterWarps = 8;
+// Rows of the transposed router weights [W_g | W_noise | 0]^T in the workspace.
+constexpr int kWtRows = 128;
+
+// Byte offsets of the sections of the caller's workspace.
+struct WsLayout {
+    size_t wt;     // router weights transposed to [nout_pad][d] (dtype)
+    size_t rpart;  // router per-CTA partial sums [blocks][2][E] f32
+    size_t hist;   // dispatch per-chunk counts, then bases, [E][chunks] int32
+    size_t total;
+};
+WsLayout ws_layout(const moe_params_t *p);
+
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+inline int ceil_div(int v, int m) { return (v + m - 1) / m; }
+
+// Launch counter shared by every launch site.
+void count_launch(int n = 1);
+// Current time limit of bounded device waits (ns).
+uint64_t wait_limit_ns();
+
+// Every launcher returns cudaSuccess or the launch error.
+cudaError_t launch_partition(const void *W1, const void *W3, const void *W2, int d, int d_ff,
+                             int E, int m, int mode, const int32_t *perm, int dtype,
+                             void *W13_e, void *W2_e, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
+                         const void *Wnoise, const float *noise, const float *bias,
+                         int32_t *idx, float *w, float *probs_sum, float *importance,
+                         char *ws, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
+                            void *x_perm, int32_t *row_token, int32_t *slot_row,
+                            int32_t *counts, int32_t *kept, int32_t *offsets, char *ws,
+                            int32_t *status, cudaStream_t s);
+
+// a3 / a4 for f32 (CUDA-core FMA)
+cudaError_t launch_up_simt(const moe_params_t *p, const float *x_perm, const int32_t *offsets,
+                           const float *W13, float *h, cudaStream_t s);
+cudaError_t launch_down_simt(const moe_params_t *p, const float *h, const int32_t *offsets,
+                             const float *W2, float *out, cudaStream_t s);
+
+// a3 / a4 for bf16 (tcgen05 tensor cores, TMA, TMEM)
+cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
+                         const void *W13, void *h, int32_t *status, cudaStream_t s);
+cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
+                           const void *W2, void *out, int32_t *status, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
+                           const float *w, void *y, cudaStream_t s);
+
+cudaError_t launch_gate_stats(const moe_params_t *p, const int32_t *counts,
+                              const float *probs_sum, float *f, float *P, float *loss,
+                              cudaStream_t s);
+
+}  // namespace moe
