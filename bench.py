@@ -1,0 +1,482 @@
+"""Throughput of the MoE-layer forward on B200 (one JSON line on stdout).
+
+A step is one pass of the whole layer (route -> dispatch -> expert GEMM 1 with
+SwiGLU -> expert GEMM 2 -> combine -> gate statistics) over one batch of seeded
+synthetic input already resident in HBM; the working set per step (x, the packed
+expert weights and the intermediates) is several times the 126 MB L2, so no flush
+is needed between steps.  Every step is issued as the six C-ABI step calls with
+CUDA events between them on the launching stream, which gives the per-kernel
+times used for the roofline line.  The end-to-end leg times ``moe_forward`` with
+the inputs copied from pinned host memory and the result read back every step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+N > 1 runs under torchrun: every rank runs an independent replica of the layer on
+its own batch (weak scaling, no data-path collective); times are the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (host cores; rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec and TFLOP/s at 1 B200; % of bf16 tensor peak / % HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes of one a3 launch (expert GEMM 1 + SwiGLU) from an ncu capture, keyed by
+# the source it was taken on; reported as null once the kernel source changes.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(rel):
+    with open(os.path.join(ROOT, rel), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_of(w: wl.Workload, C: int):
+    return {
+        "workload": w.name, "T": w.T, "d": w.d, "d_ff": w.d_ff, "E": w.E, "k": w.k, "m": w.m,
+        "router": "mixtral" if w.router == wl.MIXTRAL else "st", "noisy": w.noisy,
+        "bias": w.bias, "rescale": w.rescale, "capacity": C, "cf": w.cf,
+        "partition": "disjoint" if w.partition == wl.DISJOINT else "copy",
+        "global_batch": w.T, "seq_len": 4096,
+        "l2": "no flush: per-step working set (x, packed weights, intermediates) >> 126 MB L2",
+    }
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while it runs."""
+
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, dev_index):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            target = str(dev_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.samples:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((ts, float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        inwin = [r for r in rows if t0 <= r[0] <= t1]
+        note = "samples inside the timed region"
+        if not inwin and rows:
+            mid = 0.5 * (t0 + t1)
+            inwin = sorted(rows, key=lambda r: abs(r[0] - mid))[:3]
+            note = "timed region shorter than the sampling period: nearest samples"
+        if not inwin:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        reasons = sorted({self.NAMES[i] for r in inwin for i, v in enumerate(r[3])
+                          if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in inwin])),
+                "sm_max_mhz": max(r[2] for r in inwin), "reasons": reasons,
+                "samples": len(inwin), "note": note}
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+def oracle_sample_forward(w, x_s, eps_s, Wg, Wn, bias, OW, C, rescale):
+    """The oracle's layer forward on a sample of tokens (router, dispatch, experts,
+    combine, statistics); returns y."""
+    import oracle
+    r = oracle.router(x_s, Wg, Wn, eps_s, bias, w.k, w.router)
+    d = oracle.dispatch(r["idx"], w.E, C)
+    oracle.gate_stats(x_s.shape[0], w.k, d["counts"], r["probs_sum"], w.lam)
+    R = d["R"]
+    if R:
+        eor = np.searchsorted(d["offsets"], np.arange(R), side="right") - 1
+        out = oracle.expert_ffn(*OW, np.ascontiguousarray(x_s[d["row_token"]]), eor)
+    else:
+        out = np.zeros((1, w.d))
+    return oracle.combine(out, d["slot_row"], r["G"], (w.E / w.k) if rescale else 1.0)
+
+
+def oracle_inputs(w, inp):
+    import oracle
+    raw = wl.to_numpy_raw
+    if w.partition == wl.COPY and "W1s" in inp:
+        OW = (raw(inp["W1s"]), raw(inp["W3s"]), raw(inp["W2s"]))
+    else:
+        OW = oracle.partition(raw(inp["W1"]), raw(inp["W3"]), raw(inp["W2"]), w.E,
+                              oracle.COPY if w.partition == wl.COPY else oracle.DISJOINT,
+                              None if inp["perm"] is None else raw(inp["perm"]))
+    x = raw(inp["x"])
+    eps = None if inp["eps"] is None else raw(inp["eps"])
+    Wn = None if inp["Wnoise"] is None else raw(inp["Wnoise"])
+    bias = None if inp["bias"] is None else raw(inp["bias"])
+    return x, eps, raw(inp["Wg"]), Wn, bias, OW
+
+
+def time_oracle(w, inp, C, target_s=12.0, max_tokens=8192):
+    """Oracle tokens/s on a bounded, seeded sample of the workload's tokens."""
+    import oracle
+    x, eps, Wg, Wn, bias, OW = oracle_inputs(w, inp)
+    rng = np.random.default_rng(w.seed)
+
+    def run(n):
+        toks = np.sort(rng.choice(w.T, size=min(n, w.T), replace=False))
+        xs = np.ascontiguousarray(x[toks])
+        es = None if eps is None else np.ascontiguousarray(eps[toks])
+        t0 = time.perf_counter()
+        oracle_sample_forward(w, xs, es, Wg, Wn, bias, OW, C, w.rescale)
+        return len(toks), time.perf_counter() - t0
+
+    n0, t_probe = run(4)
+    per_tok = t_probe / max(n0, 1)
+    n = int(max(4, min(max_tokens, target_s / max(per_tok, 1e-9))))
+    n_done, t = run(n)
+    return {"value": n_done / t, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d of %d tokens of %s (seeded), full layer: router, dispatch (capacity "
+                      "%d), SwiGLU experts, combine, statistics; fp64, %.1f s" %
+                      (n_done, w.T, w.name, C, t)}
+
+
+# --------------------------------------------------------------------------- main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="moe_2of8", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="libmoe", choices=["libmoe", "reference"])
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's T (small cases for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_setup(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (n, world))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                              device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = wl.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.with_(T=args.tokens)
+    inp = wl.make_inputs(w, device="cpu")
+    C = -1 if w.cf < 0 else int(np.ceil(w.T * w.cf / w.E - 1e-12))
+    import oracle
+    x, eps, Wg, Wn, bias, OW = oracle_inputs(w, inp)
+    rng = np.random.default_rng(w.seed)
+    # size each step's sample so that warm-up + timed steps take about two minutes
+    t0 = time.perf_counter()
+    oracle_sample_forward(w, x[:2], None if eps is None else eps[:2], Wg, Wn, bias, OW, C,
+                          w.rescale)
+    per_tok = (time.perf_counter() - t0) / 2
+    n = int(max(1, min(64, 120.0 / max((args.steps + args.warmup) * per_tok, 1e-9))))
+    total_tok, total_t = 0, 0.0
+    for i in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(w.T, size=n, replace=False))
+        xs = np.ascontiguousarray(x[toks])
+        es = None if eps is None else np.ascontiguousarray(eps[toks])
+        t0 = time.perf_counter()
+        oracle_sample_forward(w, xs, es, Wg, Wn, bias, OW, C, w.rescale)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            total_tok += n
+            total_t += dt
+    v = total_tok / total_t
+    sample = ("%d seeded tokens of %s per step (full layer in fp64 on the host, "
+              "oracle as is)" % (n, w.name))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, C),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    import top_routing_grouped_noisy_b200 as moe
+
+    w = wl.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.with_(T=args.tokens)
+    inp = wl.make_inputs(w, device="cuda", seed=w.seed + 7919 * rank)
+    C = moe.moe_capacity(w.T, w.E, w.cf) if w.cf >= 0 else -1
+    dt = wl.torch_dtype(w)
+    p = moe.params(w.T, w.d, w.E, w.k, w.m, dt, w.router, C, w.rescale, w.lam)
+    ws = moe.Workspace(p)
+    if w.partition == wl.COPY and "W1s" in inp:
+        W13_e, W2_e = moe.moe_partition_experts(inp["W1s"], inp["W3s"], inp["W2s"], w.E,
+                                                moe.STACKED, ws=ws)
+    elif w.partition == wl.COPY:
+        W13_e, W2_e = moe.moe_partition_experts(inp["W1"], inp["W3"], inp["W2"], w.E, moe.COPY,
+                                                ws=ws)
+    else:
+        W13_e, W2_e = moe.moe_partition_experts(inp["W1"], inp["W3"], inp["W2"], w.E,
+                                                moe.DISJOINT, perm=inp["perm"], ws=ws)
+    b = moe.ForwardBuffers(p)
+    x, Wg, Wn, eps, bias = inp["x"], inp["Wg"], inp["Wnoise"], inp["eps"], inp["bias"]
+    stream = torch.cuda.current_stream()
+    NSEG = 6
+    SEG = ["route", "dispatch", "expert_up", "expert_down", "combine", "gate_stats"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b.topk_idx, b.topk_w, b.probs_sum,
+                      b.importance)
+        if ev is not None:
+            ev[1].record(stream)
+        moe.moe_dispatch(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
+                         b.kept, b.offsets)
+        if ev is not None:
+            ev[2].record(stream)
+        moe.moe_expert_up(p, b.x_perm, b.offsets, W13_e, b.h, ws)
+        if ev is not None:
+            ev[3].record(stream)
+        moe.moe_expert_down(p, b.h, b.offsets, W2_e, b.out, ws)
+        if ev is not None:
+            ev[4].record(stream)
+        moe.moe_combine(p, b.out, b.slot_row, b.topk_w, b.y)
+        if ev is not None:
+            ev[5].record(stream)
+        moe.moe_gate_stats(p, b.counts, b.probs_sum, b.f, b.P, b.loss)
+        if ev is not None:
+            ev[6].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = moe.moe_get_device_status(ws)
+    if status != 0:
+        raise SystemExit("device status %d after warm-up" % status)
+    R = int(b.offsets[-1])
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(NSEG + 1)]
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    launches = moe.moe_launch_count() - l0
+    time.sleep(0.15)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    status = moe.moe_get_device_status(ws)
+    if status != 0:
+        raise SystemExit("device status %d after the timed region" % status)
+    ms_local = start.elapsed_time(end)
+    seg_ms = np.zeros(NSEG)
+    for e in evs:
+        for s in range(NSEG):
+            seg_ms[s] += e[s].elapsed_time(e[s + 1])
+    seg_ms /= args.steps
+    ms = max_over_ranks(ms_local, world)
+    seg_ms = np.array([max_over_ranks(v, world) for v in seg_ms])
+    tokens = w.T * args.steps * world
+    value = tokens / (ms / 1000.0)
+    flop_step = 6.0 * w.d * w.m * R
+    tflops = flop_step * args.steps * world / (ms / 1000.0) / 1e12
+
+    # roofline of the dominant kernel (expert GEMM 1 + SwiGLU), timed inside the step loop
+    peaks, peak_src = load_peaks()
+    es = 2 if dt == torch.bfloat16 else 4
+    up_flop = 4.0 * w.d * w.m * R
+    down_flop = 2.0 * w.d * w.m * R
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    up_tf = up_flop / (seg_ms[2] / 1000.0) / 1e12
+    traffic = None
+    key = _src_hash("top_routing_grouped_noisy_b200/csrc/ffn_tc.cu")
+    if NCU_TRAFFIC.get("src") == key and NCU_TRAFFIC.get("workload") == w.name:
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    roofline = {"kernel": "grouped_gemm_kernel<SwiGLU> (expert GEMM 1, moe_expert_up)",
+                "bound": "tensor", "achieved": up_tf, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": up_tf / peak_t, "traffic": traffic,
+                "peak_source": "%s bf16_tflops_sustained (kernel timed inside the step loop)"
+                               % peak_src,
+                "algorithmic": "4*d*m FLOP per kept row x R=%d rows = %.4g FLOP per launch"
+                               % (R, up_flop)}
+    hbm = peaks["hbm_gbs"]
+    route_bytes = w.T * w.d * es + (w.T * w.E * 4 if eps is not None else 0) + w.T * w.k * 8
+    disp_bytes = w.T * w.d * es + R * w.d * es + w.T * w.k * 12
+    comb_bytes = R * w.d * es + w.T * w.d * es + w.T * w.k * 8
+    kernels = {
+        "route": {"ms": seg_ms[0], "bound": "hbm", "GB/s": route_bytes / seg_ms[0] / 1e6,
+                  "frac": route_bytes / seg_ms[0] / 1e6 / hbm},
+        "dispatch": {"ms": seg_ms[1], "bound": "hbm", "GB/s": disp_bytes / seg_ms[1] / 1e6,
+                     "frac": disp_bytes / seg_ms[1] / 1e6 / hbm},
+        "expert_up": {"ms": seg_ms[2], "bound": "tensor", "TFLOP/s": up_tf,
+                      "frac": up_tf / peak_t},
+        "expert_down": {"ms": seg_ms[3], "bound": "tensor",
+                        "TFLOP/s": down_flop / (seg_ms[3] / 1000.0) / 1e12,
+                        "frac": down_flop / (seg_ms[3] / 1000.0) / 1e12 / peak_t},
+        "combine": {"ms": seg_ms[4], "bound": "hbm", "GB/s": comb_bytes / seg_ms[4] / 1e6,
+                    "frac": comb_bytes / seg_ms[4] / 1e6 / hbm},
+        "gate_stats": {"ms": seg_ms[5]},
+    }
+
+    # end to end through moe_forward with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_h = x.cpu().pin_memory()
+        eps_h = eps.cpu().pin_memory() if eps is not None else None
+        y_h = torch.empty(b.y.shape, dtype=b.y.dtype).pin_memory()
+        loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+        x_d = torch.empty_like(x)
+        eps_d = torch.empty_like(eps) if eps is not None else None
+
+        def e2e_step():
+            x_d.copy_(x_h, non_blocking=True)
+            if eps_d is not None:
+                eps_d.copy_(eps_h, non_blocking=True)
+            moe.moe_forward(p, x_d, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps_d, bias=bias)
+            y_h.copy_(b.y, non_blocking=True)
+            loss_h.copy_(b.loss, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier(world)
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms2 = max_over_ranks(s2.elapsed_time(e2), world)
+        h2d = x.numel() * x.element_size() + (eps.numel() * 4 if eps is not None else 0)
+        d2h = b.y.numel() * b.y.element_size() + 4
+        e2e = {"value": w.T * args.steps * world / (ms2 / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms2 / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {k2: (v.cpu() if isinstance(v, torch.Tensor) else v) for k2, v in inp.items()}
+        cpu = time_oracle(w, inp_cpu, C)
+
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": dict(config_of(w, C), parallelism="dp%d replicas" % world, kept_rows=R),
+        "tflops": tflops, "tflops_frac_of_peak": tflops / peak_t,
+        "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
