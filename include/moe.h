@@ -172,6 +172,22 @@ int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx,
                  void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
                  int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* a2 without a workspace.  The pages have no counterpart: this is a service
+ * for callers that cannot allocate device memory or pass a workspace (for
+ * example a host engine whose plugin interface hands a layer only its input and
+ * output tensors and forbids allocation while work is enqueued).  Same inputs,
+ * outputs and results as moe_dispatch; `status` (device int32, may be NULL)
+ * receives MOE_ERR_DEVICE_BADINDEX like the workspace status word.
+ * Scratch: a fixed 256 KiB array inside the library image, reserved on every
+ * GPU that loads libmoe.so until the process exits; limit E * ceil(T/32) <=
+ * 65536 (T <= 32768 at E = 64), larger sizes return MOE_ERR_SHAPE.  The first
+ * call on a device looks up that array's device address (make it before any
+ * stream capture).  All calls share the array: calls that overlap on the GPU
+ * race, so serialise them.  Allocates nothing. */
+int moe_dispatch_noalloc(const moe_params_t *p, const void *x, const int32_t *topk_idx,
+                         void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
+                         int32_t *kept, int32_t *offsets, int32_t *status, void *stream);
+
 /* a3. First half of every expert's SwiGLU FFN on its kept rows
  * ["LLaMA-MoE v2", code sample, class Expert: down(silu(gate(x)) * up(x))]:
  *   h[r] = silu(x_perm[r] W1_e^T) * (x_perm[r] W3_e^T) for rows r in

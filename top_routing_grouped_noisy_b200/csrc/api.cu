@@ -132,6 +132,12 @@ static int after_launch(const char *fn, cudaError_t e)
     return ok();
 }
 
+// Accessors for entry points defined in other translation units.
+int validate_params(const char *fn, const moe_params_t *p) { return check_params(fn, p); }
+int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+int report_cuda(cudaError_t e, const char *where) { return cuda_fail(e, where); }
+int report_ok() { return ok(); }
+
 }  // namespace moe
 
 using namespace moe;

@@ -176,3 +176,100 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free dispatch.  Some callers cannot allocate device memory or hand
+// the library a workspace -- for example a host engine whose plugin interface
+// gives a layer only its input and output tensors and forbids allocation while
+// it enqueues work, or a latency-critical loop that must never enter an
+// allocator.  For them moe_dispatch_noalloc keeps the per-chunk histogram in a
+// fixed array in device memory that is part of the library image itself: it is
+// reserved on every GPU that loads libmoe.so and stays reserved until the
+// process exits.  Every call reuses the same array, so calls whose kernels
+// overlap on the GPU (different streams, different host threads) race and
+// corrupt each other's results; serialise them.  The scan kernel overwrites
+// every histogram entry a call reads, so stale contents from an earlier call
+// are never used.
+#include <mutex>
+
+namespace moe {
+
+constexpr int kNoallocHistInts = 65536;  // 256 KiB of per-(expert, chunk) counts
+constexpr int kNoallocStatusInts = 64;   // status word used when the caller passes none
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocHistInts + kNoallocStatusInts];
+
+static std::mutex g_noalloc_mu;
+static int32_t *g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device (host code must not
+// use the symbol itself: on the host it names a stand-in, not device memory).
+static cudaError_t noalloc_scratch(int32_t **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess)
+            return e;
+        g_noalloc_ptr[dev] = static_cast<int32_t *>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace moe
+
+extern "C" int moe_dispatch_noalloc(const moe_params_t *p, const void *x,
+                                    const int32_t *topk_idx, void *x_perm, int32_t *row_token,
+                                    int32_t *slot_row, int32_t *counts, int32_t *kept,
+                                    int32_t *offsets, int32_t *status, void *stream)
+{
+    using namespace moe;
+    const char *fn = "moe_dispatch_noalloc";
+    int rc = validate_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    const void *tok[] = {x, topk_idx, x_perm, row_token, slot_row};
+    const void *exp_[] = {counts, kept, offsets};
+    for (const void *q : tok)
+        if ((q == nullptr && p->T > 0) || (reinterpret_cast<uintptr_t>(q) & 15u))
+            return report_error(q == nullptr ? MOE_ERR_INVALID_ARG : MOE_ERR_ALIGN,
+                                "moe_dispatch_noalloc: a token buffer is NULL or not 16-byte "
+                                "aligned");
+    for (const void *q : exp_)
+        if (q == nullptr || (reinterpret_cast<uintptr_t>(q) & 15u))
+            return report_error(q == nullptr ? MOE_ERR_INVALID_ARG : MOE_ERR_ALIGN,
+                                "moe_dispatch_noalloc: counts/kept/offsets is NULL or not "
+                                "16-byte aligned");
+    const int64_t chunks = ceil_div(p->T > 0 ? p->T : 1, kDispatchChunk);
+    if ((int64_t)p->E * chunks > kNoallocHistInts)
+        return report_error(MOE_ERR_SHAPE,
+                            "moe_dispatch_noalloc: E * ceil(T/32) exceeds the fixed scratch of "
+                            "65536 entries (e.g. T <= 32768 at E = 64, T <= 262144 at E = 8)");
+    int32_t *scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess)
+        return report_cuda(e, fn);
+    int32_t *hist = scratch;
+    int32_t *st = status != nullptr ? status : scratch + kNoallocHistInts;
+    cudaStream_t s = (cudaStream_t)stream;
+    dispatch_scan_kernel<<<1, 1024, 0, s>>>(topk_idx, p->T, p->k, p->E, p->capacity, hist,
+                                            counts, kept, offsets, st);
+    count_launch();
+    e = cudaGetLastError();
+    if (e == cudaSuccess && p->T > 0) {
+        const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
+        dispatch_scatter_kernel<<<(unsigned)chunks, 256, 0, s>>>(
+            (const char *)x, row_bytes, topk_idx, p->T, p->k, p->E, hist, kept, offsets,
+            (char *)x_perm, row_token, slot_row);
+        count_launch();
+        e = cudaGetLastError();
+    }
+    return e == cudaSuccess ? report_ok() : report_cuda(e, fn);
+}

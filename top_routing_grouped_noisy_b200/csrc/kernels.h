@@ -31,6 +31,12 @@ WsLayout ws_layout(const moe_params_t *p);
 inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 inline int ceil_div(int v, int m) { return (v + m - 1) / m; }
 
+// Error reporting of the C ABI, for entry points outside api.cu.
+int validate_params(const char *fn, const moe_params_t *p);
+int report_error(int code, const char *msg);
+int report_cuda(cudaError_t e, const char *where);
+int report_ok();
+
 // Launch counter shared by every launch site.
 void count_launch(int n = 1);
 // Current time limit of bounded device waits (ns).
