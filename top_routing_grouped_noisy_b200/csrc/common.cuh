@@ -19,6 +19,8 @@ typedef __nv_bfloat16 bf16;
 // The first 256 bytes of the caller's workspace are a header; word 0 is the
 // device status word (0 or a MOE_ERR_DEVICE_* code; the first error sticks).
 constexpr size_t kWsHeader = 256;
+// Word 1 of the header: ticket counter of the dispatch count kernel (zero between calls).
+constexpr int kWsCounterWord = 1;
 
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {

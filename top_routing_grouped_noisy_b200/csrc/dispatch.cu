@@ -6,10 +6,10 @@
 // by expert, token-ascending inside an expert.  An assignment is kept iff its
 // rank inside its expert is < C, so the lower token index wins.
 //
-//   scan kernel (one CTA): per 32-token chunk and expert, the number of tokens
-//     of the chunk routed to the expert (one warp ballot per expert), then an
-//     exclusive scan over chunks per expert -> the rank base of each chunk;
-//     counts, kept = min(counts, C), offsets = exclusive scan of kept.
+//   count kernel: per 32-token chunk and expert, the number of tokens of the
+//     chunk routed to the expert (one warp ballot per expert); the CTA that
+//     finishes last then scans over chunks per expert -> the rank base of each
+//     chunk; counts, kept = min(counts, C), offsets = exclusive scan of kept.
 //   scatter kernel (one CTA per chunk): each assignment's rank = chunk base +
 //     ballot prefix inside the chunk; slot_row / row_token; then the chunk's x
 //     rows are read once (16-byte loads) and written to each kept row.
@@ -19,17 +19,25 @@
 
 namespace moe {
 
-__global__ void __launch_bounds__(1024) dispatch_scan_kernel(
+constexpr int kCountWarps = 8;  // chunks per count CTA
+
+// Per-chunk expert counts (one warp ballot per expert and 32-token chunk), then, in
+// whichever CTA finishes last, the exclusive scan over chunks per expert (rank base
+// of every chunk), counts, kept = min(counts, C) and offsets.  The last CTA is
+// found with a ticket counter (threadfence + atomicAdd); it resets the counter, so
+// the next launch on the stream starts from zero.  No thread ever waits on another
+// CTA, and the outputs do not depend on which CTA happens to be last.
+__global__ void __launch_bounds__(256) dispatch_count_kernel(
     const int32_t *__restrict__ idx, int T, int k, int E, int C, int32_t *__restrict__ hist,
-    int32_t *__restrict__ counts, int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
-    int32_t *status)
+    int32_t *counter, int32_t *__restrict__ counts, int32_t *__restrict__ kept,
+    int32_t *__restrict__ offsets, int32_t *status)
 {
+    __shared__ int s_last;
     __shared__ int32_t s_count[MOE_MAX_EXPERTS];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarp = blockDim.x >> 5;
     const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
-    // phase 1: per-chunk histograms, hist[e][chunk]
-    for (int c = warp; c < nch; c += nwarp) {
+    const int c = blockIdx.x * kCountWarps + warp;
+    if (c < nch) {
         const int64_t t = (int64_t)c * kDispatchChunk + lane;
         int ej[MOE_MAX_TOPK];
         for (int j = 0; j < k; ++j) {
@@ -48,34 +56,45 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
             for (int j = 0; j < k; ++j)
                 has |= ej[j] == e;
             const unsigned b = __ballot_sync(0xffffffffu, has);
-            if (lane == 0)
+            if (lane == (e & 31))
                 hist[(int64_t)e * nch + c] = __popc(b);
         }
     }
+    __threadfence();
     __syncthreads();
-    // phase 2: exclusive scan over chunks, one warp per expert
-    for (int e = warp; e < E; e += nwarp) {
-        int32_t run = 0;
+    if (threadIdx.x == 0)
+        s_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    // exclusive scan over chunks, one warp per expert; lane l owns a contiguous run
+    const int per = (nch + 31) / 32;
+    for (int e = warp; e < E; e += kCountWarps) {
         int32_t *h = hist + (int64_t)e * nch;
-        for (int base = 0; base < nch; base += 32) {
-            const int c = base + lane;
-            const int32_t v = c < nch ? h[c] : 0;
-            int32_t incl = v;
+        const int c0 = lane * per, c1 = min(nch, c0 + per);
+        int32_t sum = 0;
+#pragma unroll 8
+        for (int cc = c0; cc < c1; ++cc)
+            sum += __ldcg(h + cc);
+        int32_t incl = sum;
 #pragma unroll
-            for (int s = 1; s < 32; s <<= 1) {
-                const int32_t u = __shfl_up_sync(0xffffffffu, incl, s);
-                if (lane >= s)
-                    incl += u;
-            }
-            if (c < nch)
-                h[c] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+        for (int sh = 1; sh < 32; sh <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, incl, sh);
+            if (lane >= sh)
+                incl += u;
         }
+        int32_t run = incl - sum;
+        for (int cc = c0; cc < c1; ++cc) {
+            const int32_t v = __ldcg(h + cc);
+            h[cc] = run;
+            run += v;
+        }
+        const int32_t total = __shfl_sync(0xffffffffu, incl, 31);
         if (lane == 0)
-            s_count[e] = run;
+            s_count[e] = total;
     }
     __syncthreads();
-    // phase 3: capacity clip and expert offsets
     if (threadIdx.x == 0) {
         int32_t off = 0;
         offsets[0] = 0;
@@ -87,7 +106,15 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
             off += kp;
             offsets[e + 1] = off;
         }
+        *counter = 0;
     }
+}
+
+static unsigned count_grid(int T)
+{
+    const int nch = ceil_div(T, kDispatchChunk);
+    const int g = ceil_div(nch, kCountWarps);
+    return (unsigned)(g > 0 ? g : 1);
 }
 
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
@@ -160,8 +187,10 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
 {
     const WsLayout L = ws_layout(p);
     int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
-    dispatch_scan_kernel<<<1, 1024, 0, s>>>(idx, p->T, p->k, p->E, p->capacity, hist, counts,
-                                            kept, offsets, status);
+    int32_t *counter = reinterpret_cast<int32_t *>(ws) + kWsCounterWord;
+    dispatch_count_kernel<<<count_grid(p->T), 256, 0, s>>>(idx, p->T, p->k, p->E, p->capacity,
+                                                           hist, counter, counts, kept, offsets,
+                                                           status);
     count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p->T == 0)
@@ -187,9 +216,10 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
 // reserved on every GPU that loads libmoe.so and stays reserved until the
 // process exits.  Every call reuses the same array, so calls whose kernels
 // overlap on the GPU (different streams, different host threads) race and
-// corrupt each other's results; serialise them.  The scan kernel overwrites
+// corrupt each other's results; serialise them.  The count kernel overwrites
 // every histogram entry a call reads, so stale contents from an earlier call
-// are never used.
+// are never used, and it returns its ticket counter to zero (the array starts
+// zeroed when the library loads).
 #include <mutex>
 
 namespace moe {
@@ -258,9 +288,11 @@ extern "C" int moe_dispatch_noalloc(const moe_params_t *p, const void *x,
         return report_cuda(e, fn);
     int32_t *hist = scratch;
     int32_t *st = status != nullptr ? status : scratch + kNoallocHistInts;
+    int32_t *counter = scratch + kNoallocHistInts + 1;  // zero at load, reset by every call
     cudaStream_t s = (cudaStream_t)stream;
-    dispatch_scan_kernel<<<1, 1024, 0, s>>>(topk_idx, p->T, p->k, p->E, p->capacity, hist,
-                                            counts, kept, offsets, st);
+    dispatch_count_kernel<<<count_grid(p->T), 256, 0, s>>>(topk_idx, p->T, p->k, p->E,
+                                                           p->capacity, hist, counter, counts,
+                                                           kept, offsets, st);
     count_launch();
     e = cudaGetLastError();
     if (e == cudaSuccess && p->T > 0) {
