@@ -33,6 +33,12 @@ SMALL = {
     "k_eq_E": W("k_eq_E", T=128, d=64, d_ff=128, E=4, k=4, seed=19),
     "one_token": W("one_token", T=1, d=256, d_ff=512, E=8, k=2, noisy=True, seed=20),
     "tiny_cap": W("tiny_cap", T=200, d=64, d_ff=256, E=8, k=2, cf=0.25, seed=21),
+    # T*k >= 4096 rows: the 2-SM (cta_group::2) GEMM kernel
+    "pair_mid": W("pair_mid", T=2100, d=256, d_ff=2048, E=8, k=2, noisy=True, rescale=True,
+                  seed=24),
+    "pair_e16_odd": W("pair_e16_odd", T=1200, d=200, d_ff=1600, E=16, k=4, router=wl.ST,
+                      noisy=True, bias=True, cf=1.1, seed=25),
+    "pair_e64": W("pair_e64", T=600, d=128, d_ff=1024, E=64, k=8, noisy=True, seed=26),
     "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
                           router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
     "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",

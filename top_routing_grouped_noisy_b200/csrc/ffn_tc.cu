@@ -441,6 +441,396 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------------ 2-SM variant
+// The same grouped GEMM with cta_group::2: a cluster of two CTAs (two SMs) owns a
+// 256 x 256 output tile.  CTA r of the pair loads rows [128r, 128r+128) of the A
+// tile and rows [128r, 128r+128) of the B tile (half of N); the leader (r = 0)
+// issues tcgen05.mma.cta_group::2 with M = 256, which reads A from each CTA's own
+// shared memory and B from both, and writes each CTA's 128 accumulator rows
+// (all 256 columns) into that CTA's TMEM.  Per CTA a K slab is 32 KB instead of
+// 48 KB for the same 128 x 256 x 64 of MMA work, which relieves shared-memory
+// bandwidth, the limit of the 1-SM kernel.
+//   full[s]   leader only: the leader's producer expects both CTAs' bytes; both
+//             CTAs' TMA loads complete on it
+//   empty[s]  both CTAs: the leader's commit arrives on both (multicast commit)
+//   tfull[a]  both CTAs: the leader's commit arrives on both
+//   tempty[a] leader only: 4 epilogue warps of each CTA arrive (remote for r = 1)
+// Loads carry no multicast qualifier.
+namespace tc2 {
+
+constexpr int BM = 128;   // rows per CTA (256 per pair)
+constexpr int BN = 256;   // columns per pair tile
+constexpr int BNH = 128;  // B rows loaded by each CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int ACC = 2;
+constexpr int TMEM_COLS = ACC * BN;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BNH * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint64_t kAbortSettleNs = 200000ull;  // pause before exit after an abort
+
+struct Aux {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[ACC];
+    uint64_t tempty[ACC];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int32_t abort_flag;
+    int32_t off[MOE_MAX_EXPERTS + 1];
+    int32_t tstart[MOE_MAX_EXPERTS + 1];
+};
+constexpr int SMEM_BYTES = 1024 + TILE_BYTES + (int)sizeof(Aux);
+
+// kind::f16, D f32, A/B bf16 K-major, N = 256, M = 256 (the pair)
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cta_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_cluster_s32(uint32_t cluster_addr)
+{
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster,
+                                                 uint32_t dst, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *map, uint32_t bar_cluster,
+                                                 uint32_t dst, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
+        : "memory");
+}
+
+// arrive on the barrier at this shared offset in both CTAs of the pair
+__device__ __forceinline__ void umma_commit_both(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_own(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+struct PairTile {
+    int e, row0, row_end, n0;
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(const Aux *aux, int tile)
+{
+    PairTile t;
+    int e = 0;
+    while (tile >= aux->tstart[e + 1])
+        ++e;
+    const int local = tile - aux->tstart[e];
+    const int rows = aux->off[e + 1] - aux->off[e];
+    const int mtiles = (rows + 2 * BM - 1) / (2 * BM);
+    const int mt = local % mtiles, nt = local / mtiles;
+    t.e = e;
+    t.row0 = aux->off[e] + mt * 2 * BM;
+    t.row_end = aux->off[e + 1];
+    t.n0 = nt * BN;
+    return t;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB,
+                            const int32_t *__restrict__ offsets, int E, int N, int K,
+                            bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
+                            uint64_t wait_ns)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int32_t *abort_flag = &aux->abort_flag;
+    const uint32_t rank = cta_rank();
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(tc::smem_u32(&aux->full[s]), 1);
+            tc::mbar_init(tc::smem_u32(&aux->empty[s]), 1);
+        }
+        for (int a = 0; a < ACC; ++a) {
+            tc::mbar_init(tc::smem_u32(&aux->tfull[a]), 1);
+            tc::mbar_init(tc::smem_u32(&aux->tempty[a]), 8);
+        }
+        tc::mbar_init(tc::smem_u32(&aux->drain), 1);
+        aux->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    const int n_tiles = (N + BN - 1) / BN;
+    if (warp == 2) {
+        for (int i = lane; i <= E; i += 32)
+            aux->off[i] = offsets[i];
+        __syncwarp();
+        if (lane == 0) {
+            int acc = 0;
+            for (int e = 0; e < E; ++e) {
+                aux->tstart[e] = acc;
+                const int rows = aux->off[e + 1] - aux->off[e];
+                acc += (rows + 2 * BM - 1) / (2 * BM) * n_tiles;
+            }
+            aux->tstart[E] = acc;
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         tc::smem_u32(&aux->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc::tc_fence_before();
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+    tc::tc_fence_after();
+    const uint32_t tmem_base = aux->tmem_base;
+    const int total = aux->tstart[E];
+    const int num_kb = (K + BK - 1) / BK;
+    const uint32_t smem_base = tc::smem_u32(smem);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- TMA producer (both)
+            int stage = 0;
+            uint32_t phase = 0;
+            int64_t fills = 0;
+            for (int tile = cluster_id; tile < total && !*abort_flag; tile += nclusters) {
+                const PairTile t = decode_pair_tile(aux, tile);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!tc::mbar_wait(tc::smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns,
+                                       abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = tc::smem_u32(&aux->full[stage]);
+                    if (leader)
+                        tc::mbar_expect_tx(fb, 2 * STAGE_BYTES);
+                    const uint32_t fb0 = map_rank(fb, 0);
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    tma_load_2d_pair(&tmA, fb0, sa, kb * BK, t.row0 + (int)rank * BM);
+                    tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, kb * BK, t.n0 + (int)rank * BNH,
+                                     t.e);
+                    ++fills;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+            if (leader) {  // the leader's full barriers count both CTAs' bytes
+                for (int s = 0; s < STAGES; ++s) {
+                    const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
+                    if (n > 0)
+                        tc::mbar_drain(tc::smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------------------------------------------------- MMA issuer (leader)
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
+                if (!tc::mbar_wait(tc::smem_u32(&aux->tempty[acc]), acc_phase ^ 1u, wait_ns,
+                                   abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!tc::mbar_wait(tc::smem_u32(&aux->full[stage]), phase, wait_ns,
+                                       abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint64_t da = tc::sdesc(sa), db = tc::sdesc(sa + A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
+                                  (kb | k) != 0);
+                    umma_commit_both(tc::smem_u32(&aux->empty[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit_both(tc::smem_u32(&aux->tfull[acc]));
+                if (++acc == ACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            umma_commit_own(tc::smem_u32(&aux->drain));
+            tc::mbar_drain(tc::smem_u32(&aux->drain), 0);
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue (both)
+        const int wq = warp & 3;
+        const int lane_base = wq * 32;
+        const uint32_t tempty0 = map_rank(tc::smem_u32(&aux->tempty[0]), 0);
+        const uint32_t tempty1 = map_rank(tc::smem_u32(&aux->tempty[1]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = cluster_id; tile < total; tile += nclusters) {
+            const PairTile t = decode_pair_tile(aux, tile);
+            if (!tc::mbar_wait(tc::smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag,
+                               status))
+                break;
+            tc::tc_fence_after();
+            const int row = t.row0 + (int)rank * BM + lane_base + lane;
+            const bool rv = row < t.row_end;
+            const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tc::tmem_ld32(taddr + (uint32_t)(c * 32), v);
+                if constexpr (EPI == tc::EPI_SWIGLU) {
+                    const int nb = t.n0 / 2 + c * 16;
+                    float hv[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float g = __uint_as_float(v[i]);
+                        const float u = __uint_as_float(v[16 + i]);
+                        hv[i] = g / (1.0f + __expf(-g)) * u;
+                    }
+                    if (rv && nb < n_valid) {
+                        bf16 *dst = out + (int64_t)row * ld_out + nb;
+                        if (nb + 16 <= n_valid) {
+                            st_v4(dst, f32x8_to_bf16(hv));
+                            st_v4(dst + 8, f32x8_to_bf16(hv + 8));
+                        } else {
+                            for (int i = 0; i < 16 && nb + i < n_valid; ++i)
+                                dst[i] = __float2bfloat16_rn(hv[i]);
+                        }
+                    }
+                } else {
+                    const int col = t.n0 + c * 32;
+                    if (rv) {
+                        bf16 *dst = out + (int64_t)row * ld_out + col;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (col + q * 8 < n_valid) {
+                                float f[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    f[i] = __uint_as_float(v[q * 8 + i]);
+                                st_v4(dst + q * 8, f32x8_to_bf16(f));
+                            }
+                        }
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);
+            if (++acc == ACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    tc::tc_fence_before();
+    cluster_sync();
+    // after an abort, give copies still in flight time to land before either CTA of
+    // the pair releases its shared memory (the other CTA's loads signal the leader)
+    if (threadIdx.x == 0) {
+        const int peer_abort =
+            ld_cluster_s32(map_rank(tc::smem_u32(&aux->abort_flag), rank ^ 1u));
+        if (*abort_flag || peer_abort) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < kAbortSettleNs) {
+            }
+        }
+    }
+    cluster_sync();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace tc2
+
 // ------------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -491,12 +881,26 @@ static cudaError_t make_map(CUtensorMap *map, const void *base, int rank, const 
 
 struct DevInfo {
     int sms = 0;
-    bool attr[2] = {false, false};
+    int pair_clusters = 0;
+    bool attr[4] = {false, false, false, false};
 };
 static std::mutex g_dev_mu;
 static DevInfo g_dev[64];
 
-static cudaError_t prepare_device(int which, int *sms)
+template <typename Kern>
+static cudaError_t set_smem_attr(Kern kern, int bytes, bool &done)
+{
+    if (done)
+        return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        done = true;
+    return e;
+}
+
+// SM count, dynamic shared memory opt-in of the four GEMM kernels, and how many
+// 2-CTA clusters of the pair kernel fit at once (per device, cached).
+static cudaError_t prepare_device(DevInfo **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -511,18 +915,84 @@ static cudaError_t prepare_device(int which, int *sms)
         if (e != cudaSuccess)
             return e;
     }
-    if (!di.attr[which]) {
-        e = which == EPI_SWIGLU
-                ? cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
-                : cudaFuncSetAttribute(grouped_gemm_kernel<EPI_STORE>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if ((e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU>, SMEM_BYTES, di.attr[0])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE>, SMEM_BYTES, di.attr[1])) != cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU>, tc2::SMEM_BYTES,
+                           di.attr[2])) != cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_STORE>, tc2::SMEM_BYTES,
+                           di.attr[3])) != cudaSuccess)
+        return e;
+    if (di.pair_clusters == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (di.sms / 2));
+        cfg.blockDim = dim3(tc2::NUM_THREADS);
+        cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU>, &cfg);
         if (e != cudaSuccess)
             return e;
-        di.attr[which] = true;
+        di.pair_clusters = n > 0 ? n : 1;
     }
-    *sms = di.sms;
+    *out = &di;
     return cudaSuccess;
+}
+
+// Rows (T*k) from which the 2-SM kernel is used; below it the 1-SM kernel spreads
+// the few tiles over more SMs.
+constexpr int64_t kPairMinRows = 4096;
+
+// One grouped GEMM launch.  A: [rows][a_ld] activations (K extent a_k); B:
+// [E][b_rows][b_ld] expert weights (K extent b_k, N = b_rows); out: [rows][ld_out],
+// first n_valid columns written.
+template <int EPI>
+static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t rows,
+                               const void *B, uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
+                               const int32_t *offsets, int E, bf16 *out, int ld_out, int n_valid,
+                               int32_t *status, cudaStream_t s)
+{
+    DevInfo *di = nullptr;
+    cudaError_t e = prepare_device(&di);
+    if (e != cudaSuccess)
+        return e;
+    const bool pair = (int64_t)rows >= kPairMinRows;
+    CUtensorMap ta, tb;
+    const uint64_t da[2] = {a_k, rows}, sa[1] = {a_ld * 2};
+    const uint32_t ba[2] = {BK, BM};
+    const uint64_t db[3] = {b_k, b_rows, (uint64_t)E};
+    const uint64_t sb[2] = {b_ld * 2, b_rows * b_ld * 2};
+    const uint32_t bb[3] = {BK, pair ? (uint32_t)tc2::BNH : (uint32_t)BN, 1};
+    if ((e = make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
+        return e;
+    if ((e = make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
+        return e;
+    const uint64_t wait_ns = wait_limit_ns();
+    const int N = (int)b_rows, K = (int)a_k;
+    if (!pair) {
+        grouped_gemm_kernel<EPI><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
+            ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * di->pair_clusters);
+    cfg.blockDim = dim3(tc2::NUM_THREADS);
+    cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI>, ta, tb, offsets, E, N, K,
+                              out, ld_out, n_valid, status, wait_ns);
 }
 
 }  // namespace tc
@@ -532,51 +1002,23 @@ using namespace tc;
 cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                          const void *W13, void *h, int32_t *status, cudaStream_t s)
 {
-    const int d = p->d, m = p->m, m16 = round_up(m, 16), m8 = round_up(m, 8);
+    const uint64_t d = p->d, m = p->m, m16 = round_up(p->m, 16), m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    CUtensorMap ta, tb;
-    const uint64_t da[2] = {(uint64_t)d, rows}, sa[1] = {(uint64_t)d * 2};
-    const uint32_t ba[2] = {BK, BM};
-    const uint64_t db[3] = {(uint64_t)d, (uint64_t)2 * m16, (uint64_t)p->E};
-    const uint64_t sb[2] = {(uint64_t)d * 2, (uint64_t)2 * m16 * d * 2};
-    const uint32_t bb[3] = {BK, BN, 1};
-    cudaError_t e;
-    if ((e = make_map(&ta, x_perm, 2, da, sa, ba)) != cudaSuccess)
-        return e;
-    if ((e = make_map(&tb, W13, 3, db, sb, bb)) != cudaSuccess)
-        return e;
-    int sms = 0;
-    if ((e = prepare_device(EPI_SWIGLU, &sms)) != cudaSuccess)
-        return e;
-    grouped_gemm_kernel<EPI_SWIGLU><<<sms, NUM_THREADS, SMEM_BYTES, s>>>(
-        ta, tb, offsets, p->E, 2 * m16, d, (bf16 *)h, m8, m, status, wait_limit_ns());
+    cudaError_t e = launch_gemm<EPI_SWIGLU>(x_perm, d, d, rows, W13, d, d, 2 * m16, offsets, p->E,
+                                            (bf16 *)h, (int)m8, (int)m, status, s);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
                            const void *W2, void *out, int32_t *status, cudaStream_t s)
 {
-    const int d = p->d, m = p->m, m8 = round_up(m, 8);
+    const uint64_t d = p->d, m = p->m, m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    CUtensorMap ta, tb;
-    const uint64_t da[2] = {(uint64_t)m, rows}, sa[1] = {(uint64_t)m8 * 2};
-    const uint32_t ba[2] = {BK, BM};
-    const uint64_t db[3] = {(uint64_t)m, (uint64_t)d, (uint64_t)p->E};
-    const uint64_t sb[2] = {(uint64_t)m8 * 2, (uint64_t)d * m8 * 2};
-    const uint32_t bb[3] = {BK, BN, 1};
-    cudaError_t e;
-    if ((e = make_map(&ta, h, 2, da, sa, ba)) != cudaSuccess)
-        return e;
-    if ((e = make_map(&tb, W2, 3, db, sb, bb)) != cudaSuccess)
-        return e;
-    int sms = 0;
-    if ((e = prepare_device(EPI_STORE, &sms)) != cudaSuccess)
-        return e;
-    grouped_gemm_kernel<EPI_STORE><<<sms, NUM_THREADS, SMEM_BYTES, s>>>(
-        ta, tb, offsets, p->E, d, m, (bf16 *)out, d, d, status, wait_limit_ns());
+    cudaError_t e = launch_gemm<EPI_STORE>(h, m, m8, rows, W2, m, m8, d, offsets, p->E,
+                                           (bf16 *)out, (int)d, (int)d, status, s);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe
