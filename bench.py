@@ -233,6 +233,81 @@ def barrier(world):
     if world > 1:
         torch.distributed.barrier()
 
+def run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank, world,
+               local):
+    """Decode-shaped batches (T <= 64): the layer is launch- and weight-streaming-bound,
+    so one moe_forward is captured in a CUDA graph and the graph is replayed; the
+    figure of merit is the HBM rate of streaming the selected experts' weights."""
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps, bias=bias)
+    stream.synchronize()
+    status = moe.moe_get_device_status(ws)
+    if status != 0:
+        raise SystemExit("device status %d after warm-up" % status)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps, bias=bias)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    kept = b.kept.cpu()
+    experts_used = int((kept > 0).sum())
+    es = 2
+    w_bytes = experts_used * (2 * w.m * w.d + w.d * w.m) * es
+    io_bytes = 2 * w.T * w.d * es + w.d * w.E * es
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    t_wall0 = time.time()
+    start.record(cur)
+    for _ in range(args.steps):
+        graph.replay()
+    end.record(cur)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    time.sleep(0.15)
+    sampler.stop()
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    us = 1000.0 * ms / args.steps
+    peaks, peak_src = load_peaks()
+    gbs = (w_bytes + io_bytes) / (us * 1e-6) / 1e9
+    launches_per_forward = None
+    l1 = moe.moe_launch_count()
+    moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps, bias=bias)
+    launches_per_forward = moe.moe_launch_count() - l1
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": w.T * args.steps * world / (ms / 1000.0), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "us_per_layer": us, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(w, C), parallelism="dp%d replicas" % world,
+                       experts_streamed=experts_used, timing="CUDA graph of one moe_forward"),
+        "roofline": {"kernel": "whole layer (selected experts' weights streamed once)",
+                     "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": "%s hbm_gbs" % peak_src,
+                     "algorithmic": "%d experts x 3*d*m*2 B + x, y, W_g = %.4g B per layer"
+                                    % (experts_used, w_bytes + io_bytes)},
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": launches_per_forward * args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -337,6 +412,10 @@ def main():
         moe.moe_gate_stats(p, b.counts, b.probs_sum, b.f, b.P, b.loss)
         if ev is not None:
             ev[6].record(stream)
+
+    if w.T <= 64:
+        return run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank,
+                          world, local)
 
     for _ in range(args.warmup):
         step()

@@ -39,6 +39,13 @@ SMALL = {
     "pair_e16_odd": W("pair_e16_odd", T=1200, d=200, d_ff=1600, E=16, k=4, router=wl.ST,
                       noisy=True, bias=True, cf=1.1, seed=25),
     "pair_e64": W("pair_e64", T=600, d=128, d_ff=1024, E=64, k=8, noisy=True, seed=26),
+    # T <= 64: the weight-streaming decode kernels
+    "decode_t64_m344": W("decode_t64_m344", T=64, d=512, d_ff=8 * 344, E=8, k=2, rescale=True,
+                         seed=27),
+    "decode_skewed_rows": W("decode_skewed_rows", T=40, d=256, d_ff=4 * 96, E=4, k=2, bias=True,
+                            seed=28),
+    "decode_ragged_d": W("decode_ragged_d", T=8, d=200, d_ff=8 * 100, E=8, k=2, noisy=True,
+                         seed=29),
     "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
                           router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
     "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",
@@ -72,7 +79,11 @@ def _full_check(w, inp, rows_sample=None, tok_sample=None, capacity=None):
 def test_layer_parity_small(name):
     w = SMALL[name]
     inp = wl.make_inputs(w)
-    _full_check(w, inp)
+    if name == "decode_skewed_rows":  # two experts take (nearly) every token: > 32 rows each
+        inp["bias"] = torch.tensor([6.0, 6.0, -6.0, -6.0])
+    res = _full_check(w, inp)
+    if name == "decode_skewed_rows":
+        assert int(res["bufs"].kept.max()) > 32
 
 
 def test_tiny_fp32_workload_full():
@@ -207,7 +218,8 @@ def test_dense_equivalence_on_gpu():
 
 # ------------------------------------------------------------------ full-size workloads
 
-FULL = ["tiny_fp32", "moe_2of8", "moe_4of16", "e8t2_cf1", "e8t2_cf4"]
+FULL = ["tiny_fp32", "moe_2of8", "moe_4of16", "e8t2_cf1", "e8t2_cf4", "decode_t1", "decode_t8",
+        "decode_t64"]
 
 
 @pytest.mark.slow

@@ -106,6 +106,9 @@ WsLayout ws_layout(const moe_params_t *p)
     L.rpart = take(blocks * 2 * p->E * sizeof(float));
     const size_t chunks = (size_t)ceil_div(p->T > 0 ? p->T : 1, kDispatchChunk);
     L.hist = take(chunks * p->E * sizeof(int32_t));
+    L.rsmall = take(p->T <= kRouterSmallTokens
+                        ? (size_t)kRouterSmallSplit * (p->T > 0 ? p->T : 1) * 2 * p->E * sizeof(float)
+                        : 0);
     L.total = off;
     return L;
 }
@@ -328,6 +331,8 @@ int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offs
     cudaError_t e;
     if (p->dtype == MOE_F32)
         e = launch_up_simt(p, (const float *)x_perm, offsets, (const float *)W13_e, (float *)h, s);
+    else if (p->T <= kDecodeMaxTokens)
+        e = launch_up_decode(p, x_perm, offsets, W13_e, h, s);
     else
         e = launch_up_tc(p, x_perm, offsets, W13_e, h, reinterpret_cast<int32_t *>(ws), s);
     return after_launch(fn, e);
@@ -352,6 +357,8 @@ int moe_expert_down(const moe_params_t *p, const void *h, const int32_t *offsets
     cudaError_t e;
     if (p->dtype == MOE_F32)
         e = launch_down_simt(p, (const float *)h, offsets, (const float *)W2_e, (float *)out, s);
+    else if (p->T <= kDecodeMaxTokens)
+        e = launch_down_decode(p, h, offsets, W2_e, out, s);
     else
         e = launch_down_tc(p, h, offsets, W2_e, out, reinterpret_cast<int32_t *>(ws), s);
     return after_launch(fn, e);

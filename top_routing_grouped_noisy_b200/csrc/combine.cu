@@ -13,7 +13,7 @@
 
 namespace moe {
 
-template <typename E_T>
+template <typename E_T, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ out,
                                                       const int32_t *__restrict__ slot_row,
                                                       const float *__restrict__ w, int T, int d,
@@ -26,28 +26,38 @@ __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ ou
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = i / nv;
         const int v = (int)(i - t * nv);
+        // all k rows are requested before any is used
+        uint4 raw[KMAX];
+        float g[KMAX];
+        bool kept[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            const int32_t row = j < k ? slot_row[t * k + j] : -1;
+            kept[j] = row >= 0;
+            g[j] = kept[j] ? w[t * k + j] : 0.f;
+            raw[j] = kept[j] ? ld_nc_na(out + (int64_t)row * d + (int64_t)v * VN)
+                             : make_uint4(0, 0, 0, 0);
+        }
         float acc[VN];
 #pragma unroll
         for (int q = 0; q < VN; ++q)
             acc[q] = 0.f;
-        for (int j = 0; j < k; ++j) {
-            const int32_t row = slot_row[t * k + j];
-            if (row < 0)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (!kept[j])
                 continue;
-            const float g = w[t * k + j];
-            const uint4 raw = ld_nc_na(out + (int64_t)row * d + (int64_t)v * VN);
             float f[VN];
             if constexpr (sizeof(E_T) == 2) {
-                bf16x8_to_f32(raw, f);
+                bf16x8_to_f32(raw[j], f);
             } else {
-                f[0] = __uint_as_float(raw.x);
-                f[1] = __uint_as_float(raw.y);
-                f[2] = __uint_as_float(raw.z);
-                f[3] = __uint_as_float(raw.w);
+                f[0] = __uint_as_float(raw[j].x);
+                f[1] = __uint_as_float(raw[j].y);
+                f[2] = __uint_as_float(raw[j].z);
+                f[3] = __uint_as_float(raw[j].w);
             }
 #pragma unroll
             for (int q = 0; q < VN; ++q)
-                acc[q] = fmaf(g, f[q], acc[q]);
+                acc[q] = fmaf(g[j], f[q], acc[q]);
         }
 #pragma unroll
         for (int q = 0; q < VN; ++q)
@@ -94,12 +104,22 @@ cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t
     const int64_t items = (int64_t)p->T * (p->d / VN);
     const int64_t blocks = (items + 255) / 256;
     const unsigned grid = (unsigned)(blocks < (1 << 30) ? blocks : (1 << 30));
-    if (p->dtype == MOE_BF16)
-        combine_kernel<bf16><<<grid, 256, 0, s>>>((const bf16 *)out, slot_row, w, p->T, p->d,
-                                                  p->k, scale, (bf16 *)y);
+#define MOE_COMBINE(KM)                                                                        \
+    do {                                                                                       \
+        if (p->dtype == MOE_BF16)                                                              \
+            combine_kernel<bf16, KM><<<grid, 256, 0, s>>>((const bf16 *)out, slot_row, w, p->T, \
+                                                          p->d, p->k, scale, (bf16 *)y);       \
+        else                                                                                   \
+            combine_kernel<float, KM><<<grid, 256, 0, s>>>((const float *)out, slot_row, w,     \
+                                                           p->T, p->d, p->k, scale, (float *)y); \
+    } while (0)
+    if (p->k <= 2)
+        MOE_COMBINE(2);
+    else if (p->k <= 4)
+        MOE_COMBINE(4);
     else
-        combine_kernel<float><<<grid, 256, 0, s>>>((const float *)out, slot_row, w, p->T, p->d,
-                                                   p->k, scale, (float *)y);
+        MOE_COMBINE(8);
+#undef MOE_COMBINE
     count_launch();
     return cudaGetLastError();
 }

@@ -51,12 +51,14 @@ template <> __device__ __forceinline__ float from_f32<float>(float v) { return v
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
 
 // 16-byte global loads.  nc: read-only path, no L1 allocation (streamed once).
+// Not volatile: a pure load the compiler may hoist and batch, so unrolled loops
+// keep several loads in flight.
 __device__ __forceinline__ uint4 ld_nc_na(const void *p)
 {
     uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
     return r;
 }
 __device__ __forceinline__ uint4 ld_nc(const void *p)
@@ -91,6 +93,17 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float *f)
     v.z = pack_bf16x2(f[4], f[5]);
     v.w = pack_bf16x2(f[6], f[7]);
     return v;
+}
+
+// D += A * B on the tensor cores, m16n8k16, bf16 inputs, f32 accumulators
+// (A row-major 16x16 in a0..a3, B column-major 16x8 in b0..b1).
+__device__ __forceinline__ void mma_bf16_16816(float *c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 }  // namespace moe

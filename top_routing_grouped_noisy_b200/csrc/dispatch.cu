@@ -17,6 +17,10 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#ifndef MOE_SCATTER_U
+#define MOE_SCATTER_U 8  // row vectors loaded per thread before they are stored
+#endif
+
 namespace moe {
 
 constexpr int kCountWarps = 8;  // chunks per count CTA
@@ -60,14 +64,18 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
                 hist[(int64_t)e * nch + c] = __popc(b);
         }
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0)
-        s_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!s_last)
-        return;
-    __threadfence();
+    if (gridDim.x > 1) {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            s_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+        __syncthreads();
+        if (!s_last)
+            return;
+        __threadfence();
+    } else {
+        __syncthreads();  // one CTA: its own writes are visible after the barrier
+    }
     // exclusive scan over chunks, one warp per expert; lane l owns a contiguous run
     const int per = (nch + 31) / 32;
     for (int e = warp; e < E; e += kCountWarps) {
@@ -106,7 +114,8 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
             off += kp;
             offsets[e + 1] = off;
         }
-        *counter = 0;
+        if (gridDim.x > 1)
+            *counter = 0;
     }
 }
 
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
         }
         for (int j = 0; j < k; ++j) {
             s_row[lane][j] = rowj[j];
-            if (t < T) {
+            if (t < T && blockIdx.y == 0) {
                 slot_row[t * k + j] = rowj[j];
                 if (rowj[j] >= 0)
                     row_token[rowj[j]] = (int32_t)t;
@@ -166,18 +175,48 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     }
     __syncthreads();
     const int ntok = (int)((int64_t)T - t0 < kDispatchChunk ? (int64_t)T - t0 : kDispatchChunk);
-    const int nv = (int)(row_bytes / 16);
+    // the row's 16-byte vectors [v0, v1) of this CTA (blockIdx.y splits rows when T is small)
+    const int nv_all = (int)(row_bytes / 16);
+    const int per = (nv_all + gridDim.y - 1) / gridDim.y;
+    const int v0 = blockIdx.y * per, v1 = min(nv_all, v0 + per);
+    const int nv = v1 > v0 ? v1 - v0 : 0;
     const int items = ntok * nv;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < items; i += blockDim.x) {
-        const int l = i / nv, v = i - l * nv;
-        const uint4 val = ld_nc_na(x + (t0 + l) * row_bytes + (int64_t)v * 16);
-        for (int j = 0; j < k; ++j) {
-            const int32_t row = s_row[l][j];
-            if (row >= 0)
-                st_v4(x_perm + (int64_t)row * row_bytes + (int64_t)v * 16, val);
+    constexpr int U = MOE_SCATTER_U;  // loads in flight per thread before the stores
+    for (int base = threadIdx.x; base < items; base += blockDim.x * U) {
+        uint4 val[U];
+        int lv[U], vv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x;
+            lv[u] = -1;
+            if (i < items) {
+                lv[u] = i / nv;
+                vv[u] = v0 + (i - lv[u] * nv);
+                val[u] = ld_nc_na(x + (t0 + lv[u]) * row_bytes + (int64_t)vv[u] * 16);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (lv[u] < 0)
+                continue;
+            for (int j = 0; j < k; ++j) {
+                const int32_t row = s_row[lv[u]][j];
+                if (row >= 0)
+                    st_v4(x_perm + (int64_t)row * row_bytes + (int64_t)vv[u] * 16, val[u]);
+            }
         }
     }
+}
+
+// CTAs per chunk along the row: enough CTAs in total to cover the SMs twice.
+static unsigned scatter_split(int nch, int64_t row_bytes)
+{
+    const int64_t nv = row_bytes / 16;
+    int64_t y = (296 + nch - 1) / nch;
+    const int64_t ymax = (nv + 63) / 64;  // at least 64 vectors (1 KB) per CTA
+    if (y > ymax)
+        y = ymax;
+    return (unsigned)(y > 0 ? y : 1);
 }
 
 cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
@@ -197,9 +236,9 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
         return e;
     const int nch = ceil_div(p->T, kDispatchChunk);
     const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
-    dispatch_scatter_kernel<<<nch, 256, 0, s>>>((const char *)x, row_bytes, idx, p->T, p->k,
-                                                p->E, hist, kept, offsets, (char *)x_perm,
-                                                row_token, slot_row);
+    dispatch_scatter_kernel<<<dim3(nch, scatter_split(nch, row_bytes)), 256, 0, s>>>(
+        (const char *)x, row_bytes, idx, p->T, p->k, p->E, hist, kept, offsets, (char *)x_perm,
+        row_token, slot_row);
     count_launch();
     return cudaGetLastError();
 }
@@ -297,9 +336,10 @@ extern "C" int moe_dispatch_noalloc(const moe_params_t *p, const void *x,
     e = cudaGetLastError();
     if (e == cudaSuccess && p->T > 0) {
         const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
-        dispatch_scatter_kernel<<<(unsigned)chunks, 256, 0, s>>>(
-            (const char *)x, row_bytes, topk_idx, p->T, p->k, p->E, hist, kept, offsets,
-            (char *)x_perm, row_token, slot_row);
+        dispatch_scatter_kernel<<<dim3((unsigned)chunks, scatter_split((int)chunks, row_bytes)),
+                                  256, 0, s>>>((const char *)x, row_bytes, topk_idx, p->T, p->k,
+                                               p->E, hist, kept, offsets, (char *)x_perm,
+                                               row_token, slot_row);
         count_launch();
         e = cudaGetLastError();
     }

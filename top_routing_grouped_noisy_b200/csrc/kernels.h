@@ -18,12 +18,16 @@ constexpr int kRouterMinTokens = 8;
 constexpr int kRouterWarps = 8;
 // Rows of the transposed router weights [W_g | W_noise | 0]^T in the workspace.
 constexpr int kWtRows = 128;
+// Batches up to this many tokens use the split-K router (partials in `rsmall`).
+constexpr int kRouterSmallTokens = 64;
+constexpr int kRouterSmallSplit = 32;
 
 // Byte offsets of the sections of the caller's workspace.
 struct WsLayout {
     size_t wt;     // router weights transposed to [nout_pad][d] (dtype)
     size_t rpart;  // router per-CTA partial sums [blocks][2][E] f32
     size_t hist;   // dispatch per-chunk counts, then bases, [E][chunks] int32
+    size_t rsmall; // small-batch router partial logits [32][T][2E] f32 (T <= 64)
     size_t total;
 };
 WsLayout ws_layout(const moe_params_t *p);
@@ -68,6 +72,13 @@ cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_
                          const void *W13, void *h, int32_t *status, cudaStream_t s);
 cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
                            const void *W2, void *out, int32_t *status, cudaStream_t s);
+
+// a3 / a4 for decode-shaped bf16 batches (T <= kDecodeMaxTokens): weight streaming
+constexpr int kDecodeMaxTokens = 64;
+cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
+                             const void *W13, void *h, cudaStream_t s);
+cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32_t *offsets,
+                               const void *W2, void *out, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
                            const float *w, void *y, cudaStream_t s);

@@ -17,6 +17,17 @@
 #include "common.cuh"
 #include "kernels.h"
 
+// Tile constants (compile-time; tuned on B200).
+#ifndef MOE_ROUTER_NNT1
+#define MOE_ROUTER_NNT1 8  // token n-tiles per CTA when the router has <= 16 outputs
+#endif
+#ifndef MOE_ROUTER_U
+#define MOE_ROUTER_U 4  // k32 blocks of loads issued per round
+#endif
+#ifndef MOE_ROUTER_U_WIDE
+#define MOE_ROUTER_U_WIDE 1  // the same for 8 token n-tiles per CTA
+#endif
+
 namespace moe {
 
 
@@ -128,16 +139,6 @@ __global__ void router_transpose_kernel(const bf16 *__restrict__ Wg, const bf16 
     Wt[i] = v;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float *c, uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // NMT m-tiles of 16 router outputs x NNT n-tiles of 8 tokens per CTA.
 // Each thread (g = lane/4, q = lane%4) owns K columns [32kb + 8q, 32kb + 8q + 8) of
 // every k32 block kb it visits; the 8 columns feed two m16n8k16 steps, physical
@@ -172,31 +173,39 @@ __global__ void __launch_bounds__(256) router_bf16_kernel(
                 acc[a][b][c] = 0.f;
 
     const int nkb = (d + 31) / 32;
-#pragma unroll 2
-    for (int kb = warp; kb < nkb; kb += NW) {
-        const int c = kb * 32 + 8 * q;
-        const bool kv = c < d;
-        uint4 xb[NNT];
-        uint4 wa[NMT][2];
+    // U k32 blocks per round: all loads of a round are issued before its MMAs
+    constexpr int U = NNT >= 8 ? MOE_ROUTER_U_WIDE : MOE_ROUTER_U;
+    for (int kb0 = warp; kb0 < nkb; kb0 += NW * U) {
+        uint4 xb[U][NNT];
+        uint4 wa[U][NMT][2];
 #pragma unroll
-        for (int nt = 0; nt < NNT; ++nt) {
-            const int64_t t = tok0 + nt * 8 + g;
-            xb[nt] = (kv && t < T) ? ld_nc_na(x + t * d + c) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int mt = 0; mt < NMT; ++mt) {
-            wa[mt][0] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g) * d + c) : make_uint4(0, 0, 0, 0);
-            wa[mt][1] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g + 8) * d + c) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int mt = 0; mt < NMT; ++mt)
+        for (int u = 0; u < U; ++u) {
+            const int c = (kb0 + u * NW) * 32 + 8 * q;
+            const bool kv = c < d;
 #pragma unroll
             for (int nt = 0; nt < NNT; ++nt) {
-                mma_bf16_16816(acc[mt][nt], wa[mt][0].x, wa[mt][1].x, wa[mt][0].y, wa[mt][1].y,
-                               xb[nt].x, xb[nt].y);
-                mma_bf16_16816(acc[mt][nt], wa[mt][0].z, wa[mt][1].z, wa[mt][0].w, wa[mt][1].w,
-                               xb[nt].z, xb[nt].w);
+                const int64_t t = tok0 + nt * 8 + g;
+                xb[u][nt] = (kv && t < T) ? ld_nc_na(x + t * d + c) : make_uint4(0, 0, 0, 0);
             }
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt) {
+                wa[u][mt][0] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g) * d + c)
+                                  : make_uint4(0, 0, 0, 0);
+                wa[u][mt][1] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g + 8) * d + c)
+                                  : make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int mt = 0; mt < NMT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NNT; ++nt) {
+                    mma_bf16_16816(acc[mt][nt], wa[u][mt][0].x, wa[u][mt][1].x, wa[u][mt][0].y,
+                                   wa[u][mt][1].y, xb[u][nt].x, xb[u][nt].y);
+                    mma_bf16_16816(acc[mt][nt], wa[u][mt][0].z, wa[u][mt][1].z, wa[u][mt][0].w,
+                                   wa[u][mt][1].w, xb[u][nt].z, xb[u][nt].w);
+                }
     }
     // D fragment: c0,c1 -> (row g, cols 2q,2q+1); c2,c3 -> (row g+8, cols 2q,2q+1)
 #pragma unroll
@@ -301,6 +310,79 @@ __global__ void __launch_bounds__(1024) router_finalize_kernel(const float *__re
     }
 }
 
+
+// ---------------------------------------------------------------- T <= 64 tokens
+// Decode-sized batches: a few tokens cannot keep the split-over-warps kernel
+// busy, so K is split over kSmallKSplit CTAs instead.  Each CTA stages its K slice
+// of x and of [W_g | W_noise] (read in place, no transpose) in shared memory and
+// writes partial logits part[ks][t][o]; one finishing CTA adds the slices in a
+// fixed order, runs the per-token gate and the token sums.
+constexpr int kSmallKSplit = kRouterSmallSplit;
+
+template <typename E_T>
+__global__ void __launch_bounds__(256) router_small_partial_kernel(
+    const E_T *__restrict__ x, const E_T *__restrict__ Wg, const E_T *__restrict__ Wn, int T,
+    int d, int E, float *__restrict__ part)
+{
+    extern __shared__ float sm[];
+    const int nout = Wn ? 2 * E : E;
+    const int kc = (d + kSmallKSplit - 1) / kSmallKSplit;
+    const int k0 = blockIdx.x * kc, k1 = min(d, k0 + kc);
+    const int kn = k1 > k0 ? k1 - k0 : 0;
+    float *xs = sm;                    // [T][kc]
+    float *ws_ = sm + (size_t)T * kc;  // [kc][nout]
+    for (int i = threadIdx.x; i < T * kn; i += blockDim.x) {
+        const int t = i / kn, c = i % kn;
+        xs[t * kc + c] = to_f32(x[(int64_t)t * d + k0 + c]);
+    }
+    for (int i = threadIdx.x; i < kn * nout; i += blockDim.x) {
+        const int c = i / nout, o = i % nout;
+        ws_[c * nout + o] = o < E ? to_f32(Wg[(int64_t)(k0 + c) * E + o])
+                                  : to_f32(Wn[(int64_t)(k0 + c) * E + o - E]);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
+        const int t = i / nout, o = i % nout;
+        float acc = 0.f;
+        for (int c = 0; c < kn; ++c)
+            acc = fmaf(xs[t * kc + c], ws_[c * nout + o], acc);
+        part[((int64_t)blockIdx.x * T + t) * nout + o] = acc;
+    }
+}
+
+__global__ void __launch_bounds__(256) router_small_finish_kernel(
+    const float *__restrict__ part, int T, int E, int k, int noisy,
+    const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
+    int32_t *__restrict__ idx_out, float *__restrict__ w_out, float *__restrict__ probs_sum,
+    float *__restrict__ importance, int32_t *status)
+{
+    extern __shared__ float sm[];
+    const int nout = noisy ? 2 * E : E;
+    float *lg = sm;                          // [T][nout]
+    float *prob_s = lg + (size_t)T * nout;   // [T][E]
+    float *gw_s = prob_s + (size_t)T * E;    // [T][E]
+    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
+        float acc = 0.f;
+        for (int ks = 0; ks < kSmallKSplit; ++ks)
+            acc += part[(int64_t)ks * T * nout + i];
+        lg[i] = acc;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < T; t += blockDim.x)
+        finish_token(t, lg + (size_t)t * nout, E, k, noisy, noise, bias, router_type, idx_out,
+                     w_out, prob_s + (size_t)t * E, gw_s + (size_t)t * E, status);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        float sp = 0.f, sg = 0.f;
+        for (int t = 0; t < T; ++t) {
+            sp += prob_s[t * E + e];
+            sg += gw_s[t * E + e];
+        }
+        probs_sum[e] = sp;
+        importance[e] = sg;
+    }
+}
+
 template <int NMT, int NNT>
 static cudaError_t run_bf16(const moe_params_t *p, const bf16 *x, const bf16 *Wt, int noisy,
                             const float *noise, const float *bias, int32_t *idx, float *w,
@@ -330,6 +412,30 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
     float *part = reinterpret_cast<float *>(ws + L.rpart);
     int nblk = 0;
     cudaError_t e = cudaSuccess;
+    const int small_noisy = Wnoise != nullptr;
+    const int small_nout = small_noisy ? 2 * p->E : p->E;
+    const int small_kc = ceil_div(p->d, kSmallKSplit);
+    const size_t sm1 = sizeof(float) * ((size_t)p->T * small_kc + (size_t)small_kc * small_nout);
+    const size_t sm2 =
+        sizeof(float) * ((size_t)p->T * small_nout + 2 * (size_t)p->T * p->E);
+    if (p->T > 0 && p->T <= kRouterSmallTokens && sm1 <= 48 * 1024 && sm2 <= 48 * 1024) {
+        const int noisy = small_noisy;
+        float *sp = reinterpret_cast<float *>(ws + L.rsmall);
+        if (p->dtype == MOE_BF16)
+            router_small_partial_kernel<bf16><<<kSmallKSplit, 256, sm1, s>>>(
+                (const bf16 *)x, (const bf16 *)Wg, (const bf16 *)Wnoise, p->T, p->d, p->E, sp);
+        else
+            router_small_partial_kernel<float><<<kSmallKSplit, 256, sm1, s>>>(
+                (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E, sp);
+        count_launch();
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        router_small_finish_kernel<<<1, 256, sm2, s>>>(sp, p->T, p->E, p->k, noisy, noise, bias,
+                                                       p->router_type, idx, w, probs_sum,
+                                                       importance, status);
+        count_launch();
+        return cudaGetLastError();
+    }
     if (p->T > 0) {
         if (p->dtype == MOE_BF16) {
             const int noisy = Wnoise != nullptr;
@@ -342,7 +448,7 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
             if ((e = cudaGetLastError()) != cudaSuccess)
                 return e;
             if (nout <= 16)
-                e = run_bf16<1, 8>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
+                e = run_bf16<1, MOE_ROUTER_NNT1>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
                                    status, s, &nblk);
             else if (nout <= 32)
                 e = run_bf16<2, 4>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
