@@ -221,12 +221,19 @@ def dist_setup(n):
     return rank, world, local
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """The slowest rank's time (every rank calls it, in the same order)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def tokens_per_s(tokens_per_rank, steps, world, ms_max):
+    """Whole-job throughput of independent replicas (weak scaling): every rank's
+    tokens over the slowest rank's time."""
+    return tokens_per_rank * steps * world / (ms_max / 1000.0)
 
 
 def barrier(world):
@@ -456,8 +463,7 @@ def main():
     seg_ms /= args.steps
     ms = max_over_ranks(ms_local, world)
     seg_ms = np.array([max_over_ranks(v, world) for v in seg_ms])
-    tokens = w.T * args.steps * world
-    value = tokens / (ms / 1000.0)
+    value = tokens_per_s(w.T, args.steps, world, ms)
     flop_step = 6.0 * w.d * w.m * R
     tflops = flop_step * args.steps * world / (ms / 1000.0) / 1e12
 

@@ -1,0 +1,46 @@
+"""Failure detection on the GPU without a GPU fault: every bounded wait inside the
+tensor-core GEMM kernels is made to run out at once (wait limit 0), the kernel
+must report MOE_ERR_DEVICE_TIMEOUT through the workspace status word and return,
+and the context must stay usable (a normal layer afterwards passes parity)."""
+import numpy as np
+import pytest
+import torch
+
+import harness as H
+import top_routing_grouped_noisy_b200 as moe
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DEFAULT_LIMIT_NS = 2_000_000_000
+
+
+@pytest.mark.parametrize("T", [300, 2500], ids=["one_sm_kernel", "two_sm_kernel"])
+def test_wait_timeout_is_reported_and_context_survives(T):
+    w = wl.Workload("to", T=T, d=256, d_ff=1024, E=8, k=2, noisy=True, seed=81)
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    W13_e, W2_e = H.gpu_weights(w, inp, ws)
+    b = moe.ForwardBuffers(p)
+    dev = "cuda"
+    x, Wg, Wn, eps = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_route(p, x, Wg, Wn, eps, None, ws, b.topk_idx, b.topk_w, b.probs_sum, b.importance)
+    moe.moe_dispatch(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts, b.kept,
+                     b.offsets)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    moe.moe_set_wait_limit_ns(0)
+    try:
+        moe.moe_expert_up(p, b.x_perm, b.offsets, W13_e, b.h, ws)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert moe.moe_get_device_status(ws) == 0  # cleared by the read
+    # the same context still computes the layer correctly
+    p2, bufs, ws2, status, _ = H.run_forward(w, inp, weights=(W13_e, W2_e))
+    assert status == 0
+    r, ties = H.check_routing(w, inp, bufs, 5e-5)
+    dsp = H.check_dispatch(w, inp, p2, bufs)
+    H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0])
