@@ -393,6 +393,9 @@ def main():
     b = moe.ForwardBuffers(p)
     x, Wg, Wn, eps, bias = inp["x"], inp["Wg"], inp["Wnoise"], inp["eps"], inp["bias"]
     stream = torch.cuda.current_stream()
+    # moe_forward's path: the dispatch materialises x_perm (the row-gathering GEMM 1
+    # variant, moe_expert_up_gather, is slower on B200)
+    gather = False
     NSEG = 6
     SEG = ["route", "dispatch", "expert_up", "expert_down", "combine", "gate_stats"]
 
@@ -403,11 +406,18 @@ def main():
                       b.importance)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_dispatch(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
-                         b.kept, b.offsets)
+        if gather:
+            moe.moe_dispatch_rows(p, b.topk_idx, ws, b.row_token, b.slot_row, b.counts, b.kept,
+                                  b.offsets)
+        else:
+            moe.moe_dispatch(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
+                             b.kept, b.offsets)
         if ev is not None:
             ev[2].record(stream)
-        moe.moe_expert_up(p, b.x_perm, b.offsets, W13_e, b.h, ws)
+        if gather:
+            moe.moe_expert_up_gather(p, x, b.row_token, b.offsets, W13_e, b.h, ws)
+        else:
+            moe.moe_expert_up(p, b.x_perm, b.offsets, W13_e, b.h, ws)
         if ev is not None:
             ev[3].record(stream)
         moe.moe_expert_down(p, b.h, b.offsets, W2_e, b.out, ws)
@@ -478,7 +488,9 @@ def main():
     key = _src_hash("top_routing_grouped_noisy_b200/csrc/ffn_tc.cu")
     if NCU_TRAFFIC.get("src") == key and NCU_TRAFFIC.get("workload") == w.name:
         traffic = NCU_TRAFFIC["bytes_per_launch"]
-    roofline = {"kernel": "grouped_gemm_kernel<SwiGLU> (expert GEMM 1, moe_expert_up)",
+    roofline = {"kernel": "grouped_gemm_2sm_kernel<SwiGLU, gather> (expert GEMM 1, "
+                          "moe_expert_up_gather)" if gather else
+                "grouped_gemm_kernel<SwiGLU> (expert GEMM 1, moe_expert_up)",
                 "bound": "tensor", "achieved": up_tf, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": up_tf / peak_t, "traffic": traffic,
                 "peak_source": "%s bf16_tflops_sustained (kernel timed inside the step loop)"
@@ -487,13 +499,15 @@ def main():
                                % (R, up_flop)}
     hbm = peaks["hbm_gbs"]
     route_bytes = w.T * w.d * es + (w.T * w.E * 4 if eps is not None else 0) + w.T * w.k * 8
-    disp_bytes = w.T * w.d * es + R * w.d * es + w.T * w.k * 12
+    disp_bytes = (w.T * w.k * 12 if gather else w.T * w.d * es + R * w.d * es + w.T * w.k * 12)
     comb_bytes = R * w.d * es + w.T * w.d * es + w.T * w.k * 8
     kernels = {
         "route": {"ms": seg_ms[0], "bound": "hbm", "GB/s": route_bytes / seg_ms[0] / 1e6,
                   "frac": route_bytes / seg_ms[0] / 1e6 / hbm},
         "dispatch": {"ms": seg_ms[1], "bound": "hbm", "GB/s": disp_bytes / seg_ms[1] / 1e6,
-                     "frac": disp_bytes / seg_ms[1] / 1e6 / hbm},
+                     "frac": disp_bytes / seg_ms[1] / 1e6 / hbm,
+                     "x_perm": "not materialised (GEMM 1 gathers rows of x)" if gather
+                     else "materialised"},
         "expert_up": {"ms": seg_ms[2], "bound": "tensor", "TFLOP/s": up_tf,
                       "frac": up_tf / peak_t},
         "expert_down": {"ms": seg_ms[3], "bound": "tensor",

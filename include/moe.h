@@ -172,6 +172,13 @@ int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx,
                  void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
                  int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* a2, tables only: moe_dispatch without the permuted copy of x (x_perm).  Same
+ * counts, kept, offsets, row_token and slot_row.  For moe_expert_up_gather, which
+ * reads the rows of x through row_token itself. */
+int moe_dispatch_rows(const moe_params_t *p, const int32_t *topk_idx, int32_t *row_token,
+                      int32_t *slot_row, int32_t *counts, int32_t *kept, int32_t *offsets,
+                      void *ws, size_t ws_bytes, void *stream);
+
 /* a2 without a workspace.  The pages have no counterpart: this is a service
  * for callers that cannot allocate device memory or pass a workspace (for
  * example a host engine whose plugin interface hands a layer only its input and
@@ -196,6 +203,18 @@ int moe_dispatch_noalloc(const moe_params_t *p, const void *x, const int32_t *to
  * f32: CUDA-core FMA in f32 (no TF32).  Row tables stay on the device. */
 int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                   const void *W13_e, void *h, void *ws, size_t ws_bytes, void *stream);
+
+/* a3 reading the activations in place ["LLaMA-MoE v2", code sample, class Expert]:
+ * h[r] = silu(x[row_token[r]] W1_e^T) * (x[row_token[r]] W3_e^T) for the kept rows
+ * r of expert e.  x [T][d] (unpermuted), row_token from moe_dispatch(_rows); the
+ * tensor-core kernel gathers four rows of x per TMA instruction.  bf16 only
+ * (MOE_ERR_DTYPE otherwise).  Bit-identical to moe_expert_up on x_perm; it saves
+ * the T*k*d x_perm buffer and its copy, but the one-row TMA gathers make the GEMM
+ * about 2.8x slower on B200 (1593 vs 561 us at T=16384, d=4096, 8x1376, top-2),
+ * so moe_forward does not use it. */
+int moe_expert_up_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                         const int32_t *offsets, const void *W13_e, void *h, void *ws,
+                         size_t ws_bytes, void *stream);
 
 /* a4. Second half: out[r] = h[r] W2_e^T.  h [T*k][m8], W2_e packed, out [T*k][d]. */
 int moe_expert_down(const moe_params_t *p, const void *h, const int32_t *offsets,

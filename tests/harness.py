@@ -144,12 +144,18 @@ def check_dispatch(w, inp, p, bufs):
     return d
 
 
+def x_rows_of(inp, dsp, rows):
+    """The activations of kept rows, taken from x through the oracle's row tables."""
+    x = raw(inp["x"])
+    return np.ascontiguousarray(x[dsp["row_token"][rows]])
+
+
 def rel_err(a, b):
     den = np.abs(b).max() if b.size else 0.0
     return float(np.abs(a - b).max() / den) if den > 0 else float(np.abs(a - b).max())
 
 
-def check_expert_rows(w, bufs, dsp, OW, rows=None):
+def check_expert_rows(w, bufs, dsp, OW, rows=None, inp=None):
     """a3/a4 parity on kept rows (the GPU's x_perm through the oracle's experts)."""
     R = dsp["R"]
     if R == 0:
@@ -157,7 +163,7 @@ def check_expert_rows(w, bufs, dsp, OW, rows=None):
     if rows is None:
         rows = np.arange(R)
     expert_of_row = np.searchsorted(dsp["offsets"], rows, side="right") - 1
-    x_rows = raw(bufs.x_perm[torch.from_numpy(rows).long().cuda()])
+    x_rows = x_rows_of(inp, dsp, rows)
     out_ref, h_ref = oracle.expert_ffn(*OW, x_rows, expert_of_row, want_h=True)
     out_g = f64(bufs.out[torch.from_numpy(rows).long().cuda()])
     h_g = f64(bufs.h[torch.from_numpy(rows).long().cuda()][:, :w.m])
@@ -168,7 +174,7 @@ def check_expert_rows(w, bufs, dsp, OW, rows=None):
     return eo
 
 
-def check_y(w, bufs, r, dsp, OW, tokens):
+def check_y(w, bufs, r, dsp, OW, tokens, inp=None):
     """End-to-end y for `tokens` (non-tie tokens): y_ref from the oracle's experts and
     gate weights over the dispatch of the GPU's indices."""
     tokens = np.asarray(tokens, np.int64)
@@ -179,7 +185,7 @@ def check_y(w, bufs, r, dsp, OW, tokens):
     y_g = f64(bufs.y[torch.from_numpy(tokens).cuda()])
     if len(rows):
         expert_of_row = np.searchsorted(dsp["offsets"], rows, side="right") - 1
-        x_rows = raw(bufs.x_perm[torch.from_numpy(rows).long().cuda()])
+        x_rows = x_rows_of(inp, dsp, rows)
         out_u = oracle.expert_ffn(*OW, x_rows, expert_of_row)
         remap = {int(v): i for i, v in enumerate(rows)}
         sr_local = np.vectorize(lambda v: remap.get(int(v), -1))(sr).astype(np.int32)

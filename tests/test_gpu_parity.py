@@ -66,11 +66,11 @@ def _full_check(w, inp, rows_sample=None, tok_sample=None, capacity=None):
     rows = None
     if rows_sample is not None and dsp["R"] > rows_sample:
         rows = np.sort(np.random.default_rng(w.seed).choice(dsp["R"], rows_sample, replace=False))
-    H.check_expert_rows(w, bufs, dsp, OW, rows)
+    H.check_expert_rows(w, bufs, dsp, OW, rows, inp=inp)
     good = np.nonzero(~ties)[0]
     if tok_sample is not None and len(good) > tok_sample:
         good = np.sort(np.random.default_rng(w.seed + 1).choice(good, tok_sample, replace=False))
-    e = H.check_y(w, bufs, r, dsp, OW, good)
+    e = H.check_y(w, bufs, r, dsp, OW, good, inp=inp)
     H.check_loss(w, bufs, r)
     return dict(p=p, bufs=bufs, ws=ws, r=r, ties=ties, dsp=dsp, y_err=e, weights=weights)
 
@@ -143,6 +143,37 @@ def test_steps_reproduce_forward_bit_exactly():
         assert torch.equal(getattr(bufs, n), getattr(b2, n)), n
     assert torch.equal(bufs.out[:R], b2.out[:R])
     assert torch.equal(bufs.row_token[:R], b2.row_token[:R])
+
+
+@pytest.mark.parametrize("T", [600, 2500], ids=["one_sm_kernel", "two_sm_kernel"])
+def test_gather_gemm_equals_permuted_copy_gemm(T):
+    """moe_expert_up_gather (rows of x fetched by TMA gather through row_token) gives
+    the same bytes as moe_expert_up on the permuted copy x_perm, and
+    moe_dispatch_rows the same tables as moe_dispatch."""
+    w = W("gather", T=T, d=320, d_ff=8 * 176, E=8, k=2, noisy=True, cf=1.2, seed=45)
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    W13_e, W2_e = H.gpu_weights(w, inp, ws)
+    a, b = moe.ForwardBuffers(p), moe.ForwardBuffers(p)
+    x, Wg, Wn, eps = (inp[n].cuda() for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_route(p, x, Wg, Wn, eps, None, ws, a.topk_idx, a.topk_w, a.probs_sum, a.importance)
+    moe.moe_dispatch(p, x, a.topk_idx, ws, a.x_perm, a.row_token, a.slot_row, a.counts, a.kept,
+                     a.offsets)
+    moe.moe_dispatch_rows(p, a.topk_idx, ws, b.row_token, b.slot_row, b.counts, b.kept,
+                          b.offsets)
+    moe.moe_expert_up(p, a.x_perm, a.offsets, W13_e, a.h, ws)
+    moe.moe_expert_up_gather(p, x, b.row_token, b.offsets, W13_e, b.h, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    R = int(a.offsets[-1])
+    for n in ("counts", "kept", "offsets", "slot_row"):
+        assert torch.equal(getattr(a, n), getattr(b, n)), n
+    assert torch.equal(a.row_token[:R], b.row_token[:R])
+    m = w.m
+    assert torch.equal(a.h[:R, :m], b.h[:R, :m])
+    # and the permuted copy itself is x's rows in dispatch order
+    assert torch.equal(a.x_perm[:R], x[a.row_token[:R].long()])
 
 
 def test_empty_batch():

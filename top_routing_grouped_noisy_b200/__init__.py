@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "MoeError", "Params", "lib", "params", "moe_capacity", "moe_version", "moe_launch_count",
     "moe_partition_experts", "moe_workspace_size", "Workspace", "moe_route", "moe_dispatch",
-    "moe_dispatch_noalloc",
+    "moe_dispatch_noalloc", "moe_dispatch_rows", "moe_expert_up_gather",
     "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
     "packed_w13_elems", "packed_w2_elems", "h_ld",
@@ -94,6 +94,8 @@ def lib():
             "moe_route": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v, sz, v]),
             "moe_dispatch": (C.c_int, [P, v, v, v, v, v, v, v, v, v, sz, v]),
             "moe_dispatch_noalloc": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v]),
+            "moe_dispatch_rows": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
+            "moe_expert_up_gather": (C.c_int, [P, v, v, v, v, v, v, sz, v]),
             "moe_expert_up": (C.c_int, [P, v, v, v, v, v, sz, v]),
             "moe_expert_down": (C.c_int, [P, v, v, v, v, v, sz, v]),
             "moe_expert_ffn": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
@@ -232,6 +234,19 @@ def moe_dispatch(p, x, topk_idx, ws, x_perm, row_token, slot_row, counts, kept, 
     _check(lib().moe_dispatch(C.byref(p), _p(x), _p(topk_idx), _p(x_perm), _p(row_token),
                               _p(slot_row), _p(counts), _p(kept), _p(offsets), ws.ptr,
                               ws.nbytes, _stream(stream)))
+
+
+def moe_dispatch_rows(p, topk_idx, ws, row_token, slot_row, counts, kept, offsets, stream=None):
+    """a2 tables only (no permuted copy of x)."""
+    _check(lib().moe_dispatch_rows(C.byref(p), _p(topk_idx), _p(row_token), _p(slot_row),
+                                   _p(counts), _p(kept), _p(offsets), ws.ptr, ws.nbytes,
+                                   _stream(stream)))
+
+
+def moe_expert_up_gather(p, x, row_token, offsets, W13_e, h, ws, stream=None):
+    """a3 gathering rows of x through row_token (bf16)."""
+    _check(lib().moe_expert_up_gather(C.byref(p), _p(x), _p(row_token), _p(offsets), _p(W13_e),
+                                      _p(h), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def moe_dispatch_noalloc(p, x, topk_idx, x_perm, row_token, slot_row, counts, kept, offsets,

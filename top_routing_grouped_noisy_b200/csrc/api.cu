@@ -312,6 +312,53 @@ int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx, 
     return after_launch(fn, e);
 }
 
+int moe_dispatch_rows(const moe_params_t *p, const int32_t *topk_idx, int32_t *row_token,
+                      int32_t *slot_row, int32_t *counts, int32_t *kept, int32_t *offsets,
+                      void *ws, size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_dispatch_rows";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    REQUIRE_TOK(topk_idx);
+    REQUIRE_TOK(row_token);
+    REQUIRE_TOK(slot_row);
+    REQUIRE_PTR(counts);
+    REQUIRE_PTR(kept);
+    REQUIRE_PTR(offsets);
+    if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+        return rc;
+    char *w = static_cast<char *>(ws);
+    cudaError_t e = launch_dispatch(p, nullptr, topk_idx, nullptr, row_token, slot_row, counts,
+                                    kept, offsets, w, reinterpret_cast<int32_t *>(w),
+                                    (cudaStream_t)stream);
+    return after_launch(fn, e);
+}
+
+int moe_expert_up_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                         const int32_t *offsets, const void *W13_e, void *h, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_expert_up_gather";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    if (p->dtype != MOE_BF16)
+        return fail(MOE_ERR_DTYPE, "%s: the gathering expert GEMM is bf16 only", fn);
+    REQUIRE_TOK(x);
+    REQUIRE_TOK(row_token);
+    REQUIRE_PTR(offsets);
+    REQUIRE_PTR(W13_e);
+    REQUIRE_TOK(h);
+    if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+        return rc;
+    if (p->T == 0)
+        return ok();
+    cudaError_t e = launch_up_tc_gather(p, x, row_token, offsets, W13_e, h,
+                                        reinterpret_cast<int32_t *>(ws), (cudaStream_t)stream);
+    return after_launch(fn, e);
+}
+
 int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                   const void *W13_e, void *h, void *ws, size_t ws_bytes, void *stream)
 {

@@ -173,6 +173,8 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
             }
         }
     }
+    if (x_perm == nullptr)  // tables only: the expert GEMM gathers rows of x itself
+        return;
     __syncthreads();
     const int ntok = (int)((int64_t)T - t0 < kDispatchChunk ? (int64_t)T - t0 : kDispatchChunk);
     // the row's 16-byte vectors [v0, v1) of this CTA (blockIdx.y splits rows when T is small)
@@ -236,7 +238,8 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
         return e;
     const int nch = ceil_div(p->T, kDispatchChunk);
     const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
-    dispatch_scatter_kernel<<<dim3(nch, scatter_split(nch, row_bytes)), 256, 0, s>>>(
+    const unsigned ysplit = x_perm != nullptr ? scatter_split(nch, row_bytes) : 1u;
+    dispatch_scatter_kernel<<<dim3(nch, ysplit), 256, 0, s>>>(
         (const char *)x, row_bytes, idx, p->T, p->k, p->E, hist, kept, offsets, (char *)x_perm,
         row_token, slot_row);
     count_launch();

@@ -166,6 +166,19 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+// Four rows r0..r3 of a 2-D tensor (box one row high), 64 columns from `col`,
+// written as four consecutive 128-byte rows at dst (128-byte swizzle as a tile).
+__device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint32_t bar, uint32_t dst,
+                                            int col, int r0, int r1, int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2),
+        "r"(r3)
+        : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -224,13 +237,16 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     return t;
 }
 
-template <int EPI>
+// GATHER: tmA covers the unpermuted activations x [T][K] with a box one row high;
+// the A rows of a tile are gathered through row_token (4 rows per TMA, one TMA
+// per producer lane) instead of being read from a permuted copy.
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const int32_t *__restrict__ offsets, int E, int N, int K,
                         bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
-                        uint64_t wait_ns)
+                        uint64_t wait_ns, const int32_t *__restrict__ row_token)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -285,35 +301,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t smem_base = smem_u32(smem);
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer
-            int stage = 0;
-            uint32_t phase = 0;
-            int64_t fills = 0;
-            for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-                const Tile t = decode_tile(aux, tile, n_tiles);
-                bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns, abort_flag,
-                                   status)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = smem_u32(&aux->full[stage]);
-                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    mbar_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(&tmA, fb, sa, kb * BK, t.row0);
-                    tma_load_3d(&tmB, fb, sa + A_BYTES, kb * BK, t.n0, t.e);
-                    ++fills;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+        // -------------------------------------------------------------- TMA producer
+        // lane 0 waits for and arms each stage; in GATHER mode every lane then
+        // fetches four A rows, otherwise lane 0 copies the A box
+        int stage = 0;
+        uint32_t phase = 0;
+        int64_t fills = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, (int)*abort_flag, 0))
+                break;
+            const Tile t = decode_tile(aux, tile, n_tiles);
+            int src[4] = {0, 0, 0, 0};
+            if constexpr (GATHER) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = t.row0 + 4 * lane + i;
+                    src[i] = row_token[r < t.row_end ? r : t.row_end - 1];
                 }
-                if (!ok)
-                    break;
             }
-            // drain: the last fill of every stage has landed before the CTA may exit
+            bool ok = true;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                int w_ok = 1;
+                if (lane == 0)
+                    w_ok = mbar_wait(smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns,
+                                     abort_flag, status);
+                if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_u32(&aux->full[stage]);
+                const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                if (lane == 0)
+                    mbar_expect_tx(fb, STAGE_BYTES);
+                __syncwarp();
+                if constexpr (GATHER)
+                    tma_gather4(&tmA, fb, sa + lane * 4 * 128, kb * BK, src[0], src[1], src[2],
+                                src[3]);
+                else if (lane == 0)
+                    tma_load_2d(&tmA, fb, sa, kb * BK, t.row0);
+                if (lane == 0)
+                    tma_load_3d(&tmB, fb, sa + A_BYTES, kb * BK, t.n0, t.e);
+                ++fills;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok)
+                break;
+        }
+        // drain: the last fill of every stage has landed before the CTA may exit
+        if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
                 const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
                 if (n > 0)
@@ -543,6 +581,18 @@ __device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *map, uint32_
         : "memory");
 }
 
+__device__ __forceinline__ void tma_gather4_pair(const CUtensorMap *map, uint32_t bar_cluster,
+                                                 uint32_t dst, int col, int r0, int r1, int r2,
+                                                 int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+        "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(col), "r"(r0), "r"(r1),
+        "r"(r2), "r"(r3)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
 {
     asm volatile(
@@ -591,13 +641,13 @@ __device__ __forceinline__ PairTile decode_pair_tile(const Aux *aux, int tile)
     return t;
 }
 
-template <int EPI>
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
                             const int32_t *__restrict__ offsets, int E, int N, int K,
                             bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
-                            uint64_t wait_ns)
+                            uint64_t wait_ns, const int32_t *__restrict__ row_token)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -655,43 +705,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t smem_base = tc::smem_u32(smem);
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer (both)
-            int stage = 0;
-            uint32_t phase = 0;
-            int64_t fills = 0;
-            for (int tile = cluster_id; tile < total && !*abort_flag; tile += nclusters) {
-                const PairTile t = decode_pair_tile(aux, tile);
-                bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!tc::mbar_wait(tc::smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns,
-                                       abort_flag, status)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = tc::smem_u32(&aux->full[stage]);
-                    if (leader)
-                        tc::mbar_expect_tx(fb, 2 * STAGE_BYTES);
-                    const uint32_t fb0 = map_rank(fb, 0);
-                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+        // -------------------------------------------------------------- TMA producer (both)
+        int stage = 0;
+        uint32_t phase = 0;
+        int64_t fills = 0;
+        for (int tile = cluster_id; tile < total; tile += nclusters) {
+            if (__shfl_sync(0xffffffffu, (int)*abort_flag, 0))
+                break;
+            const PairTile t = decode_pair_tile(aux, tile);
+            int src[4] = {0, 0, 0, 0};
+            if constexpr (GATHER) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = t.row0 + (int)rank * BM + 4 * lane + i;
+                    src[i] = row_token[r < t.row_end ? r : t.row_end - 1];
+                }
+            }
+            bool ok = true;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                int w_ok = 1;
+                if (lane == 0)
+                    w_ok = tc::mbar_wait(tc::smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns,
+                                         abort_flag, status);
+                if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = tc::smem_u32(&aux->full[stage]);
+                if (lane == 0 && leader)
+                    tc::mbar_expect_tx(fb, 2 * STAGE_BYTES);
+                __syncwarp();
+                const uint32_t fb0 = map_rank(fb, 0);
+                const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                if constexpr (GATHER)
+                    tma_gather4_pair(&tmA, fb0, sa + lane * 4 * 128, kb * BK, src[0], src[1],
+                                     src[2], src[3]);
+                else if (lane == 0)
                     tma_load_2d_pair(&tmA, fb0, sa, kb * BK, t.row0 + (int)rank * BM);
+                if (lane == 0)
                     tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, kb * BK, t.n0 + (int)rank * BNH,
                                      t.e);
-                    ++fills;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                ++fills;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
-                if (!ok)
-                    break;
             }
-            if (leader) {  // the leader's full barriers count both CTAs' bytes
-                for (int s = 0; s < STAGES; ++s) {
-                    const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
-                    if (n > 0)
-                        tc::mbar_drain(tc::smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
-                }
+            if (!ok)
+                break;
+        }
+        if (lane == 0 && leader) {  // the leader's full barriers count both CTAs' bytes
+            for (int s = 0; s < STAGES; ++s) {
+                const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
+                if (n > 0)
+                    tc::mbar_drain(tc::smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
             }
         }
     } else if (warp == 1) {
@@ -882,7 +949,7 @@ static cudaError_t make_map(CUtensorMap *map, const void *base, int rank, const 
 struct DevInfo {
     int sms = 0;
     int pair_clusters = 0;
-    bool attr[4] = {false, false, false, false};
+    bool attr[8] = {false, false, false, false, false, false, false, false};
 };
 static std::mutex g_dev_mu;
 static DevInfo g_dev[64];
@@ -915,12 +982,22 @@ static cudaError_t prepare_device(DevInfo **out)
         if (e != cudaSuccess)
             return e;
     }
-    if ((e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU>, SMEM_BYTES, di.attr[0])) != cudaSuccess ||
-        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE>, SMEM_BYTES, di.attr[1])) != cudaSuccess ||
-        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU>, tc2::SMEM_BYTES,
-                           di.attr[2])) != cudaSuccess ||
-        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_STORE>, tc2::SMEM_BYTES,
-                           di.attr[3])) != cudaSuccess)
+    if ((e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, false>, SMEM_BYTES, di.attr[0])) !=
+            cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, false>, SMEM_BYTES, di.attr[1])) !=
+            cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, true>, SMEM_BYTES, di.attr[2])) !=
+            cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, true>, SMEM_BYTES, di.attr[3])) !=
+            cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU, false>, tc2::SMEM_BYTES,
+                           di.attr[4])) != cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_STORE, false>, tc2::SMEM_BYTES,
+                           di.attr[5])) != cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU, true>, tc2::SMEM_BYTES,
+                           di.attr[6])) != cudaSuccess ||
+        (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_STORE, true>, tc2::SMEM_BYTES,
+                           di.attr[7])) != cudaSuccess)
         return e;
     if (di.pair_clusters == 0) {
         cudaLaunchConfig_t cfg = {};
@@ -935,7 +1012,8 @@ static cudaError_t prepare_device(DevInfo **out)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU, false>,
+                                           &cfg);
         if (e != cudaSuccess)
             return e;
         di.pair_clusters = n > 0 ? n : 1;
@@ -948,12 +1026,14 @@ static cudaError_t prepare_device(DevInfo **out)
 // the few tiles over more SMs.
 constexpr int64_t kPairMinRows = 4096;
 
-// One grouped GEMM launch.  A: [rows][a_ld] activations (K extent a_k); B:
-// [E][b_rows][b_ld] expert weights (K extent b_k, N = b_rows); out: [rows][ld_out],
-// first n_valid columns written.
+// One grouped GEMM launch.  A: [a_rows][a_ld] activations (K extent a_k), read in
+// expert-grouped row order, or -- when row_token is given -- gathered: tile row r is
+// row row_token[r] of A; B: [E][b_rows][b_ld] expert weights (K extent b_k, N =
+// b_rows); out: [rows][ld_out], first n_valid columns written; rows = T*k.
 template <int EPI>
-static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t rows,
-                               const void *B, uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
+static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a_rows,
+                               const int32_t *row_token, uint64_t rows, const void *B,
+                               uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
                                const int32_t *offsets, int E, bf16 *out, int ld_out, int n_valid,
                                int32_t *status, cudaStream_t s)
 {
@@ -962,9 +1042,10 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     if (e != cudaSuccess)
         return e;
     const bool pair = (int64_t)rows >= kPairMinRows;
+    const bool gather = row_token != nullptr;
     CUtensorMap ta, tb;
-    const uint64_t da[2] = {a_k, rows}, sa[1] = {a_ld * 2};
-    const uint32_t ba[2] = {BK, BM};
+    const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
+    const uint32_t ba[2] = {BK, gather ? 1u : (uint32_t)BM};  // gather4 boxes are one row high
     const uint64_t db[3] = {b_k, b_rows, (uint64_t)E};
     const uint64_t sb[2] = {b_ld * 2, b_rows * b_ld * 2};
     const uint32_t bb[3] = {BK, pair ? (uint32_t)tc2::BNH : (uint32_t)BN, 1};
@@ -975,8 +1056,12 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     const uint64_t wait_ns = wait_limit_ns();
     const int N = (int)b_rows, K = (int)a_k;
     if (!pair) {
-        grouped_gemm_kernel<EPI><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
-            ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns);
+        if (gather)
+            grouped_gemm_kernel<EPI, true><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
+                ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+        else
+            grouped_gemm_kernel<EPI, false><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
+                ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
@@ -991,8 +1076,11 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI>, ta, tb, offsets, E, N, K,
-                              out, ld_out, n_valid, status, wait_ns);
+    if (gather)
+        return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, true>, ta, tb, offsets,
+                                  E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+    return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, false>, ta, tb, offsets, E,
+                              N, K, out, ld_out, n_valid, status, wait_ns, row_token);
 }
 
 }  // namespace tc
@@ -1004,8 +1092,21 @@ cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_
 {
     const uint64_t d = p->d, m = p->m, m16 = round_up(p->m, 16), m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    cudaError_t e = launch_gemm<EPI_SWIGLU>(x_perm, d, d, rows, W13, d, d, 2 * m16, offsets, p->E,
-                                            (bf16 *)h, (int)m8, (int)m, status, s);
+    cudaError_t e = launch_gemm<EPI_SWIGLU>(x_perm, d, d, rows, nullptr, rows, W13, d, d, 2 * m16,
+                                            offsets, p->E, (bf16 *)h, (int)m8, (int)m, status, s);
+    count_launch();
+    return e;
+}
+
+cudaError_t launch_up_tc_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                                const int32_t *offsets, const void *W13, void *h,
+                                int32_t *status, cudaStream_t s)
+{
+    const uint64_t d = p->d, m = p->m, m16 = round_up(p->m, 16), m8 = round_up(p->m, 8);
+    const uint64_t rows = (uint64_t)p->T * p->k;
+    cudaError_t e = launch_gemm<EPI_SWIGLU>(x, d, d, (uint64_t)p->T, row_token, rows, W13, d, d,
+                                            2 * m16, offsets, p->E, (bf16 *)h, (int)m8, (int)m,
+                                            status, s);
     count_launch();
     return e;
 }
@@ -1015,8 +1116,8 @@ cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *
 {
     const uint64_t d = p->d, m = p->m, m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    cudaError_t e = launch_gemm<EPI_STORE>(h, m, m8, rows, W2, m, m8, d, offsets, p->E,
-                                           (bf16 *)out, (int)d, (int)d, status, s);
+    cudaError_t e = launch_gemm<EPI_STORE>(h, m, m8, rows, nullptr, rows, W2, m, m8, d, offsets,
+                                           p->E, (bf16 *)out, (int)d, (int)d, status, s);
     count_launch();
     return e;
 }

@@ -70,6 +70,9 @@ cudaError_t launch_down_simt(const moe_params_t *p, const float *h, const int32_
 // a3 / a4 for bf16 (tcgen05 tensor cores, TMA, TMEM)
 cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                          const void *W13, void *h, int32_t *status, cudaStream_t s);
+cudaError_t launch_up_tc_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                                const int32_t *offsets, const void *W13, void *h,
+                                int32_t *status, cudaStream_t s);
 cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
                            const void *W2, void *out, int32_t *status, cudaStream_t s);
 
