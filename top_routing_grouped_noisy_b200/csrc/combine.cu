@@ -13,6 +13,10 @@
 
 namespace moe {
 
+// Each thread produces VPT adjacent 16-byte vectors of one token's output; all k
+// slot rows of all of them are requested before any is used.
+constexpr int kCombineVPT = 2;
+
 template <typename E_T, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ out,
                                                       const int32_t *__restrict__ slot_row,
@@ -20,14 +24,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ ou
                                                       int k, float scale, E_T *__restrict__ y)
 {
     constexpr int VN = Vec<E_T>::N;
+    constexpr int VPT = kCombineVPT;
     const int nv = d / VN;
-    const int64_t items = (int64_t)T * nv;
+    const int ng = (nv + VPT - 1) / VPT;  // vector groups per token
+    const int64_t items = (int64_t)T * ng;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = i / nv;
-        const int v = (int)(i - t * nv);
-        // all k rows are requested before any is used
-        uint4 raw[KMAX];
+        const int64_t t = i / ng;
+        const int v0 = (int)(i - t * ng) * VPT;
+        uint4 raw[KMAX][VPT];
         float g[KMAX];
         bool kept[KMAX];
 #pragma unroll
@@ -35,41 +40,49 @@ __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ ou
             const int32_t row = j < k ? slot_row[t * k + j] : -1;
             kept[j] = row >= 0;
             g[j] = kept[j] ? w[t * k + j] : 0.f;
-            raw[j] = kept[j] ? ld_nc_na(out + (int64_t)row * d + (int64_t)v * VN)
-                             : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < VPT; ++u)
+                raw[j][u] = (kept[j] && v0 + u < nv)
+                                ? ld_nc_na(out + (int64_t)row * d + (int64_t)(v0 + u) * VN)
+                                : make_uint4(0, 0, 0, 0);
         }
-        float acc[VN];
 #pragma unroll
-        for (int q = 0; q < VN; ++q)
-            acc[q] = 0.f;
+        for (int u = 0; u < VPT; ++u) {
+            if (v0 + u >= nv)
+                break;
+            float acc[VN];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (!kept[j])
-                continue;
-            float f[VN];
-            if constexpr (sizeof(E_T) == 2) {
-                bf16x8_to_f32(raw[j], f);
-            } else {
-                f[0] = __uint_as_float(raw[j].x);
-                f[1] = __uint_as_float(raw[j].y);
-                f[2] = __uint_as_float(raw[j].z);
-                f[3] = __uint_as_float(raw[j].w);
+            for (int q = 0; q < VN; ++q)
+                acc[q] = 0.f;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (!kept[j])
+                    continue;
+                float f[VN];
+                if constexpr (sizeof(E_T) == 2) {
+                    bf16x8_to_f32(raw[j][u], f);
+                } else {
+                    f[0] = __uint_as_float(raw[j][u].x);
+                    f[1] = __uint_as_float(raw[j][u].y);
+                    f[2] = __uint_as_float(raw[j][u].z);
+                    f[3] = __uint_as_float(raw[j][u].w);
+                }
+#pragma unroll
+                for (int q = 0; q < VN; ++q)
+                    acc[q] = fmaf(g[j], f[q], acc[q]);
             }
 #pragma unroll
             for (int q = 0; q < VN; ++q)
-                acc[q] = fmaf(g[j], f[q], acc[q]);
+                acc[q] *= scale;
+            uint4 o;
+            if constexpr (sizeof(E_T) == 2) {
+                o = f32x8_to_bf16(acc);
+            } else {
+                o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
+                               __float_as_uint(acc[2]), __float_as_uint(acc[3]));
+            }
+            st_v4(y + t * d + (int64_t)(v0 + u) * VN, o);
         }
-#pragma unroll
-        for (int q = 0; q < VN; ++q)
-            acc[q] *= scale;
-        uint4 o;
-        if constexpr (sizeof(E_T) == 2) {
-            o = f32x8_to_bf16(acc);
-        } else {
-            o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]),
-                           __float_as_uint(acc[2]), __float_as_uint(acc[3]));
-        }
-        st_v4(y + t * d + (int64_t)v * VN, o);
     }
 }
 
@@ -101,7 +114,7 @@ cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t
 {
     const float scale = p->rescale ? (float)p->E / (float)p->k : 1.0f;
     const int VN = p->dtype == MOE_BF16 ? 8 : 4;
-    const int64_t items = (int64_t)p->T * (p->d / VN);
+    const int64_t items = (int64_t)p->T * ((p->d / VN + kCombineVPT - 1) / kCombineVPT);
     const int64_t blocks = (items + 255) / 256;
     const unsigned grid = (unsigned)(blocks < (1 << 30) ? blocks : (1 << 30));
 #define MOE_COMBINE(KM)                                                                        \

@@ -14,11 +14,12 @@
 // in TMEM, double-buffered (2 x 256 columns), so the epilogue of one tile
 // overlaps the main loop of the next.
 //
-// Warp roles (192 threads, one CTA per SM, grid = #SMs):
-//   warp 0     TMA producer (one lane)
+// Warp roles (320 threads, one CTA per SM, grid = #SMs):
+//   warp 0     TMA producer (lane 0; every lane in the row-gathering variant)
 //   warp 1     TMEM allocator and MMA issuer (one lane)
-//   warps 2-5  epilogue: tcgen05.ld -> registers -> bf16 -> global; warp w reads
-//              TMEM lanes 32*(w%4)..+31, i.e. tile rows, one row per thread.
+//   warps 2-9  epilogue: tcgen05.ld -> registers -> bf16 -> global; warp w reads
+//              TMEM lanes 32*(w%4)..+31, i.e. tile rows, one row per thread, and
+//              half of the 256 accumulator columns (warps 2-5 the first half).
 // For a3 the packed W13 layout puts, in each 32-row group, 16 W1 rows and then the
 // 16 W3 rows of the same 16 neurons, so each 32-column TMEM load holds the gate
 // and up values of 16 neurons of the thread's row.
@@ -48,7 +49,8 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int EPI_WARPS = 8;
 constexpr uint64_t kDrainNs = 1000000000ull;  // bound of the drain waits on exit
 
 enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
@@ -199,6 +201,28 @@ __device__ __forceinline__ void umma_commit(uint32_t bar)
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_wait_ld()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 consecutive f32 accumulator columns of this thread's TMEM lane; the registers
+// are valid only after tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
@@ -213,6 +237,65 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
           "=r"(v[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Epilogue of one accumulator row held by this thread: 32-column chunks
+// [c_first, c_first + n_chunks) of the tile starting at output column n0.
+//   SwiGLU: columns 32c..32c+15 are gate and 32c+16..32c+31 up of neurons
+//           n0/2 + 16c + i; h = silu(gate) * up, rounded to bf16.
+//   Store:  the 32 columns rounded to bf16.
+// Two chunks are requested from TMEM before one wait.
+template <int EPI>
+__device__ __forceinline__ void epilogue_row(uint32_t taddr, int c_first, int n_chunks, int row,
+                                             bool rv, int n0, bf16 *__restrict__ out,
+                                             int ld_out, int n_valid)
+{
+#pragma unroll 1
+    for (int c = c_first; c < c_first + n_chunks; c += 2) {
+        uint32_t v[2][32];
+        tmem_ld32_async(taddr + (uint32_t)(c * 32), v[0]);
+        tmem_ld32_async(taddr + (uint32_t)((c + 1) * 32), v[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int cc = c + q2;
+            if constexpr (EPI == EPI_SWIGLU) {
+                const int nb = n0 / 2 + cc * 16;
+                float hv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float g = __uint_as_float(v[q2][i]);
+                    const float u = __uint_as_float(v[q2][16 + i]);
+                    hv[i] = g / (1.0f + __expf(-g)) * u;
+                }
+                if (rv && nb < n_valid) {
+                    bf16 *dst = out + (int64_t)row * ld_out + nb;
+                    if (nb + 16 <= n_valid) {
+                        st_v4(dst, f32x8_to_bf16(hv));
+                        st_v4(dst + 8, f32x8_to_bf16(hv + 8));
+                    } else {
+                        for (int i = 0; i < 16 && nb + i < n_valid; ++i)
+                            dst[i] = __float2bfloat16_rn(hv[i]);
+                    }
+                }
+            } else {
+                const int col = n0 + cc * 32;
+                if (rv) {
+                    bf16 *dst = out + (int64_t)row * ld_out + col;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (col + q * 8 < n_valid) {  // n_valid is a multiple of 8
+                            float f[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                f[i] = __uint_as_float(v[q2][q * 8 + i]);
+                            st_v4(dst + q * 8, f32x8_to_bf16(f));
+                        }
+                    }
+                }
+            }
+        }
+    }
 }
 
 struct Tile {
@@ -262,7 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int a = 0; a < ACC; ++a) {
             mbar_init(smem_u32(&aux->tfull[a]), 1);
-            mbar_init(smem_u32(&aux->tempty[a]), 4);
+            mbar_init(smem_u32(&aux->tempty[a]), EPI_WARPS);
         }
         mbar_init(smem_u32(&aux->drain), 1);
         aux->abort_flag = 0;
@@ -407,8 +490,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue
+        // warp w reads TMEM lanes 32*(w%4)..+31 (tile rows); warps 2-5 take columns
+        // 0..127 of the accumulator, warps 6-9 columns 128..255
         const int wq = warp & 3;
         const int lane_base = wq * 32;
+        const int c_first = ((warp - 2) / 4) * (BN / 64);
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -417,48 +503,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
             tc_fence_after();
             const int row = t.row0 + lane_base + lane;
-            const bool rv = row < t.row_end;
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(taddr + (uint32_t)(c * 32), v);
-                if constexpr (EPI == EPI_SWIGLU) {
-                    const int nb = t.n0 / 2 + c * 16;  // first neuron of this 32-column group
-                    float hv[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float g = __uint_as_float(v[i]);
-                        const float u = __uint_as_float(v[16 + i]);
-                        hv[i] = g / (1.0f + __expf(-g)) * u;
-                    }
-                    if (rv && nb < n_valid) {
-                        bf16 *dst = out + (int64_t)row * ld_out + nb;
-                        if (nb + 16 <= n_valid) {
-                            st_v4(dst, f32x8_to_bf16(hv));
-                            st_v4(dst + 8, f32x8_to_bf16(hv + 8));
-                        } else {
-                            for (int i = 0; i < 16 && nb + i < n_valid; ++i)
-                                dst[i] = __float2bfloat16_rn(hv[i]);
-                        }
-                    }
-                } else {
-                    const int col = t.n0 + c * 32;
-                    if (rv) {
-                        bf16 *dst = out + (int64_t)row * ld_out + col;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            if (col + q * 8 < n_valid) {  // n_valid is a multiple of 8
-                                float f[8];
-#pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    f[i] = __uint_as_float(v[q * 8 + i]);
-                                st_v4(dst + q * 8, f32x8_to_bf16(f));
-                            }
-                        }
-                    }
-                }
-            }
+            epilogue_row<EPI>(taddr, c_first, BN / 64, row, row < t.row_end, t.n0, out, ld_out,
+                              n_valid);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -507,7 +554,8 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int EPI_WARPS = 8;
 constexpr uint64_t kAbortSettleNs = 200000ull;  // pause before exit after an abort
 
 struct Aux {
@@ -666,7 +714,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int a = 0; a < ACC; ++a) {
             tc::mbar_init(tc::smem_u32(&aux->tfull[a]), 1);
-            tc::mbar_init(tc::smem_u32(&aux->tempty[a]), 8);
+            tc::mbar_init(tc::smem_u32(&aux->tempty[a]), 2 * EPI_WARPS);
         }
         tc::mbar_init(tc::smem_u32(&aux->drain), 1);
         aux->abort_flag = 0;
@@ -811,6 +859,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // -------------------------------------------------------------- epilogue (both)
         const int wq = warp & 3;
         const int lane_base = wq * 32;
+        const int c_first = ((warp - 2) / 4) * (BN / 64);
         const uint32_t tempty0 = map_rank(tc::smem_u32(&aux->tempty[0]), 0);
         const uint32_t tempty1 = map_rank(tc::smem_u32(&aux->tempty[1]), 0);
         int acc = 0;
@@ -822,48 +871,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
             tc::tc_fence_after();
             const int row = t.row0 + (int)rank * BM + lane_base + lane;
-            const bool rv = row < t.row_end;
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(taddr + (uint32_t)(c * 32), v);
-                if constexpr (EPI == tc::EPI_SWIGLU) {
-                    const int nb = t.n0 / 2 + c * 16;
-                    float hv[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float g = __uint_as_float(v[i]);
-                        const float u = __uint_as_float(v[16 + i]);
-                        hv[i] = g / (1.0f + __expf(-g)) * u;
-                    }
-                    if (rv && nb < n_valid) {
-                        bf16 *dst = out + (int64_t)row * ld_out + nb;
-                        if (nb + 16 <= n_valid) {
-                            st_v4(dst, f32x8_to_bf16(hv));
-                            st_v4(dst + 8, f32x8_to_bf16(hv + 8));
-                        } else {
-                            for (int i = 0; i < 16 && nb + i < n_valid; ++i)
-                                dst[i] = __float2bfloat16_rn(hv[i]);
-                        }
-                    }
-                } else {
-                    const int col = t.n0 + c * 32;
-                    if (rv) {
-                        bf16 *dst = out + (int64_t)row * ld_out + col;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            if (col + q * 8 < n_valid) {
-                                float f[8];
-#pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    f[i] = __uint_as_float(v[q * 8 + i]);
-                                st_v4(dst + q * 8, f32x8_to_bf16(f));
-                            }
-                        }
-                    }
-                }
-            }
+            tc::epilogue_row<EPI>(taddr, c_first, BN / 64, row, row < t.row_end, t.n0, out,
+                                  ld_out, n_valid);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0)
