@@ -66,7 +66,7 @@ struct Aux {
     int32_t off[MOE_MAX_EXPERTS + 1];
     int32_t tstart[MOE_MAX_EXPERTS + 1];
 };
-constexpr int SMEM_BYTES = 1024 + TILE_BYTES + (int)sizeof(Aux);
+constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux);
 
 // kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, N = BN, M = BM.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -181,6 +181,26 @@ __device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+// Bulk tensor store of a shared-memory box to global memory, tracked as a bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one bulk group of this thread still reads shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// every bulk group of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -239,48 +259,104 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Epilogue of one accumulator row held by this thread: 32-column chunks
+// Output staging: each epilogue warp owns two 2 KB shared-memory slots, each one
+// [32 rows][64 bytes] box laid out with the 64-byte swizzle (16-byte chunk j of row
+// r at r*64 + ((j ^ ((r >> 1) & 3)) * 16)), the layout the output tensor map's
+// SWIZZLE_64B expects; the 32 lanes write their rows without bank conflicts.
+constexpr int kStageSlotBytes = 32 * 64;
+constexpr int kEpiStageBytes = 8 /* warps */ * 2 * kStageSlotBytes;
+
+struct EpiStore {
+    const CUtensorMap *map;  // output [rows][cols], box {32 cols, 32 rows}, SWIZZLE_64B
+    uint32_t slots;          // this warp's two slots (1024-byte aligned)
+    int slot;                // slot to use next
+};
+
+// Writes 32 bf16 values (16 packed words) of this lane's row into the next slot and
+// stores the warp's 32 x 32 box at (col, row0) with one bulk tensor store.
+__device__ __forceinline__ void stage_box(EpiStore &st, const uint32_t (&pk)[16], int col, int row0)
+{
+    const int lane = threadIdx.x & 31;
+    if (lane == 0)
+        bulk_wait_read_1();  // the slot's previous store has finished reading it
+    __syncwarp();
+    const uint32_t base = st.slots + (uint32_t)(st.slot * kStageSlotBytes) + (uint32_t)(lane * 64);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        st_shared_v4(base + (uint32_t)(((j ^ ((lane >> 1) & 3)) << 4)), pk[4 * j], pk[4 * j + 1],
+                     pk[4 * j + 2], pk[4 * j + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(st.map, st.slots + (uint32_t)(st.slot * kStageSlotBytes), col, row0);
+        bulk_commit();
+    }
+    st.slot ^= 1;
+}
+
+// Epilogue of the warp's 32-row slab (one row per lane), 32-column chunks
 // [c_first, c_first + n_chunks) of the tile starting at output column n0.
 //   SwiGLU: columns 32c..32c+15 are gate and 32c+16..32c+31 up of neurons
 //           n0/2 + 16c + i; h = silu(gate) * up, rounded to bf16.
 //   Store:  the 32 columns rounded to bf16.
-// Two chunks are requested from TMEM before one wait.
+// Boxes wholly inside the expert's rows and the valid columns go out through the
+// staging slots as bulk tensor stores; the others are written per lane, masked.
 template <int EPI>
-__device__ __forceinline__ void epilogue_row(uint32_t taddr, int c_first, int n_chunks, int row,
-                                             bool rv, int n0, bf16 *__restrict__ out,
-                                             int ld_out, int n_valid)
+__device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n_chunks,
+                                              int row0, int row_end, int n0,
+                                              bf16 *__restrict__ out, int ld_out, int n_valid,
+                                              EpiStore &st)
 {
+    const int lane = threadIdx.x & 31;
+    const int row = row0 + lane;
+    const bool rv = row < row_end;
+    const bool full_rows = row0 + 32 <= row_end;
 #pragma unroll 1
     for (int c = c_first; c < c_first + n_chunks; c += 2) {
         uint32_t v[2][32];
         tmem_ld32_async(taddr + (uint32_t)(c * 32), v[0]);
         tmem_ld32_async(taddr + (uint32_t)((c + 1) * 32), v[1]);
         tmem_wait_ld();
+        if constexpr (EPI == EPI_SWIGLU) {
+            const int nb = n0 / 2 + c * 16;  // 32 neurons: 16 from each chunk
+            float hv[32];
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            const int cc = c + q2;
-            if constexpr (EPI == EPI_SWIGLU) {
-                const int nb = n0 / 2 + cc * 16;
-                float hv[16];
+            for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float g = __uint_as_float(v[q2][i]);
                     const float u = __uint_as_float(v[q2][16 + i]);
-                    hv[i] = g / (1.0f + __expf(-g)) * u;
+                    hv[q2 * 16 + i] = g / (1.0f + __expf(-g)) * u;
                 }
-                if (rv && nb < n_valid) {
-                    bf16 *dst = out + (int64_t)row * ld_out + nb;
-                    if (nb + 16 <= n_valid) {
-                        st_v4(dst, f32x8_to_bf16(hv));
-                        st_v4(dst + 8, f32x8_to_bf16(hv + 8));
-                    } else {
-                        for (int i = 0; i < 16 && nb + i < n_valid; ++i)
-                            dst[i] = __float2bfloat16_rn(hv[i]);
-                    }
+            if (full_rows && nb + 32 <= n_valid) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(hv[2 * i], hv[2 * i + 1]);
+                stage_box(st, pk, nb, row0);
+            } else if (rv && nb < n_valid) {
+                bf16 *dst = out + (int64_t)row * ld_out + nb;
+                if (nb + 32 <= n_valid) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_v4(dst + 8 * q, f32x8_to_bf16(hv + 8 * q));
+                } else {
+                    for (int i = 0; i < 32 && nb + i < n_valid; ++i)
+                        dst[i] = __float2bfloat16_rn(hv[i]);
                 }
-            } else {
-                const int col = n0 + cc * 32;
-                if (rv) {
+            }
+        } else {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int col = n0 + (c + q2) * 32;
+                if (full_rows && col + 32 <= n_valid) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(__uint_as_float(v[q2][2 * i]),
+                                            __uint_as_float(v[q2][2 * i + 1]));
+                    stage_box(st, pk, col, row0);
+                } else if (rv) {
                     bf16 *dst = out + (int64_t)row * ld_out + col;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -327,6 +403,7 @@ template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO,
                         const int32_t *__restrict__ offsets, int E, int N, int K,
                         bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
                         uint64_t wait_ns, const int32_t *__restrict__ row_token)
@@ -334,7 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES);
+    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES + kEpiStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int32_t *abort_flag = &aux->abort_flag;
 
@@ -352,6 +429,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
     }
     const int n_tiles = (N + BN - 1) / BN;
     if (warp == 2) {
@@ -495,6 +573,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int wq = warp & 3;
         const int lane_base = wq * 32;
         const int c_first = ((warp - 2) / 4) * (BN / 64);
+        EpiStore st{&tmO, smem_base + TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -502,10 +581,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!mbar_wait(smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag, status))
                 break;
             tc_fence_after();
-            const int row = t.row0 + lane_base + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-            epilogue_row<EPI>(taddr, c_first, BN / 64, row, row < t.row_end, t.n0, out, ld_out,
-                              n_valid);
+            epilogue_slab<EPI>(taddr, c_first, BN / 64, t.row0 + lane_base, t.row_end, t.n0, out,
+                               ld_out, n_valid, st);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -515,6 +593,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
+        if (lane == 0)
+            bulk_wait_all();  // this lane's output stores are done before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -569,7 +649,7 @@ struct Aux {
     int32_t off[MOE_MAX_EXPERTS + 1];
     int32_t tstart[MOE_MAX_EXPERTS + 1];
 };
-constexpr int SMEM_BYTES = 1024 + TILE_BYTES + (int)sizeof(Aux);
+constexpr int SMEM_BYTES = 1024 + TILE_BYTES + tc::kEpiStageBytes + (int)sizeof(Aux);
 
 // kind::f16, D f32, A/B bf16 K-major, N = 256, M = 256 (the pair)
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -693,6 +773,7 @@ template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
+                            const __grid_constant__ CUtensorMap tmO,
                             const int32_t *__restrict__ offsets, int E, int N, int K,
                             bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
                             uint64_t wait_ns, const int32_t *__restrict__ row_token)
@@ -700,7 +781,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES);
+    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES + tc::kEpiStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int32_t *abort_flag = &aux->abort_flag;
     const uint32_t rank = cta_rank();
@@ -721,6 +802,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
     }
     const int n_tiles = (N + BN - 1) / BN;
     if (warp == 2) {
@@ -862,6 +944,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int c_first = ((warp - 2) / 4) * (BN / 64);
         const uint32_t tempty0 = map_rank(tc::smem_u32(&aux->tempty[0]), 0);
         const uint32_t tempty1 = map_rank(tc::smem_u32(&aux->tempty[1]), 0);
+        tc::EpiStore st{&tmO,
+                        smem_base + TILE_BYTES + (uint32_t)((warp - 2) * 2 * tc::kStageSlotBytes),
+                        0};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster_id; tile < total; tile += nclusters) {
@@ -870,10 +955,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                status))
                 break;
             tc::tc_fence_after();
-            const int row = t.row0 + (int)rank * BM + lane_base + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-            tc::epilogue_row<EPI>(taddr, c_first, BN / 64, row, row < t.row_end, t.n0, out,
-                                  ld_out, n_valid);
+            tc::epilogue_slab<EPI>(taddr, c_first, BN / 64, t.row0 + (int)rank * BM + lane_base,
+                                   t.row_end, t.n0, out, ld_out, n_valid, st);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -883,6 +967,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
         }
+        if (lane == 0)
+            tc::bulk_wait_all();  // this lane's output stores are done before the CTA exits
     }
     tc::tc_fence_before();
     cluster_sync();
@@ -935,7 +1021,8 @@ static EncodeTiledFn get_encoder(cudaError_t *err)
 
 // rank-2 or rank-3 bf16 tensor map; dims/strides innermost first, strides in bytes.
 static cudaError_t make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                            const uint64_t *strides, const uint32_t *box)
+                            const uint64_t *strides, const uint32_t *box,
+                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     cudaError_t err;
     EncodeTiledFn enc = get_encoder(&err);
@@ -950,9 +1037,8 @@ static cudaError_t make_map(CUtensorMap *map, const void *base, int rank, const 
     for (int i = 0; i < rank - 1; ++i)
         gs[i] = strides[i];
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
-                     const_cast<void *>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     const_cast<void *>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -1063,15 +1149,21 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
         return e;
     if ((e = make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
         return e;
+    // output boxes of 32 columns x 32 rows written by bulk tensor stores
+    CUtensorMap to;
+    const uint64_t dout[2] = {(uint64_t)n_valid, rows}, sout[1] = {(uint64_t)ld_out * 2};
+    const uint32_t bout[2] = {32, 32};
+    if ((e = make_map(&to, out, 2, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess)
+        return e;
     const uint64_t wait_ns = wait_limit_ns();
     const int N = (int)b_rows, K = (int)a_k;
     if (!pair) {
         if (gather)
             grouped_gemm_kernel<EPI, true><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
-                ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
         else
             grouped_gemm_kernel<EPI, false><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
-                ta, tb, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
@@ -1087,10 +1179,11 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (gather)
-        return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, true>, ta, tb, offsets,
-                                  E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
-    return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, false>, ta, tb, offsets, E,
-                              N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+        return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, true>, ta, tb, to,
+                                  offsets, E, N, K, out, ld_out, n_valid, status, wait_ns,
+                                  row_token);
+    return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, false>, ta, tb, to, offsets,
+                              E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
 }
 
 }  // namespace tc
