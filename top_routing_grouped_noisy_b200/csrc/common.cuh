@@ -21,6 +21,8 @@ typedef __nv_bfloat16 bf16;
 constexpr size_t kWsHeader = 256;
 // Word 1 of the header: ticket counter of the dispatch count kernel (zero between calls).
 constexpr int kWsCounterWord = 1;
+// Word 2: ticket counter of the tensor-core router (zero between calls).
+constexpr int kWsRouterCounterWord = 2;
 
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {

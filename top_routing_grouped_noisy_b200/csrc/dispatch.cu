@@ -10,9 +10,10 @@
 //     chunk routed to the expert (one warp ballot per expert); the CTA that
 //     finishes last then scans over chunks per expert -> the rank base of each
 //     chunk; counts, kept = min(counts, C), offsets = exclusive scan of kept.
-//   scatter kernel (one CTA per chunk): each assignment's rank = chunk base +
-//     ballot prefix inside the chunk; slot_row / row_token; then the chunk's x
-//     rows are read once (16-byte loads) and written to each kept row.
+//   rank kernel (one warp per chunk): each assignment's rank = chunk base + ballot
+//     prefix inside the chunk -> slot_row / row_token.
+//   copy kernel: every x row is read once (16-byte loads) and written to each of
+//     its kept rows; equal contiguous work ranges for a grid that fills the device.
 // No atomics decide any output, so every output is bit-reproducible.
 #include "common.cuh"
 #include "kernels.h"
@@ -23,7 +24,8 @@
 
 namespace moe {
 
-constexpr int kCountWarps = 8;  // chunks per count CTA
+constexpr int kCountWarps = 8;         // chunks per count CTA
+constexpr int kCountSmemInts = 8192;   // histogram entries the last CTA scans in shared memory
 
 // Per-chunk expert counts (one warp ballot per expert and 32-token chunk), then, in
 // whichever CTA finishes last, the exclusive scan over chunks per expert (rank base
@@ -38,6 +40,7 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
 {
     __shared__ int s_last;
     __shared__ int32_t s_count[MOE_MAX_EXPERTS];
+    __shared__ int32_t s_hist[kCountSmemInts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
     const int c = blockIdx.x * kCountWarps + warp;
@@ -76,15 +79,23 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
     } else {
         __syncthreads();  // one CTA: its own writes are visible after the barrier
     }
-    // exclusive scan over chunks, one warp per expert; lane l owns a contiguous run
+    // exclusive scan over chunks, one warp per expert; lane l owns a contiguous run.
+    // The histogram is staged in shared memory with coalesced loads when it fits.
     const int per = (nch + 31) / 32;
+    const int64_t nhist = (int64_t)E * nch;
+    const bool staged = nhist <= kCountSmemInts;
+    if (staged) {
+        for (int64_t i = threadIdx.x; i < nhist; i += blockDim.x)
+            s_hist[i] = __ldcg(hist + i);
+        __syncthreads();
+    }
     for (int e = warp; e < E; e += kCountWarps) {
-        int32_t *h = hist + (int64_t)e * nch;
+        int32_t *h = staged ? s_hist + (int64_t)e * nch : hist + (int64_t)e * nch;
         const int c0 = lane * per, c1 = min(nch, c0 + per);
         int32_t sum = 0;
 #pragma unroll 8
         for (int cc = c0; cc < c1; ++cc)
-            sum += __ldcg(h + cc);
+            sum += staged ? h[cc] : __ldcg(h + cc);
         int32_t incl = sum;
 #pragma unroll
         for (int sh = 1; sh < 32; sh <<= 1) {
@@ -94,7 +105,7 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
         }
         int32_t run = incl - sum;
         for (int cc = c0; cc < c1; ++cc) {
-            const int32_t v = __ldcg(h + cc);
+            const int32_t v = staged ? h[cc] : __ldcg(h + cc);
             h[cc] = run;
             run += v;
         }
@@ -103,6 +114,9 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
             s_count[e] = total;
     }
     __syncthreads();
+    if (staged)  // the chunk bases go back to global memory for the rank kernel
+        for (int64_t i = threadIdx.x; i < nhist; i += blockDim.x)
+            hist[i] = s_hist[i];
     if (threadIdx.x == 0) {
         int32_t off = 0;
         offsets[0] = 0;
@@ -126,83 +140,99 @@ static unsigned count_grid(int T)
     return (unsigned)(g > 0 ? g : 1);
 }
 
-__global__ void __launch_bounds__(256) dispatch_scatter_kernel(
-    const char *__restrict__ x, int64_t row_bytes, const int32_t *__restrict__ idx, int T, int k,
-    int E, const int32_t *__restrict__ hist, const int32_t *__restrict__ kept,
-    const int32_t *__restrict__ offsets, char *__restrict__ x_perm,
+// Ranks of one 32-token chunk per warp: rank = chunk base + ballot prefix inside
+// the chunk; writes slot_row and row_token.
+__global__ void __launch_bounds__(256) dispatch_rank_kernel(
+    const int32_t *__restrict__ idx, int T, int k, int E, const int32_t *__restrict__ hist,
+    const int32_t *__restrict__ kept, const int32_t *__restrict__ offsets,
     int32_t *__restrict__ row_token, int32_t *__restrict__ slot_row)
 {
-    __shared__ int32_t s_row[kDispatchChunk][MOE_MAX_TOPK];
-    const int c = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
-    const int64_t t0 = (int64_t)c * kDispatchChunk;
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const int64_t t = t0 + lane;
-        const unsigned lt = (1u << lane) - 1u;
-        int ej[MOE_MAX_TOPK], rowj[MOE_MAX_TOPK];
-        for (int j = 0; j < k; ++j) {
-            int e = -1;
-            if (t < T) {
-                e = idx[t * k + j];
-                if (e < 0 || e >= E)
-                    e = -1;  // reported by the scan kernel
-            }
-            ej[j] = e;
-            rowj[j] = -1;
+    const int c = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (c >= nch)
+        return;
+    const int64_t t = (int64_t)c * kDispatchChunk + lane;
+    const unsigned lt = (1u << lane) - 1u;
+    // the chunk's rank base, kept count and first row of every expert, fetched in one
+    // round of loads (lane l holds experts l and l + 32)
+    int32_t base_l[2], kept_l[2], off_l[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int e = lane + 32 * h;
+        base_l[h] = e < E ? hist[(int64_t)e * nch + c] : 0;
+        kept_l[h] = e < E ? kept[e] : 0;
+        off_l[h] = e < E ? offsets[e] : 0;
+    }
+    int ej[MOE_MAX_TOPK], rowj[MOE_MAX_TOPK];
+    for (int j = 0; j < k; ++j) {
+        int e = -1;
+        if (t < T) {
+            e = idx[t * k + j];
+            if (e < 0 || e >= E)
+                e = -1;  // reported by the count kernel
         }
-        for (int e = 0; e < E; ++e) {
-            bool has = false;
+        ej[j] = e;
+        rowj[j] = -1;
+    }
+    for (int e = 0; e < E; ++e) {
+        bool has = false;
+        for (int j = 0; j < k; ++j)
+            has |= ej[j] == e;
+        const unsigned b = __ballot_sync(0xffffffffu, has);
+        const int h = e >> 5, src = e & 31;
+        const int32_t ebase = __shfl_sync(0xffffffffu, h ? base_l[1] : base_l[0], src);
+        const int32_t ekept = __shfl_sync(0xffffffffu, h ? kept_l[1] : kept_l[0], src);
+        const int32_t eoff = __shfl_sync(0xffffffffu, h ? off_l[1] : off_l[0], src);
+        if (has) {
+            const int32_t rank = ebase + __popc(b & lt);
+            const int32_t row = rank < ekept ? eoff + rank : -1;
             for (int j = 0; j < k; ++j)
-                has |= ej[j] == e;
-            const unsigned b = __ballot_sync(0xffffffffu, has);
-            if (has) {
-                const int32_t rank = hist[(int64_t)e * nch + c] + __popc(b & lt);
-                const int32_t row = rank < kept[e] ? offsets[e] + rank : -1;
-                for (int j = 0; j < k; ++j)
-                    if (ej[j] == e)
-                        rowj[j] = row;
-            }
-        }
-        for (int j = 0; j < k; ++j) {
-            s_row[lane][j] = rowj[j];
-            if (t < T && blockIdx.y == 0) {
-                slot_row[t * k + j] = rowj[j];
-                if (rowj[j] >= 0)
-                    row_token[rowj[j]] = (int32_t)t;
-            }
+                if (ej[j] == e)
+                    rowj[j] = row;
         }
     }
-    if (x_perm == nullptr)  // tables only: the expert GEMM gathers rows of x itself
-        return;
-    __syncthreads();
-    const int ntok = (int)((int64_t)T - t0 < kDispatchChunk ? (int64_t)T - t0 : kDispatchChunk);
-    // the row's 16-byte vectors [v0, v1) of this CTA (blockIdx.y splits rows when T is small)
-    const int nv_all = (int)(row_bytes / 16);
-    const int per = (nv_all + gridDim.y - 1) / gridDim.y;
-    const int v0 = blockIdx.y * per, v1 = min(nv_all, v0 + per);
-    const int nv = v1 > v0 ? v1 - v0 : 0;
-    const int items = ntok * nv;
-    constexpr int U = MOE_SCATTER_U;  // loads in flight per thread before the stores
-    for (int base = threadIdx.x; base < items; base += blockDim.x * U) {
+    if (t < T)
+        for (int j = 0; j < k; ++j) {
+            slot_row[t * k + j] = rowj[j];
+            if (rowj[j] >= 0)
+                row_token[rowj[j]] = (int32_t)t;
+        }
+}
+
+// x_perm[slot_row[t][j]] = x[t] for every kept slot.  The T * (row bytes / 16)
+// vector items are split into equal contiguous ranges, one per CTA of a grid that
+// fills the device once; each thread issues U loads before their stores.
+__global__ void __launch_bounds__(256) dispatch_copy_kernel(const char *__restrict__ x,
+                                                            int64_t row_bytes, int T, int k,
+                                                            const int32_t *__restrict__ slot_row,
+                                                            char *__restrict__ x_perm)
+{
+    const int64_t nv = row_bytes / 16;
+    const int64_t items = (int64_t)T * nv;
+    const int64_t per = (items + gridDim.x - 1) / gridDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * per;
+    const int64_t i1 = i0 + per < items ? i0 + per : items;
+    constexpr int U = MOE_SCATTER_U;
+    for (int64_t base = i0 + threadIdx.x; base < i1; base += (int64_t)blockDim.x * U) {
         uint4 val[U];
-        int lv[U], vv[U];
+        int tv[U], vv[U];  // token and vector of each item (T < 2^31, nv < 2^17)
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = base + u * blockDim.x;
-            lv[u] = -1;
-            if (i < items) {
-                lv[u] = i / nv;
-                vv[u] = v0 + (i - lv[u] * nv);
-                val[u] = ld_nc_na(x + (t0 + lv[u]) * row_bytes + (int64_t)vv[u] * 16);
+            const int64_t i = base + (int64_t)u * blockDim.x;
+            tv[u] = -1;
+            if (i < i1) {
+                tv[u] = (int)(i / nv);
+                vv[u] = (int)(i - (int64_t)tv[u] * nv);
+                val[u] = ld_nc_na(x + (int64_t)tv[u] * row_bytes + (int64_t)vv[u] * 16);
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (lv[u] < 0)
+            if (tv[u] < 0)
                 continue;
             for (int j = 0; j < k; ++j) {
-                const int32_t row = s_row[lv[u]][j];
+                const int32_t row = slot_row[(int64_t)tv[u] * k + j];
                 if (row >= 0)
                     st_v4(x_perm + (int64_t)row * row_bytes + (int64_t)vv[u] * 16, val[u]);
             }
@@ -210,15 +240,45 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     }
 }
 
-// CTAs per chunk along the row: enough CTAs in total to cover the SMs twice.
-static unsigned scatter_split(int nch, int64_t row_bytes)
+// CTAs of the copy kernel that fit on the device at once (cached per device).
+static unsigned copy_wave()
 {
-    const int64_t nv = row_bytes / 16;
-    int64_t y = (296 + nch - 1) / nch;
-    const int64_t ymax = (nv + 63) / 64;  // at least 64 vectors (1 KB) per CTA
-    if (y > ymax)
-        y = ymax;
-    return (unsigned)(y > 0 ? y : 1);
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (cached[dev] == 0) {
+        int sms = 0, per = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, dispatch_copy_kernel, 256, 0);
+        cached[dev] = (sms > 0 ? sms : 148) * (per > 0 ? per : 1);
+    }
+    return (unsigned)cached[dev];
+}
+
+// rank + copy launches shared by moe_dispatch and moe_dispatch_noalloc
+static cudaError_t launch_rank_copy(const moe_params_t *p, const void *x, const int32_t *idx,
+                                    const int32_t *hist, const int32_t *kept,
+                                    const int32_t *offsets, void *x_perm, int32_t *row_token,
+                                    int32_t *slot_row, cudaStream_t s)
+{
+    const int nch = ceil_div(p->T, kDispatchChunk);
+    dispatch_rank_kernel<<<ceil_div(nch, 8), 256, 0, s>>>(idx, p->T, p->k, p->E, hist, kept,
+                                                          offsets, row_token, slot_row);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || x_perm == nullptr)
+        return e;
+    const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
+    const int64_t items = (int64_t)p->T * (row_bytes / 16);
+    const int64_t min_per = 256;  // at least one vector per thread per CTA
+    int64_t grid = (items + min_per - 1) / min_per;
+    if (grid > copy_wave())
+        grid = copy_wave();
+    dispatch_copy_kernel<<<(unsigned)grid, 256, 0, s>>>((const char *)x, row_bytes, p->T, p->k,
+                                                         slot_row, (char *)x_perm);
+    count_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
@@ -236,14 +296,7 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p->T == 0)
         return e;
-    const int nch = ceil_div(p->T, kDispatchChunk);
-    const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
-    const unsigned ysplit = x_perm != nullptr ? scatter_split(nch, row_bytes) : 1u;
-    dispatch_scatter_kernel<<<dim3(nch, ysplit), 256, 0, s>>>(
-        (const char *)x, row_bytes, idx, p->T, p->k, p->E, hist, kept, offsets, (char *)x_perm,
-        row_token, slot_row);
-    count_launch();
-    return cudaGetLastError();
+    return launch_rank_copy(p, x, idx, hist, kept, offsets, x_perm, row_token, slot_row, s);
 }
 
 }  // namespace moe
@@ -337,14 +390,7 @@ extern "C" int moe_dispatch_noalloc(const moe_params_t *p, const void *x,
                                                            kept, offsets, st);
     count_launch();
     e = cudaGetLastError();
-    if (e == cudaSuccess && p->T > 0) {
-        const int64_t row_bytes = (int64_t)p->d * (p->dtype == MOE_BF16 ? 2 : 4);
-        dispatch_scatter_kernel<<<dim3((unsigned)chunks, scatter_split((int)chunks, row_bytes)),
-                                  256, 0, s>>>((const char *)x, row_bytes, topk_idx, p->T, p->k,
-                                               p->E, hist, kept, offsets, (char *)x_perm,
-                                               row_token, slot_row);
-        count_launch();
-        e = cudaGetLastError();
-    }
+    if (e == cudaSuccess && p->T > 0)
+        e = launch_rank_copy(p, x, topk_idx, hist, kept, offsets, x_perm, row_token, slot_row, s);
     return e == cudaSuccess ? report_ok() : report_cuda(e, fn);
 }

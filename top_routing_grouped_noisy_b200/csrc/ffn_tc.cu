@@ -28,13 +28,10 @@
 // MOE_ERR_DEVICE_TIMEOUT, every role stops, in-flight TMA copies and MMAs are
 // drained (bounded again) and TMEM is freed before the CTA exits.  No TMA load here
 // uses cluster multicast.
-#include <cuda.h>
-
 #include <atomic>
 #include <mutex>
 
-#include "common.cuh"
-#include "kernels.h"
+#include "tc_common.cuh"
 
 namespace moe {
 namespace tc {
@@ -51,7 +48,6 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
 constexpr int NUM_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int EPI_WARPS = 8;
-constexpr uint64_t kDrainNs = 1000000000ull;  // bound of the drain waits on exit
 
 enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
 
@@ -72,191 +68,9 @@ constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-// Shared-memory matrix descriptor of a K-major, 128B-swizzled tile whose rows are
-// 128 bytes apart (8-row core groups 1024 bytes apart); tile base 1024-aligned.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address, 16-byte units
-    d |= (uint64_t)1 << 16;                    // leading byte offset (unused for this layout)
-    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next 8-row group
-    d |= (uint64_t)1 << 46;                    // descriptor version
-    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
-    return d;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait; gives up when the limit passes or another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
-                                          volatile int32_t *abort_flag, int32_t *status)
-{
-    if (mbar_try(bar, parity))
-        return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (mbar_try(bar, parity))
-            return true;
-        if (*abort_flag)
-            return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            set_status(status, MOE_ERR_DEVICE_TIMEOUT);
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
-
-// Bounded wait used while draining on exit (ignores the abort flag).
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity)
-{
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try(bar, parity))
-        if (globaltimer_ns() - t0 > kDrainNs)
-            return;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t bar, uint32_t dst,
-                                            int c0, int c1)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar, uint32_t dst,
-                                            int c0, int c1, int c2)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// Four rows r0..r3 of a 2-D tensor (box one row high), 64 columns from `col`,
-// written as four consecutive 128-byte rows at dst (128-byte swizzle as a tile).
-__device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint32_t bar, uint32_t dst,
-                                            int col, int r0, int r1, int r2, int r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2),
-        "r"(r3)
-        : "memory");
-}
-
-// Bulk tensor store of a shared-memory box to global memory, tracked as a bulk group.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1)
-{
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// at most one bulk group of this thread still reads shared memory
-__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-// every bulk group of this thread has completed
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld()
-{
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 32 consecutive f32 accumulator columns of this thread's TMEM lane; the registers
-// are valid only after tmem_wait_ld().
-__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-          "=r"(v[31])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-          "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    umma_f16(d_tmem, a, b, kIdesc, acc);
 }
 
 // Output staging: each epilogue warp owns two 2 KB shared-memory slots, each one
@@ -995,52 +809,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace tc2
 
 // ------------------------------------------------------------------------ host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encoder(cudaError_t *err)
-{
-    static std::once_flag once;
-    static EncodeTiledFn fn = nullptr;
-    static cudaError_t e0 = cudaSuccess;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        e0 = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                              cudaEnableDefault, &q);
-        if (e0 == cudaSuccess && q != cudaDriverEntryPointSuccess)
-            e0 = cudaErrorSymbolNotFound;
-        fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    *err = e0;
-    return fn;
-}
-
-// rank-2 or rank-3 bf16 tensor map; dims/strides innermost first, strides in bytes.
-static cudaError_t make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                            const uint64_t *strides, const uint32_t *box,
-                            CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
-{
-    cudaError_t err;
-    EncodeTiledFn enc = get_encoder(&err);
-    if (enc == nullptr)
-        return err != cudaSuccess ? err : cudaErrorSymbolNotFound;
-    cuuint64_t gd[3], gs[2];
-    cuuint32_t bx[3], es[3] = {1, 1, 1};
-    for (int i = 0; i < rank; ++i) {
-        gd[i] = dims[i];
-        bx[i] = box[i];
-    }
-    for (int i = 0; i < rank - 1; ++i)
-        gs[i] = strides[i];
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
-                     const_cast<void *>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
 
 struct DevInfo {
     int sms = 0;

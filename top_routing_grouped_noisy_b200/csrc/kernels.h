@@ -2,6 +2,7 @@
 // kernel translation units of libmoe.so.  Not installed, not part of the ABI.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -55,6 +56,14 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
                          const void *Wnoise, const float *noise, const float *bias,
                          int32_t *idx, float *w, float *probs_sum, float *importance,
                          char *ws, int32_t *status, cudaStream_t s);
+
+// a1 on the tcgen05 tensor cores (bf16), token sums included (per-CTA partials in
+// `part`, added by the CTA that finishes last; `counter` is zero between calls).
+cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wg,
+                            const void *Wnoise, const float *noise, const float *bias,
+                            int32_t *idx, float *w, float *probs_sum, float *importance,
+                            float *part, int32_t *counter, __nv_bfloat16 *Wt, int32_t *status,
+                            cudaStream_t s);
 
 cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
                             void *x_perm, int32_t *row_token, int32_t *slot_row,

@@ -6,27 +6,14 @@
 //   Mixtral: G_tj = softmax over the k kept H;  ST: G_tj = softmax(H_t)[idx_tj]
 // plus per-CTA partial sums of softmax(H_t) (for P) and of G (importance).
 //
-// bf16 path: the logits x.[W_g | W_noise] are a skinny GEMM (T x d x 2E) read
-// at HBM speed; it runs on the tensor cores with mma.sync m16n8k16 (bf16 in,
-// f32 accumulate), the router weights as the M=16 operand and 8 tokens as N.
-// The K dimension is split over the 8 warps of a CTA and reduced through shared
-// memory in a fixed order (bit-deterministic).  x is streamed once with 16-byte
-// non-allocating loads.  f32 path: one warp per token on the CUDA cores.
+// Kernels here: the f32 router (one warp per token on the CUDA cores), the
+// split-K router for batches of at most 64 tokens, and the fixed-order sum of
+// per-CTA partials.  bf16 batches above that size run on the tensor cores
+// (router_tc.cu).
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
-
-// Tile constants (compile-time; tuned on B200).
-#ifndef MOE_ROUTER_NNT1
-#define MOE_ROUTER_NNT1 8  // token n-tiles per CTA when the router has <= 16 outputs
-#endif
-#ifndef MOE_ROUTER_U
-#define MOE_ROUTER_U 4  // k32 blocks of loads issued per round
-#endif
-#ifndef MOE_ROUTER_U_WIDE
-#define MOE_ROUTER_U_WIDE 1  // the same for 8 token n-tiles per CTA
-#endif
 
 namespace moe {
 
@@ -121,121 +108,6 @@ __device__ void write_partials(int ntok, int E, const float *prob_s, const float
         part[((int64_t)blockIdx.x * 2 + 0) * E + e] = sp;
         part[((int64_t)blockIdx.x * 2 + 1) * E + e] = sg;
     }
-}
-
-// Wt[o][c]: o < E -> W_g[c][o]; E <= o < 2E -> W_noise[c][o-E] (if given); else 0.
-__global__ void router_transpose_kernel(const bf16 *__restrict__ Wg, const bf16 *__restrict__ Wn,
-                                        int d, int E, int rows, bf16 *__restrict__ Wt)
-{
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)rows * d)
-        return;
-    const int o = (int)(i / d), c = (int)(i % d);
-    bf16 v = __float2bfloat16_rn(0.f);
-    if (o < E)
-        v = Wg[(int64_t)c * E + o];
-    else if (Wn != nullptr && o < 2 * E)
-        v = Wn[(int64_t)c * E + (o - E)];
-    Wt[i] = v;
-}
-
-// NMT m-tiles of 16 router outputs x NNT n-tiles of 8 tokens per CTA.
-// Each thread (g = lane/4, q = lane%4) owns K columns [32kb + 8q, 32kb + 8q + 8) of
-// every k32 block kb it visits; the 8 columns feed two m16n8k16 steps, physical
-// columns 8q+{0,1},{2,3} as logical k {2q,2q+1},{2q+8,2q+9} of the first step and
-// 8q+{4,5},{6,7} of the second.  A and B use the same map, so the dot product is
-// unchanged.
-template <int NMT, int NNT>
-__global__ void __launch_bounds__(256) router_bf16_kernel(
-    const bf16 *__restrict__ x, const bf16 *__restrict__ Wt, int T, int d, int E, int k,
-    int noisy, const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
-    int32_t *__restrict__ idx_out, float *__restrict__ w_out, float *__restrict__ part,
-    int32_t *status)
-{
-    constexpr int TOK = NNT * 8, NOUT = NMT * 16, NW = kRouterWarps;
-    extern __shared__ float smem[];
-    float *red = smem;                          // [NW][NOUT][TOK]
-    float *lg = red + NW * NOUT * TOK;          // [TOK][NOUT + 1]
-    float *prob_s = lg + TOK * (NOUT + 1);      // [TOK][E]
-    float *gw_s = prob_s + TOK * E;             // [TOK][E]
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, q = lane & 3;
-    const int64_t tok0 = (int64_t)blockIdx.x * TOK;
-
-    float acc[NMT][NNT][4];
-#pragma unroll
-    for (int a = 0; a < NMT; ++a)
-#pragma unroll
-        for (int b = 0; b < NNT; ++b)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                acc[a][b][c] = 0.f;
-
-    const int nkb = (d + 31) / 32;
-    // U k32 blocks per round: all loads of a round are issued before its MMAs
-    constexpr int U = NNT >= 8 ? MOE_ROUTER_U_WIDE : MOE_ROUTER_U;
-    for (int kb0 = warp; kb0 < nkb; kb0 += NW * U) {
-        uint4 xb[U][NNT];
-        uint4 wa[U][NMT][2];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = (kb0 + u * NW) * 32 + 8 * q;
-            const bool kv = c < d;
-#pragma unroll
-            for (int nt = 0; nt < NNT; ++nt) {
-                const int64_t t = tok0 + nt * 8 + g;
-                xb[u][nt] = (kv && t < T) ? ld_nc_na(x + t * d + c) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int mt = 0; mt < NMT; ++mt) {
-                wa[u][mt][0] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g) * d + c)
-                                  : make_uint4(0, 0, 0, 0);
-                wa[u][mt][1] = kv ? ld_nc(Wt + (int64_t)(mt * 16 + g + 8) * d + c)
-                                  : make_uint4(0, 0, 0, 0);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int mt = 0; mt < NMT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NNT; ++nt) {
-                    mma_bf16_16816(acc[mt][nt], wa[u][mt][0].x, wa[u][mt][1].x, wa[u][mt][0].y,
-                                   wa[u][mt][1].y, xb[u][nt].x, xb[u][nt].y);
-                    mma_bf16_16816(acc[mt][nt], wa[u][mt][0].z, wa[u][mt][1].z, wa[u][mt][0].w,
-                                   wa[u][mt][1].w, xb[u][nt].z, xb[u][nt].w);
-                }
-    }
-    // D fragment: c0,c1 -> (row g, cols 2q,2q+1); c2,c3 -> (row g+8, cols 2q,2q+1)
-#pragma unroll
-    for (int mt = 0; mt < NMT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NNT; ++nt) {
-            const int o0 = mt * 16 + g, t0 = nt * 8 + 2 * q;
-            red[(warp * NOUT + o0) * TOK + t0] = acc[mt][nt][0];
-            red[(warp * NOUT + o0) * TOK + t0 + 1] = acc[mt][nt][1];
-            red[(warp * NOUT + o0 + 8) * TOK + t0] = acc[mt][nt][2];
-            red[(warp * NOUT + o0 + 8) * TOK + t0 + 1] = acc[mt][nt][3];
-        }
-    __syncthreads();
-    for (int i = threadIdx.x; i < NOUT * TOK; i += blockDim.x) {
-        const int o = i / TOK, tk = i % TOK;
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w)
-            s += red[(w * NOUT + o) * TOK + tk];
-        lg[tk * (NOUT + 1) + o] = s;
-    }
-    __syncthreads();
-    const int ntok = (int)((int64_t)T - tok0 < TOK ? (int64_t)T - tok0 : TOK);
-    if (threadIdx.x < ntok) {
-        const int tk = threadIdx.x;
-        finish_token(tok0 + tk, lg + tk * (NOUT + 1), E, k, noisy, noise, bias, router_type,
-                     idx_out, w_out, prob_s + tk * E, gw_s + tk * E, status);
-    }
-    __syncthreads();
-    write_partials(ntok, E, prob_s, gw_s, part);
 }
 
 // f32 router on the CUDA cores: one warp per token, 8 tokens per CTA.
@@ -383,26 +255,6 @@ __global__ void __launch_bounds__(256) router_small_finish_kernel(
     }
 }
 
-template <int NMT, int NNT>
-static cudaError_t run_bf16(const moe_params_t *p, const bf16 *x, const bf16 *Wt, int noisy,
-                            const float *noise, const float *bias, int32_t *idx, float *w,
-                            float *part, int32_t *status, cudaStream_t s, int *nblk)
-{
-    constexpr int TOK = NNT * 8, NOUT = NMT * 16;
-    const size_t smem =
-        sizeof(float) * ((size_t)kRouterWarps * NOUT * TOK + TOK * (NOUT + 1) + 2 * TOK * p->E);
-    // E <= min(64, 16 * NMT) for this instantiation
-    static_assert(sizeof(float) * (kRouterWarps * NOUT * TOK + TOK * (NOUT + 1) +
-                                   2 * TOK * (16 * NMT < MOE_MAX_EXPERTS ? 16 * NMT
-                                                                         : MOE_MAX_EXPERTS)) <=
-                      48 * 1024,
-                  "router shared memory must fit the default 48 KB");
-    *nblk = ceil_div(p->T, TOK);
-    router_bf16_kernel<NMT, NNT><<<*nblk, 256, smem, s>>>(
-        x, Wt, p->T, p->d, p->E, p->k, noisy, noise, bias, p->router_type, idx, w, part, status);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
                          const void *Wnoise, const float *noise, const float *bias,
                          int32_t *idx, float *w, float *probs_sum, float *importance,
@@ -436,39 +288,20 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
         count_launch();
         return cudaGetLastError();
     }
+    if (p->T > 0 && p->dtype == MOE_BF16) {
+        bf16 *Wt = reinterpret_cast<bf16 *>(ws + L.wt);
+        int32_t *counter = reinterpret_cast<int32_t *>(ws) + kWsRouterCounterWord;
+        return launch_route_tc(p, x, Wg, Wnoise, noise, bias, idx, w, probs_sum, importance,
+                               part, counter, Wt, status, s);
+    }
     if (p->T > 0) {
-        if (p->dtype == MOE_BF16) {
-            const int noisy = Wnoise != nullptr;
-            const int nout = noisy ? 2 * p->E : p->E;
-            bf16 *Wt = reinterpret_cast<bf16 *>(ws + L.wt);
-            const int64_t n = (int64_t)kWtRows * p->d;
-            router_transpose_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-                (const bf16 *)Wg, (const bf16 *)Wnoise, p->d, p->E, kWtRows, Wt);
-            count_launch();
-            if ((e = cudaGetLastError()) != cudaSuccess)
-                return e;
-            if (nout <= 16)
-                e = run_bf16<1, MOE_ROUTER_NNT1>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
-                                   status, s, &nblk);
-            else if (nout <= 32)
-                e = run_bf16<2, 4>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
-                                   status, s, &nblk);
-            else if (nout <= 64)
-                e = run_bf16<4, 2>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
-                                   status, s, &nblk);
-            else
-                e = run_bf16<8, 1>(p, (const bf16 *)x, Wt, noisy, noise, bias, idx, w, part,
-                                   status, s, &nblk);
-        } else {
-            nblk = ceil_div(p->T, kRouterWarps);
-            const size_t smem = sizeof(float) * ((size_t)kRouterWarps * 4 * p->E);
-            router_f32_kernel<<<nblk, 256, smem, s>>>(
-                (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E,
-                p->k, noise, bias, p->router_type, idx, w, part, status);
-            e = cudaGetLastError();
-        }
+        nblk = ceil_div(p->T, kRouterWarps);
+        const size_t smem = sizeof(float) * ((size_t)kRouterWarps * 4 * p->E);
+        router_f32_kernel<<<nblk, 256, smem, s>>>(
+            (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E, p->k,
+            noise, bias, p->router_type, idx, w, part, status);
         count_launch();
-        if (e != cudaSuccess)
+        if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
     }
     router_finalize_kernel<<<1, 1024, 0, s>>>(part, nblk, p->E, probs_sum, importance);
