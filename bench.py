@@ -240,6 +240,41 @@ def barrier(world):
     if world > 1:
         torch.distributed.barrier()
 
+def e2e_pipeline(args, w, p, moe, x, Wg, Wn, eps, bias, W13_e, W2_e, world, depth=2):
+    """End to end through the host-buffer pipeline (moe_pipeline_*): every step copies
+    its x (and noise) in from pinned host memory and its y, L_balance and status word
+    back out; with `depth` batches in flight the copies overlap the layer.  Host wall
+    clock around the whole run, device idle on both sides, max over ranks."""
+    x_h = x.cpu().pin_memory()
+    eps_h = eps.cpu().pin_memory() if eps is not None else None
+    y_h = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for _ in range(depth)]
+    loss_h = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(depth)]
+    pl = moe.Pipeline(p, Wg, W13_e, W2_e, Wnoise=Wn, bias=bias, depth=depth)
+
+    def run(n):
+        t = None
+        for i in range(n):
+            t = pl.submit(x_h, y_h[i % depth], loss_h[i % depth], noise_host=eps_h)
+        pl.wait(t)
+
+    run(args.warmup)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    run(args.steps)
+    t1 = time.perf_counter()
+    barrier(world)
+    pl.close()
+    ms = max_over_ranks((t1 - t0) * 1000.0, world)
+    h2d = x.numel() * x.element_size() + (eps.numel() * 4 if eps is not None else 0)
+    d2h = x.numel() * x.element_size() + 4 + 4
+    return {"value": w.T * args.steps * world / (ms / 1000.0), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.steps,
+            "api": "moe_pipeline_submit/moe_pipeline_wait, %d batches in flight, host wall "
+                   "clock" % depth}
+
+
 def run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank, world,
                local):
     """Decode-shaped batches (T <= 64): the layer is launch- and weight-streaming-bound,
@@ -291,6 +326,8 @@ def run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, ran
     moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps, bias=bias)
     launches_per_forward = moe.moe_launch_count() - l1
     torch.cuda.synchronize()
+    e2e = None if args.no_e2e else e2e_pipeline(args, w, p, moe, x, Wg, Wn, eps, bias, W13_e,
+                                                W2_e, world)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
@@ -308,7 +345,7 @@ def run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, ran
                      "peak_source": "%s hbm_gbs" % peak_src,
                      "algorithmic": "%d experts x 3*d*m*2 B + x, y, W_g = %.4g B per layer"
                                     % (experts_used, w_bytes + io_bytes)},
-        "cpu_baseline": None, "e2e": None,
+        "cpu_baseline": None, "e2e": e2e,
         "gpu_launches": launches_per_forward * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
     }
@@ -488,9 +525,10 @@ def main():
     key = _src_hash("top_routing_grouped_noisy_b200/csrc/ffn_tc.cu")
     if NCU_TRAFFIC.get("src") == key and NCU_TRAFFIC.get("workload") == w.name:
         traffic = NCU_TRAFFIC["bytes_per_launch"]
-    roofline = {"kernel": "grouped_gemm_2sm_kernel<SwiGLU, gather> (expert GEMM 1, "
-                          "moe_expert_up_gather)" if gather else
-                "grouped_gemm_kernel<SwiGLU> (expert GEMM 1, moe_expert_up)",
+    kname = ("grouped_gemm_2sm_kernel" if w.T * w.k >= 4096 else "grouped_gemm_kernel")
+    kname += "<SwiGLU, gather> (expert GEMM 1, moe_expert_up_gather)" if gather else \
+        "<SwiGLU> (expert GEMM 1, moe_expert_up)"
+    roofline = {"kernel": kname,
                 "bound": "tensor", "achieved": up_tf, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": up_tf / peak_t, "traffic": traffic,
                 "peak_source": "%s bf16_tflops_sustained (kernel timed inside the step loop)"
@@ -518,41 +556,8 @@ def main():
         "gate_stats": {"ms": seg_ms[5]},
     }
 
-    # end to end through moe_forward with host buffers
-    e2e = None
-    if not args.no_e2e:
-        x_h = x.cpu().pin_memory()
-        eps_h = eps.cpu().pin_memory() if eps is not None else None
-        y_h = torch.empty(b.y.shape, dtype=b.y.dtype).pin_memory()
-        loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
-        x_d = torch.empty_like(x)
-        eps_d = torch.empty_like(eps) if eps is not None else None
-
-        def e2e_step():
-            x_d.copy_(x_h, non_blocking=True)
-            if eps_d is not None:
-                eps_d.copy_(eps_h, non_blocking=True)
-            moe.moe_forward(p, x_d, Wg, W13_e, W2_e, ws, b, Wnoise=Wn, noise=eps_d, bias=bias)
-            y_h.copy_(b.y, non_blocking=True)
-            loss_h.copy_(b.loss, non_blocking=True)
-
-        for _ in range(args.warmup):
-            e2e_step()
-        barrier(world)
-        torch.cuda.synchronize()
-        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e2.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        ms2 = max_over_ranks(s2.elapsed_time(e2), world)
-        h2d = x.numel() * x.element_size() + (eps.numel() * 4 if eps is not None else 0)
-        d2h = b.y.numel() * b.y.element_size() + 4
-        e2e = {"value": w.T * args.steps * world / (ms2 / 1000.0), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms2 / args.steps}
+    e2e = None if args.no_e2e else e2e_pipeline(args, w, p, moe, x, Wg, Wn, eps, bias, W13_e,
+                                                W2_e, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -130,3 +130,27 @@ def test_empty_batch_needs_no_token_buffers(L):
 def test_wait_limit_setter_is_host_only(L):
     moe.moe_set_wait_limit_ns(123)
     moe.moe_set_wait_limit_ns(2_000_000_000)
+
+
+def test_pipeline_rejects_bad_arguments_before_the_device(L):
+    p = moe.params(1000, 512, 8, 2, 344)
+    out = C.c_void_p(123)
+    dummy = C.c_void_p(16)
+    assert L.moe_pipeline_create(C.byref(p), dummy, None, None, dummy, dummy, 2, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pipeline_create(C.byref(p), dummy, None, None, dummy, dummy, 1,
+                                 C.byref(out)) == moe.MOE_ERR_INVALID_ARG
+    assert out.value is None
+    assert L.moe_pipeline_create(C.byref(p), dummy, None, None, dummy, dummy, 5,
+                                 C.byref(out)) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pipeline_create(C.byref(p), None, None, None, dummy, dummy, 2,
+                                 C.byref(out)) == moe.MOE_ERR_INVALID_ARG
+    p0 = moe.params(0, 512, 8, 2, 344)
+    assert L.moe_pipeline_create(C.byref(p0), dummy, None, None, dummy, dummy, 2,
+                                 C.byref(out)) == moe.MOE_ERR_INVALID_ARG
+    assert b"T must be" in L.moe_last_error_string()
+    t = C.c_int64(0)
+    assert L.moe_pipeline_submit(None, dummy, None, dummy, dummy, C.byref(t)) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pipeline_wait(None, 0) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_pipeline_destroy(None) == moe.MOE_OK

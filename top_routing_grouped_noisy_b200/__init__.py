@@ -19,7 +19,7 @@ __all__ = [
     "moe_dispatch_noalloc", "moe_dispatch_rows", "moe_expert_up_gather",
     "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
-    "packed_w13_elems", "packed_w2_elems", "h_ld",
+    "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -103,6 +103,10 @@ def lib():
             "moe_gate_stats": (C.c_int, [P, v, v, v, v, v, v]),
             "moe_forward": (C.c_int, [P, C.POINTER(_Buffers), v, sz, v]),
             "moe_get_device_status": (C.c_int, [v, C.POINTER(i32), i32, v]),
+            "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
+            "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
+            "moe_pipeline_wait": (C.c_int, [v, i64]),
+            "moe_pipeline_destroy": (C.c_int, [v]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -318,3 +322,64 @@ def moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs: ForwardBuffers, Wnoise=None, no
         setattr(b, n, _p(t))
     _check(lib().moe_forward(C.byref(p), C.byref(b), ws.ptr, ws.nbytes, _stream(stream)))
     return bufs
+
+
+def _host_ptr(t, name):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s: expected a torch.Tensor, got %r" % (name, type(t)))
+    if t.is_cuda:
+        raise ValueError("%s: the pipeline takes host tensors (pinned for overlap)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s: the pipeline takes contiguous tensors" % name)
+    return t.data_ptr() or None
+
+
+class Pipeline:
+    """Host-buffer pipeline (include/moe_pipeline.h): batches in host memory go
+    through the layer with up to ``depth`` of them in flight, copies overlapping
+    the compute.  The weights are device tensors that must outlive the pipeline."""
+
+    def __init__(self, p: Params, Wg, W13_e, W2_e, Wnoise=None, bias=None, depth=2):
+        self._p = p
+        self._keep = (Wg, W13_e, W2_e, Wnoise, bias)
+        h = C.c_void_p(None)
+        _check(lib().moe_pipeline_create(C.byref(p), _p(Wg), _p(Wnoise), _p(bias), _p(W13_e),
+                                         _p(W2_e), int(depth), C.byref(h)))
+        self._h = h
+        self._held = {}
+
+    def submit(self, x_host, y_host, loss_host, noise_host=None) -> int:
+        """Enqueue one batch; returns its ticket.  The host tensors are held until
+        wait() has returned for that ticket."""
+        t = C.c_int64(-1)
+        _check(lib().moe_pipeline_submit(self._h, _host_ptr(x_host, "x_host"),
+                                         _host_ptr(noise_host, "noise_host"),
+                                         _host_ptr(y_host, "y_host"),
+                                         _host_ptr(loss_host, "loss_host"), C.byref(t)))
+        self._held[t.value] = (x_host, noise_host, y_host, loss_host)
+        return t.value
+
+    def wait(self, ticket: int) -> None:
+        _check(lib().moe_pipeline_wait(self._h, int(ticket)))
+        for k in [k for k in self._held if k <= ticket]:
+            del self._held[k]
+
+    def close(self) -> None:
+        if self._h is not None and self._h.value is not None:
+            h, self._h = self._h, None
+            self._held.clear()
+            _check(lib().moe_pipeline_destroy(h))
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -15,8 +15,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "partition.cu", "router.cu", "router_tc.cu", "dispatch.cu", "ffn_simt.cu", "ffn_tc.cu", "decode.cu",
-           "combine.cu"]
+SOURCES = ["api.cu", "partition.cu", "router.cu", "router_tc.cu", "dispatch.cu", "ffn_simt.cu",
+           "ffn_tc.cu", "decode.cu", "combine.cu", "pipeline.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr"]
 
@@ -38,7 +38,7 @@ def _stale(obj, src, deps):
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
     os.makedirs(BUILD_DIR, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
-    headers.append(os.path.join(INCLUDE, "moe.h"))
+    headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
