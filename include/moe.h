@@ -138,7 +138,8 @@ int moe_partition_experts(const void *W1, const void *W3, const void *W2,
                           void *W13_e, void *W2_e, void *ws, void *stream);
 
 /* Bytes of workspace the calls below need for `p` (covers every call with the
- * same or smaller T, E, d).  Host-only, never fails (returns 0 on bad params). */
+ * same dtype and the same or smaller T, E, d, m).  Host-only, never fails
+ * (returns 0 on bad params). */
 size_t moe_workspace_size(const moe_params_t *p);
 
 /* Zeroes a freshly allocated workspace (status word and counters).  Call once
@@ -199,7 +200,8 @@ int moe_dispatch_noalloc(const moe_params_t *p, const void *x, const int32_t *to
  * ["LLaMA-MoE v2", code sample, class Expert: down(silu(gate(x)) * up(x))]:
  *   h[r] = silu(x_perm[r] W1_e^T) * (x_perm[r] W3_e^T) for rows r in
  *   [offsets[e], offsets[e+1]).  x_perm [T*k][d], W13_e packed, h [T*k][m8].
- * bf16: tcgen05 tensor cores, f32 accumulate, h rounded to bf16.
+ * bf16: tcgen05 tensor cores, f32 accumulate, h rounded to bf16; for T <= 16
+ * (decode-shaped batches) a weight-streaming kernel on mma.sync instead.
  * f32: CUDA-core FMA in f32 (no TF32).  Row tables stay on the device. */
 int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                   const void *W13_e, void *h, void *ws, size_t ws_bytes, void *stream);
@@ -216,7 +218,8 @@ int moe_expert_up_gather(const moe_params_t *p, const void *x, const int32_t *ro
                          const int32_t *offsets, const void *W13_e, void *h, void *ws,
                          size_t ws_bytes, void *stream);
 
-/* a4. Second half: out[r] = h[r] W2_e^T.  h [T*k][m8], W2_e packed, out [T*k][d]. */
+/* a4. Second half: out[r] = h[r] W2_e^T.  h [T*k][m8], W2_e packed, out [T*k][d].
+ * bf16 with T <= 16: the weight-streaming kernel, as for moe_expert_up. */
 int moe_expert_down(const moe_params_t *p, const void *h, const int32_t *offsets,
                     const void *W2_e, void *out, void *ws, size_t ws_bytes, void *stream);
 
@@ -273,7 +276,8 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
                 void *stream);
 
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
- * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards. */
+ * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
+ * the workspace's internal launch counters. */
 int moe_get_device_status(void *ws, int32_t *status, int32_t clear, void *stream);
 
 /* Time limit, in nanoseconds, of every bounded wait inside the kernels that

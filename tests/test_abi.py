@@ -61,6 +61,11 @@ def test_workspace_size_and_invalid_params():
     assert moe.moe_workspace_size(p) > 0
     bigger = moe.params(32768, 4096, 8, 2, 1376)
     assert moe.moe_workspace_size(bigger) >= moe.moe_workspace_size(p)
+    # non-decreasing in T across the small-batch sizes, so a workspace sized for a
+    # batch serves every smaller one
+    sizes = [moe.moe_workspace_size(moe.params(T, 4096, 8, 2, 1376))
+             for T in (1, 2, 8, 9, 63, 64, 65, 300, 16384)]
+    assert sizes == sorted(sizes), sizes
     for bad in (moe.params(16, 4096, 8, 9, 1376), moe.params(16, 4096, 65, 2, 1376),
                 moe.params(16, 100, 8, 2, 1376), moe.params(-1, 64, 8, 2, 16),
                 moe.params(16, 64, 8, 0, 16), moe.params(16, 64, 8, 2, 0)):

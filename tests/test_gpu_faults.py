@@ -44,3 +44,4 @@ def test_wait_timeout_is_reported_and_context_survives(T):
     r, ties = H.check_routing(w, inp, bufs, 5e-5)
     dsp = H.check_dispatch(w, inp, p2, bufs)
     H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)
+

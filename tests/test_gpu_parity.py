@@ -39,13 +39,15 @@ SMALL = {
     "pair_e16_odd": W("pair_e16_odd", T=1200, d=200, d_ff=1600, E=16, k=4, router=wl.ST,
                       noisy=True, bias=True, cf=1.1, seed=25),
     "pair_e64": W("pair_e64", T=600, d=128, d_ff=1024, E=64, k=8, noisy=True, seed=26),
-    # T <= 64: the weight-streaming decode kernels
+    # T <= 16: the weight-streaming decode kernels (larger small batches: tcgen05)
     "decode_t64_m344": W("decode_t64_m344", T=64, d=512, d_ff=8 * 344, E=8, k=2, rescale=True,
                          seed=27),
     "decode_skewed_rows": W("decode_skewed_rows", T=40, d=256, d_ff=4 * 96, E=4, k=2, bias=True,
                             seed=28),
     "decode_ragged_d": W("decode_ragged_d", T=8, d=200, d_ff=8 * 100, E=8, k=2, noisy=True,
                          seed=29),
+    "decode_t16_st_cap": W("decode_t16_st_cap", T=16, d=264, d_ff=8 * 120, E=8, k=3,
+                           router=wl.ST, noisy=True, bias=True, cf=1.0, rescale=True, seed=31),
     "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
                           router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
     "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",
@@ -120,14 +122,29 @@ def test_partition_parity(mode):
     assert not W2_e.view(w.E, w.d, m8)[:, :, w.m:].float().abs().sum()
 
 
-def test_steps_reproduce_forward_bit_exactly():
+STEP_CASES = {
+    "mid_st_bias_cap": SMALL["mid_st_bias_cap"],
+    # small batches (weight-streaming kernels up to 16 tokens, tcgen05 above)
+    "decode_t64_m344": SMALL["decode_t64_m344"],
+    "decode_ragged_d": SMALL["decode_ragged_d"],
+    "decode_t16_st_cap": SMALL["decode_t16_st_cap"],
+    "one_token": SMALL["one_token"],
+    "decode_st_bias_cap": W("decode_st_bias_cap", T=48, d=192, d_ff=16 * 40, E=16, k=4,
+                            router=wl.ST, noisy=True, bias=True, cf=1.0, rescale=True,
+                            lam=0.01, seed=30),
+}
+
+
+@pytest.mark.parametrize("name", list(STEP_CASES))
+def test_steps_reproduce_forward_bit_exactly(name):
     """The six step calls give the same bytes as moe_forward, and reruns are identical."""
-    w = SMALL["mid_st_bias_cap"]
+    w = STEP_CASES[name]
     inp = wl.make_inputs(w)
     p, bufs, ws, status, (W13_e, W2_e) = H.run_forward(w, inp)
-    dev = "cuda"
+    assert status == 0
     b2 = moe.ForwardBuffers(p)
-    x, Wg, Wn, eps, bias = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps", "bias"))
+    x, Wg, Wn, eps, bias = (None if inp.get(n) is None else inp[n].to("cuda")
+                            for n in ("x", "Wg", "Wnoise", "eps", "bias"))
     moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b2.topk_idx, b2.topk_w, b2.probs_sum,
                   b2.importance)
     moe.moe_dispatch(p, x, b2.topk_idx, ws, b2.x_perm, b2.row_token, b2.slot_row, b2.counts,
@@ -143,14 +160,20 @@ def test_steps_reproduce_forward_bit_exactly():
         assert torch.equal(getattr(bufs, n), getattr(b2, n)), n
     assert torch.equal(bufs.out[:R], b2.out[:R])
     assert torch.equal(bufs.row_token[:R], b2.row_token[:R])
+    assert torch.equal(bufs.x_perm[:R], b2.x_perm[:R])
+    assert torch.equal(bufs.h[:R, :w.m], b2.h[:R, :w.m])
 
 
-@pytest.mark.parametrize("T", [600, 2500], ids=["one_sm_kernel", "two_sm_kernel"])
-def test_gather_gemm_equals_permuted_copy_gemm(T):
-    """moe_expert_up_gather (rows of x fetched by TMA gather through row_token) gives
-    the same bytes as moe_expert_up on the permuted copy x_perm, and
-    moe_dispatch_rows the same tables as moe_dispatch."""
-    w = W("gather", T=T, d=320, d_ff=8 * 176, E=8, k=2, noisy=True, cf=1.2, seed=45)
+@pytest.mark.parametrize("T,d,E,k", [(600, 320, 8, 2), (2500, 320, 8, 2), (2500, 200, 8, 2),
+                                     (1100, 136, 16, 4)],
+                         ids=["one_sm_kernel", "two_sm_kernel", "two_sm_k_tail",
+                              "two_sm_e16_k_tail"])
+def test_gather_gemm_equals_permuted_copy_gemm(T, d, E, k):
+    """moe_expert_up_gather (rows of x gathered through row_token: TMA gather4 in the
+    1-SM kernel, cp.async in the 2-SM kernel) gives the same bytes as moe_expert_up
+    on the permuted copy x_perm, and moe_dispatch_rows the same tables as
+    moe_dispatch."""
+    w = W("gather", T=T, d=d, d_ff=E * 176, E=E, k=k, noisy=True, cf=1.2, seed=45)
     inp = wl.make_inputs(w)
     p = H.layer_params(w)
     ws = moe.Workspace(p)

@@ -106,9 +106,10 @@ WsLayout ws_layout(const moe_params_t *p)
     L.rpart = take(blocks * 2 * p->E * sizeof(float));
     const size_t chunks = (size_t)ceil_div(p->T > 0 ? p->T : 1, kDispatchChunk);
     L.hist = take(chunks * p->E * sizeof(int32_t));
-    L.rsmall = take(p->T <= kRouterSmallTokens
-                        ? (size_t)kRouterSmallSplit * (p->T > 0 ? p->T : 1) * 2 * p->E * sizeof(float)
-                        : 0);
+    // Sections for small batches are sized for min(T, 64) tokens even when T is
+    // larger, so that a workspace sized for T also serves every smaller batch.
+    const int t_small = p->T < kRouterSmallTokens ? (p->T > 0 ? p->T : 1) : kRouterSmallTokens;
+    L.rsmall = take((size_t)kRouterSmallSplit * t_small * 2 * p->E * sizeof(float));
     L.total = off;
     return L;
 }
@@ -214,8 +215,8 @@ int moe_get_device_status(void *ws, int32_t *status, int32_t clear, void *stream
     cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess)
         e = cudaStreamSynchronize(s);
-    if (e == cudaSuccess && clear)
-        e = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess && clear)  // status word and the launch counters
+        e = cudaMemsetAsync(ws, 0, kWsResetBytes, s);
     if (e != cudaSuccess)
         return cuda_fail(e, fn);
     *status = v;

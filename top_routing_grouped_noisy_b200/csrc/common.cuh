@@ -23,6 +23,8 @@ constexpr size_t kWsHeader = 256;
 constexpr int kWsCounterWord = 1;
 // Word 2: ticket counter of the tensor-core router (zero between calls).
 constexpr int kWsRouterCounterWord = 2;
+// Header bytes that clearing the status resets (status word and counters).
+constexpr size_t kWsResetBytes = 32;
 
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {

@@ -1,4 +1,4 @@
-// decode.cu -- a3/a4 for decode-shaped bf16 batches (T <= 64 tokens): the expert
+// decode.cu -- a3/a4 for decode-shaped bf16 batches (T <= 16 tokens): the expert
 // FFN then reads each selected expert's weights once and does little arithmetic
 // per byte, so it is bound by streaming weights from HBM.  SwiGLU expert as in
 // "LLaMA-MoE v2", code sample "代码实现示例", class Expert.
@@ -221,10 +221,8 @@ cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const in
 {
     if (p->T <= 8)
         up_dispatch<1>(p, x_perm, offsets, W13, h, s);
-    else if (p->T <= 16)
-        up_dispatch<2>(p, x_perm, offsets, W13, h, s);
     else
-        up_dispatch<4>(p, x_perm, offsets, W13, h, s);
+        up_dispatch<2>(p, x_perm, offsets, W13, h, s);
     count_launch();
     return cudaGetLastError();
 }
@@ -234,10 +232,8 @@ cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32
 {
     if (p->T <= 8)
         down_dispatch<1>(p, h, offsets, W2, out, s);
-    else if (p->T <= 16)
-        down_dispatch<2>(p, h, offsets, W2, out, s);
     else
-        down_dispatch<4>(p, h, offsets, W2, out, s);
+        down_dispatch<2>(p, h, offsets, W2, out, s);
     count_launch();
     return cudaGetLastError();
 }

@@ -85,8 +85,11 @@ cudaError_t launch_up_tc_gather(const moe_params_t *p, const void *x, const int3
 cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
                            const void *W2, void *out, int32_t *status, cudaStream_t s);
 
-// a3 / a4 for decode-shaped bf16 batches (T <= kDecodeMaxTokens): weight streaming
-constexpr int kDecodeMaxTokens = 64;
+// a3 / a4 for decode-shaped bf16 batches (T <= kDecodeMaxTokens): weight
+// streaming on the CUDA-core/mma.sync path.  Larger batches, from 17 tokens up,
+// run the tcgen05 grouped GEMMs, which stream the selected experts' weights
+// faster once each expert has a few rows.
+constexpr int kDecodeMaxTokens = 16;
 cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                              const void *W13, void *h, cudaStream_t s);
 cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32_t *offsets,

@@ -13,87 +13,11 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "gate.cuh"
 #include "kernels.h"
 
 namespace moe {
 
-
-__device__ __forceinline__ float softplus_f(float z) { return fmaxf(z, 0.f) + log1pf(expf(-fabsf(z))); }
-
-// Gate of one token from its clean logits lg[0..E) and noise logits lg[E..2E).
-// Writes the token's k (index, weight) pairs, its full softmax prob[0..E) and its
-// per-expert gate weight gw[0..E) (zero where not selected).  The routing logits
-// H overwrite lg[0..E) (each lg[e], lg[E+e] is read before H[e] is written).
-__device__ void finish_token(int64_t t, float *lg, int E, int k, int noisy,
-                             const float *__restrict__ noise, const float *__restrict__ bias,
-                             int router_type, int32_t *__restrict__ idx_out,
-                             float *__restrict__ w_out, float *prob, float *gw, int32_t *status)
-{
-    float *H = lg;
-    bool bad = false;
-    for (int e = 0; e < E; ++e) {
-        float h = lg[e];
-        if (bias)
-            h += bias[e];
-        if (noisy)
-            h += noise[t * E + e] * softplus_f(lg[E + e]);
-        bad |= !isfinite(h);
-        H[e] = h;
-        gw[e] = 0.f;
-    }
-    if (bad) {
-        set_status(status, MOE_ERR_DEVICE_BADINDEX);
-        for (int j = 0; j < k; ++j) {
-            idx_out[t * k + j] = -1;
-            w_out[t * k + j] = 0.f;
-        }
-        for (int e = 0; e < E; ++e)
-            prob[e] = 0.f;
-        return;
-    }
-    int sel[MOE_MAX_TOPK];
-    uint64_t taken = 0;
-    for (int j = 0; j < k; ++j) {
-        int bi = -1;
-        float best = 0.f;
-        for (int e = 0; e < E; ++e) {
-            if ((taken >> e) & 1ull)
-                continue;
-            if (bi < 0 || H[e] > best) {
-                best = H[e];
-                bi = e;
-            }
-        }
-        taken |= 1ull << bi;
-        sel[j] = bi;
-    }
-    const float hmax = H[sel[0]];
-    float z = 0.f;
-    for (int e = 0; e < E; ++e)
-        z += expf(H[e] - hmax);
-    const float inv = 1.f / z;
-    for (int e = 0; e < E; ++e)
-        prob[e] = expf(H[e] - hmax) * inv;
-    if (router_type == MOE_ROUTER_MIXTRAL) {
-        float zs = 0.f;
-        for (int j = 0; j < k; ++j)
-            zs += expf(H[sel[j]] - hmax);
-        const float is = 1.f / zs;
-        for (int j = 0; j < k; ++j) {
-            const float w = expf(H[sel[j]] - hmax) * is;
-            idx_out[t * k + j] = sel[j];
-            w_out[t * k + j] = w;
-            gw[sel[j]] = w;
-        }
-    } else {
-        for (int j = 0; j < k; ++j) {
-            const float w = prob[sel[j]];
-            idx_out[t * k + j] = sel[j];
-            w_out[t * k + j] = w;
-            gw[sel[j]] = w;
-        }
-    }
-}
 
 // Per-CTA partial sums over its tokens, in token order.
 __device__ void write_partials(int ntok, int E, const float *prob_s, const float *gw_s,
@@ -185,11 +109,10 @@ __global__ void __launch_bounds__(1024) router_finalize_kernel(const float *__re
 
 // ---------------------------------------------------------------- T <= 64 tokens
 // Decode-sized batches: a few tokens cannot keep the split-over-warps kernel
-// busy, so K is split over kSmallKSplit CTAs instead.  Each CTA stages its K slice
+// busy, so K is split over kRouterSmallSplit CTAs instead.  Each CTA stages its K slice
 // of x and of [W_g | W_noise] (read in place, no transpose) in shared memory and
 // writes partial logits part[ks][t][o]; one finishing CTA adds the slices in a
 // fixed order, runs the per-token gate and the token sums.
-constexpr int kSmallKSplit = kRouterSmallSplit;
 
 template <typename E_T>
 __global__ void __launch_bounds__(256) router_small_partial_kernel(
@@ -197,29 +120,7 @@ __global__ void __launch_bounds__(256) router_small_partial_kernel(
     int d, int E, float *__restrict__ part)
 {
     extern __shared__ float sm[];
-    const int nout = Wn ? 2 * E : E;
-    const int kc = (d + kSmallKSplit - 1) / kSmallKSplit;
-    const int k0 = blockIdx.x * kc, k1 = min(d, k0 + kc);
-    const int kn = k1 > k0 ? k1 - k0 : 0;
-    float *xs = sm;                    // [T][kc]
-    float *ws_ = sm + (size_t)T * kc;  // [kc][nout]
-    for (int i = threadIdx.x; i < T * kn; i += blockDim.x) {
-        const int t = i / kn, c = i % kn;
-        xs[t * kc + c] = to_f32(x[(int64_t)t * d + k0 + c]);
-    }
-    for (int i = threadIdx.x; i < kn * nout; i += blockDim.x) {
-        const int c = i / nout, o = i % nout;
-        ws_[c * nout + o] = o < E ? to_f32(Wg[(int64_t)(k0 + c) * E + o])
-                                  : to_f32(Wn[(int64_t)(k0 + c) * E + o - E]);
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
-        const int t = i / nout, o = i % nout;
-        float acc = 0.f;
-        for (int c = 0; c < kn; ++c)
-            acc = fmaf(xs[t * kc + c], ws_[c * nout + o], acc);
-        part[((int64_t)blockIdx.x * T + t) * nout + o] = acc;
-    }
+    router_small_slice(blockIdx.x, x, Wg, Wn, T, d, E, part, sm);
 }
 
 __global__ void __launch_bounds__(256) router_small_finish_kernel(
@@ -229,30 +130,8 @@ __global__ void __launch_bounds__(256) router_small_finish_kernel(
     float *__restrict__ importance, int32_t *status)
 {
     extern __shared__ float sm[];
-    const int nout = noisy ? 2 * E : E;
-    float *lg = sm;                          // [T][nout]
-    float *prob_s = lg + (size_t)T * nout;   // [T][E]
-    float *gw_s = prob_s + (size_t)T * E;    // [T][E]
-    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
-        float acc = 0.f;
-        for (int ks = 0; ks < kSmallKSplit; ++ks)
-            acc += part[(int64_t)ks * T * nout + i];
-        lg[i] = acc;
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < T; t += blockDim.x)
-        finish_token(t, lg + (size_t)t * nout, E, k, noisy, noise, bias, router_type, idx_out,
-                     w_out, prob_s + (size_t)t * E, gw_s + (size_t)t * E, status);
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        float sp = 0.f, sg = 0.f;
-        for (int t = 0; t < T; ++t) {
-            sp += prob_s[t * E + e];
-            sg += gw_s[t * E + e];
-        }
-        probs_sum[e] = sp;
-        importance[e] = sg;
-    }
+    router_small_finish(part, T, E, k, noisy, noise, bias, router_type, idx_out, w_out,
+                        probs_sum, importance, status, sm);
 }
 
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
@@ -266,7 +145,7 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
     cudaError_t e = cudaSuccess;
     const int small_noisy = Wnoise != nullptr;
     const int small_nout = small_noisy ? 2 * p->E : p->E;
-    const int small_kc = ceil_div(p->d, kSmallKSplit);
+    const int small_kc = ceil_div(p->d, kRouterSmallSplit);
     const size_t sm1 = sizeof(float) * ((size_t)p->T * small_kc + (size_t)small_kc * small_nout);
     const size_t sm2 =
         sizeof(float) * ((size_t)p->T * small_nout + 2 * (size_t)p->T * p->E);
@@ -274,10 +153,10 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
         const int noisy = small_noisy;
         float *sp = reinterpret_cast<float *>(ws + L.rsmall);
         if (p->dtype == MOE_BF16)
-            router_small_partial_kernel<bf16><<<kSmallKSplit, 256, sm1, s>>>(
+            router_small_partial_kernel<bf16><<<kRouterSmallSplit, 256, sm1, s>>>(
                 (const bf16 *)x, (const bf16 *)Wg, (const bf16 *)Wnoise, p->T, p->d, p->E, sp);
         else
-            router_small_partial_kernel<float><<<kSmallKSplit, 256, sm1, s>>>(
+            router_small_partial_kernel<float><<<kRouterSmallSplit, 256, sm1, s>>>(
                 (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E, sp);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess)
