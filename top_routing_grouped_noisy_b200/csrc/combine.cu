@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ ou
                                                       const float *__restrict__ w, int T, int d,
                                                       int k, float scale, E_T *__restrict__ y)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int VN = Vec<E_T>::N;
     constexpr int VPT = kCombineVPT;
     const int nv = d / VN;
@@ -91,6 +93,8 @@ __global__ void gate_stats_kernel(const int32_t *__restrict__ counts,
                                   float lambda, float *__restrict__ f, float *__restrict__ P,
                                   float *__restrict__ loss)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ double s_fp[MOE_MAX_EXPERTS];
     const int e = threadIdx.x;
     if (e < E) {
@@ -120,10 +124,10 @@ cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t
 #define MOE_COMBINE(KM)                                                                        \
     do {                                                                                       \
         if (p->dtype == MOE_BF16)                                                              \
-            combine_kernel<bf16, KM><<<grid, 256, 0, s>>>((const bf16 *)out, slot_row, w, p->T, \
+            launch_pdl(combine_kernel<bf16, KM>, dim3(grid), dim3(256), 0, s, (const bf16 *)out, slot_row, w, p->T, \
                                                           p->d, p->k, scale, (bf16 *)y);       \
         else                                                                                   \
-            combine_kernel<float, KM><<<grid, 256, 0, s>>>((const float *)out, slot_row, w,     \
+            launch_pdl(combine_kernel<float, KM>, dim3(grid), dim3(256), 0, s, (const float *)out, slot_row, w,     \
                                                            p->T, p->d, p->k, scale, (float *)y); \
     } while (0)
     if (p->k <= 2)
@@ -141,7 +145,7 @@ cudaError_t launch_gate_stats(const moe_params_t *p, const int32_t *counts,
                               const float *probs_sum, float *f, float *P, float *loss,
                               cudaStream_t s)
 {
-    gate_stats_kernel<<<1, MOE_MAX_EXPERTS, 0, s>>>(counts, probs_sum, p->T, p->E, p->k,
+    launch_pdl(gate_stats_kernel, dim3(1), dim3(MOE_MAX_EXPERTS), 0, s, counts, probs_sum, p->T, p->E, p->k,
                                                     p->balance_lambda, f, P, loss);
     count_launch();
     return cudaGetLastError();

@@ -26,6 +26,18 @@ constexpr int kWsRouterCounterWord = 2;
 // Header bytes that clearing the status resets (status word and counters).
 constexpr size_t kWsResetBytes = 32;
 
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialization allowed (launch_pdl): it may be scheduled
+// while the previous kernel on the stream is still running, so it calls
+// pdl_wait() before it touches global memory (the wait returns once the
+// previous grid has completed and its writes are visible), and pdl_trigger() to
+// let the next kernel be scheduled early in turn.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {
     if (status != nullptr)

@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(256) decode_up_kernel(const bf16 *__restrict__
                                                         int m, int blocks_per_expert,
                                                         bf16 *__restrict__ h)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int NJ = NNT * 8;
     __shared__ float red[kDecodeWarps * 32 * NJ];
     const int e = blockIdx.x / blocks_per_expert, blk = blockIdx.x % blocks_per_expert;
@@ -159,6 +161,8 @@ __global__ void __launch_bounds__(256) decode_down_kernel(const bf16 *__restrict
                                                           int m, int blocks_per_expert,
                                                           bf16 *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int NJ = NNT * 8;
     __shared__ float red[kDecodeWarps * 32 * NJ];
     const int e = blockIdx.x / blocks_per_expert, blk = blockIdx.x % blocks_per_expert;
@@ -202,7 +206,7 @@ static void up_dispatch(const moe_params_t *p, const void *x_perm, const int32_t
                         const void *W13, void *h, cudaStream_t s)
 {
     const int bpe = (p->m + 15) / 16;
-    decode_up_kernel<NNT><<<p->E * bpe, 256, 0, s>>>((const bf16 *)x_perm, offsets,
+    launch_pdl(decode_up_kernel<NNT>, dim3(p->E * bpe), dim3(256), 0, s, (const bf16 *)x_perm, offsets,
                                                     (const bf16 *)W13, p->d, p->m, bpe, (bf16 *)h);
 }
 
@@ -211,7 +215,7 @@ static void down_dispatch(const moe_params_t *p, const void *h, const int32_t *o
                           const void *W2, void *out, cudaStream_t s)
 {
     const int bpe = (p->d + 31) / 32;
-    decode_down_kernel<NNT><<<p->E * bpe, 256, 0, s>>>((const bf16 *)h, offsets,
+    launch_pdl(decode_down_kernel<NNT>, dim3(p->E * bpe), dim3(256), 0, s, (const bf16 *)h, offsets,
                                                       (const bf16 *)W2, p->d, p->m, bpe,
                                                       (bf16 *)out);
 }

@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(256) dispatch_count_kernel(
     int32_t *counter, int32_t *__restrict__ counts, int32_t *__restrict__ kept,
     int32_t *__restrict__ offsets, int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int s_last;
     __shared__ int32_t s_count[MOE_MAX_EXPERTS];
     __shared__ int32_t s_hist[kCountSmemInts];
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(
     const int32_t *__restrict__ kept, const int32_t *__restrict__ offsets,
     int32_t *__restrict__ row_token, int32_t *__restrict__ slot_row)
 {
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
     const int c = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -208,6 +212,8 @@ __global__ void __launch_bounds__(256) dispatch_copy_kernel(const char *__restri
                                                             const int32_t *__restrict__ slot_row,
                                                             char *__restrict__ x_perm)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t nv = row_bytes / 16;
     const int64_t items = (int64_t)T * nv;
     const int64_t per = (items + gridDim.x - 1) / gridDim.x;
@@ -263,7 +269,7 @@ static cudaError_t launch_rank_copy(const moe_params_t *p, const void *x, const 
                                     int32_t *slot_row, cudaStream_t s)
 {
     const int nch = ceil_div(p->T, kDispatchChunk);
-    dispatch_rank_kernel<<<ceil_div(nch, 8), 256, 0, s>>>(idx, p->T, p->k, p->E, hist, kept,
+    launch_pdl(dispatch_rank_kernel, dim3(ceil_div(nch, 8)), dim3(256), 0, s, idx, p->T, p->k, p->E, hist, kept,
                                                           offsets, row_token, slot_row);
     count_launch();
     cudaError_t e = cudaGetLastError();
@@ -275,7 +281,7 @@ static cudaError_t launch_rank_copy(const moe_params_t *p, const void *x, const 
     int64_t grid = (items + min_per - 1) / min_per;
     if (grid > copy_wave())
         grid = copy_wave();
-    dispatch_copy_kernel<<<(unsigned)grid, 256, 0, s>>>((const char *)x, row_bytes, p->T, p->k,
+    launch_pdl(dispatch_copy_kernel, dim3((unsigned)grid), dim3(256), 0, s, (const char *)x, row_bytes, p->T, p->k,
                                                          slot_row, (char *)x_perm);
     count_launch();
     return cudaGetLastError();
@@ -289,7 +295,7 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
     const WsLayout L = ws_layout(p);
     int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
     int32_t *counter = reinterpret_cast<int32_t *>(ws) + kWsCounterWord;
-    dispatch_count_kernel<<<count_grid(p->T), 256, 0, s>>>(idx, p->T, p->k, p->E, p->capacity,
+    launch_pdl(dispatch_count_kernel, dim3(count_grid(p->T)), dim3(256), 0, s, idx, p->T, p->k, p->E, p->capacity,
                                                            hist, counter, counts, kept, offsets,
                                                            status);
     count_launch();
@@ -385,7 +391,7 @@ extern "C" int moe_dispatch_noalloc(const moe_params_t *p, const void *x,
     int32_t *st = status != nullptr ? status : scratch + kNoallocHistInts;
     int32_t *counter = scratch + kNoallocHistInts + 1;  // zero at load, reset by every call
     cudaStream_t s = (cudaStream_t)stream;
-    dispatch_count_kernel<<<count_grid(p->T), 256, 0, s>>>(topk_idx, p->T, p->k, p->E,
+    launch_pdl(dispatch_count_kernel, dim3(count_grid(p->T)), dim3(256), 0, s, topk_idx, p->T, p->k, p->E,
                                                            p->capacity, hist, counter, counts,
                                                            kept, offsets, st);
     count_launch();

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(256) up_simt_kernel(const float *__restrict__ 
                                                       const float *__restrict__ W13, int E,
                                                       int d, int m, float *__restrict__ h)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int BM = kSimtBM, BK = 16, BP = 64;  // BP packed rows = 32 neurons
     __shared__ float As[BK][BM + 4];
     __shared__ float Bs[BK][BP + 4];
@@ -107,6 +109,8 @@ __global__ void __launch_bounds__(256) down_simt_kernel(const float *__restrict_
                                                         const float *__restrict__ W2, int E,
                                                         int d, int m, float *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int BM = kSimtBM, BK = 16, BN = 64;
     __shared__ float As[BK][BM + 4];
     __shared__ float Bs[BK][BN + 4];
@@ -182,7 +186,7 @@ cudaError_t launch_up_simt(const moe_params_t *p, const float *x_perm, const int
                            const float *W13, float *h, cudaStream_t s)
 {
     dim3 grid(max_mtiles(p, kSimtBM), ceil_div(p->m, 32));
-    up_simt_kernel<<<grid, 256, 0, s>>>(x_perm, offsets, W13, p->E, p->d, p->m, h);
+    launch_pdl(up_simt_kernel, dim3(grid), dim3(256), 0, s, x_perm, offsets, W13, p->E, p->d, p->m, h);
     count_launch();
     return cudaGetLastError();
 }
@@ -191,7 +195,7 @@ cudaError_t launch_down_simt(const moe_params_t *p, const float *h, const int32_
                              const float *W2, float *out, cudaStream_t s)
 {
     dim3 grid(max_mtiles(p, kSimtBM), ceil_div(p->d, 64));
-    down_simt_kernel<<<grid, 256, 0, s>>>(h, offsets, W2, p->E, p->d, p->m, out);
+    launch_pdl(down_simt_kernel, dim3(grid), dim3(256), 0, s, h, offsets, W2, p->E, p->d, p->m, out);
     count_launch();
     return cudaGetLastError();
 }

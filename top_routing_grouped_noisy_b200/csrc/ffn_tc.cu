@@ -222,6 +222,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
                         uint64_t wait_ns, const int32_t *__restrict__ row_token)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -592,6 +594,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
                             uint64_t wait_ns, const int32_t *__restrict__ row_token)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -927,25 +931,27 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     const int N = (int)b_rows, K = (int)a_k;
     if (!pair) {
         if (gather)
-            grouped_gemm_kernel<EPI, true><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
+            launch_pdl(grouped_gemm_kernel<EPI, true>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s, 
                 ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
         else
-            grouped_gemm_kernel<EPI, false><<<di->sms, NUM_THREADS, SMEM_BYTES, s>>>(
+            launch_pdl(grouped_gemm_kernel<EPI, false>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s, 
                 ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(2 * di->pair_clusters);
     cfg.blockDim = dim3(tc2::NUM_THREADS);
     cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (gather)
         return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, true>, ta, tb, to,
                                   offsets, E, N, K, out, ld_out, n_valid, status, wait_ns,

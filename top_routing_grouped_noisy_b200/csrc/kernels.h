@@ -42,6 +42,26 @@ int report_error(int code, const char *msg);
 int report_cuda(cudaError_t e, const char *where);
 int report_ok();
 
+// Launches `kern` with programmatic stream serialization allowed: the kernel
+// may be scheduled while the previous kernel on `s` finishes (it waits for that
+// kernel with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Launch counter shared by every launch site.
 void count_launch(int n = 1);
 // Current time limit of bounded device waits (ns).

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(128) partition_w13_kernel(
     int m16, int mode, const int32_t *__restrict__ perm, E_T *__restrict__ W13,
     int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;
     const int e = (int)(row / (2 * m16));
     const int r = (int)(row % (2 * m16));
@@ -55,6 +57,8 @@ __global__ void __launch_bounds__(256) partition_w2_kernel(
     const E_T *__restrict__ W2, int d, int d_ff, int E, int m, int m8, int mode,
     const int32_t *__restrict__ perm, E_T *__restrict__ W2e, int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t row = blockIdx.x;  // e * d + o
     const int e = (int)(row / d);
     const int o = (int)(row % d);
@@ -86,16 +90,16 @@ cudaError_t launch_partition(const void *W1, const void *W3, const void *W2, int
     const unsigned g13 = (unsigned)((int64_t)E * 2 * m16);
     const unsigned g2 = (unsigned)((int64_t)E * d);
     if (dtype == MOE_BF16) {
-        partition_w13_kernel<bf16><<<g13, 128, 0, s>>>(
+        launch_pdl(partition_w13_kernel<bf16>, dim3(g13), dim3(128), 0, s, 
             (const bf16 *)W1, (const bf16 *)W3, d, d_ff, E, m, m16, mode, perm, (bf16 *)W13_e,
             status);
-        partition_w2_kernel<bf16><<<g2, 256, 0, s>>>((const bf16 *)W2, d, d_ff, E, m, m8, mode,
+        launch_pdl(partition_w2_kernel<bf16>, dim3(g2), dim3(256), 0, s, (const bf16 *)W2, d, d_ff, E, m, m8, mode,
                                                      perm, (bf16 *)W2_e, status);
     } else {
-        partition_w13_kernel<float><<<g13, 128, 0, s>>>(
+        launch_pdl(partition_w13_kernel<float>, dim3(g13), dim3(128), 0, s, 
             (const float *)W1, (const float *)W3, d, d_ff, E, m, m16, mode, perm,
             (float *)W13_e, status);
-        partition_w2_kernel<float><<<g2, 256, 0, s>>>((const float *)W2, d, d_ff, E, m, m8,
+        launch_pdl(partition_w2_kernel<float>, dim3(g2), dim3(256), 0, s, (const float *)W2, d, d_ff, E, m, m8,
                                                       mode, perm, (float *)W2_e, status);
     }
     count_launch(2);

@@ -41,6 +41,8 @@ __global__ void __launch_bounds__(256) router_f32_kernel(
     int router_type, int32_t *__restrict__ idx_out, float *__restrict__ w_out,
     float *__restrict__ part, int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int TOK = kRouterWarps;
     extern __shared__ float smem[];
     const int nout = Wn ? 2 * E : E;
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(1024) router_finalize_kernel(const float *__re
                                                                float *__restrict__ probs_sum,
                                                                float *__restrict__ importance)
 {
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int o = warp; o < 2 * E; o += blockDim.x / 32) {
         const int which = o / E, e = o % E;
@@ -119,6 +123,8 @@ __global__ void __launch_bounds__(256) router_small_partial_kernel(
     const E_T *__restrict__ x, const E_T *__restrict__ Wg, const E_T *__restrict__ Wn, int T,
     int d, int E, float *__restrict__ part)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float sm[];
     router_small_slice(blockIdx.x, x, Wg, Wn, T, d, E, part, sm);
 }
@@ -129,6 +135,8 @@ __global__ void __launch_bounds__(256) router_small_finish_kernel(
     int32_t *__restrict__ idx_out, float *__restrict__ w_out, float *__restrict__ probs_sum,
     float *__restrict__ importance, int32_t *status)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ float sm[];
     router_small_finish(part, T, E, k, noisy, noise, bias, router_type, idx_out, w_out,
                         probs_sum, importance, status, sm);
@@ -153,15 +161,15 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
         const int noisy = small_noisy;
         float *sp = reinterpret_cast<float *>(ws + L.rsmall);
         if (p->dtype == MOE_BF16)
-            router_small_partial_kernel<bf16><<<kRouterSmallSplit, 256, sm1, s>>>(
+            launch_pdl(router_small_partial_kernel<bf16>, dim3(kRouterSmallSplit), dim3(256), sm1, s, 
                 (const bf16 *)x, (const bf16 *)Wg, (const bf16 *)Wnoise, p->T, p->d, p->E, sp);
         else
-            router_small_partial_kernel<float><<<kRouterSmallSplit, 256, sm1, s>>>(
+            launch_pdl(router_small_partial_kernel<float>, dim3(kRouterSmallSplit), dim3(256), sm1, s, 
                 (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E, sp);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
-        router_small_finish_kernel<<<1, 256, sm2, s>>>(sp, p->T, p->E, p->k, noisy, noise, bias,
+        launch_pdl(router_small_finish_kernel, dim3(1), dim3(256), sm2, s, sp, p->T, p->E, p->k, noisy, noise, bias,
                                                        p->router_type, idx, w, probs_sum,
                                                        importance, status);
         count_launch();
@@ -176,14 +184,14 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
     if (p->T > 0) {
         nblk = ceil_div(p->T, kRouterWarps);
         const size_t smem = sizeof(float) * ((size_t)kRouterWarps * 4 * p->E);
-        router_f32_kernel<<<nblk, 256, smem, s>>>(
+        launch_pdl(router_f32_kernel, dim3(nblk), dim3(256), smem, s, 
             (const float *)x, (const float *)Wg, (const float *)Wnoise, p->T, p->d, p->E, p->k,
             noise, bias, p->router_type, idx, w, part, status);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess)
             return e;
     }
-    router_finalize_kernel<<<1, 1024, 0, s>>>(part, nblk, p->E, probs_sum, importance);
+    launch_pdl(router_finalize_kernel, dim3(1), dim3(1024), 0, s, part, nblk, p->E, probs_sum, importance);
     count_launch();
     return cudaGetLastError();
 }

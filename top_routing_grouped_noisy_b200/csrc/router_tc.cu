@@ -110,6 +110,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      float *__restrict__ probs_sum, float *__restrict__ importance,
                      int32_t *status, uint64_t wait_ns)
 {
+    pdl_wait();
+    pdl_trigger();
     using C = Cfg<NOUT>;
     constexpr int STAGES = C::STAGES;
     constexpr int EMAX = NOISY ? NOUT / 2 : NOUT;
@@ -399,6 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 __global__ void router_pack_tc_kernel(const bf16 *__restrict__ Wg, const bf16 *__restrict__ Wn,
                                       int d, int E, int rows, bf16 *__restrict__ Wt)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)rows * d)
         return;
@@ -450,7 +454,7 @@ static cudaError_t run(const moe_params_t *p, const void *x, const bf16 *Wt, con
         return e;
     const int n_tiles = ceil_div(p->T, BM);
     const int grid = n_tiles < sms_cached[dev] ? n_tiles : sms_cached[dev];
-    router_tc_kernel<NOUT, NOISY><<<grid, NUM_THREADS, SMEM, s>>>(
+    launch_pdl(router_tc_kernel<NOUT, NOISY>, dim3(grid), dim3(NUM_THREADS), SMEM, s, 
         tx, tw, p->T, p->d, p->E, p->k, noise, bias, p->router_type, idx, w, part, counter,
         probs_sum, importance, status, wait_limit_ns());
     return cudaGetLastError();
@@ -469,7 +473,7 @@ cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wg
     const int nout = noisy ? 2 * p->E : p->E;
     const int rows = nout <= 16 ? 16 : nout <= 32 ? 32 : nout <= 64 ? 64 : 128;
     const int64_t n = (int64_t)rows * p->d;
-    rtc::router_pack_tc_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+    launch_pdl(rtc::router_pack_tc_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 
         (const bf16 *)Wg, (const bf16 *)Wnoise, p->d, p->E, rows, Wt);
     count_launch();
     cudaError_t e = cudaGetLastError();
