@@ -468,6 +468,44 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
     REQUIRE_PTR(b->loss);
     REQUIRE_PTR(b->f);
     REQUIRE_PTR(b->P);
+    if (small_forward_fits(p, b->Wnoise != nullptr)) {
+        // decode-shaped batch: router slices, then router finish + dispatch tables +
+        // gate statistics in one CTA, GEMM 1 gathering rows of x, GEMM 2, combine
+        REQUIRE_PTR(b->x);
+        REQUIRE_PTR(b->Wg);
+        OPTIONAL_PTR(b->Wnoise);
+        OPTIONAL_PTR(b->noise);
+        OPTIONAL_PTR(b->bias);
+        REQUIRE_PTR(b->W13_e);
+        REQUIRE_PTR(b->W2_e);
+        REQUIRE_PTR(b->counts);
+        REQUIRE_PTR(b->importance);
+        REQUIRE_PTR(b->topk_idx);
+        REQUIRE_PTR(b->topk_w);
+        REQUIRE_PTR(b->probs_sum);
+        REQUIRE_PTR(b->x_perm);
+        REQUIRE_PTR(b->row_token);
+        REQUIRE_PTR(b->slot_row);
+        REQUIRE_PTR(b->kept);
+        REQUIRE_PTR(b->offsets);
+        REQUIRE_PTR(b->h);
+        REQUIRE_PTR(b->out);
+        if (b->Wnoise != nullptr && b->noise == nullptr)
+            return fail(MOE_ERR_INVALID_ARG, "%s: Wnoise given without the noise draws", fn);
+        if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+            return rc;
+        char *w = static_cast<char *>(ws);
+        cudaStream_t s = (cudaStream_t)stream;
+        cudaError_t e = launch_route_dispatch_small(p, b, w, reinterpret_cast<int32_t *>(w), s);
+        if (e == cudaSuccess)
+            e = launch_up_decode_gather(p, b->x, b->row_token, b->offsets, b->W13_e, b->h,
+                                        b->x_perm, s);
+        if (e == cudaSuccess)
+            e = launch_down_decode(p, b->h, b->offsets, b->W2_e, b->out, s);
+        if (e == cudaSuccess)
+            e = launch_combine(p, b->out, b->slot_row, b->topk_w, b->y, s);
+        return after_launch(fn, e);
+    }
     if ((rc = moe_route(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx, b->topk_w,
                         b->probs_sum, b->importance, ws, ws_bytes, stream)) != MOE_OK)
         return rc;

@@ -20,17 +20,24 @@ namespace moe {
 constexpr int kDecodeWarps = 8;
 
 // acc += W[0..32) . X[0..n_rows)^T over K; weight rows >= w_rows and activation
-// columns >= k_valid_x read as zero.
+// columns >= k_valid_x read as zero.  Activation row r is Xrows + r x_ld, or,
+// with a row table, Xrows + rtok[r] x_ld (rows of x gathered in dispatch order).
 template <int NNT>
 __device__ __forceinline__ void decode_mma_block(const bf16 *__restrict__ Wrows, int64_t w_ld,
                                                  int w_rows, const bf16 *__restrict__ Xrows,
                                                  int64_t x_ld, int n_rows, int K, int k_valid_x,
-                                                 float (&acc)[2][NNT][4])
+                                                 float (&acc)[2][NNT][4],
+                                                 const int32_t *__restrict__ rtok = nullptr)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
-    const int nnt = (n_rows + 7) >> 3;
     const int nkb = (K + 31) / 32;
+    const bf16 *xrow[NNT];
+#pragma unroll
+    for (int nt = 0; nt < NNT; ++nt) {
+        const int r = nt * 8 + g;
+        xrow[nt] = r < n_rows ? Xrows + (rtok ? (int64_t)rtok[r] : (int64_t)r) * x_ld : nullptr;
+    }
     // U k32 blocks per round: every load of the round is issued before its MMAs
     constexpr int U = NNT >= 4 ? 2 : 4;
     for (int kb0 = warp; kb0 < nkb; kb0 += kDecodeWarps * U) {
@@ -50,10 +57,8 @@ __device__ __forceinline__ void decode_mma_block(const bf16 *__restrict__ Wrows,
             }
 #pragma unroll
             for (int nt = 0; nt < NNT; ++nt) {
-                const int r = nt * 8 + g;
-                xb[u][nt] = (kv && nt < nnt && r < n_rows)
-                                ? ld_nc(Xrows + (int64_t)r * x_ld + c)
-                                : make_uint4(0, 0, 0, 0);
+                xb[u][nt] = (kv && xrow[nt] != nullptr) ? ld_nc(xrow[nt] + c)
+                                                        : make_uint4(0, 0, 0, 0);
                 if (c + 8 > k_valid_x) {  // activation columns past the valid K are not data
                     uint32_t *wv = reinterpret_cast<uint32_t *>(&xb[u][nt]);
 #pragma unroll
@@ -73,7 +78,7 @@ __device__ __forceinline__ void decode_mma_block(const bf16 *__restrict__ Wrows,
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                 for (int nt = 0; nt < NNT; ++nt) {
-                    if (nt < nnt) {
+                    if (nt * 8 < n_rows) {
                         mma_bf16_16816(acc[mt][nt], wa[u][mt][0].x, wa[u][mt][1].x,
                                        wa[u][mt][0].y, wa[u][mt][1].y, xb[u][nt].x,
                                        xb[u][nt].y);
@@ -105,17 +110,30 @@ __device__ __forceinline__ void decode_store_partials(float *red, const float (&
         }
 }
 
+// x_rows: x_perm (expert-ordered rows), or, when row_token is given, x itself,
+// whose rows are gathered through row_token; then CTA r < R also writes x_perm
+// row r (x_perm_out) for inspection.
 template <int NNT>
-__global__ void __launch_bounds__(256) decode_up_kernel(const bf16 *__restrict__ x_perm,
+__global__ void __launch_bounds__(256) decode_up_kernel(const bf16 *__restrict__ x_rows,
                                                         const int32_t *__restrict__ offsets,
                                                         const bf16 *__restrict__ W13, int d,
                                                         int m, int blocks_per_expert,
-                                                        bf16 *__restrict__ h)
+                                                        bf16 *__restrict__ h,
+                                                        const int32_t *__restrict__ row_token,
+                                                        bf16 *__restrict__ x_perm_out, int E)
 {
     pdl_wait();
     pdl_trigger();
     constexpr int NJ = NNT * 8;
     __shared__ float red[kDecodeWarps * 32 * NJ];
+    if (row_token != nullptr && (int)blockIdx.x < offsets[E]) {
+        const int r = blockIdx.x;
+        const int64_t src = (int64_t)row_token[r] * d;
+        for (int v = threadIdx.x; v < d / 8; v += blockDim.x)
+            st_v4(x_perm_out + (int64_t)r * d + 8 * v, ld_nc(x_rows + src + 8 * v));
+    }
+    if ((int)blockIdx.x >= E * blocks_per_expert)  // extra CTAs of the copy only
+        return;
     const int e = blockIdx.x / blocks_per_expert, blk = blockIdx.x % blocks_per_expert;
     const int r0 = offsets[e], n_rows = offsets[e + 1] - r0;
     if (n_rows <= 0)
@@ -132,7 +150,10 @@ __global__ void __launch_bounds__(256) decode_up_kernel(const bf16 *__restrict__
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     acc[a][b][c] = 0.f;
-        decode_mma_block<NNT>(W, d, 32, x_perm + (int64_t)(r0 + rg) * d, d, nr, d, d, acc);
+        if (row_token != nullptr)
+            decode_mma_block<NNT>(W, d, 32, x_rows, d, nr, d, d, acc, row_token + r0 + rg);
+        else
+            decode_mma_block<NNT>(W, d, 32, x_rows + (int64_t)(r0 + rg) * d, d, nr, d, d, acc);
         if (rg > 0)
             __syncthreads();
         decode_store_partials<NNT>(red, acc);
@@ -203,11 +224,14 @@ __global__ void __launch_bounds__(256) decode_down_kernel(const bf16 *__restrict
 
 template <int NNT>
 static void up_dispatch(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
-                        const void *W13, void *h, cudaStream_t s)
+                        const void *W13, void *h, cudaStream_t s,
+                        const int32_t *row_token = nullptr, void *x_perm_out = nullptr)
 {
     const int bpe = (p->m + 15) / 16;
-    launch_pdl(decode_up_kernel<NNT>, dim3(p->E * bpe), dim3(256), 0, s, (const bf16 *)x_perm, offsets,
-                                                    (const bf16 *)W13, p->d, p->m, bpe, (bf16 *)h);
+    const int grid = row_token ? max(p->E * bpe, p->T * p->k) : p->E * bpe;
+    launch_pdl(decode_up_kernel<NNT>, dim3(grid), dim3(256), 0, s, (const bf16 *)x_perm, offsets,
+               (const bf16 *)W13, p->d, p->m, bpe, (bf16 *)h, row_token, (bf16 *)x_perm_out,
+               p->E);
 }
 
 template <int NNT>
@@ -227,6 +251,18 @@ cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const in
         up_dispatch<1>(p, x_perm, offsets, W13, h, s);
     else
         up_dispatch<2>(p, x_perm, offsets, W13, h, s);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_up_decode_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                                    const int32_t *offsets, const void *W13, void *h,
+                                    void *x_perm_out, cudaStream_t s)
+{
+    if (p->T <= 8)
+        up_dispatch<1>(p, x, offsets, W13, h, s, row_token, x_perm_out);
+    else
+        up_dispatch<2>(p, x, offsets, W13, h, s, row_token, x_perm_out);
     count_launch();
     return cudaGetLastError();
 }

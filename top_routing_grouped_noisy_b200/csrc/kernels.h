@@ -114,6 +114,15 @@ cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const in
                              const void *W13, void *h, cudaStream_t s);
 cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32_t *offsets,
                                const void *W2, void *out, cudaStream_t s);
+// a3 reading rows of x through row_token, writing x_perm alongside (moe_forward)
+cudaError_t launch_up_decode_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
+                                    const int32_t *offsets, const void *W13, void *h,
+                                    void *x_perm_out, cudaStream_t s);
+// a1 finish + a2 + a6 for at most kDecodeMaxTokens tokens in one CTA, after the
+// split-K router slices (moe_forward); false when the batch does not qualify.
+bool small_forward_fits(const moe_params_t *p, bool noisy);
+cudaError_t launch_route_dispatch_small(const moe_params_t *p, const moe_buffers_t *b, char *ws,
+                                        int32_t *status, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
                            const float *w, void *y, cudaStream_t s);

@@ -142,6 +142,132 @@ __global__ void __launch_bounds__(256) router_small_finish_kernel(
                         probs_sum, importance, status, sm);
 }
 
+// ---------------------------------------------------------------- small-batch forward
+// For at most kDecodeMaxTokens tokens moe_forward finishes the split-K router,
+// builds the dispatch tables and computes the gate statistics in ONE CTA (three
+// launches fewer on a path that is bound by launch latency).  The arithmetic is
+// that of router_small_finish_kernel, dispatch_count/rank_kernel ("Llama 3 Meets
+// MoE", section 3 "容量因子": stable by token, assignments past the capacity
+// dropped) and gate_stats_kernel ("LLaMA-MoE v2", section "门控机制设计"), so
+// moe_forward gives the same bits as the step calls.  x_perm is written by the
+// GEMM 1 kernel, which reads the rows of x through row_token.
+__global__ void __launch_bounds__(256) route_dispatch_small_kernel(
+    const float *__restrict__ part, int T, int E, int k, int C, int noisy,
+    const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
+    float lambda, int32_t *__restrict__ idx, float *__restrict__ w_out,
+    float *__restrict__ probs_sum, float *__restrict__ importance, int32_t *__restrict__ counts,
+    int32_t *__restrict__ kept, int32_t *__restrict__ offsets, int32_t *__restrict__ row_token,
+    int32_t *__restrict__ slot_row, float *__restrict__ f, float *__restrict__ P,
+    float *__restrict__ loss, int32_t *status)
+{
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ float sm[];
+    __shared__ int32_t s_idx[kDecodeMaxTokens * MOE_MAX_TOPK];
+    __shared__ int32_t s_cnt[MOE_MAX_EXPERTS], s_kept[MOE_MAX_EXPERTS];
+    __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
+    __shared__ double s_fp[MOE_MAX_EXPERTS];
+    router_small_finish(part, T, E, k, noisy, noise, bias, router_type, idx, w_out, probs_sum,
+                        importance, status, sm);
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x)
+        s_idx[i] = idx[i];
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+        for (int i = 0; i < T * k; ++i)
+            c += s_idx[i] == e;
+        s_cnt[e] = c;
+        s_kept[e] = C < 0 ? c : min(c, C);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int e = 0; e < E; ++e) {
+            s_off[e] = acc;
+            acc += s_kept[e];
+        }
+        s_off[E] = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        counts[e] = s_cnt[e];
+        kept[e] = s_kept[e];
+    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x)
+        offsets[e] = s_off[e];
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+        const int t = i / k, e = s_idx[i];
+        int row = -1;
+        if (e < 0 || e >= E) {
+            set_status(status, MOE_ERR_DEVICE_BADINDEX);
+        } else {
+            int rank = 0;  // the expert's assignments of earlier tokens
+            for (int i2 = 0; i2 < t * k; ++i2)
+                rank += s_idx[i2] == e;
+            if (rank < s_kept[e]) {
+                row = s_off[e] + rank;
+                row_token[row] = t;
+            }
+        }
+        slot_row[i] = row;
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const double fe = (double)s_cnt[e] / ((double)T * k);
+        const double pe = (double)probs_sum[e] / (double)T;
+        f[e] = (float)fe;
+        P[e] = (float)pe;
+        s_fp[e] = fe * pe;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double sfp = 0.0;
+        for (int i = 0; i < E; ++i)
+            sfp += s_fp[i];
+        loss[0] = (float)(lambda * sfp);
+    }
+}
+
+static void small_router_smem(const moe_params_t *p, bool noisy, size_t *sm1, size_t *sm2)
+{
+    const int nout = noisy ? 2 * p->E : p->E;
+    const int kc = ceil_div(p->d, kRouterSmallSplit);
+    *sm1 = sizeof(float) * ((size_t)p->T * kc + (size_t)kc * nout);
+    *sm2 = sizeof(float) * ((size_t)p->T * nout + 2 * (size_t)p->T * p->E);
+}
+
+bool small_forward_fits(const moe_params_t *p, bool noisy)
+{
+    if (p->dtype != MOE_BF16 || p->T < 1 || p->T > kDecodeMaxTokens)
+        return false;
+    size_t sm1, sm2;
+    small_router_smem(p, noisy, &sm1, &sm2);
+    return sm1 <= 48 * 1024 && sm2 <= 48 * 1024;
+}
+
+cudaError_t launch_route_dispatch_small(const moe_params_t *p, const moe_buffers_t *b, char *ws,
+                                        int32_t *status, cudaStream_t s)
+{
+    const WsLayout L = ws_layout(p);
+    float *sp = reinterpret_cast<float *>(ws + L.rsmall);
+    const bool noisy = b->Wnoise != nullptr;
+    size_t sm1, sm2;
+    small_router_smem(p, noisy, &sm1, &sm2);
+    cudaError_t e = launch_pdl(router_small_partial_kernel<bf16>, dim3(kRouterSmallSplit),
+                               dim3(256), sm1, s, (const bf16 *)b->x, (const bf16 *)b->Wg,
+                               (const bf16 *)b->Wnoise, p->T, p->d, p->E, sp);
+    count_launch();
+    if (e != cudaSuccess)
+        return e;
+    e = launch_pdl(route_dispatch_small_kernel, dim3(1), dim3(256), sm2, s, (const float *)sp,
+                   p->T, p->E, p->k, p->capacity, noisy ? 1 : 0, b->noise, b->bias,
+                   p->router_type, p->balance_lambda, b->topk_idx, b->topk_w, b->probs_sum,
+                   b->importance, b->counts, b->kept, b->offsets, b->row_token, b->slot_row,
+                   b->f, b->P, b->loss, status);
+    count_launch();
+    return e;
+}
+
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
                          const void *Wnoise, const float *noise, const float *bias,
                          int32_t *idx, float *w, float *probs_sum, float *importance,
