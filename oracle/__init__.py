@@ -249,3 +249,40 @@ def forward(x, Wg, W1e, W3e, W2e, k, router_type=MIXTRAL, Wnoise=None, eps=None,
     y = combine(out_u, sr_local, r["G"][toks], scale)
     return dict(router=r, dispatch=dsp, f=f, P=P, L=L, tokens=toks, y=y, out_rows=out_u,
                 rows=uniq)
+
+
+# --------------------------------------------------------------------------- residual MoE
+# "LLaMA-MoE v2", section "共享神经元划分" (Shared Neuron Partitioning): the neurons of a
+# set S are shared by all experts, the rest are split into E equal disjoint experts.
+# The pages give no output formula; the layer is read as a residual block every token
+# passes through next to the routed experts:
+#     y = FFN_S(x) + s * sum_j G_j E_j(x)
+# (FFN_S the SwiGLU FFN on the neurons of S, unscaled, applied to dropped tokens too).
+
+def partition_residual(W1, W3, W2, E: int, shared_idx, perm_rest):
+    """a0 of the residual MoE: the shared block (W1, W3 rows and W2 columns of S) and
+    E disjoint experts over perm_rest (expert e gets perm_rest[e m, (e+1) m))."""
+    shared = np.asarray(shared_idx, np.int64)
+    rest = np.asarray(perm_rest, np.int64)
+    W1, W3, W2 = np.asarray(W1), np.asarray(W3), np.asarray(W2)
+    blk = (np.ascontiguousarray(W1[shared]), np.ascontiguousarray(W3[shared]),
+           np.ascontiguousarray(W2[:, shared]))
+    experts = partition(np.ascontiguousarray(W1[rest]), np.ascontiguousarray(W3[rest]),
+                        np.ascontiguousarray(W2[:, rest]), E, DISJOINT,
+                        np.arange(len(rest), dtype=np.int32))
+    return experts, blk
+
+
+def forward_residual(x, Wg, experts, shared_block, k, router_type=MIXTRAL, Wnoise=None,
+                     eps=None, bias=None, capacity_rows=-1, rescale=False, lam=0.0,
+                     tokens=None):
+    """The residual MoE layer: forward() over the routed experts plus FFN_S(x) for
+    every token evaluated.  Adds ``y_shared`` to the returned dict."""
+    r = forward(x, Wg, *experts, k, router_type, Wnoise, eps, bias, capacity_rows, rescale,
+                lam, tokens)
+    xs = np.ascontiguousarray(np.asarray(x)[r["tokens"]])
+    ys = dense_ffn(*shared_block, xs)
+    r["y_moe"] = r["y"]
+    r["y_shared"] = ys
+    r["y"] = r["y"] + ys
+    return r

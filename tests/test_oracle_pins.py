@@ -424,3 +424,61 @@ def test_forward_sample_equals_full(orc):
     part = orc.forward(x, Wg, W1e, W3e, W2e, k, capacity_rows=10, tokens=toks)
     np.testing.assert_array_equal(part["y"], full["y"][toks])
     assert full["dispatch"]["R"] < T * k  # some assignments dropped
+
+
+# --------------------------------------------------------------------------- residual MoE
+
+def _residual_split(seed, d_ff, m_s):
+    perm = _rng(seed).permutation(d_ff).astype(np.int32)
+    return perm[:m_s], perm[m_s:]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_residual_all_experts_selected_equal_dense(orc, dtype):
+    """Shared block plus every disjoint expert at gate weight 1 (no rescale) is the
+    dense FFN: S and the experts together regroup all intermediate neurons."""
+    T, d, d_ff, E, m_s = 9, 32, 72, 4, 8
+    x, W1, W3, W2, Wg, _ = _layer(21, T, d, d_ff, E, dtype)
+    shared, rest = _residual_split(22, d_ff, m_s)
+    (W1e, W3e, W2e), blk = orc.partition_residual(W1, W3, W2, E, shared, rest)
+    idx = np.tile(np.arange(E, dtype=np.int32), (T, 1))
+    dsp = orc.dispatch(idx, E, -1)
+    eor = np.searchsorted(dsp["offsets"], np.arange(dsp["R"]), side="right") - 1
+    out = orc.expert_ffn(W1e, W3e, W2e, x[dsp["row_token"]], eor)
+    y = orc.combine(out, dsp["slot_row"], np.ones((T, E)), 1.0) + orc.dense_ffn(*blk, x)
+    ref = _numpy_dense_ffn(W1, W3, W2, x)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-11 * np.abs(ref).max())
+
+
+def test_residual_capacity_zero_leaves_the_shared_block(orc):
+    """With capacity 0 every routed assignment is dropped: y is exactly the shared
+    block, the SwiGLU FFN restricted to the neurons of S (numpy)."""
+    T, d, d_ff, E, k, m_s = 10, 24, 40, 4, 2, 8
+    x, W1, W3, W2, Wg, _ = _layer(23, T, d, d_ff, E)
+    shared, rest = _residual_split(24, d_ff, m_s)
+    experts, blk = orc.partition_residual(W1, W3, W2, E, shared, rest)
+    r = orc.forward_residual(x, Wg, experts, blk, k, capacity_rows=0, rescale=True)
+    ref = _numpy_dense_ffn(W1[shared], W3[shared], W2[:, shared], x)
+    assert (r["dispatch"]["slot_row"] == -1).all()
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
+
+
+def test_residual_is_shared_block_plus_routed_layer(orc):
+    """The routed part of the residual layer is the plain MoE layer over the
+    non-shared neurons; E/k rescale applies to it and not to the shared block."""
+    T, d, d_ff, E, k, m_s = 12, 16, 56, 4, 2, 16
+    x, W1, W3, W2, Wg, _ = _layer(25, T, d, d_ff, E)
+    shared, rest = _residual_split(26, d_ff, m_s)
+    experts, blk = orc.partition_residual(W1, W3, W2, E, shared, rest)
+    r = orc.forward_residual(x, Wg, experts, blk, k, rescale=True)
+    # the routed experts rebuilt independently from the numpy weights
+    m = (d_ff - m_s) // E
+    y_moe = np.zeros((T, d))
+    G = r["router"]["G"]
+    for t in range(T):
+        for j in range(k):
+            e = int(r["router"]["idx"][t, j])
+            cols = rest[e * m:(e + 1) * m]
+            y_moe[t] += G[t, j] * _numpy_dense_ffn(W1[cols], W3[cols], W2[:, cols], x[t:t + 1])[0]
+    ref = _numpy_dense_ffn(W1[shared], W3[shared], W2[:, shared], x) + (E / k) * y_moe
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-10, atol=1e-11 * np.abs(ref).max())
