@@ -62,6 +62,7 @@ def config_of(w: wl.Workload, C: int):
         "router": "mixtral" if w.router == wl.MIXTRAL else "st", "noisy": w.noisy,
         "bias": w.bias, "rescale": w.rescale, "capacity": C, "cf": w.cf,
         "partition": "disjoint" if w.partition == wl.DISJOINT else "copy",
+        "shared_neurons": w.shared,
         "global_batch": w.T, "seq_len": 4096,
         "l2": "no flush: per-step working set (x, packed weights, intermediates) >> 126 MB L2",
     }
@@ -425,54 +426,69 @@ def main():
     elif w.partition == wl.COPY:
         W13_e, W2_e = moe.moe_partition_experts(inp["W1"], inp["W3"], inp["W2"], w.E, moe.COPY,
                                                 ws=ws)
+    elif w.shared > 0:  # residual MoE: shared block plus disjoint experts
+        W13_e, W2_e, W13_s, W2_s = moe.moe_partition_residual(
+            inp["W1"], inp["W3"], inp["W2"], w.E, inp["shared_idx"], inp["perm_rest"], ws=ws)
     else:
         W13_e, W2_e = moe.moe_partition_experts(inp["W1"], inp["W3"], inp["W2"], w.E,
                                                 moe.DISJOINT, perm=inp["perm"], ws=ws)
+    res = w.shared > 0
+    if res:
+        ps = moe.params(w.T, w.d, 1, 1, w.shared, dt, w.router, -1, w.rescale, w.lam)
+        tok_range = torch.tensor([0, w.T], dtype=torch.int32, device="cuda")
+        h_s = torch.empty(w.T, moe.h_ld(w.shared), dtype=dt, device="cuda")
+        out_s = torch.empty(w.T, w.d, dtype=dt, device="cuda")
     b = moe.ForwardBuffers(p)
     x, Wg, Wn, eps, bias = inp["x"], inp["Wg"], inp["Wnoise"], inp["eps"], inp["bias"]
     stream = torch.cuda.current_stream()
     # moe_forward's path: the dispatch materialises x_perm (the row-gathering GEMM 1
     # variant, moe_expert_up_gather, is slower on B200)
     gather = False
-    NSEG = 6
-    SEG = ["route", "dispatch", "expert_up", "expert_down", "combine", "gate_stats"]
+    SEG = ["route", "dispatch", "expert_up", "expert_down"] + (["shared"] if res else []) + \
+        ["combine", "gate_stats"]
+    NSEG = len(SEG)
 
     def step(ev=None, up_only=None):
-        # ev: events between all six steps; up_only: a (start, end) pair around
-        # expert GEMM 1 alone (the roofline kernel), for the timed loop
-        if ev is not None:
-            ev[0].record(stream)
+        # ev: events between all steps; up_only: a (start, end) pair around expert
+        # GEMM 1 alone (the roofline kernel), for the timed loop
+        seg = iter(range(NSEG + 1))
+
+        def mark():
+            i = next(seg)
+            if ev is not None:
+                ev[i].record(stream)
+
+        mark()
         moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b.topk_idx, b.topk_w, b.probs_sum,
                       b.importance)
-        if ev is not None:
-            ev[1].record(stream)
+        mark()
         if gather:
             moe.moe_dispatch_rows(p, b.topk_idx, ws, b.row_token, b.slot_row, b.counts, b.kept,
                                   b.offsets)
         else:
             moe.moe_dispatch(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
                              b.kept, b.offsets)
-        if ev is not None:
-            ev[2].record(stream)
+        mark()
         if up_only is not None:
             up_only[0].record(stream)
         if gather:
             moe.moe_expert_up_gather(p, x, b.row_token, b.offsets, W13_e, b.h, ws)
         else:
             moe.moe_expert_up(p, b.x_perm, b.offsets, W13_e, b.h, ws)
-        if ev is not None:
-            ev[3].record(stream)
         if up_only is not None:
             up_only[1].record(stream)
+        mark()
         moe.moe_expert_down(p, b.h, b.offsets, W2_e, b.out, ws)
-        if ev is not None:
-            ev[4].record(stream)
-        moe.moe_combine(p, b.out, b.slot_row, b.topk_w, b.y)
-        if ev is not None:
-            ev[5].record(stream)
+        mark()
+        if res:  # the shared block: one expert over every token
+            moe.moe_expert_ffn(ps, x, tok_range, W13_s, W2_s, h_s, out_s, ws)
+            mark()
+            moe.moe_combine_residual(p, b.out, b.slot_row, b.topk_w, out_s, b.y)
+        else:
+            moe.moe_combine(p, b.out, b.slot_row, b.topk_w, b.y)
+        mark()
         moe.moe_gate_stats(p, b.counts, b.probs_sum, b.f, b.P, b.loss)
-        if ev is not None:
-            ev[6].record(stream)
+        mark()
 
     if w.T <= 64:
         return run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank,
@@ -530,7 +546,7 @@ def main():
     ms = max_over_ranks(ms_local, world)
     seg_ms = np.array([max_over_ranks(v, world) for v in seg_ms])
     value = tokens_per_s(w.T, args.steps, world, ms)
-    flop_step = 6.0 * w.d * w.m * R
+    flop_step = 6.0 * w.d * w.m * R + (6.0 * w.d * w.shared * w.T if res else 0.0)
     tflops = flop_step * args.steps * world / (ms / 1000.0) / 1e12
 
     # roofline of the dominant kernel (expert GEMM 1 + SwiGLU), timed inside the step loop
@@ -559,6 +575,7 @@ def main():
     route_bytes = w.T * w.d * es + (w.T * w.E * 4 if eps is not None else 0) + w.T * w.k * 8
     disp_bytes = (w.T * w.k * 12 if gather else w.T * w.d * es + R * w.d * es + w.T * w.k * 12)
     comb_bytes = R * w.d * es + w.T * w.d * es + w.T * w.k * 8
+    sm = dict(zip(SEG, seg_ms))
     kernels = {
         "route": {"ms": seg_ms[0], "bound": "hbm", "GB/s": route_bytes / seg_ms[0] / 1e6,
                   "frac": route_bytes / seg_ms[0] / 1e6 / hbm},
@@ -573,16 +590,26 @@ def main():
         "expert_down": {"ms": seg_ms[3], "bound": "tensor",
                         "TFLOP/s": down_flop / (seg_ms[3] / 1000.0) / 1e12,
                         "frac": down_flop / (seg_ms[3] / 1000.0) / 1e12 / peak_t},
-        "combine": {"ms": seg_ms[4], "bound": "hbm", "GB/s": comb_bytes / seg_ms[4] / 1e6,
-                    "frac": comb_bytes / seg_ms[4] / 1e6 / hbm},
-        "gate_stats": {"ms": seg_ms[5]},
+        "combine": {"ms": sm["combine"], "bound": "hbm",
+                    "GB/s": comb_bytes / sm["combine"] / 1e6,
+                    "frac": comb_bytes / sm["combine"] / 1e6 / hbm},
+        "gate_stats": {"ms": sm["gate_stats"]},
     }
+    if res:
+        sh_flop = 6.0 * w.d * w.shared * w.T
+        kernels["shared"] = {"ms": sm["shared"], "bound": "tensor",
+                             "TFLOP/s": sh_flop / (sm["shared"] / 1000.0) / 1e12,
+                             "frac": sh_flop / (sm["shared"] / 1000.0) / 1e12 / peak_t,
+                             "what": "shared block FFN_S: GEMM 1 + SwiGLU and GEMM 2 over all "
+                                     "%d tokens, %d shared neurons" % (w.T, w.shared)}
 
-    e2e = None if args.no_e2e else e2e_pipeline(args, w, p, moe, x, Wg, Wn, eps, bias, W13_e,
-                                                W2_e, world)
+    # the host pipeline runs moe_forward (no shared block): no end-to-end figure for
+    # a residual layer
+    e2e = None if (args.no_e2e or res) else e2e_pipeline(args, w, p, moe, x, Wg, Wn, eps, bias,
+                                                          W13_e, W2_e, world)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not res:
         inp_cpu = {k2: (v.cpu() if isinstance(v, torch.Tensor) else v) for k2, v in inp.items()}
         cpu = time_oracle(w, inp_cpu, C)
 

@@ -275,6 +275,45 @@ typedef struct {
 int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t ws_bytes,
                 void *stream);
 
+/* ---- residual MoE: shared neurons plus disjoint experts ------------------
+ * "LLaMA-MoE v2", section "共享神经元划分" (Shared Neuron Partitioning): a set S
+ * of the dense FFN's intermediate neurons is shared by all experts and the
+ * remaining neurons are split into E equal disjoint experts; the hub page "从大炼
+ * 到巧炼" lists the residual MoE module that holds it.  The pages give no output
+ * formula; the layer computed here is the plain reading of a residual block that
+ * every token passes through next to the routed experts:
+ *     y_t = FFN_S(x_t) + s * sum_j G_tj E_{idx_tj}(x_t)
+ * with FFN_S the SwiGLU FFN restricted to the neurons of S (not scaled by s,
+ * applied to dropped tokens too) and E_e the experts over the other neurons.
+ * Choosing S (importance scores from gradients) is out of scope: the caller
+ * supplies it. */
+
+/* a0 for the residual MoE.  shared_idx [m_s] (device int32): the neurons of S;
+ * perm_rest [d_ff - m_s] (device int32): the other neurons in expert order
+ * (expert e gets perm_rest[e m, (e+1) m), m = (d_ff - m_s) / E).  Outputs the
+ * packed experts W13_e / W2_e (E experts of width m) and the packed shared
+ * block W13_s / W2_s (one "expert" of width m_s), layouts as above.  Entries
+ * outside [0, d_ff) write zero neurons and set MOE_ERR_DEVICE_BADINDEX in ws.
+ * Errors: MOE_ERR_SHAPE unless 1 <= m_s < d_ff and E divides d_ff - m_s. */
+int moe_partition_residual(const void *W1, const void *W3, const void *W2, int32_t d,
+                           int32_t d_ff, int32_t E, const int32_t *shared_idx, int32_t m_s,
+                           const int32_t *perm_rest, int32_t dtype, void *W13_e, void *W2_e,
+                           void *W13_s, void *W2_s, void *ws, void *stream);
+
+/* a5 with the residual term: y[t] = s * sum_j topk_w[t][j] out[slot_row[t][j]]
+ * + resid[t] (the scaled sum in slot order in f32, then resid added, rounded
+ * once).  resid [T][d] in dtype. */
+int moe_combine_residual(const moe_params_t *p, const void *out, const int32_t *slot_row,
+                         const float *topk_w, const void *resid, void *y, void *stream);
+
+/* The residual MoE layer: a1, a2, a3, a4 for the routed experts (p->m = their
+ * width), then the shared block FFN_S over all T tokens as a one-expert grouped
+ * GEMM (h_s [T][m_s8], out_s [T][d], caller-owned; out_s = FFN_S(x)), then
+ * moe_combine_residual and a6.  The workspace must be sized for p. */
+int moe_forward_residual(const moe_params_t *p, const moe_buffers_t *b, const void *W13_s,
+                         const void *W2_s, int32_t m_s, void *h_s, void *out_s, void *ws,
+                         size_t ws_bytes, void *stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
  * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
  * the workspace's internal launch counters. */

@@ -19,7 +19,8 @@ __all__ = [
     "moe_dispatch_noalloc", "moe_dispatch_rows", "moe_expert_up_gather",
     "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
-    "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline",
+    "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline", "moe_partition_residual",
+    "moe_combine_residual", "moe_forward_residual",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -103,6 +104,11 @@ def lib():
             "moe_gate_stats": (C.c_int, [P, v, v, v, v, v, v]),
             "moe_forward": (C.c_int, [P, C.POINTER(_Buffers), v, sz, v]),
             "moe_get_device_status": (C.c_int, [v, C.POINTER(i32), i32, v]),
+            "moe_partition_residual": (C.c_int, [v, v, v, i32, i32, i32, v, i32, v, i32, v, v,
+                                                 v, v, v, v]),
+            "moe_combine_residual": (C.c_int, [P, v, v, v, v, v, v]),
+            "moe_forward_residual": (C.c_int, [P, C.POINTER(_Buffers), v, v, i32, v, v, v, sz,
+                                               v]),
             "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
             "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
             "moe_pipeline_wait": (C.c_int, [v, i64]),
@@ -321,6 +327,41 @@ def moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs: ForwardBuffers, Wnoise=None, no
         t = vals[n] if n in vals else getattr(bufs, n)
         setattr(b, n, _p(t))
     _check(lib().moe_forward(C.byref(p), C.byref(b), ws.ptr, ws.nbytes, _stream(stream)))
+    return bufs
+
+
+def moe_partition_residual(W1, W3, W2, E, shared_idx, perm_rest, ws=None, stream=None):
+    """a0 of the residual MoE: E disjoint experts over perm_rest and the shared block
+    over shared_idx; returns (W13_e, W2_e, W13_s, W2_s) (include/moe.h)."""
+    dt = _dtype_code(W1.dtype)
+    d_ff, d = W1.shape
+    m_s = shared_idx.numel()
+    m = (d_ff - m_s) // E
+    mk = lambda n: torch.empty(n, dtype=W1.dtype, device=W1.device)
+    W13_e, W2_e = mk(packed_w13_elems(E, m, d)), mk(packed_w2_elems(E, m, d))
+    W13_s, W2_s = mk(packed_w13_elems(1, m_s, d)), mk(packed_w2_elems(1, m_s, d))
+    _check(lib().moe_partition_residual(_p(W1), _p(W3), _p(W2), d, d_ff, E, _p(shared_idx), m_s,
+                                        _p(perm_rest), dt, _p(W13_e), _p(W2_e), _p(W13_s),
+                                        _p(W2_s), ws.ptr if ws is not None else None,
+                                        _stream(stream)))
+    return W13_e, W2_e, W13_s, W2_s
+
+
+def moe_combine_residual(p, out, slot_row, topk_w, resid, y, stream=None):
+    _check(lib().moe_combine_residual(C.byref(p), _p(out), _p(slot_row), _p(topk_w), _p(resid),
+                                      _p(y), _stream(stream)))
+
+
+def moe_forward_residual(p, x, Wg, W13_e, W2_e, W13_s, W2_s, m_s, ws, bufs: ForwardBuffers, h_s,
+                         out_s, Wnoise=None, noise=None, bias=None, stream=None):
+    """The residual MoE layer: routed experts plus the shared block (include/moe.h)."""
+    b = _Buffers()
+    vals = dict(x=x, Wg=Wg, Wnoise=Wnoise, noise=noise, bias=bias, W13_e=W13_e, W2_e=W2_e)
+    for n in _BUF_FIELDS:
+        t = vals[n] if n in vals else getattr(bufs, n)
+        setattr(b, n, _p(t))
+    _check(lib().moe_forward_residual(C.byref(p), C.byref(b), _p(W13_s), _p(W2_s), int(m_s),
+                                      _p(h_s), _p(out_s), ws.ptr, ws.nbytes, _stream(stream)))
     return bufs
 
 

@@ -520,4 +520,118 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
     return moe_gate_stats(p, b->counts, b->probs_sum, b->f, b->P, b->loss, stream);
 }
 
+// ---------------------------------------------------------------- residual MoE
+
+int moe_partition_residual(const void *W1, const void *W3, const void *W2, int32_t d,
+                           int32_t d_ff, int32_t E, const int32_t *shared_idx, int32_t m_s,
+                           const int32_t *perm_rest, int32_t dtype, void *W13_e, void *W2_e,
+                           void *W13_s, void *W2_s, void *ws, void *stream)
+{
+    const char *fn = "moe_partition_residual";
+    REQUIRE_PTR(W1);
+    REQUIRE_PTR(W3);
+    REQUIRE_PTR(W2);
+    REQUIRE_PTR(shared_idx);
+    REQUIRE_PTR(perm_rest);
+    REQUIRE_PTR(W13_e);
+    REQUIRE_PTR(W2_e);
+    REQUIRE_PTR(W13_s);
+    REQUIRE_PTR(W2_s);
+    OPTIONAL_PTR(ws);
+    if (dtype != MOE_BF16 && dtype != MOE_F32)
+        return fail(MOE_ERR_DTYPE, "%s: dtype=%d", fn, dtype);
+    if (E < 1 || E > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_INVALID_ARG, "%s: E=%d outside [1,%d]", fn, E, MOE_MAX_EXPERTS);
+    if (d < 8 || d % 8 != 0)
+        return fail(MOE_ERR_SHAPE, "%s: d=%d is not a positive multiple of 8", fn, d);
+    if (d_ff < 2 || d_ff > (1 << 22))
+        return fail(MOE_ERR_SHAPE, "%s: d_ff=%d", fn, d_ff);
+    if (m_s < 1 || m_s >= d_ff || (d_ff - m_s) % E != 0)
+        return fail(MOE_ERR_SHAPE,
+                    "%s: need 1 <= m_s < d_ff and (d_ff - m_s) divisible by E (m_s=%d, d_ff=%d, "
+                    "E=%d)",
+                    fn, m_s, d_ff, E);
+    const int m = (d_ff - m_s) / E;
+    int32_t *status = reinterpret_cast<int32_t *>(ws);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_partition(W1, W3, W2, d, d_ff, E, m, MOE_PARTITION_DISJOINT, perm_rest,
+                                     dtype, W13_e, W2_e, status, s);
+    if (e == cudaSuccess)
+        e = launch_partition(W1, W3, W2, d, d_ff, 1, m_s, MOE_PARTITION_DISJOINT, shared_idx,
+                             dtype, W13_s, W2_s, status, s);
+    return after_launch(fn, e);
+}
+
+int moe_combine_residual(const moe_params_t *p, const void *out, const int32_t *slot_row,
+                         const float *topk_w, const void *resid, void *y, void *stream)
+{
+    const char *fn = "moe_combine_residual";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    REQUIRE_TOK(out);
+    REQUIRE_TOK(slot_row);
+    REQUIRE_TOK(topk_w);
+    REQUIRE_TOK(resid);
+    REQUIRE_TOK(y);
+    if (p->T == 0)
+        return ok();
+    cudaError_t e = launch_combine(p, out, slot_row, topk_w, y, (cudaStream_t)stream, resid);
+    return after_launch(fn, e);
+}
+
+int moe_forward_residual(const moe_params_t *p, const moe_buffers_t *b, const void *W13_s,
+                         const void *W2_s, int32_t m_s, void *h_s, void *out_s, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_forward_residual";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    if (b == nullptr)
+        return fail(MOE_ERR_INVALID_ARG, "%s: buffers is NULL", fn);
+    if (m_s < 1 || m_s > 1 << 20)
+        return fail(MOE_ERR_SHAPE, "%s: m_s=%d", fn, m_s);
+    REQUIRE_PTR(W13_s);
+    REQUIRE_PTR(W2_s);
+    REQUIRE_TOK(h_s);
+    REQUIRE_TOK(out_s);
+    REQUIRE_TOK(b->y);
+    REQUIRE_PTR(b->loss);
+    REQUIRE_PTR(b->f);
+    REQUIRE_PTR(b->P);
+    if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+        return rc;
+    // the shared block: one expert of width m_s that every token goes to
+    moe_params_t ps = *p;
+    ps.E = 1;
+    ps.k = 1;
+    ps.m = m_s;
+    ps.capacity = -1;
+    if ((rc = check_params(fn, &ps)) != MOE_OK || (rc = check_ws(fn, &ps, ws, ws_bytes)) != MOE_OK)
+        return rc;
+    if ((rc = moe_route(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx, b->topk_w,
+                        b->probs_sum, b->importance, ws, ws_bytes, stream)) != MOE_OK)
+        return rc;
+    if ((rc = moe_dispatch(p, b->x, b->topk_idx, b->x_perm, b->row_token, b->slot_row,
+                           b->counts, b->kept, b->offsets, ws, ws_bytes, stream)) != MOE_OK)
+        return rc;
+    if ((rc = moe_expert_ffn(p, b->x_perm, b->offsets, b->W13_e, b->W2_e, b->h, b->out, ws,
+                             ws_bytes, stream)) != MOE_OK)
+        return rc;
+    if (p->T > 0) {
+        int32_t *range = reinterpret_cast<int32_t *>(ws) + kWsTokenRangeWord;
+        cudaError_t e = launch_token_range(range, p->T, (cudaStream_t)stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, fn);
+        if ((rc = moe_expert_ffn(&ps, b->x, range, W13_s, W2_s, h_s, out_s, ws, ws_bytes,
+                                 stream)) != MOE_OK)
+            return rc;
+    }
+    if ((rc = moe_combine_residual(p, b->out, b->slot_row, b->topk_w, out_s, b->y, stream)) !=
+        MOE_OK)
+        return rc;
+    return moe_gate_stats(p, b->counts, b->probs_sum, b->f, b->P, b->loss, stream);
+}
+
 }  // extern "C"

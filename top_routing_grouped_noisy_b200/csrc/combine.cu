@@ -17,11 +17,14 @@ namespace moe {
 // slot rows of all of them are requested before any is used.
 constexpr int kCombineVPT = 2;
 
+// resid (may be NULL): a dense [T][d] term added after the scaled sum (the shared
+// block of a residual MoE: y = s sum_j G_j out_j + resid).
 template <typename E_T, int KMAX>
 __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ out,
                                                       const int32_t *__restrict__ slot_row,
                                                       const float *__restrict__ w, int T, int d,
-                                                      int k, float scale, E_T *__restrict__ y)
+                                                      int k, float scale, E_T *__restrict__ y,
+                                                      const E_T *__restrict__ resid)
 {
     pdl_wait();
     pdl_trigger();
@@ -76,6 +79,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const E_T *__restrict__ ou
 #pragma unroll
             for (int q = 0; q < VN; ++q)
                 acc[q] *= scale;
+            if (resid != nullptr) {
+                const uint4 rv = ld_nc_na(resid + t * d + (int64_t)(v0 + u) * VN);
+                float rf[VN];
+                if constexpr (sizeof(E_T) == 2) {
+                    bf16x8_to_f32(rv, rf);
+                } else {
+                    rf[0] = __uint_as_float(rv.x);
+                    rf[1] = __uint_as_float(rv.y);
+                    rf[2] = __uint_as_float(rv.z);
+                    rf[3] = __uint_as_float(rv.w);
+                }
+#pragma unroll
+                for (int q = 0; q < VN; ++q)
+                    acc[q] += rf[q];
+            }
             uint4 o;
             if constexpr (sizeof(E_T) == 2) {
                 o = f32x8_to_bf16(acc);
@@ -114,7 +132,7 @@ __global__ void gate_stats_kernel(const int32_t *__restrict__ counts,
 }
 
 cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
-                           const float *w, void *y, cudaStream_t s)
+                           const float *w, void *y, cudaStream_t s, const void *resid)
 {
     const float scale = p->rescale ? (float)p->E / (float)p->k : 1.0f;
     const int VN = p->dtype == MOE_BF16 ? 8 : 4;
@@ -125,10 +143,12 @@ cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t
     do {                                                                                       \
         if (p->dtype == MOE_BF16)                                                              \
             launch_pdl(combine_kernel<bf16, KM>, dim3(grid), dim3(256), 0, s, (const bf16 *)out, slot_row, w, p->T, \
-                                                          p->d, p->k, scale, (bf16 *)y);       \
+                                                          p->d, p->k, scale, (bf16 *)y,        \
+                       (const bf16 *)resid);                                                   \
         else                                                                                   \
             launch_pdl(combine_kernel<float, KM>, dim3(grid), dim3(256), 0, s, (const float *)out, slot_row, w,     \
-                                                           p->T, p->d, p->k, scale, (float *)y); \
+                                                           p->T, p->d, p->k, scale, (float *)y, \
+                       (const float *)resid);                                                  \
     } while (0)
     if (p->k <= 2)
         MOE_COMBINE(2);
@@ -137,6 +157,23 @@ cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t
     else
         MOE_COMBINE(8);
 #undef MOE_COMBINE
+    count_launch();
+    return cudaGetLastError();
+}
+
+__global__ void token_range_kernel(int32_t *offsets2, int T)
+{
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x == 0) {
+        offsets2[0] = 0;
+        offsets2[1] = T;
+    }
+}
+
+cudaError_t launch_token_range(int32_t *offsets2, int T, cudaStream_t s)
+{
+    launch_pdl(token_range_kernel, dim3(1), dim3(32), 0, s, offsets2, T);
     count_launch();
     return cudaGetLastError();
 }

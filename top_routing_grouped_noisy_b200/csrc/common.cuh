@@ -25,6 +25,8 @@ constexpr int kWsCounterWord = 1;
 constexpr int kWsRouterCounterWord = 2;
 // Header bytes that clearing the status resets (status word and counters).
 constexpr size_t kWsResetBytes = 32;
+// Words 8-9: offsets {0, T} of the shared block's one-expert GEMMs (residual MoE).
+constexpr int kWsTokenRangeWord = 8;
 
 // Programmatic dependent launch.  Every kernel of the library is launched with
 // programmatic stream serialization allowed (launch_pdl): it may be scheduled

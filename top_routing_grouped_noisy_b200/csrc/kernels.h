@@ -125,7 +125,9 @@ cudaError_t launch_route_dispatch_small(const moe_params_t *p, const moe_buffers
                                         int32_t *status, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
-                           const float *w, void *y, cudaStream_t s);
+                           const float *w, void *y, cudaStream_t s, const void *resid = nullptr);
+// offsets {0, T} of a one-expert grouped GEMM over all tokens (the shared block)
+cudaError_t launch_token_range(int32_t *offsets2, int T, cudaStream_t s);
 
 cudaError_t launch_gate_stats(const moe_params_t *p, const int32_t *counts,
                               const float *probs_sum, float *f, float *P, float *loss,

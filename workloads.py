@@ -14,6 +14,10 @@ Workloads (shapes of the models on the pages; data is synthetic):
   e8t2_cf1/_cf4   T=32768, d=4096, 8 copies of d_ff=14336 (+ N(0,1e-3) per expert), top-2
                   Mixtral, capacity factor 1 or 4 with overflow dropping
   decode_t{1,8,64} T in {1,8,64}, d=4096, 8 x 1376, top-2, no noise, rescale E/k
+  moe_res_2of8    residual MoE: T=16384, d=4096, d_ff=11008 -> 1376 shared neurons +
+                  8 x 1204 experts, noisy top-2 Mixtral, rescale E/k
+With ``shared`` > 0 (residual MoE) the seeded permutation also chooses the shared
+neurons: perm[:shared] is the shared set, perm[shared:] the experts' neurons in order.
 """
 from dataclasses import dataclass, replace
 from typing import Optional
@@ -45,10 +49,13 @@ class Workload:
     partition: int = DISJOINT    # DISJOINT, or COPY (upcycling)
     perturb: float = 0.0         # std of the per-expert perturbation of copies
     seed: int = 1000
+    shared: int = 0              # > 0: residual MoE with this many shared neurons
 
     @property
     def m(self) -> int:
-        return self.d_ff // self.E if self.partition == DISJOINT else self.d_ff
+        if self.partition != DISJOINT:
+            return self.d_ff
+        return (self.d_ff - self.shared) // self.E
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -71,6 +78,8 @@ WORKLOADS = {
                           seed=1004),
     "decode_t64": Workload("decode_t64", T=64, d=4096, d_ff=11008, E=8, k=2, rescale=True,
                            seed=1004),
+    "moe_res_2of8": Workload("moe_res_2of8", T=16384, d=4096, d_ff=11008, E=8, k=2, noisy=True,
+                             rescale=True, shared=1376, seed=1005),
 }
 
 
@@ -108,6 +117,9 @@ def make_inputs(w: Workload, device: str = "cpu", seed: Optional[int] = None):
     out["bias"] = randn(w.E) if w.bias else None
     if w.partition == DISJOINT:
         out["perm"] = torch.randperm(w.d_ff, generator=g, device=device).to(torch.int32)
+        if w.shared > 0:  # residual MoE: the permutation's head is the shared set
+            out["shared_idx"] = out["perm"][:w.shared].contiguous()
+            out["perm_rest"] = out["perm"][w.shared:].contiguous()
     else:
         out["perm"] = None
     if w.partition == COPY and w.perturb > 0:
