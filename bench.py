@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes of one a3 launch (expert GEMM 1 + SwiGLU) from an ncu capture, keyed by
 # the source it was taken on; reported as null once the kernel source changes.
-NCU_TRAFFIC = {"src": "1de7c203599a0b20", "workload": "moe_2of8",
-               "bytes_per_launch": 609.73e6 + 119.16e6}
+NCU_TRAFFIC = {"src": "96ed2dffb627d991", "workload": "moe_2of8",
+               "bytes_per_launch": 589.66e6 + 110.52e6}
 
 
 def _src_hash(rel):
