@@ -45,6 +45,7 @@ def lib():
         _lib.oracle_combine.argtypes = [i, i, i, p, p, p, d, p]
         _lib.oracle_gate_stats.argtypes = [i, i, i, p, p, d, p, p, p]
         _lib.oracle_balance_sketch.argtypes = [i, i, i, p, p, p, p]
+        _lib.oracle_cluster.argtypes = [p, i, i, i, i, i, p, p, p, p]
     return _lib
 
 
@@ -286,3 +287,19 @@ def forward_residual(x, Wg, experts, shared_block, k, router_type=MIXTRAL, Wnois
     r["y_shared"] = ys
     r["y"] = r["y"] + ys
     return r
+
+
+def cluster(F, E: int, n_iter: int, init):
+    """f4: balanced k-means partition of the rows of F [d_ff][d] into E clusters
+    of d_ff/E neurons.  Returns (assign [d_ff] int32, centers [E][d] float64,
+    perm [d_ff] int32)."""
+    F = _c(F)
+    dt = _dt(F)
+    d_ff, d = F.shape
+    ini = _c(np.asarray(init), np.int32)
+    assign = np.empty(d_ff, np.int32)
+    centers = np.empty((E, d), np.float64)
+    perm = np.empty(d_ff, np.int32)
+    _check(lib().oracle_cluster(_ptr(F), dt, d, d_ff, E, n_iter, _ptr(ini), _ptr(assign),
+                                _ptr(centers), _ptr(perm)), "cluster")
+    return assign, centers, perm

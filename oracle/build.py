@@ -1,10 +1,11 @@
 """Builds the CPU oracle (``oracle/liboracle.so``) with gcc.
 
 The oracle is test infrastructure: only the tests, the package smoke check and
-the benchmark's CPU-baseline leg load it.  Built with -O2, no fast-math (so the
-double arithmetic is the plain IEEE arithmetic the formulas ask for), with
-OpenMP so loops over independent tokens/rows may use several host cores; the
-per-row arithmetic does not depend on the thread count.
+the benchmark's CPU-baseline leg load it.  Built with -O2, no fast-math and no
+floating-point contraction (so the double arithmetic is the plain IEEE
+arithmetic the formulas ask for, one rounding per operation), with OpenMP so
+loops over independent tokens/rows may use several host cores; the per-row
+arithmetic does not depend on the thread count.
 """
 import os
 import subprocess
@@ -20,7 +21,7 @@ def build(force: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-           "-fno-fast-math", "-Wall", "-o", tmp, SRC, "-lm"]
+           "-fno-fast-math", "-ffp-contract=off", "-Wall", "-o", tmp, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -496,3 +496,129 @@ int oracle_balance_sketch(int T, int E, int k, const int32_t *idx, const double 
     free(w);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* f4. Clustering partition [V2 "专家构建方法", IndependentClustering: k-means
+ * over the neurons' weight vectors, the neurons of one cluster form one expert;
+ * the subsets are of equal size m = d_ff / E].
+ *
+ * Readings (the page names k-means and equal sizes, nothing more):
+ *  - the feature of neuron i is row i of F [d_ff][d] (the caller passes W1);
+ *  - the E initial centers are the features of E distinct caller-chosen neurons;
+ *  - one iteration = assignment step, then center step;
+ *  - distance D[i][e] = sum over c of (F[i][c] - C[e][c])^2, summed in
+ *    ascending c, each difference, square and sum rounded (no fused multiply-add);
+ *  - the assignment step keeps every cluster at m neurons: in rounds, every
+ *    unassigned neuron proposes to its nearest cluster that is not full (ties
+ *    to the lower cluster index); a cluster with room r accepts its r proposals
+ *    of smallest (D, neuron index) and its acceptances are final; repeat until
+ *    every neuron is placed (at most E rounds: a round either places every
+ *    proposer or fills a cluster);
+ *  - the center step sets C[e] to the mean of its m members' features, summed in
+ *    ascending neuron index, then divided by m.
+ * Outputs after n_iter iterations: assign[i] (cluster of neuron i in the last
+ * assignment), centers [E][d] (after the last center step, so the means of
+ * that assignment), perm [d_ff] (cluster 0's neurons ascending, then cluster
+ * 1's, ...: the permutation a0 takes). */
+static const double *orc_sort_keys;
+
+static int orc_cmp_key(const void *a, const void *b)
+{
+    int i = *(const int32_t *)a, j = *(const int32_t *)b;
+    double di = orc_sort_keys[i], dj = orc_sort_keys[j];
+    if (di < dj)
+        return -1;
+    if (di > dj)
+        return 1;
+    return (i > j) - (i < j);
+}
+
+int oracle_cluster(const void *F, int dt, int d, int d_ff, int E, int n_iter,
+                   const int32_t *init, int32_t *assign, double *centers, int32_t *perm)
+{
+    if (d <= 0 || d_ff <= 0 || E <= 0 || n_iter < 1 || d_ff % E != 0)
+        return ORC_EINVAL;
+    const int m = d_ff / E;
+    for (int e = 0; e < E; ++e) {
+        if (init[e] < 0 || init[e] >= d_ff)
+            return ORC_EINVAL;
+        for (int f = 0; f < e; ++f)
+            if (init[f] == init[e])
+                return ORC_EINVAL;
+    }
+    double *D = (double *)malloc((size_t)d_ff * E * sizeof(double));
+    double *key = (double *)malloc((size_t)d_ff * sizeof(double));
+    int32_t *target = (int32_t *)malloc((size_t)d_ff * sizeof(int32_t));
+    int32_t *cand = (int32_t *)malloc((size_t)d_ff * sizeof(int32_t));
+    int *fill = (int *)malloc((size_t)E * sizeof(int));
+    if (!D || !key || !target || !cand || !fill) {
+        free(D), free(key), free(target), free(cand), free(fill);
+        return ORC_EINVAL;
+    }
+    for (int e = 0; e < E; ++e)
+        for (int c = 0; c < d; ++c)
+            centers[(size_t)e * d + c] = orc_load(F, dt, (size_t)init[e] * d + c);
+
+    for (int it = 0; it < n_iter; ++it) {
+        /* distances */
+#pragma omp parallel for schedule(static)
+        for (int i = 0; i < d_ff; ++i)
+            for (int e = 0; e < E; ++e) {
+                double s = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    double diff = orc_load(F, dt, (size_t)i * d + c) - centers[(size_t)e * d + c];
+                    double sq = diff * diff;
+                    s = s + sq;
+                }
+                D[(size_t)i * E + e] = s;
+            }
+        /* balanced assignment in rounds */
+        for (int i = 0; i < d_ff; ++i)
+            assign[i] = -1;
+        for (int e = 0; e < E; ++e)
+            fill[e] = 0;
+        int left = d_ff;
+        while (left > 0) {
+            for (int i = 0; i < d_ff; ++i) {
+                target[i] = -1;
+                if (assign[i] >= 0)
+                    continue;
+                for (int e = 0; e < E; ++e)
+                    if (fill[e] < m && (target[i] < 0 || D[(size_t)i * E + e] < D[(size_t)i * E + target[i]]))
+                        target[i] = e;
+            }
+            for (int e = 0; e < E; ++e) {
+                int n = 0;
+                for (int i = 0; i < d_ff; ++i)
+                    if (target[i] == e) {
+                        cand[n++] = i;
+                        key[i] = D[(size_t)i * E + e];
+                    }
+                orc_sort_keys = key;
+                qsort(cand, (size_t)n, sizeof(int32_t), orc_cmp_key);
+                int room = m - fill[e];
+                for (int r = 0; r < n && r < room; ++r) {
+                    assign[cand[r]] = e;
+                    fill[e] += 1;
+                    left -= 1;
+                }
+            }
+        }
+        /* centers: mean of the members, ascending neuron index */
+        for (int e = 0; e < E; ++e)
+            for (int c = 0; c < d; ++c) {
+                double s = 0.0;
+                for (int i = 0; i < d_ff; ++i)
+                    if (assign[i] == e)
+                        s = s + orc_load(F, dt, (size_t)i * d + c);
+                centers[(size_t)e * d + c] = s / (double)m;
+            }
+    }
+    int pos = 0;
+    for (int e = 0; e < E; ++e)
+        for (int i = 0; i < d_ff; ++i)
+            if (assign[i] == e)
+                perm[pos++] = i;
+    free(D), free(key), free(target), free(cand), free(fill);
+    return 0;
+}

@@ -482,3 +482,119 @@ def test_residual_is_shared_block_plus_routed_layer(orc):
             y_moe[t] += G[t, j] * _numpy_dense_ffn(W1[cols], W3[cols], W2[:, cols], x[t:t + 1])[0]
     ref = _numpy_dense_ffn(W1[shared], W3[shared], W2[:, shared], x) + (E / k) * y_moe
     np.testing.assert_allclose(r["y"], ref, rtol=1e-10, atol=1e-11 * np.abs(ref).max())
+
+
+# --------------------------------------------------------------------------- clustering
+
+def _load_cluster_golden():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "cluster_hand.txt")) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, rest = line.partition(" ")
+            if key == "case":
+                cur = {"name": rest}
+                cases.append(cur)
+            elif key == "centers":
+                cur[key] = [int(n) / int(q) for n, q in (v.split("/") for v in rest.split())]
+            else:
+                cur[key] = [int(v) for v in rest.split()]
+    return cases
+
+
+def test_cluster_golden(orc):
+    cases = _load_cluster_golden()
+    assert len(cases) == 7
+    for c in cases:
+        d, E = c["d"][0], c["E"][0]
+        F = np.array(c["F"], np.float32).reshape(-1, d)
+        assign, centers, perm = orc.cluster(F, E, c["iters"][0], c["init"])
+        assert assign.tolist() == c["assign"], c["name"]
+        assert perm.tolist() == c["perm"], c["name"]
+        assert centers.ravel().tolist() == c["centers"], c["name"]
+
+
+def _separated_groups(seed, E, m, d):
+    """E groups of m neurons around far-apart anchors, rows shuffled."""
+    r = _rng(seed)
+    anchors = 10.0 * r.standard_normal((E, d))
+    label = np.repeat(np.arange(E), m)
+    F = anchors[label] + 0.05 * r.standard_normal((E * m, d))
+    order = r.permutation(E * m)
+    return F[order].astype(np.float32), label[order]
+
+
+@pytest.mark.parametrize("E,m,d", [(4, 6, 16), (8, 5, 24)])
+def test_cluster_separated_groups_match_lloyd(orc, E, m, d):
+    """When the nearest-center assignment is already balanced, the balanced
+    k-means is Lloyd's k-means: compare with scikit-learn's, started from the
+    same centers."""
+    from sklearn.cluster import KMeans
+    F, label = _separated_groups(31 + E, E, m, d)
+    r = _rng(7)
+    init = np.array([r.choice(np.flatnonzero(label == g)) for g in r.permutation(E)], np.int32)
+    assign, centers, perm = orc.cluster(F, E, 3, init)
+    km = KMeans(n_clusters=E, init=F[init].astype(np.float64), n_init=1, max_iter=3,
+                algorithm="lloyd", tol=0.0).fit(F.astype(np.float64))
+    assert assign.tolist() == km.labels_.tolist()
+    np.testing.assert_allclose(centers, km.cluster_centers_, rtol=1e-12, atol=1e-12)
+    # the groups come back whole: cluster e is the group of its initial neuron
+    for e in range(E):
+        assert set(np.flatnonzero(assign == e)) == set(np.flatnonzero(label == label[init[e]]))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_cluster_invariants_and_first_round(orc, dtype):
+    """Balance, permutation layout, centers = numpy mean of the members; and for
+    one iteration, the first round of the assignment against scipy distances:
+    a cluster whose nearest-neuron set fits keeps all of it, one that overflows
+    keeps its m nearest."""
+    from scipy.spatial.distance import cdist
+    E, m, d = 6, 7, 20
+    r = _rng(41)
+    F = r.standard_normal((E * m, d)).astype(np.float32)
+    if dtype == "bf16":
+        F = _bf16_bits(F)
+    F64 = orc.to_f64(F)
+    init = r.choice(E * m, E, replace=False).astype(np.int32)
+    for iters in (1, 4):
+        assign, centers, perm = orc.cluster(F, E, iters, init)
+        assert np.bincount(assign, minlength=E).tolist() == [m] * E
+        assert sorted(perm.tolist()) == list(range(E * m))
+        for e in range(E):
+            seg = perm[e * m:(e + 1) * m]
+            assert (np.diff(seg) > 0).all() and (assign[seg] == e).all()
+            np.testing.assert_allclose(centers[e], F64[seg].mean(axis=0), rtol=1e-13, atol=1e-15)
+    assign, _, _ = orc.cluster(F, E, 1, init)
+    D = cdist(F64, F64[init], "sqeuclidean")
+    near = D.argmin(axis=1)
+    for e in range(E):
+        P = np.flatnonzero(near == e)
+        kept = P if len(P) <= m else P[np.argsort(D[P, e], kind="stable")[:m]]
+        assert (assign[kept] == e).all(), e
+        if len(P) > m:
+            assert (assign[np.setdiff1d(P, kept)] != e).all(), e
+
+
+def test_cluster_special_cases(orc):
+    r = _rng(43)
+    F = r.standard_normal((12, 5)).astype(np.float32)
+    # E = 1: one cluster, its center the mean of all rows
+    assign, centers, perm = orc.cluster(F, 1, 2, [4])
+    assert (assign == 0).all() and perm.tolist() == list(range(12))
+    np.testing.assert_allclose(centers[0], F.astype(np.float64).mean(axis=0), rtol=1e-13)
+    # m = 1: every neuron is the center of its own cluster
+    init = r.permutation(12).astype(np.int32)
+    assign, centers, perm = orc.cluster(F, 12, 1, init)
+    assert perm.tolist() == init.tolist()
+    assert assign[init].tolist() == list(range(12))
+    np.testing.assert_array_equal(centers, F[init].astype(np.float64))
+
+
+def test_cluster_rejects_bad_arguments(orc):
+    F = np.zeros((8, 4), np.float32)
+    for E, it, init in ((3, 1, [0, 1, 2]), (2, 0, [0, 1]), (2, 1, [1, 1]), (2, 1, [0, 8])):
+        with pytest.raises(ValueError):
+            orc.cluster(F, E, it, init)
