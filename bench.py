@@ -206,6 +206,10 @@ def parse():
                     help="override the workload's T (small cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cluster", action="store_true",
+                    help="time the clustering partition (balanced k-means of the W1 rows) "
+                         "of the workload's FFN instead of the layer")
+    ap.add_argument("--cluster-iters", type=int, default=10)
     return ap.parse_args()
 
 
@@ -355,6 +359,126 @@ def run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, ran
     return 0
 
 
+# FP64 lanes per SM on B200: NVIDIA's published 37-40 TFLOP/s FP64 over
+# (2 FLOP per FMA x 148 SMs x 1.965 GHz) gives 64-69; 64 is the power of two.
+FP64_LANES_PER_SM = 64
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+
+
+def run_cluster(args, rank, world, local):
+    """The clustering partition (balanced k-means over the W1 rows, E clusters of
+    d_ff/E neurons, --cluster-iters iterations) on the workload's FFN.  One step =
+    one whole moe_cluster_partition call.  F (W1) is below the 126 MB L2, so a
+    256 MB buffer is written between timed calls.  The roofline kernel is the
+    distance step (f64 ALU bound), timed alone with the same L2 flush."""
+    import top_routing_grouped_noisy_b200 as moe
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w, device="cuda", seed=w.seed + 7919 * rank)
+    F = inp["W1"]
+    del inp
+    n_iter = args.cluster_iters
+    init = wl.make_cluster_init(w.d_ff, w.E, w.seed + rank).cuda()
+    nbytes = moe.moe_cluster_workspace_size(w.d, w.d_ff, w.E)
+    ws = moe.Workspace(None, device="cuda", nbytes=nbytes)
+    assign = torch.empty(w.d_ff, dtype=torch.int32, device="cuda")
+    perm = torch.empty(w.d_ff, dtype=torch.int32, device="cuda")
+    centers = torch.empty(w.E, w.d, dtype=torch.float64, device="cuda")
+    D = torch.empty(w.d_ff, w.E, dtype=torch.float64, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    lib = moe.lib()
+    dt = moe.MOE_BF16 if F.dtype == torch.bfloat16 else moe.MOE_F32
+
+    def call():
+        rc = lib.moe_cluster_partition(F.data_ptr(), w.d, w.d_ff, w.E, dt, n_iter,
+                                       init.data_ptr(), assign.data_ptr(), centers.data_ptr(),
+                                       perm.data_ptr(), ws.ptr, ws.nbytes, stream.cuda_stream)
+        if rc != 0:
+            raise SystemExit("moe_cluster_partition: %s" % lib.moe_last_error_string().decode())
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    if moe.moe_get_device_status(ws) != 0:
+        raise SystemExit("device status set by the clustering")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    t_wall0 = time.time()
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    launches = moe.moe_launch_count() - l0
+    # the distance step alone, same flush
+    devs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for a, b in devs:
+        flush.fill_(1)
+        a.record(stream)
+        moe.moe_cluster_distances(F, centers, out=D)
+        b.record(stream)
+    torch.cuda.synchronize()
+    time.sleep(0.15)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+    dist_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in devs) / args.steps, world)
+    counts = torch.bincount(assign.long(), minlength=w.E).tolist()
+    if counts != [w.d_ff // w.E] * w.E:
+        raise SystemExit("unbalanced clusters %s" % counts)
+
+    ops = 3.0 * w.d_ff * w.E * w.d  # subtract, multiply, add per (neuron, center, column)
+    achieved = ops / (dist_ms / 1000.0) / 1e12
+    peak = SM_COUNT * FP64_LANES_PER_SM * SM_MAX_MHZ * 1e6 / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        Fh = wl.to_numpy_raw(F)
+        it_s = 2
+        t0 = time.time()
+        oracle.cluster(Fh, w.E, it_s, init.cpu().numpy())
+        t1 = time.time()
+        cpu = {"value": (t1 - t0) * 1000.0 * n_iter / it_s, "unit": "ms", "cores":
+               oracle.num_threads(), "kind": "oracle",
+               "sample": "%d of the %d iterations on the same W1, scaled to %d" %
+                         (it_s, n_iter, n_iter)}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "clustering partition time (balanced k-means over the W1 rows)",
+        "value": ms, "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "cluster_%s_w1" % w.name, "d": w.d, "d_ff": w.d_ff, "E": w.E,
+                   "n_iter": n_iter, "features": "W1 [d_ff][d] %s" % wl.torch_dtype(w),
+                   "parallelism": "dp%d replicas" % world,
+                   "l2": "256 MB buffer written between timed calls"},
+        "roofline": {"kernel": "cluster_dist_kernel (distance step, moe_cluster_distances)",
+                     "bound": "alu", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s (f64 add/sub/mul)", "frac": achieved / peak,
+                     "traffic": None,
+                     "peak_source": "derived: %d SMs x %d FP64 lanes x %.0f MHz" %
+                                    (SM_COUNT, FP64_LANES_PER_SM, SM_MAX_MHZ),
+                     "algorithmic": "3 f64 ops per (neuron, center, column) = %.4g per launch"
+                                    % ops},
+        "kernels": {"distance_step_ms": dist_ms, "per_iteration_ms": ms / n_iter},
+        "cpu_baseline": cpu, "e2e": None, "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -410,6 +534,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
+    if args.cluster:
+        return run_cluster(args, rank, world, local)
     import top_routing_grouped_noisy_b200 as moe
 
     w = wl.WORKLOADS[args.workload]

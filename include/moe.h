@@ -314,6 +314,46 @@ int moe_forward_residual(const moe_params_t *p, const moe_buffers_t *b, const vo
                          const void *W2_s, int32_t m_s, void *h_s, void *out_s, void *ws,
                          size_t ws_bytes, void *stream);
 
+/* ---- clustering partition (an alternative source of a0's perm) ------------
+ * ["LLaMA-MoE v2", section "专家构建方法", IndependentClustering: the neurons are
+ * grouped by k-means over their weight vectors and each cluster becomes one
+ * expert; the index set is split into E subsets of equal size m = d_ff / E.]
+ * Balanced k-means over the rows of F [d_ff][d] (dtype; the caller passes W1,
+ * the gate projection):
+ *   start:      C[e] = F[init_idx[e]] (E distinct neuron indices, device int32);
+ *   iteration:  D[i][e] = sum over c of (F[i][c] - C[e][c])^2;  in rounds, every
+ *               unplaced neuron proposes to its nearest cluster that is not full
+ *               (ties to the lower cluster index) and a cluster with room r keeps
+ *               its r proposals of smallest (D, neuron index), until all d_ff
+ *               neurons are placed (each cluster then holds m);  C[e] = mean of
+ *               the features of its members.
+ * All arithmetic is f64, one rounding per operation, sums in ascending column
+ * and neuron order: the result is that of the sequential definition, bit for bit.
+ * Outputs (device, caller-allocated): assign [d_ff] int32 (cluster of each neuron
+ * in the last assignment), centers [E][d] f64 (the means of that assignment),
+ * perm [d_ff] int32 (cluster 0's neurons in ascending order, then cluster 1's,
+ * ...; pass it to moe_partition_experts in DISJOINT mode).
+ * ws: moe_cluster_workspace_size bytes, zeroed once with moe_workspace_init.
+ * An init index out of range or repeated sets MOE_ERR_DEVICE_BADINDEX in the
+ * status word of ws (read it with moe_get_device_status) and gives a zero center.
+ * Errors: MOE_ERR_INVALID_ARG (NULL pointer, E outside 1..64, n_iter < 1),
+ * MOE_ERR_SHAPE (d % 8, d_ff % E), MOE_ERR_DTYPE, MOE_ERR_ALIGN (F, centers and ws
+ * 16-byte, index arrays 4-byte), MOE_ERR_WORKSPACE, MOE_ERR_CUDA.
+ * Launches 1 + n_iter * (2E + 3) kernels on `stream`. */
+size_t moe_cluster_workspace_size(int32_t d, int32_t d_ff, int32_t E);
+int moe_cluster_partition(const void *F, int32_t d, int32_t d_ff, int32_t E, int32_t dtype,
+                          int32_t n_iter, const int32_t *init_idx, int32_t *assign,
+                          double *centers, int32_t *perm, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* The distance step of the clustering alone: D [d_ff][E] f64 (device) receives
+ * sum over c of (F[i][c] - centers[e][c])^2 for F [d_ff][d] (dtype) and centers
+ * [E][d] f64, with the arithmetic of moe_cluster_partition (one launch).
+ * Errors: MOE_ERR_INVALID_ARG, MOE_ERR_SHAPE (d % 8), MOE_ERR_DTYPE,
+ * MOE_ERR_ALIGN (F and centers 16-byte, D 8-byte), MOE_ERR_CUDA. */
+int moe_cluster_distances(const void *F, int32_t d, int32_t d_ff, int32_t E, int32_t dtype,
+                          const double *centers, double *D, void *stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
  * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
  * the workspace's internal launch counters. */

@@ -46,6 +46,7 @@ def lib():
         _lib.oracle_gate_stats.argtypes = [i, i, i, p, p, d, p, p, p]
         _lib.oracle_balance_sketch.argtypes = [i, i, i, p, p, p, p]
         _lib.oracle_cluster.argtypes = [p, i, i, i, i, i, p, p, p, p]
+        _lib.oracle_sqdist.argtypes = [p, i, i, i, i, p, p]
     return _lib
 
 
@@ -303,3 +304,14 @@ def cluster(F, E: int, n_iter: int, init):
     _check(lib().oracle_cluster(_ptr(F), dt, d, d_ff, E, n_iter, _ptr(ini), _ptr(assign),
                                 _ptr(centers), _ptr(perm)), "cluster")
     return assign, centers, perm
+
+
+def sqdist(F, C):
+    """D [d_ff][E] float64: squared Euclidean distances of the rows of F to the rows of C."""
+    F = _c(F)
+    Cc = _c(C, np.float64)
+    d_ff, d = F.shape
+    E = Cc.shape[0]
+    D = np.empty((d_ff, E), np.float64)
+    _check(lib().oracle_sqdist(_ptr(F), _dt(F), d, d_ff, E, _ptr(Cc), _ptr(D)), "sqdist")
+    return D

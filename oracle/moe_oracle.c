@@ -520,6 +520,26 @@ int oracle_balance_sketch(int T, int E, int k, const int32_t *idx, const double 
  * assignment), centers [E][d] (after the last center step, so the means of
  * that assignment), perm [d_ff] (cluster 0's neurons ascending, then cluster
  * 1's, ...: the permutation a0 takes). */
+/* Squared Euclidean distance of every feature row to every center, summed in
+ * ascending column order: D[i][e] = sum_c (F[i][c] - C[e][c])^2. */
+int oracle_sqdist(const void *F, int dt, int d, int d_ff, int E, const double *C, double *D)
+{
+    if (d <= 0 || d_ff <= 0 || E <= 0)
+        return ORC_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int i = 0; i < d_ff; ++i)
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double diff = orc_load(F, dt, (size_t)i * d + c) - C[(size_t)e * d + c];
+                double sq = diff * diff;
+                s = s + sq;
+            }
+            D[(size_t)i * E + e] = s;
+        }
+    return 0;
+}
+
 static const double *orc_sort_keys;
 
 static int orc_cmp_key(const void *a, const void *b)
@@ -560,18 +580,7 @@ int oracle_cluster(const void *F, int dt, int d, int d_ff, int E, int n_iter,
             centers[(size_t)e * d + c] = orc_load(F, dt, (size_t)init[e] * d + c);
 
     for (int it = 0; it < n_iter; ++it) {
-        /* distances */
-#pragma omp parallel for schedule(static)
-        for (int i = 0; i < d_ff; ++i)
-            for (int e = 0; e < E; ++e) {
-                double s = 0.0;
-                for (int c = 0; c < d; ++c) {
-                    double diff = orc_load(F, dt, (size_t)i * d + c) - centers[(size_t)e * d + c];
-                    double sq = diff * diff;
-                    s = s + sq;
-                }
-                D[(size_t)i * E + e] = s;
-            }
+        oracle_sqdist(F, dt, d, d_ff, E, centers, D);
         /* balanced assignment in rounds */
         for (int i = 0; i < d_ff; ++i)
             assign[i] = -1;

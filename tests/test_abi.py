@@ -159,3 +159,26 @@ def test_pipeline_rejects_bad_arguments_before_the_device(L):
         moe.MOE_ERR_INVALID_ARG
     assert L.moe_pipeline_wait(None, 0) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_pipeline_destroy(None) == moe.MOE_OK
+
+
+def test_cluster_rejects_bad_arguments_before_the_device(L):
+    a = C.c_void_p(256)
+    n = L.moe_cluster_workspace_size(4096, 11008, 8)
+    assert n > 11008 * 8 * 8 and L.moe_cluster_workspace_size(4096, 11008, 7) == 0
+    assert L.moe_cluster_workspace_size(4096, 11008, 65) == 0
+    assert L.moe_cluster_workspace_size(4096, 11008, 4) < n  # monotone in E
+    call = lambda F=a, d=64, d_ff=32, E=4, dt=moe.MOE_BF16, it=1, init=a, asg=a, cen=a, perm=a, \
+        ws=a, nb=1 << 20: L.moe_cluster_partition(F, d, d_ff, E, dt, it, init, asg, cen, perm, ws,
+                                                  nb, None)
+    assert call(F=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(perm=None) == moe.MOE_ERR_INVALID_ARG
+    assert call(F=C.c_void_p(258)) == moe.MOE_ERR_ALIGN
+    assert call(cen=C.c_void_p(264)) == moe.MOE_ERR_ALIGN
+    assert call(dt=7) == moe.MOE_ERR_DTYPE
+    assert call(E=0) == moe.MOE_ERR_INVALID_ARG
+    assert call(E=65, d_ff=65 * 2) == moe.MOE_ERR_INVALID_ARG
+    assert call(it=0) == moe.MOE_ERR_INVALID_ARG
+    assert call(d=60) == moe.MOE_ERR_SHAPE
+    assert call(d_ff=30) == moe.MOE_ERR_SHAPE
+    assert call(nb=100) == moe.MOE_ERR_WORKSPACE
+    assert b"workspace" in L.moe_last_error_string()

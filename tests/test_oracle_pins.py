@@ -598,3 +598,15 @@ def test_cluster_rejects_bad_arguments(orc):
     for E, it, init in ((3, 1, [0, 1, 2]), (2, 0, [0, 1]), (2, 1, [1, 1]), (2, 1, [0, 8])):
         with pytest.raises(ValueError):
             orc.cluster(F, E, it, init)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sqdist_matches_scipy(orc, dtype):
+    from scipy.spatial.distance import cdist
+    r = _rng(47)
+    F = r.standard_normal((37, 29)).astype(np.float32)
+    if dtype == "bf16":
+        F = _bf16_bits(F)
+    Cc = r.standard_normal((5, 29))
+    D = orc.sqdist(F, Cc)
+    np.testing.assert_allclose(D, cdist(orc.to_f64(F), Cc, "sqeuclidean"), rtol=1e-13)

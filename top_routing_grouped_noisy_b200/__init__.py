@@ -20,7 +20,8 @@ __all__ = [
     "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
     "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline", "moe_partition_residual",
-    "moe_combine_residual", "moe_forward_residual",
+    "moe_combine_residual", "moe_forward_residual", "moe_cluster_workspace_size",
+    "moe_cluster_partition", "moe_cluster_distances",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -109,6 +110,10 @@ def lib():
             "moe_combine_residual": (C.c_int, [P, v, v, v, v, v, v]),
             "moe_forward_residual": (C.c_int, [P, C.POINTER(_Buffers), v, v, i32, v, v, v, sz,
                                                v]),
+            "moe_cluster_workspace_size": (sz, [i32, i32, i32]),
+            "moe_cluster_partition": (C.c_int, [v, i32, i32, i32, i32, i32, v, v, v, v, v, sz,
+                                                v]),
+            "moe_cluster_distances": (C.c_int, [v, i32, i32, i32, i32, v, v, v]),
             "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
             "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
             "moe_pipeline_wait": (C.c_int, [v, i64]),
@@ -424,3 +429,38 @@ class Pipeline:
             self.close()
         except Exception:
             pass
+
+
+def moe_cluster_workspace_size(d, d_ff, E) -> int:
+    return int(lib().moe_cluster_workspace_size(d, d_ff, E))
+
+
+def moe_cluster_partition(F, E, n_iter, init_idx, ws=None, stream=None):
+    """Balanced k-means partition of the rows of F [d_ff][d] into E clusters of
+    d_ff/E neurons (include/moe.h).  Returns (assign, centers, perm, ws); ws is a
+    Workspace-like object whose status word records a bad init index."""
+    dt = _dtype_code(F.dtype)
+    d_ff, d = F.shape
+    dev = F.device
+    if ws is None:
+        n = moe_cluster_workspace_size(d, d_ff, E)
+        if n <= 0:
+            raise MoeError(MOE_ERR_SHAPE, "invalid shape for the clustering workspace")
+        ws = Workspace(None, device=dev, nbytes=n)
+    assign = torch.empty(d_ff, dtype=torch.int32, device=dev)
+    perm = torch.empty(d_ff, dtype=torch.int32, device=dev)
+    centers = torch.empty(E, d, dtype=torch.float64, device=dev)
+    _check(lib().moe_cluster_partition(_p(F), d, d_ff, E, dt, n_iter, _p(init_idx), _p(assign),
+                                       _p(centers), _p(perm), ws.ptr, ws.nbytes,
+                                       _stream(stream)))
+    return assign, centers, perm, ws
+
+
+def moe_cluster_distances(F, centers, out=None, stream=None):
+    """D [d_ff][E] f64: squared distances of the rows of F to the centers (f64)."""
+    d_ff, d = F.shape
+    E = centers.shape[0]
+    D = out if out is not None else torch.empty(d_ff, E, dtype=torch.float64, device=F.device)
+    _check(lib().moe_cluster_distances(_p(F), d, d_ff, E, _dtype_code(F.dtype), _p(centers),
+                                       _p(D), _stream(stream)))
+    return D

@@ -16,7 +16,8 @@ LIB = os.path.join(PKG, "libmoe.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["api.cu", "partition.cu", "router.cu", "router_tc.cu", "dispatch.cu", "ffn_simt.cu",
-           "ffn_tc.cu", "decode.cu", "combine.cu", "pipeline.cu"]
+           "ffn_tc.cu", "decode.cu", "combine.cu", "pipeline.cu",
+           "cluster.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr"]
 

@@ -145,3 +145,11 @@ def to_numpy_raw(t: torch.Tensor):
     if t.dtype in (torch.int32, torch.int64):
         return t.numpy()
     raise TypeError(t.dtype)
+
+
+def make_cluster_init(d_ff: int, E: int, seed: int) -> torch.Tensor:
+    """E distinct neuron indices drawn uniformly (the initial k-means centers of the
+    clustering partition), int32 on the CPU."""
+    g = torch.Generator()
+    g.manual_seed(seed)
+    return torch.randperm(d_ff, generator=g)[:E].to(torch.int32).contiguous()
