@@ -47,6 +47,11 @@ def lib():
         _lib.oracle_balance_sketch.argtypes = [i, i, i, p, p, p, p]
         _lib.oracle_cluster.argtypes = [p, i, i, i, i, i, p, p, p, p]
         _lib.oracle_sqdist.argtypes = [p, i, i, i, i, p, p]
+        _lib.oracle_combine_backward.argtypes = [i, i, i, p, p, p, d, p, p, p]
+        _lib.oracle_expert_ffn_backward.argtypes = [i, i, i, p, p, p, i, p, i, p, i, p, p, p, p,
+                                                    p, p, p, p]
+        _lib.oracle_router_backward.argtypes = [i, i, i, i, i, p, i, p, p, p, p, p, p, p, p, d,
+                                                d, p, p, p, p, p, p]
     return _lib
 
 
@@ -315,3 +320,107 @@ def sqdist(F, C):
     D = np.empty((d_ff, E), np.float64)
     _check(lib().oracle_sqdist(_ptr(F), _dt(F), d, d_ff, E, _ptr(Cc), _ptr(D)), "sqdist")
     return D
+
+
+# --------------------------------------------------------------------------- backward (f1)
+
+def combine_backward(out_rows, slot_row, G, scale: float, dy):
+    """d_out [R][d] and dG [T][k] of y = s sum_j G_j out_{r(t,j)}."""
+    out_rows = _c(out_rows, np.float64)
+    slot_row = _c(slot_row, np.int32)
+    G = _c(G, np.float64)
+    dy = _c(dy, np.float64)
+    T, k = slot_row.shape
+    d = dy.shape[1]
+    R = out_rows.shape[0]
+    d_out = np.zeros((max(R, 1), d), np.float64)
+    dG = np.empty((T, k), np.float64)
+    src = out_rows if R > 0 else np.zeros((1, d))
+    _check(lib().oracle_combine_backward(T, d, k, _ptr(src), _ptr(slot_row), _ptr(G),
+                                         float(scale), _ptr(dy), _ptr(d_out), _ptr(dG)),
+           "combine_backward")
+    return d_out[:R], dG
+
+
+def expert_ffn_backward(W1e, W3e, W2e, x_rows, expert_of_row, d_out):
+    """Expert backward for the given rows: dx_rows [n][d], dW1e / dW3e [E][m][d],
+    dW2e [E][d][m], and the per-row dh, dg, du [n][m] (all float64)."""
+    W1e, W3e, W2e = _c(W1e), _c(W3e), _c(W2e)
+    E, m, d = W1e.shape
+    x_rows = _c(x_rows)
+    eor = _c(expert_of_row, np.int32)
+    d_out = _c(d_out, np.float64)
+    n = x_rows.shape[0]
+    dx = np.zeros((max(n, 1), d), np.float64)
+    dW1 = np.empty((E, m, d), np.float64)
+    dW3 = np.empty((E, m, d), np.float64)
+    dW2 = np.empty((E, d, m), np.float64)
+    dh = np.empty((max(n, 1), m), np.float64)
+    dg = np.empty((max(n, 1), m), np.float64)
+    du = np.empty((max(n, 1), m), np.float64)
+    xr = x_rows if n > 0 else np.zeros((1, d), x_rows.dtype)
+    dor = d_out if n > 0 else np.zeros((1, d))
+    _check(lib().oracle_expert_ffn_backward(d, m, E, _ptr(W1e), _ptr(W3e), _ptr(W2e), _dt(W1e),
+                                            _ptr(xr), _dt(xr), _ptr(eor), n, _ptr(dor), _ptr(dx),
+                                            _ptr(dW1), _ptr(dW3), _ptr(dW2), _ptr(dh), _ptr(dg),
+                                            _ptr(du)), "expert_ffn_backward")
+    return dict(dx_rows=dx[:n], dW1e=dW1, dW3e=dW3, dW2e=dW2, dh=dh[:n], dg=dg[:n], du=du[:n])
+
+
+def router_backward(x, Wg, idx, G, dG, counts, k, router_type=MIXTRAL, Wnoise=None, eps=None,
+                    bias=None, lam=0.0, dLb=1.0, dx=None):
+    """Router backward; adds W_g dL + W_noise dN to dx (a new zero array when None)."""
+    x, Wg = _c(x), _c(Wg)
+    dt = _dt(x)
+    T, d = x.shape
+    E = Wg.shape[1]
+    Wn = None if Wnoise is None else _c(Wnoise)
+    ep = None if eps is None else _c(eps, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    idx = _c(idx, np.int32)
+    G = _c(G, np.float64)
+    dG = _c(dG, np.float64)
+    counts = _c(counts, np.int32)
+    dx = np.zeros((T, d), np.float64) if dx is None else dx
+    assert dx.dtype == np.float64 and dx.flags.c_contiguous
+    dWg = np.empty((d, E), np.float64)
+    dWn = np.empty((d, E), np.float64) if Wnoise is not None else None
+    db = np.empty(E, np.float64) if bias is not None else None
+    dH = np.empty((T, E), np.float64)
+    dN = np.empty((T, E), np.float64)
+    _check(lib().oracle_router_backward(T, d, E, k, router_type, _ptr(x), dt, _ptr(Wg), _ptr(Wn),
+                                        _ptr(ep), _ptr(b), _ptr(idx), _ptr(G), _ptr(dG),
+                                        _ptr(counts), float(lam), float(dLb), _ptr(dx),
+                                        _ptr(dWg), _ptr(dWn), _ptr(db), _ptr(dH), _ptr(dN)),
+           "router_backward")
+    return dict(dx=dx, dWg=dWg, dWnoise=dWn, dbias=db, dH=dH, dN=dN)
+
+
+def backward(x, Wg, W1e, W3e, W2e, k, dy, router_type=MIXTRAL, Wnoise=None, eps=None,
+             bias=None, capacity_rows=-1, rescale=False, lam=0.0, dLb=1.0):
+    """Gradients of l(y) + dLb * L_balance for the whole layer, given dy = dl/dy:
+    dx, dWg, dWnoise, dbias, dW1e, dW3e, dW2e, plus every intermediate (d_out,
+    dG, dh, dg, du, dx_rows, dH, dN) and the forward pass (key 'fwd')."""
+    E = Wg.shape[1]
+    T = x.shape[0]
+    f = forward(x, Wg, W1e, W3e, W2e, k, router_type, Wnoise, eps, bias, capacity_rows,
+                rescale, lam)
+    r, dsp = f["router"], f["dispatch"]
+    scale = (E / k) if rescale else 1.0
+    d_out, dG = combine_backward(f["out_rows"], dsp["slot_row"], r["G"], scale, dy)
+    R = dsp["R"]
+    expert_of_row = np.searchsorted(dsp["offsets"], np.arange(R), side="right") - 1
+    x_rows = np.ascontiguousarray(np.asarray(x)[dsp["row_token"]])
+    eb = expert_ffn_backward(W1e, W3e, W2e, x_rows, expert_of_row, d_out)
+    dx = np.zeros((T, x.shape[1]), np.float64)
+    for t in range(T):
+        for j in range(k):
+            row = dsp["slot_row"][t, j]
+            if row >= 0:
+                dx[t] += eb["dx_rows"][row]
+    rb = router_backward(x, Wg, r["idx"], r["G"], dG, dsp["counts"], k, router_type, Wnoise,
+                         eps, bias, lam, dLb, dx)
+    return dict(dx=dx, dWg=rb["dWg"], dWnoise=rb["dWnoise"], dbias=rb["dbias"],
+                dW1e=eb["dW1e"], dW3e=eb["dW3e"], dW2e=eb["dW2e"], d_out=d_out, dG=dG,
+                dh=eb["dh"], dg=eb["dg"], du=eb["du"], dx_rows=eb["dx_rows"], dH=rb["dH"],
+                dN=rb["dN"], fwd=f)

@@ -631,3 +631,269 @@ int oracle_cluster(const void *F, int dt, int d, int d_ff, int E, int n_iter,
     free(D), free(key), free(target), free(cand), free(fill);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* f1. Backward of the layer.  The loss is l(y) + c * L_balance; the caller gives
+ * dy = dl/dy [T][d] and c.  Every function below is the chain rule of one forward
+ * step written out in f64 loops, in the forward's notation:
+ *   combine   y_t = s sum_j G_tj out_{r(t,j)}
+ *   expert    g = W1_e x, u = W3_e x, h = silu(g) * u, out = W2_e h
+ *   router    L = x W_g + b, N = x W_noise, H = L + eps * softplus(N),
+ *             G = softmax over the k selected H (Mixtral) or softmax(H)_idx (ST),
+ *             P_e = mean_t softmax(H_t)_e, L_balance = lambda sum_e f_e P_e
+ * The top-k choice, the dispatch and f_e (counts) are piecewise constant and
+ * carry no gradient; a dropped slot gets dG = 0. */
+
+/* Combine backward: for every kept slot (t, j) with row r = slot_row[t][j]:
+ *   d_out[r] = s * G_tj * dy_t,   dG_tj = s * <dy_t, out_r>;   dropped: dG_tj = 0.
+ * out_rows / d_out [R][d], dy [T][d], G / dG [T][k]. */
+int oracle_combine_backward(int T, int d, int k, const double *out_rows, const int32_t *slot_row,
+                            const double *G, double scale, const double *dy, double *d_out,
+                            double *dG)
+{
+    if (T < 0 || d <= 0 || k <= 0)
+        return ORC_EINVAL;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            size_t a = (size_t)t * k + j;
+            int r = slot_row[a];
+            if (r < 0) {
+                dG[a] = 0.0;
+                continue;
+            }
+            double dot = 0.0;
+            for (int o = 0; o < d; ++o) {
+                dot += dy[(size_t)t * d + o] * out_rows[(size_t)r * d + o];
+                d_out[(size_t)r * d + o] = scale * G[a] * dy[(size_t)t * d + o];
+            }
+            dG[a] = scale * dot;
+        }
+    return 0;
+}
+
+/* Derivative of silu: sigma(z) (1 + z (1 - sigma(z))). */
+static double orc_dsilu(double z)
+{
+    double s = 1.0 / (1.0 + exp(-z));
+    return s * (1.0 + z * (1.0 - s));
+}
+
+/* Expert backward for n rows (row r belongs to expert expert_of_row[r]):
+ *   dh = W2_e^T d_out,  du = dh * silu(g),  dg = dh * u * silu'(g),
+ *   dx_r = W1_e^T dg + W3_e^T du,
+ *   dW2_e += d_out h^T,  dW1_e += dg x^T,  dW3_e += du x^T  (rows summed in ascending r).
+ * Layouts as oracle_expert_ffn: W1e, W3e, dW1e, dW3e [E][m][d]; W2e, dW2e [E][d][m];
+ * x_rows [n][d] (type xdt); d_out, dx_rows [n][d]; optional dh, dg, du [n][m]. */
+int oracle_expert_ffn_backward(int d, int m, int E, const void *W1e, const void *W3e,
+                               const void *W2e, int dt, const void *x_rows, int xdt,
+                               const int32_t *expert_of_row, int n, const double *d_out,
+                               double *dx_rows, double *dW1e, double *dW3e, double *dW2e,
+                               double *dh_out, double *dg_out, double *du_out)
+{
+    if (d <= 0 || m <= 0 || E <= 0 || n < 0)
+        return ORC_EINVAL;
+    for (int r = 0; r < n; ++r)
+        if (expert_of_row[r] < 0 || expert_of_row[r] >= E)
+            return ORC_EINVAL;
+    double *X = (double *)malloc(sizeof(double) * ((size_t)n * d + 1));
+    double *Hh = (double *)malloc(sizeof(double) * ((size_t)n * m + 1));
+    double *Dg = (double *)malloc(sizeof(double) * ((size_t)n * m + 1));
+    double *Du = (double *)malloc(sizeof(double) * ((size_t)n * m + 1));
+    if (!X || !Hh || !Dg || !Du) {
+        free(X), free(Hh), free(Dg), free(Du);
+        return ORC_EINVAL;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < n; ++r) {
+        int e = expert_of_row[r];
+        double *xr = X + (size_t)r * d;
+        for (int c = 0; c < d; ++c)
+            xr[c] = orc_load(x_rows, xdt, (size_t)r * d + c);
+        for (int i = 0; i < m; ++i) {
+            double g = 0.0, u = 0.0, dh = 0.0;
+            size_t base = ((size_t)e * m + i) * d;
+            for (int c = 0; c < d; ++c) {
+                g += orc_load(W1e, dt, base + c) * xr[c];
+                u += orc_load(W3e, dt, base + c) * xr[c];
+            }
+            for (int o = 0; o < d; ++o)
+                dh += orc_load(W2e, dt, ((size_t)e * d + o) * m + i) * d_out[(size_t)r * d + o];
+            Hh[(size_t)r * m + i] = oracle_silu(g) * u;
+            Du[(size_t)r * m + i] = dh * oracle_silu(g);
+            Dg[(size_t)r * m + i] = dh * u * orc_dsilu(g);
+            if (dh_out)
+                dh_out[(size_t)r * m + i] = dh;
+        }
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int i = 0; i < m; ++i) {
+                size_t w = ((size_t)e * m + i) * d + c;
+                acc += orc_load(W1e, dt, w) * Dg[(size_t)r * m + i] +
+                       orc_load(W3e, dt, w) * Du[(size_t)r * m + i];
+            }
+            dx_rows[(size_t)r * d + c] = acc;
+        }
+    }
+    /* weight gradients: each entry sums its rows in ascending order */
+#pragma omp parallel for schedule(static)
+    for (int e = 0; e < E; ++e) {
+        for (int i = 0; i < m; ++i)
+            for (int c = 0; c < d; ++c) {
+                double a1 = 0.0, a3 = 0.0;
+                for (int r = 0; r < n; ++r)
+                    if (expert_of_row[r] == e) {
+                        a1 += Dg[(size_t)r * m + i] * X[(size_t)r * d + c];
+                        a3 += Du[(size_t)r * m + i] * X[(size_t)r * d + c];
+                    }
+                dW1e[((size_t)e * m + i) * d + c] = a1;
+                dW3e[((size_t)e * m + i) * d + c] = a3;
+            }
+        for (int o = 0; o < d; ++o)
+            for (int i = 0; i < m; ++i) {
+                double a2 = 0.0;
+                for (int r = 0; r < n; ++r)
+                    if (expert_of_row[r] == e)
+                        a2 += d_out[(size_t)r * d + o] * Hh[(size_t)r * m + i];
+                dW2e[((size_t)e * d + o) * m + i] = a2;
+            }
+    }
+    if (dg_out)
+        memcpy(dg_out, Dg, sizeof(double) * (size_t)n * m);
+    if (du_out)
+        memcpy(du_out, Du, sizeof(double) * (size_t)n * m);
+    free(X), free(Hh), free(Dg), free(Du);
+    return 0;
+}
+
+/* Router backward.  Recomputes L, N, H and p = softmax(H) per token (as
+ * oracle_router), then with dG [T][k] (from the combine backward), the forward's
+ * idx / G [T][k], counts [E] (routed, pre-drop) and c = dLb:
+ *   Mixtral: S = sum_j G_j dG_j,  dH[idx_j] += G_j (dG_j - S)
+ *   ST:      g_e = dG_j if e = idx_j else 0,  S = sum_e p_e g_e,  dH_e += p_e (g_e - S)
+ *   balance: b_e = c lambda f_e / T,  B = sum_e p_e b_e,  dH_e += p_e (b_e - B)
+ *   dL = dH,  dN = dH * eps * sigmoid(N)
+ *   dx_t += W_g dL_t + W_noise dN_t,  dW_g = x^T dL,  dW_noise = x^T dN,  db = sum_t dL_t
+ * dx [T][d] is ADDED to; dWg, dWnoise [d][E], dbias [E] are written (NULL when the
+ * input is absent); dH_out [T][E] and dN_out [T][E] optional. */
+int oracle_router_backward(int T, int d, int E, int k, int router_type, const void *x, int dt,
+                           const void *Wg, const void *Wnoise, const float *eps, const float *bias,
+                           const int32_t *idx, const double *G, const double *dG,
+                           const int32_t *counts, double lambda, double dLb, double *dx,
+                           double *dWg, double *dWnoise, double *dbias, double *dH_out,
+                           double *dN_out)
+{
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
+        return ORC_EINVAL;
+    if (Wnoise != NULL && eps == NULL)
+        return ORC_EINVAL;
+    double *DL = (double *)calloc((size_t)T * E + 1, sizeof(double));
+    double *DN = (double *)calloc((size_t)T * E + 1, sizeof(double));
+    if (!DL || !DN) {
+        free(DL), free(DN);
+        return ORC_EINVAL;
+    }
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double *L = (double *)malloc(sizeof(double) * (size_t)E * 5);
+        double *N = L + E, *H = N + E, *p = H + E, *dH = p + E;
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0, accn = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double xv = orc_load(x, dt, (size_t)t * d + c);
+                acc += xv * orc_load(Wg, dt, (size_t)c * E + e);
+                if (Wnoise)
+                    accn += xv * orc_load(Wnoise, dt, (size_t)c * E + e);
+            }
+            if (bias)
+                acc += (double)bias[e];
+            L[e] = acc;
+            N[e] = accn;
+            H[e] = Wnoise ? acc + (double)eps[(size_t)t * E + e] * oracle_softplus(accn) : acc;
+        }
+        double hmax = H[0];
+        for (int e = 1; e < E; ++e)
+            if (H[e] > hmax)
+                hmax = H[e];
+        double z = 0.0;
+        for (int e = 0; e < E; ++e)
+            z += exp(H[e] - hmax);
+        for (int e = 0; e < E; ++e) {
+            p[e] = exp(H[e] - hmax) / z;
+            dH[e] = 0.0;
+        }
+        const int32_t *it = idx + (size_t)t * k;
+        const double *Gt = G + (size_t)t * k, *dGt = dG + (size_t)t * k;
+        if (router_type == ORC_MIXTRAL) {
+            double S = 0.0;
+            for (int j = 0; j < k; ++j)
+                S += Gt[j] * dGt[j];
+            for (int j = 0; j < k; ++j)
+                if (it[j] >= 0 && it[j] < E)
+                    dH[it[j]] += Gt[j] * (dGt[j] - S);
+        } else {
+            double S = 0.0;
+            for (int j = 0; j < k; ++j)
+                if (it[j] >= 0 && it[j] < E)
+                    S += p[it[j]] * dGt[j];
+            for (int e = 0; e < E; ++e) {
+                double ge = 0.0;
+                for (int j = 0; j < k; ++j)
+                    if (it[j] == e)
+                        ge += dGt[j];
+                dH[e] += p[e] * (ge - S);
+            }
+        }
+        if (lambda != 0.0 && dLb != 0.0 && T > 0) {
+            double B = 0.0;
+            for (int e = 0; e < E; ++e)
+                B += p[e] * (dLb * lambda * ((double)counts[e] / ((double)T * k)) / (double)T);
+            for (int e = 0; e < E; ++e) {
+                double be = dLb * lambda * ((double)counts[e] / ((double)T * k)) / (double)T;
+                dH[e] += p[e] * (be - B);
+            }
+        }
+        for (int e = 0; e < E; ++e) {
+            DL[(size_t)t * E + e] = dH[e];
+            if (Wnoise) {
+                double sg = 1.0 / (1.0 + exp(-N[e]));
+                DN[(size_t)t * E + e] = dH[e] * (double)eps[(size_t)t * E + e] * sg;
+            }
+            if (dH_out)
+                dH_out[(size_t)t * E + e] = dH[e];
+            if (dN_out)
+                dN_out[(size_t)t * E + e] = DN[(size_t)t * E + e];
+        }
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int e = 0; e < E; ++e) {
+                acc += orc_load(Wg, dt, (size_t)c * E + e) * DL[(size_t)t * E + e];
+                if (Wnoise)
+                    acc += orc_load(Wnoise, dt, (size_t)c * E + e) * DN[(size_t)t * E + e];
+            }
+            dx[(size_t)t * d + c] += acc;
+        }
+        free(L);
+    }
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c)
+        for (int e = 0; e < E; ++e) {
+            double a = 0.0, an = 0.0;
+            for (int t = 0; t < T; ++t) {
+                double xv = orc_load(x, dt, (size_t)t * d + c);
+                a += xv * DL[(size_t)t * E + e];
+                an += xv * DN[(size_t)t * E + e];
+            }
+            dWg[(size_t)c * E + e] = a;
+            if (dWnoise)
+                dWnoise[(size_t)c * E + e] = an;
+        }
+    if (dbias)
+        for (int e = 0; e < E; ++e) {
+            double a = 0.0;
+            for (int t = 0; t < T; ++t)
+                a += DL[(size_t)t * E + e];
+            dbias[e] = a;
+        }
+    free(DL), free(DN);
+    return 0;
+}
