@@ -210,6 +210,8 @@ def parse():
                     help="time the clustering partition (balanced k-means of the W1 rows) "
                          "of the workload's FFN instead of the layer")
     ap.add_argument("--cluster-iters", type=int, default=10)
+    ap.add_argument("--backward", action="store_true",
+                    help="time a training step (forward + backward) of the layer")
     return ap.parse_args()
 
 
@@ -479,6 +481,147 @@ def run_cluster(args, rank, world, local):
     return 0
 
 
+def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp, rank,
+              world, local):
+    """A training step of the layer: the forward (the six step calls) and the backward
+    (combine, expert GEMM 2, expert GEMM 1 + SwiGLU, router + input) for l(y) + L_balance
+    with a seeded dl/dy.  The roofline figure is moe_expert_up_backward, timed inside the
+    step loop: three tcgen05 GEMMs (g/u recompute with the SwiGLU backward, dgrad,
+    wgrad) plus the transposes that feed the weight-gradient GEMM."""
+    if w.dtype != "bf16" or w.shared > 0:
+        raise SystemExit("--backward runs bf16 layers without a shared block")
+    stream = torch.cuda.current_stream()
+    dy = wl.make_grad_output(w, w.seed + 1 + 7919 * rank, device="cuda")
+    g = moe.BackwardBuffers(p, Wn is not None, bias is not None)
+    wsb = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
+    SEG = ["forward", "combine_bwd", "down_bwd", "up_bwd", "route_bwd"]
+
+    def step(ev=None, up=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        fwd_step()
+        mark(1)
+        moe.moe_combine_backward(p, dy, b.out, b.slot_row, b.topk_w, g.d_out, g.dG)
+        mark(2)
+        moe.moe_expert_down_backward(p, g.d_out, b.h, b.offsets, W2_e, g.dh, g.dW2_e, wsb)
+        mark(3)
+        if up is not None:
+            up[0].record(stream)
+        moe.moe_expert_up_backward(p, b.x_perm, g.dh, b.offsets, W13_e, g.dx_perm, g.dW13_e, wsb)
+        if up is not None:
+            up[1].record(stream)
+        mark(4)
+        moe.moe_route_backward(p, x, Wg, b.topk_idx, b.topk_w, g.dG, b.counts, g.dx_perm,
+                               b.slot_row, g.dx, g.dWg, wsb, Wnoise=Wn, noise=eps, bias=bias,
+                               dWnoise=g.dWnoise, dbias=g.dbias, dLb=1.0)
+        mark(5)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = moe.moe_get_device_status(wsb)
+    if st != 0:
+        raise SystemExit("device status %d after warm-up" % st)
+    R = int(b.offsets[-1])
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    up_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(up=up_evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    launches = moe.moe_launch_count() - l0
+    time.sleep(0.15)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    if moe.moe_get_device_status(wsb) != 0:
+        raise SystemExit("device status set in the timed region")
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    up_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in up_evs) / args.steps, world)
+    nseg = min(args.steps, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(SEG) + 1)]
+           for _ in range(nseg)]
+    for i in range(nseg):
+        step(evs[i])
+    torch.cuda.synchronize()
+    seg = np.zeros(len(SEG))
+    for e in evs:
+        for k2 in range(len(SEG)):
+            seg[k2] += e[k2].elapsed_time(e[k2 + 1])
+    seg = [max_over_ranks(v / nseg, world) for v in seg]
+    value = tokens_per_s(w.T, args.steps, world, ms)
+    dmr = float(w.d) * w.m * R
+    flop_step = 22.0 * dmr  # forward 6, GEMM 2 backward 4, GEMM 1 backward 12 (with recompute)
+    peaks, peak_src = load_peaks()
+    peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    up_tf = 12.0 * dmr / (up_ms / 1000.0) / 1e12
+    kernels = {n: {"ms": v} for n, v in zip(SEG, seg)}
+    kernels["down_bwd"]["TFLOP/s"] = 4.0 * dmr / (seg[2] / 1000.0) / 1e12
+    kernels["up_bwd"]["TFLOP/s"] = 12.0 * dmr / (seg[3] / 1000.0) / 1e12
+    kernels["forward"]["TFLOP/s"] = 6.0 * dmr / (seg[0] / 1000.0) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        n_s = 128
+        sub = {k2: (v[:n_s].cpu() if k2 in ("x", "eps") and v is not None else
+                    (v.cpu() if isinstance(v, torch.Tensor) else v)) for k2, v in inp.items()}
+        if w.partition == wl.COPY:
+            W1e, W3e, W2e = oracle.partition(wl.to_numpy_raw(sub["W1"]), wl.to_numpy_raw(
+                sub["W3"]), wl.to_numpy_raw(sub["W2"]), w.E, oracle.COPY)
+        else:
+            W1e, W3e, W2e = oracle.partition(wl.to_numpy_raw(sub["W1"]), wl.to_numpy_raw(
+                sub["W3"]), wl.to_numpy_raw(sub["W2"]), w.E, oracle.DISJOINT,
+                wl.to_numpy_raw(sub["perm"]))
+        dy_s = dy[:n_s].cpu().to(torch.float64).numpy()
+        C_s = moe.moe_capacity(n_s, w.E, w.cf) if w.cf >= 0 else -1
+        t0 = time.time()
+        oracle.backward(wl.to_numpy_raw(sub["x"]), wl.to_numpy_raw(sub["Wg"]), W1e, W3e, W2e,
+                        w.k, dy_s, w.router, None if sub["Wnoise"] is None else
+                        wl.to_numpy_raw(sub["Wnoise"]), None if sub["eps"] is None else
+                        sub["eps"].numpy(), None if sub["bias"] is None else sub["bias"].numpy(),
+                        C_s, w.rescale, w.lam, 1.0)
+        el = time.time() - t0
+        cpu = {"value": n_s / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+               "kind": "oracle", "sample": "forward + backward of the first %d tokens (same "
+               "weights, capacity for %d tokens), %.1f s" % (n_s, n_s, el)}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "MoE-layer training step (forward + backward) tokens/s at 1 B200",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(w, C), parallelism="dp%d replicas" % world, kept_rows=R,
+                       loss="sum(y * dy) + L_balance, dy ~ N(0,1) seeded"),
+        "tflops": flop_step * args.steps * world / (ms / 1000.0) / 1e12,
+        "roofline": {"kernel": "moe_expert_up_backward: bwd_gemm_kernel x3 (recompute + SwiGLU "
+                               "backward, dgrad, wgrad) + 3 transposes",
+                     "bound": "tensor", "achieved": up_tf, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": up_tf / peak_t, "traffic": None,
+                     "peak_source": "%s bf16_tflops_sustained" % peak_src,
+                     "algorithmic": "12*d*m FLOP per kept row x R=%d = %.4g FLOP per call"
+                                    % (R, 12.0 * dmr)},
+        "kernels": kernels, "cpu_baseline": cpu, "e2e": None, "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -616,6 +759,9 @@ def main():
         moe.moe_gate_stats(p, b.counts, b.probs_sum, b.f, b.P, b.loss)
         mark()
 
+    if args.backward:
+        return run_train(args, w, p, moe, step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp,
+                         rank, world, local)
     if w.T <= 64:
         return run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank,
                           world, local)

@@ -354,6 +354,76 @@ int moe_cluster_partition(const void *F, int32_t d, int32_t d_ff, int32_t E, int
 int moe_cluster_distances(const void *F, int32_t d, int32_t d_ff, int32_t E, int32_t dtype,
                           const double *centers, double *D, void *stream);
 
+/* ---- backward of the layer (bf16 layers, T >= 1) ---------------------------
+ * Gradients of l(y) + c * L_balance for a scalar loss l, given dy = dl/dy and c
+ * (dLb below); the chain rule of each forward step ("Llama 3 Meets MoE",
+ * section 3: the noisy Top-k router and the combine; "LLaMA-MoE v2": the SwiGLU
+ * expert of the code sample, L_balance = lambda sum f_i P_i in "门控机制设计"):
+ *   combine  d_out[r] = s G_tj dy_t,  dG_tj = s <dy_t, out_r>  (dropped slot: 0)
+ *   expert   dh = W2_e^T d_out, du = dh silu(g), dg = dh u silu'(g),
+ *            dx_perm = W1_e^T dg + W3_e^T du, dW2_e = sum d_out h^T,
+ *            dW1_e = sum dg x^T, dW3_e = sum du x^T (over the expert's rows)
+ *   router   Mixtral: dH[idx_j] = G_j (dG_j - sum_l G_l dG_l);
+ *            ST: dH_e = p_e (g_e - sum_l p_l g_l), g the dG of the selected experts;
+ *            balance: dH_e += p_e (b_e - sum_l p_l b_l), b_e = c lambda f_e / T;
+ *            dL = dH, dN = dH eps sigmoid(N);  dW_g = x^T dL, dW_noise = x^T dN,
+ *            db = sum_t dL
+ *   input    dx_t = sum_j dx_perm[slot_row[t][j]] + W_g dL_t + W_noise dN_t
+ * The top-k choice, the dispatch and the counts f carry no gradient.  The forward
+ * intermediates (moe_buffers_t of the same batch) are inputs.  bf16 gradients
+ * are rounded once from f32 sums; router weight gradients are f32.  g and u are
+ * recomputed (x_perm W13_e^T), not stored by the forward.
+ * The workspace (moe_backward_workspace_size bytes, zeroed once with
+ * moe_workspace_init) holds the transposed weights and activations the
+ * weight-gradient GEMMs read (about 1.2 GB at T=16384, d=4096, 8 x 1376, k=2). */
+typedef struct {
+    const void *dy;    /* [T][d] dl/dy */
+    void *dx;          /* [T][d] out: dl/dx (complete: experts and router) */
+    float *dWg;        /* [d][E] out */
+    float *dWnoise;    /* [d][E] out, NULL iff the layer has no noise term */
+    float *dbias;      /* [E] out, NULL iff the layer has no bias */
+    void *dW13_e;      /* out, packed like W13_e */
+    void *dW2_e;       /* out, packed like W2_e */
+    void *d_out;       /* [T*k][d] intermediate: dl/d out */
+    float *dG;         /* [T][k] intermediate: dl/d topk_w */
+    void *dh;          /* [T*k][m8] intermediate: dl/dh */
+    void *dx_perm;     /* [T*k][d] intermediate: the experts' part of dl/dx, per row */
+} moe_bwd_buffers_t;
+
+size_t moe_backward_workspace_size(const moe_params_t *p);
+
+/* Combine backward: d_out [T*k][d] (rows of kept slots) and dG [T][k] f32. */
+int moe_combine_backward(const moe_params_t *p, const void *dy, const void *out,
+                         const int32_t *slot_row, const float *topk_w, void *d_out, float *dG,
+                         void *stream);
+
+/* Expert GEMM 2 backward: dh [T*k][m8] and dW2_e (packed).  Transposes W2_e and
+ * the activations into the workspace for the tensor-core GEMMs. */
+int moe_expert_down_backward(const moe_params_t *p, const void *d_out, const void *h,
+                             const int32_t *offsets, const void *W2_e, void *dh, void *dW2_e,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/* Expert GEMM 1 + SwiGLU backward: recomputes g, u, forms dg, du, then
+ * dx_perm [T*k][d] and dW13_e (packed). */
+int moe_expert_up_backward(const moe_params_t *p, const void *x_perm, const void *dh,
+                           const int32_t *offsets, const void *W13_e, void *dx_perm,
+                           void *dW13_e, void *ws, size_t ws_bytes, void *stream);
+
+/* Router backward and the input gradient: dx [T][d] (overwritten with the full
+ * gradient: expert rows through slot_row plus the router term), dWg, dWnoise,
+ * dbias (f32).  Wnoise, noise and dWnoise are given together or all NULL; bias
+ * and dbias likewise.  counts [E] are the routed counts of the forward. */
+int moe_route_backward(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
+                       const float *noise, const float *bias, const int32_t *topk_idx,
+                       const float *topk_w, const float *dG, const int32_t *counts, float dLb,
+                       const void *dx_perm, const int32_t *slot_row, void *dx, float *dWg,
+                       float *dWnoise, float *dbias, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole backward: combine, GEMM 2, GEMM 1 + SwiGLU, router and input, on one
+ * stream.  b holds the forward's inputs and intermediates of the same batch. */
+int moe_backward(const moe_params_t *p, const moe_buffers_t *b, const moe_bwd_buffers_t *g,
+                 float dLb, void *ws, size_t ws_bytes, void *stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
  * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
  * the workspace's internal launch counters. */

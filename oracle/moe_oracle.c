@@ -734,29 +734,43 @@ int oracle_expert_ffn_backward(int d, int m, int E, const void *W1e, const void 
             dx_rows[(size_t)r * d + c] = acc;
         }
     }
-    /* weight gradients: each entry sums its rows in ascending order */
-#pragma omp parallel for schedule(static)
-    for (int e = 0; e < E; ++e) {
-        for (int i = 0; i < m; ++i)
+    /* weight gradients: each entry sums the rows of its expert in ascending order */
+    int32_t *rows_of = (int32_t *)malloc(sizeof(int32_t) * ((size_t)n + 1));
+    int32_t *start = (int32_t *)calloc((size_t)E + 1, sizeof(int32_t));
+    if (!rows_of || !start) {
+        free(X), free(Hh), free(Dg), free(Du), free(rows_of), free(start);
+        return ORC_EINVAL;
+    }
+    for (int e = 0, pos = 0; e < E; ++e) {
+        start[e] = pos;
+        for (int r = 0; r < n; ++r)
+            if (expert_of_row[r] == e)
+                rows_of[pos++] = r;
+        start[e + 1] = pos;
+    }
+#pragma omp parallel for schedule(static) collapse(2)
+    for (int e = 0; e < E; ++e)
+        for (int i = 0; i < m; ++i) {
             for (int c = 0; c < d; ++c) {
                 double a1 = 0.0, a3 = 0.0;
-                for (int r = 0; r < n; ++r)
-                    if (expert_of_row[r] == e) {
-                        a1 += Dg[(size_t)r * m + i] * X[(size_t)r * d + c];
-                        a3 += Du[(size_t)r * m + i] * X[(size_t)r * d + c];
-                    }
+                for (int q = start[e]; q < start[e + 1]; ++q) {
+                    int r = rows_of[q];
+                    a1 += Dg[(size_t)r * m + i] * X[(size_t)r * d + c];
+                    a3 += Du[(size_t)r * m + i] * X[(size_t)r * d + c];
+                }
                 dW1e[((size_t)e * m + i) * d + c] = a1;
                 dW3e[((size_t)e * m + i) * d + c] = a3;
             }
-        for (int o = 0; o < d; ++o)
-            for (int i = 0; i < m; ++i) {
+            for (int o = 0; o < d; ++o) {
                 double a2 = 0.0;
-                for (int r = 0; r < n; ++r)
-                    if (expert_of_row[r] == e)
-                        a2 += d_out[(size_t)r * d + o] * Hh[(size_t)r * m + i];
+                for (int q = start[e]; q < start[e + 1]; ++q) {
+                    int r = rows_of[q];
+                    a2 += d_out[(size_t)r * d + o] * Hh[(size_t)r * m + i];
+                }
                 dW2e[((size_t)e * d + o) * m + i] = a2;
             }
-    }
+        }
+    free(rows_of), free(start);
     if (dg_out)
         memcpy(dg_out, Dg, sizeof(double) * (size_t)n * m);
     if (du_out)

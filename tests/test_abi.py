@@ -182,3 +182,26 @@ def test_cluster_rejects_bad_arguments_before_the_device(L):
     assert call(d_ff=30) == moe.MOE_ERR_SHAPE
     assert call(nb=100) == moe.MOE_ERR_WORKSPACE
     assert b"workspace" in L.moe_last_error_string()
+
+
+def test_backward_rejects_bad_arguments_before_the_device(L):
+    p = moe.params(64, 256, 8, 2, 128)
+    a = C.c_void_p(256)
+    n = L.moe_backward_workspace_size(C.byref(p))
+    assert n > 0
+    assert L.moe_backward_workspace_size(C.byref(moe.params(128, 256, 8, 2, 128))) > n
+    assert L.moe_backward_workspace_size(C.byref(moe.params(0, 256, 8, 2, 128))) == 0
+    pf = moe.params(64, 256, 8, 2, 128, dtype=moe.MOE_F32)
+    assert L.moe_combine_backward(C.byref(pf), a, a, a, a, a, a, None) == moe.MOE_ERR_DTYPE
+    assert L.moe_combine_backward(C.byref(p), None, a, a, a, a, a, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine_backward(C.byref(p), C.c_void_p(258), a, a, a, a, a, None) == \
+        moe.MOE_ERR_ALIGN
+    assert L.moe_expert_down_backward(C.byref(p), a, a, a, a, a, a, a, n - 1, None) == \
+        moe.MOE_ERR_WORKSPACE
+    assert L.moe_expert_up_backward(C.byref(p), a, a, a, a, a, None, a, n, None) == \
+        moe.MOE_ERR_INVALID_ARG
+    # noise inputs and their gradient go together
+    assert L.moe_route_backward(C.byref(p), a, a, a, None, None, a, a, a, a, C.c_float(1.0), a,
+                                a, a, a, None, None, a, n, None) == moe.MOE_ERR_INVALID_ARG
+    assert b"together" in L.moe_last_error_string()

@@ -1,0 +1,146 @@
+"""Backward of the MoE layer on the GPU against the fp64 oracle's backward (itself
+pinned by finite differences): the gradient of l(y) + c L_balance given dy, for the
+combine, the two expert GEMMs with the SwiGLU backward, the router (Mixtral / ST,
+softplus noise, balance term) and the input.  bf16 gradients: max|err| / max|ref|
+<= 2e-2 (bf16 rounding of out, h, d_out, dh, dGU on the GPU against f64)."""
+import numpy as np
+import pytest
+import torch
+
+import harness as H
+import oracle
+import top_routing_grouped_noisy_b200 as moe
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+W = wl.Workload
+CASES = {
+    "bwd_mid": W("bwd_mid", T=1000, d=512, d_ff=2752, E=8, k=2, noisy=True, rescale=True,
+                 lam=0.01, seed=80),
+    "bwd_st_bias_cap": W("bwd_st_bias_cap", T=700, d=256, d_ff=1024, E=8, k=2, router=wl.ST,
+                         noisy=True, bias=True, cf=1.0, rescale=True, lam=0.05, seed=81),
+    "bwd_ragged": W("bwd_ragged", T=333, d=200, d_ff=400, E=4, k=2, noisy=True, seed=82),
+    "bwd_decode": W("bwd_decode", T=8, d=256, d_ff=1088, E=8, k=2, rescale=True, seed=83),
+    "bwd_e16k4": W("bwd_e16k4", T=512, d=256, d_ff=1024, E=16, k=4, router=wl.ST, noisy=True,
+                   bias=True, lam=0.01, seed=84),
+    "bwd_copy": W("bwd_copy", T=256, d=128, d_ff=256, E=4, k=2, partition=wl.COPY, seed=85),
+    "bwd_e64": W("bwd_e64", T=300, d=128, d_ff=1024, E=64, k=2, noisy=True, bias=True, lam=0.05,
+                 seed=87),
+    "bwd_e12_ragged_d": W("bwd_e12_ragged_d", T=150, d=72, d_ff=480, E=12, k=3, router=wl.ST,
+                          noisy=True, seed=88),
+}
+
+
+def rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
+
+
+def _run(w, inp, dLb=1.0):
+    dev = "cuda"
+    p, bufs, ws, st, (W13_e, W2_e) = H.run_forward(w, inp)
+    assert st == 0
+    g = lambda n: None if inp.get(n) is None else inp[n].to(dev)
+    dy = wl.make_grad_output(w, w.seed + 1).to(dev)
+    gb = moe.BackwardBuffers(p, w.noisy, w.bias)
+    wsb = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
+    moe.moe_backward(p, g("x"), g("Wg"), W13_e, W2_e, bufs, gb, dy, wsb, Wnoise=g("Wnoise"),
+                     noise=g("eps"), bias=g("bias"), dLb=dLb)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(wsb) == 0
+    return p, bufs, gb, dy
+
+
+def _oracle(w, inp, dy, dLb=1.0):
+    W1e, W3e, W2e = H.oracle_weights(w, inp)
+    r = lambda n: None if inp.get(n) is None else H.raw(inp[n])
+    eps = None if inp.get("eps") is None else inp["eps"].numpy()
+    bias = None if inp.get("bias") is None else inp["bias"].numpy()
+    rt = oracle.MIXTRAL if w.router == wl.MIXTRAL else oracle.ST
+    return oracle.backward(H.raw(inp["x"]), H.raw(inp["Wg"]), W1e, W3e, W2e, w.k, H.f64(dy), rt,
+                           r("Wnoise"), eps, bias, H.capacity_of(w), w.rescale, w.lam, dLb)
+
+
+def _check(w, inp, p, bufs, gb, dy, dLb=1.0):
+    ref = _oracle(w, inp, dy.cpu(), dLb)
+    fwd = ref["fwd"]
+    idx = bufs.topk_idx.cpu().numpy()
+    assert (idx == fwd["router"]["idx"]).all(), "routing differs: pick a seed without near ties"
+    R = int(fwd["dispatch"]["R"])
+    assert int(bufs.offsets[-1]) == R
+    m, d, E = w.m, w.d, w.E
+    errs = {
+        "dG": rel(gb.dG.cpu().numpy(), ref["dG"]),
+        "d_out": rel(H.f64(gb.d_out[:R]), ref["d_out"]),
+        "dh": rel(H.f64(gb.dh[:R, :m]), ref["dh"]),
+        "dx_perm": rel(H.f64(gb.dx_perm[:R]), ref["dx_rows"]),
+        "dx": rel(H.f64(gb.dx), ref["dx"]),
+        "dWg": rel(gb.dWg.cpu().numpy(), ref["dWg"]),
+    }
+    dW1, dW3 = H.unpack_w13(gb.dW13_e, E, m, d)
+    errs["dW1e"] = rel(H.f64(dW1), ref["dW1e"])
+    errs["dW3e"] = rel(H.f64(dW3), ref["dW3e"])
+    errs["dW2e"] = rel(H.f64(H.unpack_w2(gb.dW2_e, E, m, d)), ref["dW2e"])
+    if gb.dWnoise is not None:
+        errs["dWnoise"] = rel(gb.dWnoise.cpu().numpy(), ref["dWnoise"])
+    if gb.dbias is not None:
+        errs["dbias"] = rel(gb.dbias.cpu().numpy(), ref["dbias"])
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, (w.name, errs)
+    # the padding of the packed gradients is zero, like the packed weights
+    m16, m8 = (m + 15) // 16 * 16, (m + 7) // 8 * 8
+    A = gb.dW13_e.view(E, m16 // 16, 2, 16, d).permute(0, 2, 1, 3, 4).reshape(E, 2, m16, d)
+    assert (A[:, :, m:] == 0).all()
+    assert (gb.dW2_e.view(E, d, m8)[:, :, m:] == 0).all()
+    return errs
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_parity(name):
+    w = CASES[name]
+    inp = wl.make_inputs(w)
+    p, bufs, gb, dy = _run(w, inp)
+    _check(w, inp, p, bufs, gb, dy)
+
+
+def test_expert_without_rows_gets_zero_gradient():
+    """A large negative bias keeps the last expert unselected: its weight gradient
+    (the K-grouped GEMM with no K blocks) is zero, the others match the oracle."""
+    w = W("bwd_idle", T=300, d=256, d_ff=1024, E=8, k=2, noisy=True, bias=True, lam=0.02,
+          seed=86)
+    inp = wl.make_inputs(w)
+    inp["bias"][w.E - 1] = -1.0e4
+    p, bufs, gb, dy = _run(w, inp)
+    assert int(bufs.counts[w.E - 1]) == 0
+    dW1, dW3 = H.unpack_w13(gb.dW13_e, w.E, w.m, w.d)
+    assert (dW1[w.E - 1] == 0).all() and (dW3[w.E - 1] == 0).all()
+    assert (H.unpack_w2(gb.dW2_e, w.E, w.m, w.d)[w.E - 1] == 0).all()
+    _check(w, inp, p, bufs, gb, dy)
+
+
+def test_steps_equal_the_whole_backward():
+    """The step calls in order give bit-identical results to moe_backward."""
+    w = CASES["bwd_st_bias_cap"]
+    inp = wl.make_inputs(w)
+    p, bufs, gb, dy = _run(w, inp)
+    dev = "cuda"
+    g = lambda n: None if inp.get(n) is None else inp[n].to(dev)
+    W13_e, W2_e = H.gpu_weights(w, inp)
+    s = moe.BackwardBuffers(p, w.noisy, w.bias)
+    ws = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
+    moe.moe_combine_backward(p, dy, bufs.out, bufs.slot_row, bufs.topk_w, s.d_out, s.dG)
+    moe.moe_expert_down_backward(p, s.d_out, bufs.h, bufs.offsets, W2_e, s.dh, s.dW2_e, ws)
+    moe.moe_expert_up_backward(p, bufs.x_perm, s.dh, bufs.offsets, W13_e, s.dx_perm, s.dW13_e,
+                               ws)
+    moe.moe_route_backward(p, g("x"), g("Wg"), bufs.topk_idx, bufs.topk_w, s.dG, bufs.counts,
+                           s.dx_perm, bufs.slot_row, s.dx, s.dWg, ws, Wnoise=g("Wnoise"),
+                           noise=g("eps"), bias=g("bias"), dWnoise=s.dWnoise, dbias=s.dbias)
+    torch.cuda.synchronize()
+    for n in ("dx", "dWg", "dWnoise", "dbias", "dW13_e", "dW2_e", "dG"):
+        assert torch.equal(getattr(s, n), getattr(gb, n)), n
+    R = int(bufs.offsets[-1])  # row buffers: rows past R are unused
+    for n in ("d_out", "dh", "dx_perm"):
+        assert torch.equal(getattr(s, n)[:R], getattr(gb, n)[:R]), n

@@ -21,7 +21,9 @@ __all__ = [
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
     "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline", "moe_partition_residual",
     "moe_combine_residual", "moe_forward_residual", "moe_cluster_workspace_size",
-    "moe_cluster_partition", "moe_cluster_distances",
+    "moe_cluster_partition", "moe_cluster_distances", "moe_backward_workspace_size",
+    "moe_combine_backward", "moe_expert_down_backward", "moe_expert_up_backward",
+    "moe_route_backward", "moe_backward", "BackwardBuffers",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -66,6 +68,14 @@ _BUF_FIELDS = ["x", "Wg", "Wnoise", "noise", "bias", "W13_e", "W2_e", "y", "loss
 
 class _Buffers(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in _BUF_FIELDS]
+
+
+_BWD_FIELDS = ["dy", "dx", "dWg", "dWnoise", "dbias", "dW13_e", "dW2_e", "d_out", "dG", "dh",
+               "dx_perm"]
+
+
+class _BwdBuffers(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in _BWD_FIELDS]
 
 
 _lib = None
@@ -114,6 +124,14 @@ def lib():
             "moe_cluster_partition": (C.c_int, [v, i32, i32, i32, i32, i32, v, v, v, v, v, sz,
                                                 v]),
             "moe_cluster_distances": (C.c_int, [v, i32, i32, i32, i32, v, v, v]),
+            "moe_backward_workspace_size": (sz, [P]),
+            "moe_combine_backward": (C.c_int, [P, v, v, v, v, v, v, v]),
+            "moe_expert_down_backward": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
+            "moe_expert_up_backward": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
+            "moe_route_backward": (C.c_int, [P, v, v, v, v, v, v, v, v, v, C.c_float, v, v, v,
+                                             v, v, v, v, sz, v]),
+            "moe_backward": (C.c_int, [P, C.POINTER(_Buffers), C.POINTER(_BwdBuffers),
+                                       C.c_float, v, sz, v]),
             "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
             "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
             "moe_pipeline_wait": (C.c_int, [v, i64]),
@@ -464,3 +482,70 @@ def moe_cluster_distances(F, centers, out=None, stream=None):
     _check(lib().moe_cluster_distances(_p(F), d, d_ff, E, _dtype_code(F.dtype), _p(centers),
                                        _p(D), _stream(stream)))
     return D
+
+
+# --------------------------------------------------------------------------- backward
+
+def moe_backward_workspace_size(p) -> int:
+    return int(lib().moe_backward_workspace_size(C.byref(p)))
+
+
+class BackwardBuffers:
+    """Outputs and intermediates of moe_backward for layer p (include/moe.h)."""
+
+    def __init__(self, p: Params, noisy: bool, biased: bool, device="cuda"):
+        T, d, E, k = p.T, p.d, p.E, p.k
+        dt = torch.bfloat16
+        f32 = dict(dtype=torch.float32, device=device)
+        rows = max(T * k, 1)
+        self.dx = torch.empty(T, d, dtype=dt, device=device)
+        self.dWg = torch.empty(d, E, **f32)
+        self.dWnoise = torch.empty(d, E, **f32) if noisy else None
+        self.dbias = torch.empty(E, **f32) if biased else None
+        self.dW13_e = torch.empty(packed_w13_elems(E, p.m, d), dtype=dt, device=device)
+        self.dW2_e = torch.empty(packed_w2_elems(E, p.m, d), dtype=dt, device=device)
+        self.d_out = torch.empty(rows, d, dtype=dt, device=device)
+        self.dG = torch.empty(T, k, **f32)
+        self.dh = torch.empty(rows, h_ld(p.m), dtype=dt, device=device)
+        self.dx_perm = torch.empty(rows, d, dtype=dt, device=device)
+
+
+def moe_combine_backward(p, dy, out, slot_row, topk_w, d_out, dG, stream=None):
+    _check(lib().moe_combine_backward(C.byref(p), _p(dy), _p(out), _p(slot_row), _p(topk_w),
+                                      _p(d_out), _p(dG), _stream(stream)))
+
+
+def moe_expert_down_backward(p, d_out, h, offsets, W2_e, dh, dW2_e, ws, stream=None):
+    _check(lib().moe_expert_down_backward(C.byref(p), _p(d_out), _p(h), _p(offsets), _p(W2_e),
+                                          _p(dh), _p(dW2_e), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def moe_expert_up_backward(p, x_perm, dh, offsets, W13_e, dx_perm, dW13_e, ws, stream=None):
+    _check(lib().moe_expert_up_backward(C.byref(p), _p(x_perm), _p(dh), _p(offsets), _p(W13_e),
+                                        _p(dx_perm), _p(dW13_e), ws.ptr, ws.nbytes,
+                                        _stream(stream)))
+
+
+def moe_route_backward(p, x, Wg, topk_idx, topk_w, dG, counts, dx_perm, slot_row, dx, dWg, ws,
+                       Wnoise=None, noise=None, bias=None, dWnoise=None, dbias=None, dLb=1.0,
+                       stream=None):
+    _check(lib().moe_route_backward(C.byref(p), _p(x), _p(Wg), _p(Wnoise), _p(noise), _p(bias),
+                                    _p(topk_idx), _p(topk_w), _p(dG), _p(counts), float(dLb),
+                                    _p(dx_perm), _p(slot_row), _p(dx), _p(dWg), _p(dWnoise),
+                                    _p(dbias), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def moe_backward(p, x, Wg, W13_e, W2_e, fwd: "ForwardBuffers", g: BackwardBuffers, dy, ws,
+                 Wnoise=None, noise=None, bias=None, dLb=1.0, stream=None):
+    """The whole backward of the batch whose forward filled `fwd` (include/moe.h)."""
+    b = _Buffers()
+    vals = dict(x=x, Wg=Wg, Wnoise=Wnoise, noise=noise, bias=bias, W13_e=W13_e, W2_e=W2_e)
+    for n in _BUF_FIELDS:
+        t = vals[n] if n in vals else getattr(fwd, n)
+        setattr(b, n, _p(t))
+    gb = _BwdBuffers()
+    for n in _BWD_FIELDS:
+        setattr(gb, n, _p(dy if n == "dy" else getattr(g, n)))
+    _check(lib().moe_backward(C.byref(p), C.byref(b), C.byref(gb), float(dLb), ws.ptr, ws.nbytes,
+                              _stream(stream)))
+    return g

@@ -153,3 +153,10 @@ def make_cluster_init(d_ff: int, E: int, seed: int) -> torch.Tensor:
     g = torch.Generator()
     g.manual_seed(seed)
     return torch.randperm(d_ff, generator=g)[:E].to(torch.int32).contiguous()
+
+
+def make_grad_output(w: Workload, seed: int, device: str = "cpu") -> torch.Tensor:
+    """dl/dy for the backward pass: N(0, 1) entries [T][d] in the workload's dtype."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn(w.T, w.d, generator=g, device=device).to(torch_dtype(w))
