@@ -481,20 +481,32 @@ def run_cluster(args, rank, world, local):
     return 0
 
 
-def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp, rank,
-              world, local):
+def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp, shared,
+              rank, world, local):
     """A training step of the layer: the forward (the six step calls) and the backward
     (combine, expert GEMM 2, expert GEMM 1 + SwiGLU, router + input) for l(y) + L_balance
     with a seeded dl/dy.  The roofline figure is moe_expert_up_backward, timed inside the
     step loop: three tcgen05 GEMMs (g/u recompute with the SwiGLU backward, dgrad,
-    wgrad) plus the transposes that feed the weight-gradient GEMM."""
-    if w.dtype != "bf16" or w.shared > 0:
-        raise SystemExit("--backward runs bf16 layers without a shared block")
+    wgrad) plus the transposes that feed the weight-gradient GEMM.  For a residual layer
+    (shared neurons) the backward is the one call moe_backward_residual, which is then
+    the roofline figure (its 16 d m R + 16 d m_s T FLOP)."""
+    if w.dtype != "bf16":
+        raise SystemExit("--backward runs bf16 layers")
     stream = torch.cuda.current_stream()
     dy = wl.make_grad_output(w, w.seed + 1 + 7919 * rank, device="cuda")
     g = moe.BackwardBuffers(p, Wn is not None, bias is not None)
-    wsb = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
-    SEG = ["forward", "combine_bwd", "down_bwd", "up_bwd", "route_bwd"]
+    res = shared is not None
+    if res:
+        W13_s, W2_s, h_s = shared
+        dh_s = torch.empty_like(h_s)
+        dx_s = torch.empty(w.T, w.d, dtype=torch.bfloat16, device="cuda")
+        dW13_s = torch.empty_like(W13_s)
+        dW2_s = torch.empty_like(W2_s)
+        wsb = moe.Workspace(p, nbytes=moe.moe_backward_residual_workspace_size(p, w.shared))
+    else:
+        wsb = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
+    SEG = ["forward", "backward"] if res else ["forward", "combine_bwd", "down_bwd", "up_bwd",
+                                              "route_bwd"]
 
     def step(ev=None, up=None):
         def mark(i):
@@ -503,6 +515,16 @@ def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C
         mark(0)
         fwd_step()
         mark(1)
+        if res:
+            if up is not None:
+                up[0].record(stream)
+            moe.moe_backward_residual(p, x, Wg, W13_e, W2_e, W13_s, W2_s, w.shared, h_s, b, g,
+                                      dy, dh_s, dx_s, dW13_s, dW2_s, wsb, Wnoise=Wn, noise=eps,
+                                      bias=bias, dLb=1.0)
+            if up is not None:
+                up[1].record(stream)
+            mark(2)
+            return
         moe.moe_combine_backward(p, dy, b.out, b.slot_row, b.topk_w, g.d_out, g.dG)
         mark(2)
         moe.moe_expert_down_backward(p, g.d_out, b.h, b.offsets, W2_e, g.dh, g.dW2_e, wsb)
@@ -562,18 +584,23 @@ def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C
     seg = [max_over_ranks(v / nseg, world) for v in seg]
     value = tokens_per_s(w.T, args.steps, world, ms)
     dmr = float(w.d) * w.m * R
-    flop_step = 22.0 * dmr  # forward 6, GEMM 2 backward 4, GEMM 1 backward 12 (with recompute)
+    dms = float(w.d) * w.shared * w.T  # shared block (residual layer), every token
+    # forward 6, GEMM 2 backward 4, GEMM 1 backward 12 (with recompute); same for the block
+    flop_step = 22.0 * (dmr + dms)
     peaks, peak_src = load_peaks()
     peak_t = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    up_tf = 12.0 * dmr / (up_ms / 1000.0) / 1e12
+    up_flop = 16.0 * (dmr + dms) if res else 12.0 * dmr
+    up_tf = up_flop / (up_ms / 1000.0) / 1e12
     kernels = {n: {"ms": v} for n, v in zip(SEG, seg)}
-    kernels["down_bwd"]["TFLOP/s"] = 4.0 * dmr / (seg[2] / 1000.0) / 1e12
-    kernels["up_bwd"]["TFLOP/s"] = 12.0 * dmr / (seg[3] / 1000.0) / 1e12
-    kernels["forward"]["TFLOP/s"] = 6.0 * dmr / (seg[0] / 1000.0) / 1e12
+    kernels["forward"]["TFLOP/s"] = 6.0 * (dmr + dms) / (seg[0] / 1000.0) / 1e12
+    if res:
+        kernels["backward"]["TFLOP/s"] = up_tf
+    else:
+        kernels["down_bwd"]["TFLOP/s"] = 4.0 * dmr / (seg[2] / 1000.0) / 1e12
+        kernels["up_bwd"]["TFLOP/s"] = 12.0 * dmr / (seg[3] / 1000.0) / 1e12
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not res:
         import oracle
-        sys.path.insert(0, os.path.join(ROOT, "tests"))
         n_s = 128
         sub = {k2: (v[:n_s].cpu() if k2 in ("x", "eps") and v is not None else
                     (v.cpu() if isinstance(v, torch.Tensor) else v)) for k2, v in inp.items()}
@@ -608,13 +635,16 @@ def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C
         "config": dict(config_of(w, C), parallelism="dp%d replicas" % world, kept_rows=R,
                        loss="sum(y * dy) + L_balance, dy ~ N(0,1) seeded"),
         "tflops": flop_step * args.steps * world / (ms / 1000.0) / 1e12,
-        "roofline": {"kernel": "moe_expert_up_backward: bwd_gemm_kernel x3 (recompute + SwiGLU "
-                               "backward, dgrad, wgrad) + 3 transposes",
+        "roofline": {"kernel": ("moe_backward_residual: the routed and the shared block's "
+                                "backward GEMMs + transposes + router" if res else
+                                "moe_expert_up_backward: bwd_gemm_kernel x3 (recompute + SwiGLU "
+                                "backward, dgrad, wgrad) + 3 transposes"),
                      "bound": "tensor", "achieved": up_tf, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": up_tf / peak_t, "traffic": None,
                      "peak_source": "%s bf16_tflops_sustained" % peak_src,
-                     "algorithmic": "12*d*m FLOP per kept row x R=%d = %.4g FLOP per call"
-                                    % (R, 12.0 * dmr)},
+                     "algorithmic": ("16*d*(m*R + m_s*T) = %.4g FLOP per call" % up_flop
+                                     if res else "12*d*m FLOP per kept row x R=%d = %.4g FLOP "
+                                     "per call" % (R, up_flop))},
         "kernels": kernels, "cpu_baseline": cpu, "e2e": None, "gpu_launches": launches,
         "clocks": clocks,
     }
@@ -761,7 +791,7 @@ def main():
 
     if args.backward:
         return run_train(args, w, p, moe, step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp,
-                         rank, world, local)
+                         (W13_s, W2_s, h_s) if res else None, rank, world, local)
     if w.T <= 64:
         return run_decode(args, w, p, moe, ws, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, rank,
                           world, local)

@@ -424,6 +424,20 @@ int moe_route_backward(const moe_params_t *p, const void *x, const void *Wg, con
 int moe_backward(const moe_params_t *p, const moe_buffers_t *b, const moe_bwd_buffers_t *g,
                  float dLb, void *ws, size_t ws_bytes, void *stream);
 
+/* Backward of the residual MoE layer y = FFN_S(x) + s sum_j G_j E_j(x) (see
+ * moe_forward_residual): the routed part as moe_backward, and the shared block
+ * FFN_S, whose output gradient is dy itself, as the backward of a one-expert layer
+ * over all T tokens.  b and g as for moe_backward (b->x, b->out etc. of the routed
+ * part of the same forward); h_s [T][m_s8] is the shared block's forward
+ * activation; outputs dh_s [T][m_s8], dx_s [T][d] (the shared block's part of dx;
+ * g->dx receives the whole input gradient), dW13_s / dW2_s (packed like W13_s /
+ * W2_s).  ws: moe_backward_residual_workspace_size(p, m_s) bytes. */
+size_t moe_backward_residual_workspace_size(const moe_params_t *p, int32_t m_s);
+int moe_backward_residual(const moe_params_t *p, const moe_buffers_t *b,
+                          const moe_bwd_buffers_t *g, const void *W13_s, const void *W2_s,
+                          int32_t m_s, const void *h_s, void *dh_s, void *dx_s, void *dW13_s,
+                          void *dW2_s, float dLb, void *ws, size_t ws_bytes, void *stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
  * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
  * the workspace's internal launch counters. */

@@ -424,3 +424,22 @@ def backward(x, Wg, W1e, W3e, W2e, k, dy, router_type=MIXTRAL, Wnoise=None, eps=
                 dW1e=eb["dW1e"], dW3e=eb["dW3e"], dW2e=eb["dW2e"], d_out=d_out, dG=dG,
                 dh=eb["dh"], dg=eb["dg"], du=eb["du"], dx_rows=eb["dx_rows"], dH=rb["dH"],
                 dN=rb["dN"], fwd=f)
+
+
+def backward_residual(x, Wg, experts, shared_block, k, dy, router_type=MIXTRAL, Wnoise=None,
+                      eps=None, bias=None, capacity_rows=-1, rescale=False, lam=0.0, dLb=1.0):
+    """Gradients of the residual MoE layer y = FFN_S(x) + s sum_j G_j E_j(x): the routed
+    layer's backward() plus the shared block's (an expert over every token whose output
+    gradient is dy).  Adds dx_s, dW1s, dW3s, dW2s, dh_s to backward()'s dict; dx is the
+    total."""
+    g = backward(x, Wg, *experts, k, dy, router_type, Wnoise, eps, bias, capacity_rows,
+                 rescale, lam, dLb)
+    W1s, W3s, W2s = shared_block
+    T = x.shape[0]
+    sb = expert_ffn_backward(np.ascontiguousarray(W1s)[None], np.ascontiguousarray(W3s)[None],
+                             np.ascontiguousarray(W2s)[None], x, np.zeros(T, np.int32), dy)
+    g["dx_s"] = sb["dx_rows"]
+    g["dx"] = g["dx"] + sb["dx_rows"]
+    g["dW1s"], g["dW3s"], g["dW2s"] = sb["dW1e"][0], sb["dW3e"][0], sb["dW2e"][0]
+    g["dh_s"] = sb["dh"]
+    return g

@@ -144,3 +144,72 @@ def test_steps_equal_the_whole_backward():
     R = int(bufs.offsets[-1])  # row buffers: rows past R are unused
     for n in ("d_out", "dh", "dx_perm"):
         assert torch.equal(getattr(s, n)[:R], getattr(gb, n)[:R]), n
+
+
+# --------------------------------------------------------------------------- residual layer
+
+RES_CASES = {
+    "res_bwd_mid": W("res_bwd_mid", T=600, d=256, d_ff=1152, E=8, k=2, noisy=True, rescale=True,
+                     shared=128, lam=0.02, seed=90),
+    "res_bwd_st_cap": W("res_bwd_st_cap", T=400, d=200, d_ff=840, E=4, k=2, router=wl.ST,
+                        noisy=True, bias=True, cf=1.0, shared=40, seed=91),
+}
+
+
+@pytest.mark.parametrize("name", list(RES_CASES))
+def test_residual_backward_parity(name):
+    """y = FFN_S(x) + s sum G E(x): the routed gradients, the shared block's weight
+    gradients and the total dx against the oracle."""
+    w = RES_CASES[name]
+    inp = wl.make_inputs(w)
+    dev = "cuda"
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    g = lambda n: None if inp.get(n) is None else inp[n].to(dev)
+    W13_e, W2_e, W13_s, W2_s = moe.moe_partition_residual(
+        g("W1"), g("W3"), g("W2"), w.E, g("shared_idx"), g("perm_rest"), ws=ws)
+    b = moe.ForwardBuffers(p)
+    h_s = torch.empty(w.T, moe.h_ld(w.shared), dtype=torch.bfloat16, device=dev)
+    out_s = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
+    moe.moe_forward_residual(p, g("x"), g("Wg"), W13_e, W2_e, W13_s, W2_s, w.shared, ws, b, h_s,
+                             out_s, Wnoise=g("Wnoise"), noise=g("eps"), bias=g("bias"))
+    dy = wl.make_grad_output(w, w.seed + 1).to(dev)
+    gb = moe.BackwardBuffers(p, w.noisy, w.bias)
+    dh_s = torch.empty(w.T, moe.h_ld(w.shared), dtype=torch.bfloat16, device=dev)
+    dx_s = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=dev)
+    dW13_s = torch.empty(moe.packed_w13_elems(1, w.shared, w.d), dtype=torch.bfloat16,
+                         device=dev)
+    dW2_s = torch.empty(moe.packed_w2_elems(1, w.shared, w.d), dtype=torch.bfloat16, device=dev)
+    wsb = moe.Workspace(p, nbytes=moe.moe_backward_residual_workspace_size(p, w.shared))
+    moe.moe_backward_residual(p, g("x"), g("Wg"), W13_e, W2_e, W13_s, W2_s, w.shared, h_s, b, gb,
+                              dy, dh_s, dx_s, dW13_s, dW2_s, wsb, Wnoise=g("Wnoise"),
+                              noise=g("eps"), bias=g("bias"))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(wsb) == 0
+    raw = H.raw
+    experts, blk = oracle.partition_residual(raw(inp["W1"]), raw(inp["W3"]), raw(inp["W2"]),
+                                             w.E, raw(inp["shared_idx"]), raw(inp["perm_rest"]))
+    opt = lambda n: None if inp.get(n) is None else raw(inp[n])
+    ref = oracle.backward_residual(raw(inp["x"]), raw(inp["Wg"]), experts, blk, w.k,
+                                   H.f64(dy), w.router, opt("Wnoise"),
+                                   None if inp.get("eps") is None else inp["eps"].numpy(),
+                                   None if inp.get("bias") is None else inp["bias"].numpy(),
+                                   p.capacity, w.rescale, w.lam, 1.0)
+    assert (b.topk_idx.cpu().numpy() == ref["fwd"]["router"]["idx"]).all()
+    m_s, m, d, E = w.shared, w.m, w.d, w.E
+    dW1s, dW3s = H.unpack_w13(dW13_s, 1, m_s, d)
+    dW1, dW3 = H.unpack_w13(gb.dW13_e, E, m, d)
+    errs = {
+        "dx": rel(H.f64(gb.dx), ref["dx"]),
+        "dx_s": rel(H.f64(dx_s), ref["dx_s"]),
+        "dh_s": rel(H.f64(dh_s[:, :m_s]), ref["dh_s"]),
+        "dW1s": rel(H.f64(dW1s[0]), ref["dW1s"]),
+        "dW3s": rel(H.f64(dW3s[0]), ref["dW3s"]),
+        "dW2s": rel(H.f64(H.unpack_w2(dW2_s, 1, m_s, d)[0]), ref["dW2s"]),
+        "dW1e": rel(H.f64(dW1), ref["dW1e"]),
+        "dW3e": rel(H.f64(dW3), ref["dW3e"]),
+        "dW2e": rel(H.f64(H.unpack_w2(gb.dW2_e, E, m, d)), ref["dW2e"]),
+        "dWg": rel(gb.dWg.cpu().numpy(), ref["dWg"]),
+    }
+    bad = {k2: v for k2, v in errs.items() if not v <= TOL}
+    assert not bad, (name, errs)

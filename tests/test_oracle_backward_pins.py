@@ -126,3 +126,53 @@ def test_balance_gradient_closed_form(orc):
     np.testing.assert_allclose(g["dH"], ref, rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(g["dWg"], P["x"].astype(np.float64).T @ ref, rtol=1e-11,
                                atol=1e-14)
+
+
+def test_residual_backward_matches_central_differences(orc):
+    """Residual layer y = FFN_S(x) + s sum G E(x): finite differences of the oracle's
+    forward_residual for x, the router and both the shared and the routed weights."""
+    r = _rng(61)
+    f32 = np.float32
+    T, d, d_ff, E, k, m_s = 5, 8, 24, 4, 2, 8
+    x = r.standard_normal((T, d)).astype(f32)
+    Wg = (0.6 * r.standard_normal((d, E))).astype(f32)
+    W1 = (0.5 * r.standard_normal((d_ff, d))).astype(f32)
+    W3 = (0.5 * r.standard_normal((d_ff, d))).astype(f32)
+    W2 = (0.5 * r.standard_normal((d, d_ff))).astype(f32)
+    perm = r.permutation(d_ff).astype(np.int32)
+    shared, rest = perm[:m_s], perm[m_s:]
+    experts, blk = orc.partition_residual(W1, W3, W2, E, shared, rest)
+    experts = [e.astype(f32) for e in experts]
+    blk = [np.ascontiguousarray(b, f32) for b in blk]
+    dy = r.standard_normal((T, d))
+    lam, c = 0.2, 0.5
+
+    def loss(x_, Wg_, ex, bl):
+        f = orc.forward_residual(x_, Wg_, ex, bl, k, rescale=True, lam=lam)
+        return float((f["y"] * dy).sum() + c * f["L"])
+
+    g = orc.backward_residual(x, Wg, experts, blk, k, dy, rescale=True, lam=lam, dLb=c)
+    checks = [("x", x, g["dx"]), ("Wg", Wg, g["dWg"]), ("W1e", experts[0], g["dW1e"]),
+              ("W2e", experts[2], g["dW2e"]), ("W1s", blk[0], g["dW1s"]),
+              ("W3s", blk[1], g["dW3s"]), ("W2s", blk[2], g["dW2s"])]
+    for name, arr, G in checks:
+        for _ in range(5):
+            i = tuple(int(r.integers(0, s)) for s in arr.shape)
+            v = float(arr[i])
+            h = 2.0 ** -12 * max(1.0, abs(v))
+            vals = []
+            for vv in (np.float32(v + h), np.float32(v - h)):
+                a2 = arr.copy()
+                a2[i] = vv
+                args = {"x": x, "Wg": Wg, "ex": list(experts), "bl": list(blk)}
+                if name == "x":
+                    args["x"] = a2
+                elif name == "Wg":
+                    args["Wg"] = a2
+                elif name.endswith("e"):
+                    args["ex"][{"W1e": 0, "W2e": 2}[name]] = a2
+                else:
+                    args["bl"][{"W1s": 0, "W3s": 1, "W2s": 2}[name]] = a2
+                vals.append(loss(args["x"], args["Wg"], args["ex"], args["bl"]))
+            fd = (vals[0] - vals[1]) / (float(np.float32(v + h)) - float(np.float32(v - h)))
+            assert abs(fd - G[i]) <= 1e-6 * max(1.0, abs(fd)), (name, i, fd, G[i])

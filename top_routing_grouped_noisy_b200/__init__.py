@@ -24,6 +24,7 @@ __all__ = [
     "moe_cluster_partition", "moe_cluster_distances", "moe_backward_workspace_size",
     "moe_combine_backward", "moe_expert_down_backward", "moe_expert_up_backward",
     "moe_route_backward", "moe_backward", "BackwardBuffers",
+    "moe_backward_residual_workspace_size", "moe_backward_residual",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -132,6 +133,9 @@ def lib():
                                              v, v, v, v, sz, v]),
             "moe_backward": (C.c_int, [P, C.POINTER(_Buffers), C.POINTER(_BwdBuffers),
                                        C.c_float, v, sz, v]),
+            "moe_backward_residual_workspace_size": (sz, [P, i32]),
+            "moe_backward_residual": (C.c_int, [P, C.POINTER(_Buffers), C.POINTER(_BwdBuffers), v,
+                                                v, i32, v, v, v, v, v, C.c_float, v, sz, v]),
             "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
             "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
             "moe_pipeline_wait": (C.c_int, [v, i64]),
@@ -548,4 +552,26 @@ def moe_backward(p, x, Wg, W13_e, W2_e, fwd: "ForwardBuffers", g: BackwardBuffer
         setattr(gb, n, _p(dy if n == "dy" else getattr(g, n)))
     _check(lib().moe_backward(C.byref(p), C.byref(b), C.byref(gb), float(dLb), ws.ptr, ws.nbytes,
                               _stream(stream)))
+    return g
+
+
+def moe_backward_residual_workspace_size(p, m_s) -> int:
+    return int(lib().moe_backward_residual_workspace_size(C.byref(p), int(m_s)))
+
+
+def moe_backward_residual(p, x, Wg, W13_e, W2_e, W13_s, W2_s, m_s, h_s, fwd: "ForwardBuffers",
+                          g: BackwardBuffers, dy, dh_s, dx_s, dW13_s, dW2_s, ws, Wnoise=None,
+                          noise=None, bias=None, dLb=1.0, stream=None):
+    """Backward of the residual MoE layer (include/moe.h)."""
+    b = _Buffers()
+    vals = dict(x=x, Wg=Wg, Wnoise=Wnoise, noise=noise, bias=bias, W13_e=W13_e, W2_e=W2_e)
+    for n in _BUF_FIELDS:
+        t = vals[n] if n in vals else getattr(fwd, n)
+        setattr(b, n, _p(t))
+    gb = _BwdBuffers()
+    for n in _BWD_FIELDS:
+        setattr(gb, n, _p(dy if n == "dy" else getattr(g, n)))
+    _check(lib().moe_backward_residual(C.byref(p), C.byref(b), C.byref(gb), _p(W13_s), _p(W2_s),
+                                       int(m_s), _p(h_s), _p(dh_s), _p(dx_s), _p(dW13_s),
+                                       _p(dW2_s), float(dLb), ws.ptr, ws.nbytes, _stream(stream)))
     return g

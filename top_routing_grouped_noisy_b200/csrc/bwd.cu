@@ -409,7 +409,8 @@ __global__ void __launch_bounds__(256) router_backward_wreduce_kernel(
 // [NE2][d] (16-byte loads) into Ws [ne][cols] bf16; thread (token group tg,
 // column group ct) owns columns 8 ct .. 8 ct + 7 and tokens tg, tg + 256 / (cols
 // / 8), ...  Per element: the k expert rows in slot order, then the router term
-// over e2 ascending; f32, rounded to bf16 once.
+// over e2 ascending, then (residual layer) the shared block's input gradient; f32,
+// rounded to bf16 once.
 constexpr int kIgTokens = 128;
 
 __host__ __device__ inline int input_grad_cols(int E) { return E <= 24 ? 512 : (E <= 48 ? 256 : 128); }
@@ -417,7 +418,7 @@ __host__ __device__ inline int input_grad_cols(int E) { return E <= 24 ? 512 : (
 __global__ void __launch_bounds__(256) input_grad_kernel(
     const bf16 *__restrict__ dx_perm, const int32_t *__restrict__ slot_row,
     const bf16 *__restrict__ WT, int ne, const float *__restrict__ dLN, int T, int d, int E,
-    int k, bf16 *__restrict__ dx)
+    int k, const bf16 *__restrict__ resid, bf16 *__restrict__ dx)
 {
     pdl_wait();
     pdl_trigger();
@@ -472,6 +473,13 @@ __global__ void __launch_bounds__(256) input_grad_kernel(
 #pragma unroll
             for (int u = 0; u < 8; ++u)
                 a[u] += gl * wf[u];
+        }
+        if (resid != nullptr) {  // the shared block's input gradient (residual layer)
+            float f[8];
+            bf16x8_to_f32(ld_nc_na(resid + (int64_t)t * d + c), f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                a[u] += f[u];
         }
         st_v4(dx + (int64_t)t * d + c, f32x8_to_bf16(a));
     }
@@ -685,14 +693,15 @@ extern "C" int moe_expert_up_backward(const moe_params_t *p, const void *x_perm,
     return finish(fn, e);
 }
 
-extern "C" int moe_route_backward(const moe_params_t *p, const void *x, const void *Wg,
-                                  const void *Wnoise, const float *noise, const float *bias,
-                                  const int32_t *topk_idx, const float *topk_w, const float *dG,
-                                  const int32_t *counts, float dLb, const void *dx_perm,
-                                  const int32_t *slot_row, void *dx, float *dWg, float *dWnoise,
-                                  float *dbias, void *ws, size_t ws_bytes, void *stream)
+namespace {
+
+static int route_backward(const char *fn, const moe_params_t *p, const void *x, const void *Wg,
+                          const void *Wnoise, const float *noise, const float *bias,
+                          const int32_t *topk_idx, const float *topk_w, const float *dG,
+                          const int32_t *counts, float dLb, const void *dx_perm,
+                          const int32_t *slot_row, const void *resid, void *dx, float *dWg,
+                          float *dWnoise, float *dbias, void *ws, size_t ws_bytes, void *stream)
 {
-    const char *fn = "moe_route_backward";
     int rc = check_bwd(fn, p);
     if (rc != MOE_OK || (rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
         return rc;
@@ -706,6 +715,7 @@ extern "C" int moe_route_backward(const moe_params_t *p, const void *x, const vo
     NEED(slot_row);
     NEED(dx);
     NEED(dWg);
+    MAYBE(resid);
     MAYBE(Wnoise);
     MAYBE(noise);
     MAYBE(bias);
@@ -743,10 +753,24 @@ extern "C" int moe_route_backward(const moe_params_t *p, const void *x, const vo
                                dim3((p->d + cols - 1) / cols, (p->T + kIgTokens - 1) / kIgTokens),
                                dim3(256), smem, s, (const bf16 *)dx_perm, slot_row,
                                (const bf16 *)(w + L.wt), ne, (const float *)dLN, p->T, p->d,
-                               p->E, p->k, (bf16 *)dx);
+                               p->E, p->k, (const bf16 *)resid, (bf16 *)dx);
         }
     }
     return finish(fn, e);
+}
+
+}  // namespace
+
+extern "C" int moe_route_backward(const moe_params_t *p, const void *x, const void *Wg,
+                                  const void *Wnoise, const float *noise, const float *bias,
+                                  const int32_t *topk_idx, const float *topk_w, const float *dG,
+                                  const int32_t *counts, float dLb, const void *dx_perm,
+                                  const int32_t *slot_row, void *dx, float *dWg, float *dWnoise,
+                                  float *dbias, void *ws, size_t ws_bytes, void *stream)
+{
+    return route_backward("moe_route_backward", p, x, Wg, Wnoise, noise, bias, topk_idx, topk_w,
+                          dG, counts, dLb, dx_perm, slot_row, nullptr, dx, dWg, dWnoise, dbias,
+                          ws, ws_bytes, stream);
 }
 
 extern "C" int moe_backward(const moe_params_t *p, const moe_buffers_t *b,
@@ -768,5 +792,89 @@ extern "C" int moe_backward(const moe_params_t *p, const moe_buffers_t *b,
         rc = moe_route_backward(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx,
                                 b->topk_w, g->dG, b->counts, dLb, g->dx_perm, b->slot_row, g->dx,
                                 g->dWg, g->dWnoise, g->dbias, ws, ws_bytes, stream);
+    return rc;
+}
+
+// ---------------------------------------------------------------- residual layer
+// y = FFN_S(x) + s sum_j G_j E_j(x): the shared block's output gradient is dy
+// itself; its backward is the expert backward of a one-expert layer over all T
+// tokens (offsets {0, T}), and its input gradient joins dx in the input-gradient
+// kernel.
+
+namespace {
+
+moe_params_t shared_params(const moe_params_t *p, int32_t m_s)
+{
+    moe_params_t ps = *p;
+    ps.E = 1;
+    ps.k = 1;
+    ps.m = m_s;
+    ps.capacity = -1;
+    ps.rescale = 0;
+    return ps;
+}
+
+// words 8-9 of the backward workspace header: the offsets {0, T} of the shared block
+constexpr int kBwdTokenRangeWord = 8;
+
+}  // namespace
+
+extern "C" size_t moe_backward_residual_workspace_size(const moe_params_t *p, int32_t m_s)
+{
+    if (validate_params("moe_backward_residual_workspace_size", p) != MOE_OK || p->T < 1 ||
+        m_s < 1)
+        return 0;
+    const moe_params_t ps = shared_params(p, m_s);
+    const size_t a = bwd_layout(p).total, b = bwd_layout(&ps).total;
+    return a > b ? a : b;
+}
+
+extern "C" int moe_backward_residual(const moe_params_t *p, const moe_buffers_t *b,
+                                     const moe_bwd_buffers_t *g, const void *W13_s,
+                                     const void *W2_s, int32_t m_s, const void *h_s, void *dh_s,
+                                     void *dx_s, void *dW13_s, void *dW2_s, float dLb, void *ws,
+                                     size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_backward_residual";
+    if (b == nullptr || g == nullptr)
+        return fail_msg(MOE_ERR_INVALID_ARG, "%s: %s", fn, "buffers are NULL");
+    int rc = check_bwd(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    if (m_s < 1)
+        return fail_msg(MOE_ERR_SHAPE, "%s: %s", fn, "m_s must be >= 1");
+    NEED(ws);
+    if (ws_bytes < moe_backward_residual_workspace_size(p, m_s))
+        return fail_msg(MOE_ERR_WORKSPACE, "%s: %s", fn,
+                        "workspace smaller than moe_backward_residual_workspace_size()");
+    NEED(W13_s);
+    NEED(W2_s);
+    NEED(h_s);
+    NEED(dh_s);
+    NEED(dx_s);
+    NEED(dW13_s);
+    NEED(dW2_s);
+    const moe_params_t ps = shared_params(p, m_s);
+    int32_t *tok = reinterpret_cast<int32_t *>(ws) + kBwdTokenRangeWord;
+    cudaError_t e = launch_token_range(tok, p->T, (cudaStream_t)stream);
+    if (e != cudaSuccess)
+        return finish(fn, e);
+    rc = moe_expert_down_backward(&ps, g->dy, h_s, tok, W2_s, dh_s, dW2_s, ws, ws_bytes, stream);
+    if (rc == MOE_OK)
+        rc = moe_expert_up_backward(&ps, b->x, dh_s, tok, W13_s, dx_s, dW13_s, ws, ws_bytes,
+                                    stream);
+    if (rc == MOE_OK)
+        rc = moe_combine_backward(p, g->dy, b->out, b->slot_row, b->topk_w, g->d_out, g->dG,
+                                  stream);
+    if (rc == MOE_OK)
+        rc = moe_expert_down_backward(p, g->d_out, b->h, b->offsets, b->W2_e, g->dh, g->dW2_e, ws,
+                                      ws_bytes, stream);
+    if (rc == MOE_OK)
+        rc = moe_expert_up_backward(p, b->x_perm, g->dh, b->offsets, b->W13_e, g->dx_perm,
+                                    g->dW13_e, ws, ws_bytes, stream);
+    if (rc == MOE_OK)
+        rc = route_backward(fn, p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx,
+                            b->topk_w, g->dG, b->counts, dLb, g->dx_perm, b->slot_row, dx_s, g->dx,
+                            g->dWg, g->dWnoise, g->dbias, ws, ws_bytes, stream);
     return rc;
 }
