@@ -548,8 +548,10 @@ def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C
         raise SystemExit("device status %d after warm-up" % st)
     R = int(b.offsets[-1])
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # events around the roofline call on every 8th step only (an event between two
+    # kernels keeps the second from starting early under programmatic dependent launch)
     up_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+              if i % 8 == 0 else None for i in range(args.steps)]
     sampler = ClockSampler(local)
     time.sleep(0.3)
     barrier(world)
@@ -570,7 +572,8 @@ def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C
     if moe.moe_get_device_status(wsb) != 0:
         raise SystemExit("device status set in the timed region")
     ms = max_over_ranks(start.elapsed_time(end), world)
-    up_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in up_evs) / args.steps, world)
+    up_pairs = [ev for ev in up_evs if ev is not None]
+    up_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in up_pairs) / len(up_pairs), world)
     nseg = min(args.steps, 50)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(SEG) + 1)]
            for _ in range(nseg)]
@@ -804,11 +807,14 @@ def main():
         raise SystemExit("device status %d after warm-up" % status)
     R = int(b.offsets[-1])
 
-    # the timed loop: K whole steps back to back; the only events inside a step
-    # bracket expert GEMM 1 (its time is the roofline figure)
+    # the timed loop: K whole steps back to back; the only events inside it bracket
+    # expert GEMM 1 (its time is the roofline figure) on every UP_EVERY-th step -- an
+    # event recorded between two kernels keeps the second from starting early under
+    # programmatic dependent launch, so bracketing every step would slow the loop
+    UP_EVERY = 8
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     up_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+              if i % UP_EVERY == 0 else None for i in range(args.steps)]
     sampler = ClockSampler(local)
     time.sleep(0.3)
     barrier(world)
@@ -844,7 +850,8 @@ def main():
         for s in range(NSEG):
             seg_ms[s] += e[s].elapsed_time(e[s + 1])
     seg_ms /= nseg_steps
-    up_ms_timed = sum(a.elapsed_time(b) for a, b in up_evs) / args.steps
+    up_pairs = [ev for ev in up_evs if ev is not None]
+    up_ms_timed = sum(a.elapsed_time(b) for a, b in up_pairs) / len(up_pairs)
     ms = max_over_ranks(ms_local, world)
     seg_ms = np.array([max_over_ranks(v, world) for v in seg_ms])
     value = tokens_per_s(w.T, args.steps, world, ms)

@@ -52,6 +52,9 @@ def lib():
                                                     p, p, p, p]
         _lib.oracle_router_backward.argtypes = [i, i, i, i, i, p, i, p, p, p, p, p, p, p, p, d,
                                                 d, p, p, p, p, p, p]
+        _lib.oracle_router_backward_norm.argtypes = [i, i, i, i, i, i, p, i, p, p, p, p, p, p, p,
+                                                     p, d, d, p, p, p, p, p, p]
+        _lib.oracle_neuron_wgrad.argtypes = [i, i, i, p, p, p, i, p, i, i, p, p, p, p]
     return _lib
 
 
@@ -443,3 +446,45 @@ def backward_residual(x, Wg, experts, shared_block, k, dy, router_type=MIXTRAL, 
     g["dW1s"], g["dW3s"], g["dW2s"] = sb["dW1e"][0], sb["dW3e"][0], sb["dW2e"][0]
     g["dh_s"] = sb["dh"]
     return g
+
+
+def router_backward_tokens(x, Wg, idx, G, dG, counts, k, T_norm, router_type=MIXTRAL,
+                           Wnoise=None, eps=None, bias=None, lam=0.0, dLb=1.0):
+    """Router backward for some of a batch's tokens (rows of x etc. are those tokens;
+    counts and T_norm are the whole batch's).  Returns the router term of dx and dL/dN."""
+    x, Wg = _c(x), _c(Wg)
+    T, d = x.shape
+    E = Wg.shape[1]
+    Wn = None if Wnoise is None else _c(Wnoise)
+    ep = None if eps is None else _c(eps, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    dx = np.zeros((T, d), np.float64)
+    dWg = np.empty((d, E), np.float64)
+    dWn = np.empty((d, E), np.float64)
+    db = np.empty(E, np.float64)
+    dH = np.empty((T, E), np.float64)
+    dN = np.empty((T, E), np.float64)
+    _check(lib().oracle_router_backward_norm(
+        T, int(T_norm), d, E, k, router_type, _ptr(x), _dt(x), _ptr(Wg), _ptr(Wn), _ptr(ep),
+        _ptr(b), _ptr(_c(idx, np.int32)), _ptr(_c(G, np.float64)), _ptr(_c(dG, np.float64)),
+        _ptr(_c(counts, np.int32)), float(lam), float(dLb), _ptr(dx), _ptr(dWg),
+        _ptr(dWn if Wnoise is not None else None), _ptr(db if bias is not None else None),
+        _ptr(dH), _ptr(dN)), "router_backward_norm")
+    return dict(dx=dx, dH=dH, dN=dN)
+
+
+def neuron_wgrad(W1e, W3e, W2e, e: int, i: int, x_rows, d_out):
+    """Gradients of neuron i of expert e over the given rows of that expert:
+    (dW1 row [d], dW3 row [d], dW2 column [d]), float64."""
+    W1e, W3e, W2e = _c(W1e), _c(W3e), _c(W2e)
+    E, m, d = W1e.shape
+    x_rows = _c(x_rows)
+    d_out = _c(d_out, np.float64)
+    out = [np.empty(d, np.float64) for _ in range(3)]
+    w1 = np.ascontiguousarray(W1e[e, i])
+    w3 = np.ascontiguousarray(W3e[e, i])
+    w2 = np.ascontiguousarray(W2e[e])
+    _check(lib().oracle_neuron_wgrad(d, m, i, _ptr(w1), _ptr(w3), _ptr(w2), _dt(W1e),
+                                     _ptr(x_rows), _dt(x_rows), x_rows.shape[0], _ptr(d_out),
+                                     _ptr(out[0]), _ptr(out[1]), _ptr(out[2])), "neuron_wgrad")
+    return out

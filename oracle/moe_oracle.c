@@ -789,12 +789,34 @@ int oracle_expert_ffn_backward(int d, int m, int E, const void *W1e, const void 
  *   dx_t += W_g dL_t + W_noise dN_t,  dW_g = x^T dL,  dW_noise = x^T dN,  db = sum_t dL_t
  * dx [T][d] is ADDED to; dWg, dWnoise [d][E], dbias [E] are written (NULL when the
  * input is absent); dH_out [T][E] and dN_out [T][E] optional. */
+int oracle_router_backward_norm(int T, int T_norm, int d, int E, int k, int router_type,
+                                const void *x, int dt, const void *Wg, const void *Wnoise,
+                                const float *eps, const float *bias, const int32_t *idx,
+                                const double *G, const double *dG, const int32_t *counts,
+                                double lambda, double dLb, double *dx, double *dWg,
+                                double *dWnoise, double *dbias, double *dH_out, double *dN_out);
+
 int oracle_router_backward(int T, int d, int E, int k, int router_type, const void *x, int dt,
                            const void *Wg, const void *Wnoise, const float *eps, const float *bias,
                            const int32_t *idx, const double *G, const double *dG,
                            const int32_t *counts, double lambda, double dLb, double *dx,
                            double *dWg, double *dWnoise, double *dbias, double *dH_out,
                            double *dN_out)
+{
+    return oracle_router_backward_norm(T, T, d, E, k, router_type, x, dt, Wg, Wnoise, eps, bias,
+                                       idx, G, dG, counts, lambda, dLb, dx, dWg, dWnoise, dbias,
+                                       dH_out, dN_out);
+}
+
+/* The same for a subset of the batch's tokens: the T rows given are some of the
+ * T_norm tokens of the batch, whose counts f_e = counts_e / (T_norm k) and 1/T_norm
+ * the balance term uses.  (The weight-gradient outputs then cover only these rows.) */
+int oracle_router_backward_norm(int T, int T_norm, int d, int E, int k, int router_type,
+                                const void *x, int dt, const void *Wg, const void *Wnoise,
+                                const float *eps, const float *bias, const int32_t *idx,
+                                const double *G, const double *dG, const int32_t *counts,
+                                double lambda, double dLb, double *dx, double *dWg,
+                                double *dWnoise, double *dbias, double *dH_out, double *dN_out)
 {
     if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E)
         return ORC_EINVAL;
@@ -857,12 +879,14 @@ int oracle_router_backward(int T, int d, int E, int k, int router_type, const vo
                 dH[e] += p[e] * (ge - S);
             }
         }
-        if (lambda != 0.0 && dLb != 0.0 && T > 0) {
+        if (lambda != 0.0 && dLb != 0.0 && T_norm > 0) {
             double B = 0.0;
             for (int e = 0; e < E; ++e)
-                B += p[e] * (dLb * lambda * ((double)counts[e] / ((double)T * k)) / (double)T);
+                B += p[e] * (dLb * lambda * ((double)counts[e] / ((double)T_norm * k)) /
+                             (double)T_norm);
             for (int e = 0; e < E; ++e) {
-                double be = dLb * lambda * ((double)counts[e] / ((double)T * k)) / (double)T;
+                double be = dLb * lambda * ((double)counts[e] / ((double)T_norm * k)) /
+                            (double)T_norm;
                 dH[e] += p[e] * (be - B);
             }
         }
@@ -909,5 +933,42 @@ int oracle_router_backward(int T, int d, int E, int k, int router_type, const vo
             dbias[e] = a;
         }
     free(DL), free(DN);
+    return 0;
+}
+
+/* One neuron's weight gradients over the n rows of one expert (a sample of what
+ * oracle_expert_ffn_backward computes for every neuron):
+ *   dW1[c] = sum_r dg_r x_r[c],  dW3[c] = sum_r du_r x_r[c],  dW2[o] = sum_r d_out_r[o] h_r
+ * with g = W1_i . x_r, u = W3_i . x_r, h = silu(g) u, dh = sum_o W2[o][i] d_out_r[o],
+ * du = dh silu(g), dg = dh u silu'(g), rows in ascending order.  W1i, W3i [d] and
+ * the column W2[:, i] given as W2e [d][m] with the neuron index i (element type dt);
+ * x_rows [n][d] (type xdt); d_out [n][d] f64. */
+int oracle_neuron_wgrad(int d, int m, int i, const void *W1i, const void *W3i, const void *W2e,
+                        int dt, const void *x_rows, int xdt, int n, const double *d_out,
+                        double *dW1, double *dW3, double *dW2)
+{
+    if (d <= 0 || m <= 0 || i < 0 || i >= m || n < 0)
+        return ORC_EINVAL;
+    for (int c = 0; c < d; ++c)
+        dW1[c] = dW3[c] = dW2[c] = 0.0;
+    for (int r = 0; r < n; ++r) {
+        double g = 0.0, u = 0.0, dh = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double xv = orc_load(x_rows, xdt, (size_t)r * d + c);
+            g += orc_load(W1i, dt, (size_t)c) * xv;
+            u += orc_load(W3i, dt, (size_t)c) * xv;
+        }
+        for (int o = 0; o < d; ++o)
+            dh += orc_load(W2e, dt, (size_t)o * m + i) * d_out[(size_t)r * d + o];
+        double h = oracle_silu(g) * u;
+        double du = dh * oracle_silu(g);
+        double dg = dh * u * orc_dsilu(g);
+        for (int c = 0; c < d; ++c) {
+            double xv = orc_load(x_rows, xdt, (size_t)r * d + c);
+            dW1[c] = dW1[c] + dg * xv;
+            dW3[c] = dW3[c] + du * xv;
+            dW2[c] = dW2[c] + d_out[(size_t)r * d + c] * h;
+        }
+    }
     return 0;
 }

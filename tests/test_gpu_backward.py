@@ -213,3 +213,65 @@ def test_residual_backward_parity(name):
     }
     bad = {k2: v for k2, v in errs.items() if not v <= TOL}
     assert not bad, (name, errs)
+
+
+# --------------------------------------------------------------------------- full size
+
+def test_full_size_sampled_backward():
+    """moe_2of8 (T=16384, d=4096, 8 x 1376, top-2 noisy Mixtral, rescale, lambda=0.01) in the
+    bench's launch configuration; the oracle routes the whole batch and then computes
+    one by one: dx of 16 sampled tokens (their expert rows and the router term,
+    normalised by the whole batch), and for 6 sampled (expert, neuron) pairs the rows of
+    dW1 / dW3 and the column of dW2 summed over all of that expert's rows."""
+    w = wl.WORKLOADS["moe_2of8"]
+    inp = wl.make_inputs(w)
+    p, bufs, gb, dy = _run(w, inp)
+    raw = H.raw
+    x, Wg, Wn = raw(inp["x"]), raw(inp["Wg"]), raw(inp["Wnoise"])
+    eps = inp["eps"].numpy()
+    r = oracle.router(x, Wg, Wn, eps, None, w.k, oracle.MIXTRAL)
+    ties = H.near_tie_tokens(r["H"], w.k)
+    gidx = bufs.topk_idx.cpu().numpy()
+    assert ((gidx == r["idx"]).all(axis=1) | ties).all()
+    assert ties.sum() < 32
+    dsp = oracle.dispatch(r["idx"], w.E, -1)
+    W1e, W3e, W2e = H.oracle_weights(w, inp)
+    s = w.E / w.k
+    dy64 = H.f64(dy)
+    rng = np.random.default_rng(3)
+    m, d, E, k = w.m, w.d, w.E, w.k
+    # -- dx of sampled tokens
+    toks = np.sort(rng.choice(np.nonzero(~ties)[0], 16, replace=False))
+    sr = dsp["slot_row"][toks]
+    rows = sr[sr >= 0]
+    eor = np.searchsorted(dsp["offsets"], rows, side="right") - 1
+    xr = x[dsp["row_token"][rows]]
+    out_rows = oracle.expert_ffn(W1e, W3e, W2e, xr, eor)
+    local = np.full(sr.shape, -1, np.int32)
+    local[sr >= 0] = np.arange(len(rows))
+    d_out, dG = oracle.combine_backward(out_rows, local, r["G"][toks], s, dy64[toks])
+    eb = oracle.expert_ffn_backward(W1e, W3e, W2e, xr, eor, d_out)
+    rb = oracle.router_backward_tokens(x[toks], Wg, r["idx"][toks], r["G"][toks], dG,
+                                       dsp["counts"], k, w.T, oracle.MIXTRAL, Wn, eps[toks], None,
+                                       w.lam, 1.0)
+    dx_ref = rb["dx"].copy()
+    for a, (t_i, j) in enumerate(zip(*np.nonzero(sr >= 0))):
+        dx_ref[t_i] += eb["dx_rows"][local[t_i, j]]
+    e_dx = rel(H.f64(gb.dx[torch.from_numpy(toks).cuda()]), dx_ref)
+    assert e_dx <= TOL, e_dx
+    # -- sampled neurons of three experts
+    dW1, dW3 = H.unpack_w13(gb.dW13_e, E, m, d)
+    dW2 = H.unpack_w2(gb.dW2_e, E, m, d)
+    worst = 0.0
+    for e in rng.choice(E, 3, replace=False):
+        rows_e = np.arange(dsp["offsets"][e], dsp["offsets"][e + 1])
+        loc = np.full(dsp["slot_row"].shape, -1, np.int32)
+        hit = (dsp["slot_row"] >= dsp["offsets"][e]) & (dsp["slot_row"] < dsp["offsets"][e + 1])
+        loc[hit] = dsp["slot_row"][hit] - dsp["offsets"][e]
+        d_out_e, _ = oracle.combine_backward(np.zeros((len(rows_e), d)), loc, r["G"], s, dy64)
+        xr_e = x[dsp["row_token"][rows_e]]
+        for i in rng.choice(m, 2, replace=False):
+            d1, d3, d2 = oracle.neuron_wgrad(W1e, W3e, W2e, int(e), int(i), xr_e, d_out_e)
+            worst = max(worst, rel(H.f64(dW1[e, i]), d1), rel(H.f64(dW3[e, i]), d3),
+                        rel(H.f64(dW2[e, :, i]), d2))
+    assert worst <= TOL, worst

@@ -176,3 +176,29 @@ def test_residual_backward_matches_central_differences(orc):
                 vals.append(loss(args["x"], args["Wg"], args["ex"], args["bl"]))
             fd = (vals[0] - vals[1]) / (float(np.float32(v + h)) - float(np.float32(v - h)))
             assert abs(fd - G[i]) <= 1e-6 * max(1.0, abs(fd)), (name, i, fd, G[i])
+
+
+def test_sampled_backward_pieces_equal_the_full_backward(orc):
+    """The sampling helpers the full-size parity test uses reproduce the full
+    backward: the per-neuron weight gradient, and the router backward of a token
+    subset normalised by the whole batch."""
+    P = _problem(71, T=9, d=8, m=5, E=3, k=2, noisy=True, bias=True)
+    lam, c = 0.3, 0.7
+    g = orc.backward(P["x"], P["Wg"], P["W1e"], P["W3e"], P["W2e"], 2, P["dy"], orc.MIXTRAL,
+                     P["Wnoise"], P["eps"], P["bias"], -1, True, lam, c)
+    f = g["fwd"]
+    dsp = f["dispatch"]
+    for e in range(3):
+        rows = np.arange(dsp["offsets"][e], dsp["offsets"][e + 1])
+        xr = P["x"][dsp["row_token"][rows]]
+        for i in range(5):
+            d1, d3, d2 = orc.neuron_wgrad(P["W1e"], P["W3e"], P["W2e"], e, i, xr,
+                                          g["d_out"][rows])
+            np.testing.assert_allclose(d1, g["dW1e"][e, i], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(d3, g["dW3e"][e, i], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(d2, g["dW2e"][e][:, i], rtol=1e-12, atol=1e-14)
+    toks = np.array([1, 4, 7])
+    rb = orc.router_backward_tokens(P["x"][toks], P["Wg"], f["router"]["idx"][toks],
+                                    f["router"]["G"][toks], g["dG"][toks], dsp["counts"], 2, 9,
+                                    orc.MIXTRAL, P["Wnoise"], P["eps"][toks], P["bias"], lam, c)
+    np.testing.assert_allclose(rb["dH"], g["dH"][toks], rtol=1e-12, atol=1e-15)

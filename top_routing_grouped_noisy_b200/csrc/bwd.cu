@@ -538,7 +538,7 @@ using namespace moe;
 
 namespace {
 
-char g_msg[320];
+thread_local char g_msg[320];  // per host thread, like the library's last-error string
 
 int fail_msg(int code, const char *fmt, const char *fn, const char *what)
 {
