@@ -30,6 +30,11 @@ CASES = {
                  seed=87),
     "bwd_e12_ragged_d": W("bwd_e12_ragged_d", T=150, d=72, d_ff=480, E=12, k=3, router=wl.ST,
                           noisy=True, seed=88),
+    # T*k >= 4096: the 2-SM (cta_group::2) backward GEMMs
+    "bwd_pair_st_cap": W("bwd_pair_st_cap", T=2100, d=256, d_ff=1024, E=8, k=2, router=wl.ST,
+                         noisy=True, bias=True, cf=1.0, rescale=True, lam=0.05, seed=92),
+    "bwd_pair_e16k4": W("bwd_pair_e16k4", T=2048, d=136, d_ff=576, E=16, k=4, noisy=True,
+                        seed=93),
 }
 
 

@@ -436,6 +436,360 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------------ 2-SM variant
+// The same GEMMs with cta_group::2 (the forward's pair kernel, with the two tile
+// orders and the epilogues above): a cluster of two CTAs owns a 256-row output
+// tile; CTA r loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of
+// the B tile, the leader issues M=256 MMAs reading A from each CTA and B from both,
+// and every CTA drains its own 128 accumulator rows.  Barriers as in the forward
+// pair kernel (full: leader counts both CTAs' bytes; empty/tfull: multicast
+// commits; tempty: both CTAs' epilogue warps arrive on the leader).  Loads carry no
+// multicast qualifier.
+namespace pair {
+
+constexpr int BM = 128;   // rows per CTA
+constexpr int BNH = 128;  // B rows per CTA
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BNH * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TILE_BYTES = STAGES * STAGE_BYTES;
+constexpr uint64_t kAbortSettleNs = 200000ull;
+
+struct Aux {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[ACC];
+    uint64_t tempty[ACC];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int32_t abort_flag;
+    int32_t off[MOE_MAX_EXPERTS + 1];
+    int32_t tstart[MOE_MAX_EXPERTS + 1];
+};
+constexpr int SMEM_BYTES = 1024 + TILE_BYTES + kEpiStageBytes + (int)sizeof(Aux);
+
+// kind::f16, D f32, A/B bf16 K-major, N = 256, M = 256 (the pair)
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cta_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+__device__ __forceinline__ int32_t ld_cluster_s32(uint32_t cluster_addr)
+{
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster,
+                                                 uint32_t dst, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *map, uint32_t bar_cluster,
+                                                 uint32_t dst, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc2), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_both(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_own(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+// Pair tiles: row-grouped, 256 rows of an expert per tile; K-grouped, 256 of the M
+// rows of every expert per tile.  row0 / a_row: the pair's first row (rank 0).
+template <bool KG>
+__device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tiles, int M,
+                                            int num_kb)
+{
+    Tile t;
+    int e = 0;
+    while (tile >= aux->tstart[e + 1])
+        ++e;
+    const int local = tile - aux->tstart[e];
+    t.e = e;
+    if constexpr (KG) {
+        const int mtiles = (M + 2 * BM - 1) / (2 * BM);
+        const int mt = local % mtiles, nt = local / mtiles;
+        t.a_row = mt * 2 * BM;
+        t.row0 = e * M + mt * 2 * BM;
+        t.row_end = e * M + M;
+        t.n0 = nt * BN;
+        t.k0 = aux->off[e];
+        t.nkb = (aux->off[e + 1] - aux->off[e]) / BK;
+    } else {
+        const int rows = aux->off[e + 1] - aux->off[e];
+        const int mtiles = (rows + 2 * BM - 1) / (2 * BM);
+        const int mt = local % mtiles, nt = local / mtiles;
+        t.a_row = aux->off[e] + mt * 2 * BM;
+        t.row0 = t.a_row;
+        t.row_end = aux->off[e + 1];
+        t.n0 = nt * BN;
+        t.k0 = 0;
+        t.nkb = num_kb;
+    }
+    return t;
+}
+
+template <int EPI, bool KG>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO,
+                        const int32_t *__restrict__ offsets, int E, int N, int K, int M,
+                        bf16 *__restrict__ out, int ld_out, int n_valid,
+                        const bf16 *__restrict__ dh, int ld_dh, int32_t *status, uint64_t wait_ns)
+{
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES + kEpiStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int32_t *abort_flag = &aux->abort_flag;
+    const uint32_t rank = cta_rank();
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&aux->full[s]), 1);
+            mbar_init(smem_u32(&aux->empty[s]), 1);
+        }
+        for (int a = 0; a < ACC; ++a) {
+            mbar_init(smem_u32(&aux->tfull[a]), 1);
+            mbar_init(smem_u32(&aux->tempty[a]), 2 * EPI_WARPS);
+        }
+        mbar_init(smem_u32(&aux->drain), 1);
+        aux->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
+    }
+    const int n_tiles = (N + BN - 1) / BN;
+    if (warp == 2 && lane == 0) {
+        int acc = 0, kacc = 0;
+        for (int e = 0; e < E; ++e) {
+            const int rows = offsets[e + 1] - offsets[e];
+            aux->tstart[e] = acc;
+            if constexpr (KG) {
+                aux->off[e] = kacc;
+                kacc += (rows + BK - 1) / BK * BK;
+                acc += (M + 2 * BM - 1) / (2 * BM) * n_tiles;
+            } else {
+                aux->off[e] = offsets[e];
+                acc += (rows + 2 * BM - 1) / (2 * BM) * n_tiles;
+            }
+        }
+        aux->off[E] = KG ? kacc : offsets[E];
+        aux->tstart[E] = acc;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&aux->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+    tc_fence_after();
+    const uint32_t tmem_base = aux->tmem_base;
+    const int total = aux->tstart[E];
+    const int num_kb = (K + BK - 1) / BK;
+    const uint32_t smem_base = smem_u32(smem);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------- TMA producer (both)
+            int stage = 0;
+            uint32_t phase = 0;
+            int64_t fills = 0;
+            bool ok = true;
+            for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
+                if (*abort_flag)
+                    break;
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb);
+                for (int kb = 0; kb < t.nkb; ++kb) {
+                    if (!mbar_wait(smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns, abort_flag,
+                                   status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&aux->full[stage]);
+                    if (leader)
+                        mbar_expect_tx(fb, 2 * STAGE_BYTES);
+                    const uint32_t fb0 = map_rank(fb, 0);
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const int kc = t.k0 + kb * BK;
+                    tma_load_2d_pair(&tmA, fb0, sa, kc, t.a_row + (int)rank * BM);
+                    if constexpr (KG)
+                        tma_load_2d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH);
+                    else
+                        tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH,
+                                         t.e);
+                    ++fills;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (leader) {  // the leader's full barriers count both CTAs' bytes
+                for (int s = 0; s < STAGES; ++s) {
+                    const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
+                    if (n > 0)
+                        mbar_drain(smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------------- MMA issuer (leader)
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb);
+                if (!mbar_wait(smem_u32(&aux->tempty[acc]), acc_phase ^ 1u, wait_ns, abort_flag,
+                               status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < t.nkb; ++kb) {
+                    if (!mbar_wait(smem_u32(&aux->full[stage]), phase, wait_ns, abort_flag,
+                                   status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint64_t da = sdesc(sa), db = sdesc(sa + A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
+                                  (kb | k) != 0);
+                    umma_commit_both(smem_u32(&aux->empty[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit_both(smem_u32(&aux->tfull[acc]));  // also with no MMA (zero tile)
+                if (++acc == ACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            umma_commit_own(smem_u32(&aux->drain));
+            mbar_drain(smem_u32(&aux->drain), 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both)
+        const int wq = warp & 3;
+        const int lane_base = wq * 32;
+        const int c_first = ((warp - 2) / 4) * (BN / 64);
+        const uint32_t tempty0 = map_rank(smem_u32(&aux->tempty[0]), 0);
+        const uint32_t tempty1 = map_rank(smem_u32(&aux->tempty[1]), 0);
+        EpiStore st{&tmO, smem_base + TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = cluster_id; tile < total; tile += nclusters) {
+            const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb);
+            if (!mbar_wait(smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag, status))
+                break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
+            epilogue_slab<EPI>(taddr, c_first, BN / 64, t.row0 + (int)rank * BM + lane_base,
+                               t.row_end, t.n0, t.nkb == 0, out, ld_out, n_valid, dh, ld_dh, st);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);
+            if (++acc == ACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0)
+            bulk_wait_all();
+    }
+    tc_fence_before();
+    cluster_sync();
+    if (threadIdx.x == 0) {
+        const int peer_abort = ld_cluster_s32(map_rank(smem_u32(&aux->abort_flag), rank ^ 1u));
+        if (*abort_flag || peer_abort) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < kAbortSettleNs) {
+            }
+        }
+    }
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace pair
+
 // ------------------------------------------------------------------------ transposes
 // Both transposes move 8 x 8 bf16 blocks through registers: a thread loads 8 rows
 // of 8 columns (8 x 16 bytes), transposes them with byte permutes and stores 8
@@ -565,18 +919,19 @@ __global__ void __launch_bounds__(256) transpose_weights_kernel(const bf16 *__re
 
 struct DevInfo {
     int sms = 0;
-    bool attr[4] = {false, false, false, false};
+    int pair_clusters = 0;
+    bool attr[6] = {false, false, false, false, false, false};
 };
 static std::mutex g_mu;
 static DevInfo g_dev[64];
 
 template <typename Kern>
-static cudaError_t set_attr(Kern kern, bool &done)
+static cudaError_t set_attr(Kern kern, bool &done, int bytes = SMEM_BYTES)
 {
     if (done)
         return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+                                         bytes);
     if (e == cudaSuccess)
         done = true;
     return e;
@@ -597,11 +952,38 @@ static cudaError_t prepare(DevInfo **out)
         return e;
     if ((e = set_attr(bwd_gemm_kernel<EPI_STORE, false>, di.attr[0])) != cudaSuccess ||
         (e = set_attr(bwd_gemm_kernel<EPI_SWIGLU_BWD, false>, di.attr[1])) != cudaSuccess ||
-        (e = set_attr(bwd_gemm_kernel<EPI_STORE, true>, di.attr[2])) != cudaSuccess)
+        (e = set_attr(bwd_gemm_kernel<EPI_STORE, true>, di.attr[2])) != cudaSuccess ||
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, false>, di.attr[3],
+                      pair::SMEM_BYTES)) != cudaSuccess ||
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_SWIGLU_BWD, false>, di.attr[4],
+                      pair::SMEM_BYTES)) != cudaSuccess ||
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, true>, di.attr[5],
+                      pair::SMEM_BYTES)) != cudaSuccess)
         return e;
+    if (di.pair_clusters == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (di.sms / 2));
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, pair::bwd_gemm_2sm_kernel<EPI_STORE, false>, &cfg);
+        if (e != cudaSuccess)
+            return e;
+        di.pair_clusters = n > 0 ? n : 1;
+    }
     *out = &di;
     return cudaSuccess;
 }
+
+// Rows (T*k) from which the 2-SM kernels are used, as in the forward.
+constexpr int64_t kPairMinRows = 4096;
 
 // One backward GEMM.  A [a_rows][a_ld] (K extent a_k); B: row-grouped [E][b_rows][b_ld],
 // K-grouped [b_rows][b_ld] (K extent b_k); out [out_rows][ld_out], n_valid columns.
@@ -610,7 +992,7 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
                           const void *B, uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
                           const int32_t *offsets, int E, int M, bf16 *out, int ld_out,
                           uint64_t out_rows, int n_valid, const bf16 *dh, int ld_dh,
-                          int32_t *status, cudaStream_t s)
+                          int32_t *status, cudaStream_t s, bool use_pair)
 {
     DevInfo *di = nullptr;
     cudaError_t e = prepare(&di);
@@ -619,17 +1001,18 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     CUtensorMap ta, tb, to;
     const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
     const uint32_t ba[2] = {BK, BM};
+    const uint32_t b_box = use_pair ? (uint32_t)pair::BNH : (uint32_t)BN;
     if ((e = tc::make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
         return e;
     if constexpr (KG) {
         const uint64_t db[2] = {b_k, b_rows}, sb[1] = {b_ld * 2};
-        const uint32_t bb[2] = {BK, BN};
+        const uint32_t bb[2] = {BK, b_box};
         if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
             return e;
     } else {
         const uint64_t db[3] = {b_k, b_rows, (uint64_t)E};
         const uint64_t sb[2] = {b_ld * 2, b_rows * b_ld * 2};
-        const uint32_t bb[3] = {BK, BN, 1};
+        const uint32_t bb[3] = {BK, b_box, 1};
         if ((e = tc::make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
             return e;
     }
@@ -639,9 +1022,27 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
         cudaSuccess)
         return e;
     count_launch();
-    return launch_pdl(bwd_gemm_kernel<EPI, KG>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s,
-                      ta, tb, to, offsets, E, (int)b_rows, (int)a_k, M, out, ld_out, n_valid, dh,
-                      ld_dh, status, wait_limit_ns());
+    if (!use_pair)
+        return launch_pdl(bwd_gemm_kernel<EPI, KG>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES,
+                          s, ta, tb, to, offsets, E, (int)b_rows, (int)a_k, M, out, ld_out,
+                          n_valid, dh, ld_dh, status, wait_limit_ns());
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(2 * di->pair_clusters);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, pair::bwd_gemm_2sm_kernel<EPI, KG>, ta, tb, to, offsets, E,
+                              (int)b_rows, (int)a_k, M, out, ld_out, n_valid, dh, ld_dh, status,
+                              wait_limit_ns());
 }
 
 }  // namespace bwd
@@ -655,7 +1056,8 @@ cudaError_t launch_bwd_dh(const moe_params_t *p, const void *d_out, const int32_
     const uint64_t d = p->d, m8 = round_up(p->m, 8), m16 = round_up(p->m, 16);
     const uint64_t rows = (uint64_t)p->T * p->k;
     return launch<EPI_STORE, false>(d_out, d, d, rows, W2T, d, d, m16, offsets, p->E, 0,
-                                    (bf16 *)dh, (int)m8, rows, (int)m8, nullptr, 0, status, s);
+                                    (bf16 *)dh, (int)m8, rows, (int)m8, nullptr, 0, status, s,
+                                    (int64_t)rows >= kPairMinRows);
 }
 
 // dGU [rows][2 m16] = SwiGLU backward of (x_perm x W13_e^T) with dh [rows][m8]
@@ -667,7 +1069,8 @@ cudaError_t launch_bwd_dgu(const moe_params_t *p, const void *x_perm, const int3
     const uint64_t rows = (uint64_t)p->T * p->k;
     return launch<EPI_SWIGLU_BWD, false>(x_perm, d, d, rows, W13, d, d, 2 * m16, offsets, p->E,
                                          0, (bf16 *)dgu, (int)(2 * m16), rows, (int)(2 * m16),
-                                         (const bf16 *)dh, (int)m8, status, s);
+                                         (const bf16 *)dh, (int)m8, status, s,
+                                         (int64_t)rows >= kPairMinRows);
 }
 
 // dx_perm [rows][d] = dGU [rows][2 m16] x W13T_e [d][2 m16]^T
@@ -678,7 +1081,7 @@ cudaError_t launch_bwd_dx(const moe_params_t *p, const void *dgu, const int32_t 
     const uint64_t rows = (uint64_t)p->T * p->k;
     return launch<EPI_STORE, false>(dgu, 2 * m16, 2 * m16, rows, W13T, 2 * m16, 2 * m16, d,
                                     offsets, p->E, 0, (bf16 *)dx_perm, (int)d, rows, (int)d,
-                                    nullptr, 0, status, s);
+                                    nullptr, 0, status, s, (int64_t)rows >= kPairMinRows);
 }
 
 // dW [E][M][n_valid]: A^T [M][kmax] and B^T [b_rows][kmax] in the padded K order
@@ -688,7 +1091,8 @@ cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *AT, int M, const
 {
     return launch<EPI_STORE, true>(AT, kmax, kmax, (uint64_t)M, BT, kmax, kmax, (uint64_t)b_rows,
                                    offsets, p->E, M, (bf16 *)dW, ld_dw, (uint64_t)p->E * M,
-                                   n_valid, nullptr, 0, status, s);
+                                   n_valid, nullptr, 0, status, s,
+                                   (int64_t)p->T * p->k >= kPairMinRows);
 }
 
 cudaError_t launch_transpose_rows(const void *src, int ld_src, const int32_t *offsets, int E,
