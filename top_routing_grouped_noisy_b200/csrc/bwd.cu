@@ -84,7 +84,10 @@ BwdLayout bwd_layout(const moe_params_t *p)
 }  // namespace
 
 // ---------------------------------------------------------------- combine backward
-// One warp per token; lanes stride over the 16-byte vectors of the row.
+// One warp per token; lanes stride over the 16-byte vectors of the row, two vectors
+// per step so that the loads of both are in flight together.  KMAX = k rounded up
+// to 2, 4 or 8 sizes the per-slot registers.
+template <int KMAX>
 __global__ void __launch_bounds__(256) combine_backward_kernel(
     const bf16 *__restrict__ dy, const bf16 *__restrict__ out, const int32_t *__restrict__ slot_row,
     const float *__restrict__ topk_w, int T, int d, int k, float scale, bf16 *__restrict__ d_out,
@@ -96,34 +99,56 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T)
         return;
-    int row[MOE_MAX_TOPK];
-    float w[MOE_MAX_TOPK], dot[MOE_MAX_TOPK];
+    int row[KMAX];
+    float w[KMAX], dot[KMAX];
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         row[j] = j < k ? slot_row[(int64_t)t * k + j] : -1;
         w[j] = j < k ? scale * topk_w[(int64_t)t * k + j] : 0.f;
         dot[j] = 0.f;
     }
     const int nv = d / 8;
-    for (int v = lane; v < nv; v += 32) {
-        float fy[8];
-        bf16x8_to_f32(ld_nc_na(dy + (int64_t)t * d + 8 * v), fy);
+    for (int v0 = lane; v0 < nv; v0 += 64) {
+        const int v1 = v0 + 32;
+        const bool has1 = v1 < nv;
+        const uint4 y0 = ld_nc_na(dy + (int64_t)t * d + 8 * v0);
+        const uint4 y1 = has1 ? ld_nc_na(dy + (int64_t)t * d + 8 * v1) : make_uint4(0, 0, 0, 0);
+        uint4 o0[KMAX], o1[KMAX];
 #pragma unroll
-        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+        for (int j = 0; j < KMAX; ++j) {
+            o0[j] = row[j] >= 0 ? ld_nc_na(out + (int64_t)row[j] * d + 8 * v0)
+                                : make_uint4(0, 0, 0, 0);
+            o1[j] = (row[j] >= 0 && has1) ? ld_nc_na(out + (int64_t)row[j] * d + 8 * v1)
+                                          : make_uint4(0, 0, 0, 0);
+        }
+        float fy0[8], fy1[8];
+        bf16x8_to_f32(y0, fy0);
+        bf16x8_to_f32(y1, fy1);
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
             if (row[j] < 0)
                 continue;
             float fo[8], g[8];
-            bf16x8_to_f32(ld_nc_na(out + (int64_t)row[j] * d + 8 * v), fo);
+            bf16x8_to_f32(o0[j], fo);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                dot[j] += fy[i] * fo[i];
-                g[i] = w[j] * fy[i];
+                dot[j] += fy0[i] * fo[i];
+                g[i] = w[j] * fy0[i];
             }
-            st_v4(d_out + (int64_t)row[j] * d + 8 * v, f32x8_to_bf16(g));
+            st_v4(d_out + (int64_t)row[j] * d + 8 * v0, f32x8_to_bf16(g));
+            if (has1) {
+                bf16x8_to_f32(o1[j], fo);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    dot[j] += fy1[i] * fo[i];
+                    g[i] = w[j] * fy1[i];
+                }
+                st_v4(d_out + (int64_t)row[j] * d + 8 * v1, f32x8_to_bf16(g));
+            }
         }
     }
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    for (int j = 0; j < KMAX; ++j) {
         float s = dot[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
@@ -413,8 +438,9 @@ __global__ void __launch_bounds__(256) router_backward_wreduce_kernel(
 // rounded to bf16 once.
 constexpr int kIgTokens = 128;
 
-__host__ __device__ inline int input_grad_cols(int E) { return E <= 24 ? 512 : (E <= 48 ? 256 : 128); }
+__host__ __device__ inline int input_grad_cols(int E) { return E <= 16 ? 512 : (E <= 32 ? 256 : 128); }
 
+template <int KMAX>
 __global__ void __launch_bounds__(256) input_grad_kernel(
     const bf16 *__restrict__ dx_perm, const int32_t *__restrict__ slot_row,
     const bf16 *__restrict__ WT, int ne, const float *__restrict__ dLN, int T, int d, int E,
@@ -442,46 +468,63 @@ __global__ void __launch_bounds__(256) input_grad_kernel(
         return;
     const int t0 = blockIdx.y * kIgTokens;
     const int t1 = min(T, t0 + kIgTokens);
-    for (int t = t0 + tg; t < t1; t += ntg) {
-        float a[8];
+    // two tokens per step: all their expert rows are requested before any is summed,
+    // and each weight vector read from shared memory serves both
+    for (int tp = t0 + tg; tp < t1; tp += 2 * ntg) {
+        const int tt[2] = {tp, tp + ntg};
+        const bool v1 = tt[1] < t1;
+        uint4 rv[2][KMAX];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            a[u] = 0.f;
-        // all k rows requested before any is summed
-        uint4 rv[MOE_MAX_TOPK];
+        for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-            const int r = j < k ? slot_row[(int64_t)t * k + j] : -1;
-            rv[j] = r >= 0 ? ld_nc_na(dx_perm + (int64_t)r * d + c) : make_uint4(0, 0, 0, 0);
-        }
+            for (int j = 0; j < KMAX; ++j) {
+                const int r = (j < k && tt[q] < t1) ? slot_row[(int64_t)tt[q] * k + j] : -1;
+                rv[q][j] = r >= 0 ? ld_nc_na(dx_perm + (int64_t)r * d + c) : make_uint4(0, 0, 0, 0);
+            }
+        float a[2][8];
 #pragma unroll
-        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-            if (j >= k)
-                break;
-            float f[8];
-            bf16x8_to_f32(rv[j], f);
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                a[u] += f[u];
+                a[q][u] = 0.f;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j >= k)
+                    break;
+                float f[8];
+                bf16x8_to_f32(rv[q][j], f);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    a[q][u] += f[u];
+            }
         }
-        const float *dl = dLN + (int64_t)t * E2;
+        const float *dl0 = dLN + (int64_t)tt[0] * E2;
+        const float *dl1 = dLN + (int64_t)(v1 ? tt[1] : tt[0]) * E2;
         for (int e2 = 0; e2 < ne; ++e2) {
-            const float gl = dl[e2];
+            const float g0 = dl0[e2], g1 = dl1[e2];
             float wf[8];
             bf16x8_to_f32(*reinterpret_cast<const uint4 *>(ig_ws + (size_t)e2 * cols + 8 * ct),
                           wf);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                a[u] += gl * wf[u];
+            for (int u = 0; u < 8; ++u) {
+                a[0][u] += g0 * wf[u];
+                a[1][u] += g1 * wf[u];
+            }
         }
-        if (resid != nullptr) {  // the shared block's input gradient (residual layer)
-            float f[8];
-            bf16x8_to_f32(ld_nc_na(resid + (int64_t)t * d + c), f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                a[u] += f[u];
+        for (int q = 0; q < 2; ++q) {
+            if (q == 1 && !v1)
+                break;
+            const int t = tt[q];
+            if (resid != nullptr) {  // the shared block's input gradient (residual layer)
+                float f[8];
+                bf16x8_to_f32(ld_nc_na(resid + (int64_t)t * d + c), f);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    a[q][u] += f[u];
+            }
+            st_v4(dx + (int64_t)t * d + c, f32x8_to_bf16(a[q]));
         }
-        st_v4(dx + (int64_t)t * d + c, f32x8_to_bf16(a));
     }
 }
 
@@ -619,9 +662,11 @@ extern "C" int moe_combine_backward(const moe_params_t *p, const void *dy, const
     NEED(dG);
     const float scale = p->rescale ? (float)p->E / (float)p->k : 1.0f;
     count_launch();
-    return finish(fn, launch_pdl(combine_backward_kernel, dim3((p->T + 7) / 8), dim3(256), 0,
-                                 (cudaStream_t)stream, (const bf16 *)dy, (const bf16 *)out,
-                                 slot_row, topk_w, p->T, p->d, p->k, scale, (bf16 *)d_out, dG));
+    auto kern = p->k <= 2 ? combine_backward_kernel<2>
+                          : (p->k <= 4 ? combine_backward_kernel<4> : combine_backward_kernel<8>);
+    return finish(fn, launch_pdl(kern, dim3((p->T + 7) / 8), dim3(256), 0, (cudaStream_t)stream,
+                                 (const bf16 *)dy, (const bf16 *)out, slot_row, topk_w, p->T,
+                                 p->d, p->k, scale, (bf16 *)d_out, dG));
 }
 
 extern "C" int moe_expert_down_backward(const moe_params_t *p, const void *d_out, const void *h,
@@ -745,11 +790,13 @@ static int route_backward(const char *fn, const moe_params_t *p, const void *x, 
             const int cols = input_grad_cols(p->E);
             const int ne = Wnoise != nullptr ? 2 * p->E : p->E;
             const size_t smem = (size_t)ne * cols * sizeof(bf16);
+            auto kern = p->k <= 2 ? input_grad_kernel<2>
+                                  : (p->k <= 4 ? input_grad_kernel<4> : input_grad_kernel<8>);
             if (smem > 48 * 1024)
-                e = cudaFuncSetAttribute(input_grad_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
             if (e == cudaSuccess)
-                e = launch_pdl(input_grad_kernel,
+                e = launch_pdl(kern,
                                dim3((p->d + cols - 1) / cols, (p->T + kIgTokens - 1) / kIgTokens),
                                dim3(256), smem, s, (const bf16 *)dx_perm, slot_row,
                                (const bf16 *)(w + L.wt), ne, (const float *)dLN, p->T, p->d,
