@@ -45,3 +45,43 @@ def test_wait_timeout_is_reported_and_context_survives(T):
     dsp = H.check_dispatch(w, inp, p2, bufs)
     H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)
 
+
+
+@pytest.mark.parametrize("T", [300, 2500], ids=["one_sm_kernels", "two_sm_kernels"])
+def test_backward_wait_timeout_is_reported_and_context_survives(T):
+    """The backward GEMMs (row-grouped with the SwiGLU-backward epilogue, dgrad and the
+    K-grouped wgrad, 1-SM and 2-SM forms) give up at a wait limit of 0, report
+    MOE_ERR_DEVICE_TIMEOUT and return; a normal backward afterwards is correct."""
+    import oracle
+    w = wl.Workload("to_bwd", T=T, d=256, d_ff=1024, E=8, k=2, noisy=True, seed=82)
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, (W13_e, W2_e) = H.run_forward(w, inp)
+    assert status == 0
+    dev = "cuda"
+    dy = wl.make_grad_output(w, 5).to(dev)
+    g = moe.BackwardBuffers(p, True, False)
+    wsb = moe.Workspace(p, nbytes=moe.moe_backward_workspace_size(p))
+    moe.moe_combine_backward(p, dy, bufs.out, bufs.slot_row, bufs.topk_w, g.d_out, g.dG)
+    torch.cuda.synchronize()
+    moe.moe_set_wait_limit_ns(0)
+    try:
+        moe.moe_expert_down_backward(p, g.d_out, bufs.h, bufs.offsets, W2_e, g.dh, g.dW2_e, wsb)
+        moe.moe_expert_up_backward(p, bufs.x_perm, g.dh, bufs.offsets, W13_e, g.dx_perm,
+                                   g.dW13_e, wsb)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    assert moe.moe_get_device_status(wsb) == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert moe.moe_get_device_status(wsb) == 0
+    # the same context then runs the whole backward correctly
+    x, Wg, Wn, eps = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_backward(p, x, Wg, W13_e, W2_e, bufs, g, dy, wsb, Wnoise=Wn, noise=eps)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(wsb) == 0
+    W1e, W3e, W2e = H.oracle_weights(w, inp)
+    ref = oracle.backward(H.raw(inp["x"]), H.raw(inp["Wg"]), W1e, W3e, W2e, w.k, H.f64(dy.cpu()),
+                          oracle.MIXTRAL, H.raw(inp["Wnoise"]), inp["eps"].numpy(), None, -1,
+                          False, w.lam, 1.0)
+    assert (bufs.topk_idx.cpu().numpy() == ref["fwd"]["router"]["idx"]).all()
+    dx = H.f64(g.dx)
+    assert np.abs(dx - ref["dx"]).max() <= 2e-2 * np.abs(ref["dx"]).max()
