@@ -38,7 +38,6 @@ cudaError_t launch_transpose_weights(const void *src, int a, int ld_src, int b_v
 
 namespace {
 
-constexpr int kWChunk = 128;     // router weight columns staged per step
 constexpr int kPartChunks = 64;  // token chunks of the router weight-gradient partials
 
 // Sections of the backward workspace (after the 256-byte header).
