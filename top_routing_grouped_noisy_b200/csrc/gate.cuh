@@ -98,20 +98,61 @@ __device__ inline void router_small_slice(int ks, const E_T *__restrict__ x,
                                           const E_T *__restrict__ Wn, int T, int d, int E,
                                           float *__restrict__ part, float *sm)
 {
+    constexpr int VN = 16 / sizeof(E_T);  // elements per 16-byte load
     const int nout = Wn ? 2 * E : E;
-    const int kc = (d + kRouterSmallSplit - 1) / kRouterSmallSplit;
+    const int kc = router_small_kc(d);
     const int k0 = ks * kc, k1 = min(d, k0 + kc);
-    const int kn = k1 > k0 ? k1 - k0 : 0;
+    const int kn = k1 > k0 ? k1 - k0 : 0;  // a multiple of 8 (d % 8 == 0)
     float *xs = sm;                    // [T][kc]
     float *ws_ = sm + (size_t)T * kc;  // [kc][nout]
-    for (int i = threadIdx.x; i < T * kn; i += blockDim.x) {
-        const int t = i / kn, c = i % kn;
-        xs[t * kc + c] = to_f32(x[(int64_t)t * d + k0 + c]);
+    // x slice: 16-byte loads, four in flight per thread before any is stored
+    const int nvx = kn / VN;
+    for (int i0 = threadIdx.x; i0 < T * nvx; i0 += 4 * blockDim.x) {
+        uint4 u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * blockDim.x;
+            u[j] = make_uint4(0, 0, 0, 0);
+            if (i < T * nvx)
+                u[j] = ld_nc(x + (int64_t)(i / nvx) * d + k0 + (i % nvx) * VN);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j * blockDim.x;
+            if (i < T * nvx) {
+                const E_T *v = reinterpret_cast<const E_T *>(&u[j]);
+                float *dst = xs + (size_t)(i / nvx) * kc + (i % nvx) * VN;
+#pragma unroll
+                for (int q = 0; q < VN; ++q)
+                    dst[q] = to_f32(v[q]);
+            }
+        }
     }
-    for (int i = threadIdx.x; i < kn * nout; i += blockDim.x) {
-        const int c = i / nout, o = i % nout;
-        ws_[c * nout + o] = o < E ? to_f32(Wg[(int64_t)(k0 + c) * E + o])
-                                  : to_f32(Wn[(int64_t)(k0 + c) * E + o - E]);
+    // rows k0..k1 of W_g (and W_noise) are contiguous: kn * E elements from k0 * E
+    const int nvw = kn * E / VN;  // kn % 8 == 0, so kn * E % VN == 0
+    for (int h = 0; h < (Wn ? 2 : 1); ++h) {
+        const E_T *W = h == 0 ? Wg : Wn;
+        for (int i0 = threadIdx.x; i0 < nvw; i0 += 4 * blockDim.x) {
+            uint4 u[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j * blockDim.x;
+                u[j] = i < nvw ? ld_nc(W + (int64_t)k0 * E + (int64_t)i * VN)
+                               : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j * blockDim.x;
+                if (i < nvw) {
+                    const E_T *v = reinterpret_cast<const E_T *>(&u[j]);
+#pragma unroll
+                    for (int q = 0; q < VN; ++q) {
+                        const int f = i * VN + q;  // flat index in the slice: (c, o)
+                        ws_[(f / E) * nout + h * E + f % E] = to_f32(v[q]);
+                    }
+                }
+            }
+        }
     }
     __syncthreads();
     for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {

@@ -22,6 +22,12 @@ constexpr int kWtRows = 128;
 // Batches up to this many tokens use the split-K router (partials in `rsmall`).
 constexpr int kRouterSmallTokens = 64;
 constexpr int kRouterSmallSplit = 32;
+// Columns of x per split-K slice: d / kRouterSmallSplit rounded up to a multiple of 8,
+// so every slice starts on a 16-byte boundary of a row (d % 8 == 0).
+__host__ __device__ inline int router_small_kc(int d)
+{
+    return ((d + kRouterSmallSplit - 1) / kRouterSmallSplit + 7) / 8 * 8;
+}
 
 // Byte offsets of the sections of the caller's workspace.
 struct WsLayout {

@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(256) route_dispatch_small_kernel(
 static void small_router_smem(const moe_params_t *p, bool noisy, size_t *sm1, size_t *sm2)
 {
     const int nout = noisy ? 2 * p->E : p->E;
-    const int kc = ceil_div(p->d, kRouterSmallSplit);
+    const int kc = router_small_kc(p->d);
     *sm1 = sizeof(float) * ((size_t)p->T * kc + (size_t)kc * nout);
     *sm2 = sizeof(float) * ((size_t)p->T * nout + 2 * (size_t)p->T * p->E);
 }
@@ -279,7 +279,7 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
     cudaError_t e = cudaSuccess;
     const int small_noisy = Wnoise != nullptr;
     const int small_nout = small_noisy ? 2 * p->E : p->E;
-    const int small_kc = ceil_div(p->d, kRouterSmallSplit);
+    const int small_kc = router_small_kc(p->d);
     const size_t sm1 = sizeof(float) * ((size_t)p->T * small_kc + (size_t)small_kc * small_nout);
     const size_t sm2 =
         sizeof(float) * ((size_t)p->T * small_nout + 2 * (size_t)p->T * p->E);
