@@ -1,6 +1,8 @@
-"""Python binding of libmoe.so, the B200 (sm_100a) forward pass of a sparse
-Mixture-of-Experts SwiGLU FFN layer (noisy Top-K routing, capacity dispatch,
-grouped expert GEMMs on tcgen05 tensor cores, gate-weighted combine).
+"""Python binding of libmoe.so, the B200 (sm_100a) sparse Mixture-of-Experts SwiGLU
+FFN layer: the forward pass (noisy Top-K routing, capacity dispatch, grouped expert
+GEMMs on tcgen05 tensor cores, gate-weighted combine, gate statistics), its backward
+(moe_backward and its steps), the residual layer with shared neurons, the expert
+construction (moe_partition_*) and the clustering partition (moe_cluster_partition).
 
 The functions mirror the C ABI in ``include/moe.h`` one to one and only marshal
 arguments: torch tensors are passed as device pointers together with torch's
