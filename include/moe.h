@@ -438,6 +438,65 @@ int moe_backward_residual(const moe_params_t *p, const moe_buffers_t *b,
                           int32_t m_s, const void *h_s, void *dh_s, void *dx_s, void *dW13_s,
                           void *dW2_s, float dLb, void *ws, size_t ws_bytes, void *stream);
 
+/* ---- expert parallelism --------------------------------------------------
+ * "Llama 3 Meets MoE", section "训练框架" (5-D hybrid parallelism: Expert
+ * Parallelism places the experts of the MoE layer on different devices; the
+ * training configuration uses 8-way expert parallelism).  N ranks, rank r holds
+ * T_r tokens and the experts [r E/N, (r+1) E/N) (packed weights of those E/N
+ * experts only).  One layer step on rank r:
+ *   1. moe_route and moe_dispatch on its own tokens with capacity < 0 (dropless);
+ *   2. all ranks gather every rank's counts [E] into counts_all [N][E] and sum
+ *      probs_sum and importance (collectives of the caller, e.g. NCCL);
+ *   3. moe_ep_plan (host) on counts_all; moe_ep_mask_slots marks the dropped
+ *      assignments in slot_row;
+ *   4. run send_cnt[e] rows from x_perm row send_row[e] go to rank e / (E/N);
+ *      run i = p (E/N) + l from rank p lands at xin row recv_row[i] (recv_cnt[i]
+ *      rows); the runs between one pair of ranks pair up in expert order;
+ *   5. moe_expert_ffn on xin with E/N experts, k = 1, T = in_offsets[E/N] rows,
+ *      offsets in_offsets (copied to the device);
+ *   6. the same runs travel back (out rows from recv_row to send_row);
+ *   7. moe_combine with the masked slot_row; moe_ep_gate_stats. */
+enum { MOE_EP_CAPACITY_GLOBAL = 0, MOE_EP_CAPACITY_LOCAL = 1 };
+
+/* The exchange plan of rank `rank`.  Host-only; every rank computes the same
+ * keep_all from the same counts_all.
+ *   counts_all [N][E] (host int32): routed (pre-drop) rows of rank p for expert e.
+ *   capacity: rows an expert keeps (< 0: no limit).  scope GLOBAL: an expert's
+ *     assignments are ranked over the ranks' batches concatenated in rank order
+ *     (the layer then equals the one-device layer on that batch); LOCAL: each
+ *     rank's batch has its own capacity.  Inside a rank, lower tokens first
+ *     ("Llama 3 Meets MoE", section 3 "容量因子").
+ * Outputs (host int32, caller-allocated):
+ *   keep_all [N][E]  rows of rank p kept for expert e;
+ *   send_row [E], send_cnt [E]  this rank's run for expert e: dispatch-output
+ *     rows [send_row[e], send_row[e] + send_cnt[e]) (send_row is the prefix sum
+ *     of this rank's dropless counts);
+ *   recv_row [E], recv_cnt [E]  entry p (E/N) + l: the run of rank p for local
+ *     expert l lands at rows [recv_row, recv_row + recv_cnt) of xin;
+ *   in_offsets [E/N + 1]  expert-major offsets of xin (ranks ascending inside an
+ *     expert); in_offsets[E/N] = rows received.
+ * Errors: MOE_ERR_INVALID_ARG (NULL, rank outside [0,N), a negative count, bad
+ * scope), MOE_ERR_SHAPE (E outside 1..64, N not dividing E, row totals above
+ * 2^30). */
+int moe_ep_plan(const int32_t *counts_all, int32_t N, int32_t E, int32_t rank,
+                int32_t capacity, int32_t scope, int32_t *keep_all, int32_t *send_row,
+                int32_t *send_cnt, int32_t *recv_row, int32_t *recv_cnt, int32_t *in_offsets);
+
+/* Marks the assignments the capacity drops: slot_row[t][j] = -1 where
+ * slot_row[t][j] - offsets[topk_idx[t][j]] >= keep[topk_idx[t][j]].  p: this
+ * rank's layer (T = its tokens); topk_idx, offsets, slot_row from a dropless
+ * moe_dispatch (device); keep [E] host int32 (row `rank` of keep_all).  Entries
+ * already -1 or with an index outside [0,E) stay untouched. */
+int moe_ep_mask_slots(const moe_params_t *p, const int32_t *topk_idx, const int32_t *offsets,
+                      const int32_t *keep, int32_t *slot_row, void *stream);
+
+/* a6 over all ranks: counts[e] = sum_p counts_all[p][e] (device [N][E] -> [E]),
+ * then f, P and loss as moe_gate_stats with p->T = the tokens of all ranks and
+ * probs_sum the sum over ranks. */
+int moe_ep_gate_stats(const moe_params_t *p, const int32_t *counts_all, int32_t N,
+                      const float *probs_sum, int32_t *counts, float *f, float *P, float *loss,
+                      void *stream);
+
 /* Reads the device status word of `ws` (synchronises `stream`): *status is 0 or
  * one of MOE_ERR_DEVICE_*; clear != 0 resets it to 0 afterwards, together with
  * the workspace's internal launch counters. */

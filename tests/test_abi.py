@@ -205,3 +205,25 @@ def test_backward_rejects_bad_arguments_before_the_device(L):
     assert L.moe_route_backward(C.byref(p), a, a, a, None, None, a, a, a, a, C.c_float(1.0), a,
                                 a, a, a, None, None, a, n, None) == moe.MOE_ERR_INVALID_ARG
     assert b"together" in L.moe_last_error_string()
+
+
+def test_expert_parallel_calls_reject_bad_arguments_before_the_device(L):
+    a = C.c_void_p(256)
+    p = moe.params(64, 256, 8, 2, 128)
+    keep = (C.c_int32 * 8)(*([3] * 8))
+    mask = lambda pp=p, idx=a, off=a, kp=keep, sr=a: L.moe_ep_mask_slots(
+        C.byref(pp), idx, off, kp, sr, None)
+    assert mask(idx=None) == moe.MOE_ERR_INVALID_ARG
+    assert mask(kp=None) == moe.MOE_ERR_INVALID_ARG
+    assert mask(pp=moe.params(64, 256, 8, 9, 128)) == moe.MOE_ERR_INVALID_ARG
+    neg = (C.c_int32 * 8)(*([3] * 7 + [-1]))
+    assert mask(kp=neg) == moe.MOE_ERR_INVALID_ARG
+    assert mask(pp=moe.params(0, 256, 8, 2, 128)) == moe.MOE_OK  # nothing to mark
+    stats = lambda pp=p, ca=a, N=2, ps=a, out=a: L.moe_ep_gate_stats(
+        C.byref(pp), ca, N, ps, out, a, a, a, None)
+    assert stats(ca=None) == moe.MOE_ERR_INVALID_ARG
+    assert stats(out=None) == moe.MOE_ERR_INVALID_ARG
+    assert stats(N=3) == moe.MOE_ERR_SHAPE
+    assert stats(N=0) == moe.MOE_ERR_SHAPE
+    assert stats(N=16) == moe.MOE_ERR_SHAPE
+    assert b"N must divide E" in L.moe_last_error_string()

@@ -1,0 +1,230 @@
+"""Expert-parallel layer on the CPU: the exchange plan of libmoe (host code, no GPU)
+against a brute-force recount, and the layer's multi-rank data path (the plan plus
+``expert_parallel.exchange_runs`` over gloo, world size 2 and 4) with the fp64
+oracle doing each rank's arithmetic, against the oracle's one-process layer on the
+ranks' batches concatenated in rank order ("Llama 3 Meets MoE", section "训练框架",
+Expert Parallelism; section 3 "容量因子" for the capacity)."""
+import json
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import top_routing_grouped_noisy_b200 as moe  # noqa: E402
+
+GLOBAL, LOCAL = moe.EP_CAPACITY_GLOBAL, moe.EP_CAPACITY_LOCAL
+
+
+def _brute_keep(counts_all, capacity, scope):
+    """Rank every (rank, expert) assignment in the order the layer sees them and keep
+    those below the capacity (one list entry per assignment)."""
+    N, E = counts_all.shape
+    keep = np.zeros((N, E), np.int64)
+    for e in range(E):
+        seen = 0
+        for p in range(N):
+            local = 0
+            for _ in range(int(counts_all[p, e])):
+                pos = seen if scope == GLOBAL else local
+                if capacity < 0 or pos < capacity:
+                    keep[p, e] += 1
+                seen += 1
+                local += 1
+    return keep
+
+
+@pytest.mark.parametrize("N,E", [(1, 8), (2, 8), (4, 8), (8, 8), (4, 16), (8, 64), (3, 12)])
+@pytest.mark.parametrize("capacity", [-1, 0, 3, 11, 1000])
+@pytest.mark.parametrize("scope", [GLOBAL, LOCAL])
+def test_plan_matches_recount_and_pairs_up(N, E, capacity, scope):
+    rng = np.random.default_rng(N * 1000 + E * 10 + capacity + 7 * scope)
+    counts = rng.integers(0, 9, size=(N, E)).astype(np.int32)
+    counts[rng.random((N, E)) < 0.2] = 0
+    plans = [moe.moe_ep_plan(torch.from_numpy(counts), r, capacity, scope) for r in range(N)]
+    want = _brute_keep(counts, capacity, scope)
+    El = E // N
+    for r, pl in enumerate(plans):
+        assert np.array_equal(pl.keep_all.numpy(), want)
+        # sends: the kept prefix of each expert's block of the dropless dispatch output
+        blocks = np.concatenate([[0], np.cumsum(counts[r])])
+        assert np.array_equal(pl.send_row.numpy(), blocks[:E])
+        assert np.array_equal(pl.send_cnt.numpy(), want[r])
+        # receives tile [0, rows_in) expert-major, ranks ascending inside an expert
+        runs = pl.recv_runs()
+        pos = 0
+        for l in range(El):
+            assert int(pl.in_offsets[l]) == pos
+            for p in range(N):
+                peer, row, n, e = runs[p * El + l]
+                assert (peer, e) == (p, r * El + l)
+                assert row == pos and n == want[p, r * El + l]
+                pos += n
+        assert int(pl.in_offsets[El]) == pos == pl.rows_in
+    # between every pair, the non-empty runs one sends pair with those the other receives
+    for q in range(N):
+        for p in range(N):
+            sent = [(n, e) for (peer, _, n, e) in plans[q].send_runs() if peer == p and n > 0]
+            got = [(n, e) for (peer, _, n, e) in plans[p].recv_runs() if peer == q and n > 0]
+            assert sent == got
+
+
+def test_plan_global_capacity_totals():
+    counts = np.array([[5, 0, 2, 9], [4, 3, 0, 1], [6, 6, 6, 6], [0, 1, 2, 3]], np.int32)
+    pl = moe.moe_ep_plan(torch.from_numpy(counts), 0, capacity=7, scope=GLOBAL)
+    kept = pl.keep_all.numpy().sum(0)
+    assert np.array_equal(kept, np.minimum(counts.sum(0), 7))
+    pl = moe.moe_ep_plan(torch.from_numpy(counts), 0, capacity=7, scope=LOCAL)
+    assert np.array_equal(pl.keep_all.numpy(), np.minimum(counts, 7))
+
+
+@pytest.mark.parametrize("counts,rank,scope,code", [
+    ([[1, 2, 3]], 0, GLOBAL, moe.MOE_OK),
+    ([[1, 2, 3], [1, 1, 1]], 0, GLOBAL, moe.MOE_ERR_SHAPE),        # 2 ranks, 3 experts
+    ([[1, 2], [1, 1]], 2, GLOBAL, moe.MOE_ERR_INVALID_ARG),        # rank outside [0, N)
+    ([[1, -2], [1, 1]], 0, GLOBAL, moe.MOE_ERR_INVALID_ARG),       # negative count
+    ([[1, 2], [1, 1]], 0, 5, moe.MOE_ERR_INVALID_ARG),             # scope
+    ([[1] * 66, [1] * 66], 0, GLOBAL, moe.MOE_ERR_SHAPE),          # E > 64
+    ([[2 ** 30, 2 ** 30]], 0, GLOBAL, moe.MOE_ERR_SHAPE),          # too many rows
+])
+def test_plan_errors(counts, rank, scope, code):
+    c = torch.tensor(counts, dtype=torch.int32)
+    if code == moe.MOE_OK:
+        moe.moe_ep_plan(c, rank, -1, scope)
+        return
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_plan(c, rank, -1, scope)
+    assert ei.value.code == code
+
+
+# --------------------------------------------------------------------------- gloo layer
+
+def _layer_inputs(Ts, d, E, m, seed):
+    g = torch.Generator().manual_seed(seed)
+    Tall = sum(Ts)
+    x = torch.randn(Tall, d, generator=g)
+    Wg = torch.randn(d, E, generator=g) * 0.3
+    Wn = torch.randn(d, E, generator=g) * 0.3
+    eps = torch.randn(Tall, E, generator=g)
+    W1 = torch.randn(E, m, d, generator=g) * 0.2
+    W3 = torch.randn(E, m, d, generator=g) * 0.2
+    W2 = torch.randn(E, d, m, generator=g) * 0.2
+    f = lambda t: t.numpy().astype(np.float32)
+    return dict(x=f(x), Wg=f(Wg), Wn=f(Wn), eps=f(eps), W1=f(W1), W3=f(W3), W2=f(W2))
+
+
+def _ep_worker(rank, world, port, out_dir, cfg):
+    sys.path.insert(0, ROOT)
+    import oracle
+    from top_routing_grouped_noisy_b200 import moe_ep_plan
+    from top_routing_grouped_noisy_b200.expert_parallel import DistTransport
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
+                            world_size=world)
+    try:
+        Ts, d, E, k, m = cfg["Ts"], cfg["d"], cfg["E"], cfg["k"], cfg["m"]
+        inp = _layer_inputs(Ts, d, E, m, cfg["seed"])
+        a = sum(Ts[:rank])
+        T = Ts[rank]
+        x, eps = inp["x"][a:a + T], inp["eps"][a:a + T]
+        El = E // world
+        lo = rank * El
+        tr = DistTransport()
+        # step 1: route and dispatch this rank's tokens, no capacity
+        r = oracle.router(x, inp["Wg"], inp["Wn"], eps, None, k, cfg["router"])
+        dsp = oracle.dispatch(r["idx"], E, -1)
+        counts_T = torch.tensor(list(dsp["counts"]) + [T], dtype=torch.int32)
+        # step 2: collectives
+        counts_all = tr.all_gather(counts_T)
+        sums = torch.from_numpy(np.concatenate([r["probs_sum"], r["importance"]]))
+        tr.all_reduce_sum(sums)
+        # step 3: plan and the drop mask (slot position inside its expert's block >= keep)
+        plan = moe_ep_plan(counts_all[:, :E].contiguous(), rank, cfg["capacity"], cfg["scope"])
+        keep = plan.keep_all[rank].numpy()
+        sr = dsp["slot_row"].copy()
+        for t in range(T):
+            for j in range(k):
+                if sr[t, j] >= 0:
+                    e = r["idx"][t, j]
+                    if sr[t, j] - dsp["offsets"][e] >= keep[e]:
+                        sr[t, j] = -1
+        # step 4: rows to the experts' owners
+        x_perm = torch.from_numpy(np.ascontiguousarray(x[dsp["row_token"]])) if dsp["R"] else \
+            torch.zeros(1, d)
+        xin = torch.zeros(max(plan.rows_in, 1), d)
+        tr.exchange(x_perm, plan.send_runs(), xin, plan.recv_runs())
+        # step 5: the local experts (fp64 oracle)
+        R_in = plan.rows_in
+        off = plan.in_offsets.numpy()
+        eor = (np.searchsorted(off, np.arange(R_in), side="right") - 1).astype(np.int32)
+        if R_in:
+            out_loc = oracle.expert_ffn(inp["W1"][lo:lo + El], inp["W3"][lo:lo + El],
+                                        inp["W2"][lo:lo + El], xin[:R_in].numpy(), eor)
+        else:
+            out_loc = np.zeros((1, d))
+        # step 6: outputs back
+        out = torch.zeros(max(T * k, 1), d, dtype=torch.float64)
+        tr.exchange(torch.from_numpy(np.ascontiguousarray(out_loc)), plan.recv_runs(), out,
+                    plan.send_runs())
+        # step 7: combine
+        scale = E / k if cfg["rescale"] else 1.0
+        y = oracle.combine(out.numpy(), sr, r["G"], scale)
+        np.save(os.path.join(out_dir, "y%d.npy" % rank), y)
+        with open(os.path.join(out_dir, "r%d.json" % rank), "w") as fh:
+            json.dump({"counts_all": counts_all.tolist(), "sums": sums.tolist(),
+                       "keep_all": plan.keep_all.tolist(), "slot_row": sr.tolist()}, fh)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,Ts,E,k,capacity,scope,router,rescale", [
+    (2, [37, 20], 4, 2, -1, GLOBAL, 0, False),
+    (2, [37, 20], 4, 2, 9, GLOBAL, 0, True),
+    (2, [30, 41], 8, 3, 5, LOCAL, 1, True),
+    (4, [13, 0, 21, 8], 8, 2, 4, GLOBAL, 0, False),
+    (4, [16, 16, 16, 16], 4, 1, 6, GLOBAL, 1, False),
+])
+def test_ep_layer_over_gloo_equals_one_process_layer(tmp_path, world, Ts, E, k, capacity, scope,
+                                                      router, rescale):
+    import oracle
+    cfg = dict(Ts=Ts, d=16, E=E, k=k, m=8, capacity=capacity, scope=scope, router=router,
+               rescale=rescale, seed=sum(Ts) + E)
+    port = 29700 + (os.getpid() * 7 + world + E) % 900
+    mp.spawn(_ep_worker, args=(world, port, str(tmp_path), cfg), nprocs=world, join=True)
+    inp = _layer_inputs(Ts, 16, E, 8, cfg["seed"])
+    res = [json.load(open(tmp_path / ("r%d.json" % i))) for i in range(world)]
+    ys = [np.load(tmp_path / ("y%d.npy" % i)) for i in range(world)]
+    counts_all = np.array(res[0]["counts_all"])[:, :E]
+    if scope == GLOBAL:
+        full = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k, router,
+                              inp["Wn"], inp["eps"], None, capacity, rescale, 0.01)
+        want = [full["y"][sum(Ts[:i]):sum(Ts[:i + 1])] for i in range(world)]
+        assert np.array_equal(counts_all.sum(0), full["dispatch"]["counts"])
+        assert np.array_equal(np.array(res[0]["keep_all"]).sum(0), full["dispatch"]["kept"])
+        s = np.array(res[0]["sums"])
+        np.testing.assert_allclose(s[:E], full["router"]["probs_sum"], rtol=1e-12)
+        np.testing.assert_allclose(s[E:], full["router"]["importance"], rtol=1e-12)
+        _, _, L = oracle.gate_stats(sum(Ts), k, counts_all.sum(0), s[:E], 0.01)
+        assert L == pytest.approx(full["L"], rel=1e-12)
+    else:
+        want = []
+        for i in range(world):
+            a, b = sum(Ts[:i]), sum(Ts[:i + 1])
+            want.append(oracle.forward(inp["x"][a:b], inp["Wg"], inp["W1"], inp["W3"], inp["W2"],
+                                       k, router, inp["Wn"], inp["eps"][a:b], None, capacity,
+                                       rescale, 0.01)["y"])
+    for i in range(world):
+        # every rank's rows equal those of the one-process layer exactly: the same
+        # per-row fp64 arithmetic, only the rows' places differ
+        assert ys[i].shape == want[i].shape
+        assert np.array_equal(ys[i], want[i])
+    # every rank got the same plan
+    for i in range(1, world):
+        assert res[i]["keep_all"] == res[0]["keep_all"]
+    if capacity >= 0:
+        assert any(v == -1 for rr in res for row in rr["slot_row"] for v in row)

@@ -2,7 +2,9 @@
 FFN layer: the forward pass (noisy Top-K routing, capacity dispatch, grouped expert
 GEMMs on tcgen05 tensor cores, gate-weighted combine, gate statistics), its backward
 (moe_backward and its steps), the residual layer with shared neurons, the expert
-construction (moe_partition_*) and the clustering partition (moe_cluster_partition).
+construction (moe_partition_*), the clustering partition (moe_cluster_partition) and
+the non-collective steps of the expert-parallel layer (moe_ep_*; the layer itself is
+``expert_parallel.ExpertParallelMoE``).
 
 The functions mirror the C ABI in ``include/moe.h`` one to one and only marshal
 arguments: torch tensors are passed as device pointers together with torch's
@@ -26,7 +28,8 @@ __all__ = [
     "moe_cluster_partition", "moe_cluster_distances", "moe_backward_workspace_size",
     "moe_combine_backward", "moe_expert_down_backward", "moe_expert_up_backward",
     "moe_route_backward", "moe_backward", "BackwardBuffers",
-    "moe_backward_residual_workspace_size", "moe_backward_residual",
+    "moe_backward_residual_workspace_size", "moe_backward_residual", "EpPlan", "moe_ep_plan",
+    "moe_ep_mask_slots", "moe_ep_gate_stats", "EP_CAPACITY_GLOBAL", "EP_CAPACITY_LOCAL",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +53,8 @@ ST = 1
 DISJOINT = 0
 COPY = 1
 STACKED = 2
+EP_CAPACITY_GLOBAL = 0
+EP_CAPACITY_LOCAL = 1
 
 
 class MoeError(RuntimeError):
@@ -138,6 +143,9 @@ def lib():
             "moe_backward_residual_workspace_size": (sz, [P, i32]),
             "moe_backward_residual": (C.c_int, [P, C.POINTER(_Buffers), C.POINTER(_BwdBuffers), v,
                                                 v, i32, v, v, v, v, v, C.c_float, v, sz, v]),
+            "moe_ep_plan": (C.c_int, [v, i32, i32, i32, i32, i32, v, v, v, v, v, v]),
+            "moe_ep_mask_slots": (C.c_int, [P, v, v, v, v, v]),
+            "moe_ep_gate_stats": (C.c_int, [P, v, i32, v, v, v, v, v, v]),
             "moe_pipeline_create": (C.c_int, [P, v, v, v, v, v, i32, C.POINTER(v)]),
             "moe_pipeline_submit": (C.c_int, [v, v, v, v, v, C.POINTER(i64)]),
             "moe_pipeline_wait": (C.c_int, [v, i64]),
@@ -319,6 +327,71 @@ def moe_combine(p, out, slot_row, topk_w, y, stream=None):
 def moe_gate_stats(p, counts, probs_sum, f, P, loss, stream=None):
     _check(lib().moe_gate_stats(C.byref(p), _p(counts), _p(probs_sum), _p(f), _p(P), _p(loss),
                                 _stream(stream)))
+
+
+class EpPlan:
+    """Exchange plan of one rank of the expert-parallel layer (host int32 tensors):
+    keep_all [N][E], send_row/send_cnt [E] (indexed by expert), recv_row/recv_cnt [E]
+    (entry p*(E/N)+l: rank p's run for local expert l), in_offsets [E/N+1]."""
+
+    def __init__(self, N, E, rank, keep_all, send_row, send_cnt, recv_row, recv_cnt, in_offsets):
+        self.N, self.E, self.rank = N, E, rank
+        self.E_local = E // N
+        self.keep_all, self.send_row, self.send_cnt = keep_all, send_row, send_cnt
+        self.recv_row, self.recv_cnt, self.in_offsets = recv_row, recv_cnt, in_offsets
+
+    @property
+    def rows_in(self) -> int:
+        return int(self.in_offsets[-1])
+
+    def send_runs(self):
+        """(peer, first row, rows, expert) of the run this rank sends for each expert."""
+        El = self.E_local
+        return [(e // El, int(self.send_row[e]), int(self.send_cnt[e]), e)
+                for e in range(self.E)]
+
+    def recv_runs(self):
+        """(peer, first row, rows, expert) of every run this rank receives, grouped by
+        peer and in expert order inside a peer (the order the peer sends them in)."""
+        El = self.E_local
+        return [(i // El, int(self.recv_row[i]), int(self.recv_cnt[i]), self.rank * El + i % El)
+                for i in range(self.E)]
+
+
+def _host_i32(t, name):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.int32 or \
+            not t.is_contiguous():
+        raise ValueError("%s must be a contiguous host int32 tensor" % name)
+    return t.data_ptr()
+
+
+def moe_ep_plan(counts_all, rank, capacity=-1, scope=EP_CAPACITY_GLOBAL) -> EpPlan:
+    """counts_all: host int32 [N][E] (every rank's routed counts).  Runs on the host."""
+    c = torch.as_tensor(counts_all, dtype=torch.int32).contiguous()
+    if c.dim() != 2:
+        raise ValueError("counts_all must be [N][E]")
+    N, E = c.shape
+    El = E // N if N > 0 and E >= N else 0
+    z = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    keep, srow, scnt, rrow, rcnt, ioff = z(N, E), z(E), z(E), z(E), z(E), z(El + 1)
+    _check(lib().moe_ep_plan(_host_i32(c, "counts_all"), N, E, int(rank), int(capacity),
+                             int(scope), keep.data_ptr(), srow.data_ptr(), scnt.data_ptr(),
+                             rrow.data_ptr(), rcnt.data_ptr(), ioff.data_ptr()))
+    return EpPlan(N, E, int(rank), keep, srow, scnt, rrow, rcnt, ioff)
+
+
+def moe_ep_mask_slots(p, topk_idx, offsets, keep, slot_row, stream=None):
+    """keep: host int32 [E] (this rank's row of EpPlan.keep_all)."""
+    keep = torch.as_tensor(keep, dtype=torch.int32).contiguous()
+    if keep.numel() < p.E:
+        raise ValueError("keep needs E entries")
+    _check(lib().moe_ep_mask_slots(C.byref(p), _p(topk_idx), _p(offsets),
+                                   _host_i32(keep, "keep"), _p(slot_row), _stream(stream)))
+
+
+def moe_ep_gate_stats(p, counts_all, N, probs_sum, counts, f, P, loss, stream=None):
+    _check(lib().moe_ep_gate_stats(C.byref(p), _p(counts_all), int(N), _p(probs_sum),
+                                   _p(counts), _p(f), _p(P), _p(loss), _stream(stream)))
 
 
 class ForwardBuffers:

@@ -17,7 +17,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["api.cu", "partition.cu", "router.cu", "router_tc.cu", "dispatch.cu", "ffn_simt.cu",
            "ffn_tc.cu", "decode.cu", "combine.cu", "pipeline.cu",
-           "cluster.cu", "bwd_tc.cu", "bwd.cu"]
+           "cluster.cu", "bwd_tc.cu", "bwd.cu", "ep.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "--expt-relaxed-constexpr"]
 
