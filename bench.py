@@ -210,6 +210,9 @@ def parse():
                     help="time the clustering partition (balanced k-means of the W1 rows) "
                          "of the workload's FFN instead of the layer")
     ap.add_argument("--cluster-iters", type=int, default=10)
+    ap.add_argument("--expert-parallel", action="store_true",
+                    help="time the expert-parallel layer: each of the N ranks holds the "
+                         "workload's T tokens and E/N experts, rows move over NCCL")
     ap.add_argument("--backward", action="store_true",
                     help="time a training step (forward + backward) of the layer")
     return ap.parse_args()
@@ -481,6 +484,127 @@ def run_cluster(args, rank, world, local):
     return 0
 
 
+def run_expert_parallel(args, rank, world, local):
+    """The expert-parallel layer (expert_parallel.ExpertParallelMoE over NCCL): rank r
+    routes its own T tokens over all E experts and runs the grouped GEMMs of experts
+    [r E/N, (r+1) E/N) on the rows every rank sends it.  Capacity (if the workload has
+    one) over all ranks' tokens.  One step = one whole layer forward, host plan and
+    row exchanges included; weak scaling (T tokens per rank).  With N = 1 the group
+    has one rank and the exchanges are local copies."""
+    import datetime
+
+    import top_routing_grouped_noisy_b200 as moe
+    from top_routing_grouped_noisy_b200.expert_parallel import ExpertParallelMoE
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(29300 + os.getpid() % 600))
+        torch.distributed.init_process_group("nccl", rank=0, world_size=1,
+                                              timeout=datetime.timedelta(seconds=120),
+                                              device_id=torch.device("cuda", local))
+    w = wl.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.with_(T=args.tokens)
+    if w.E % world != 0 or w.shared > 0 or w.partition != wl.DISJOINT:
+        raise SystemExit("--expert-parallel needs a disjoint workload whose E divides N")
+    dt = wl.torch_dtype(w)
+    # the model (weights, router) is the same on every rank; the tokens differ
+    inp = wl.make_inputs(w, device="cuda", seed=w.seed)
+    tok = wl.make_inputs(w, device="cuda", seed=w.seed + 7919 * rank)
+    x, eps = tok["x"], tok["eps"]
+    del tok
+    C = moe.moe_capacity(w.T * world, w.E, w.cf) if w.cf >= 0 else -1
+    p = moe.params(w.T, w.d, w.E, w.k, w.m, dt, w.router, C, w.rescale, w.lam)
+    ws = moe.Workspace(p)
+    W13_e, W2_e = moe.moe_partition_experts(inp["W1"], inp["W3"], inp["W2"], w.E, moe.DISJOINT,
+                                            perm=inp["perm"], ws=ws)
+    El = w.E // world
+    lo = rank * El
+    W13_l = W13_e.view(w.E, -1)[lo:lo + El].clone().reshape(-1)
+    W2_l = W2_e.view(w.E, -1)[lo:lo + El].clone().reshape(-1)
+    del W13_e, W2_e
+    L = ExpertParallelMoE(w.d, w.E, w.k, w.m, W13_l, W2_l, inp["Wg"], inp["Wnoise"], inp["bias"],
+                          dt, w.router, C, moe.EP_CAPACITY_GLOBAL, w.rescale, w.lam)
+    for n in ("W1", "W3", "W2", "x", "eps"):
+        inp.pop(n, None)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        s = L.begin(x, eps)
+        L.gather_counts(s)
+        L.plan(s)
+        L.send_rows(s)
+        if ev is not None:
+            ev[0].record(stream)
+        L.experts(s)
+        if ev is not None:
+            ev[1].record(stream)
+        L.return_rows(s)
+        return L.finish(s)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    exp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    l0 = moe.moe_launch_count()
+    t_wall0 = time.time()
+    rows = 0
+    for (a, b), e in zip(evs, exp):
+        a.record(stream)
+        s = step(e)
+        b.record(stream)
+        rows += s.R_in
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall1 = time.time()
+    launches = moe.moe_launch_count() - l0
+    time.sleep(0.15)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    for wsx in (L._ws_route, L._ws_ffn):
+        if wsx is not None and moe.moe_get_device_status(wsx) != 0:
+            raise SystemExit("device status set by the expert-parallel layer")
+    # every step waits on the host for the counts (the plan), so the device time of a
+    # step is bracketed by its own events; the sum over the steps is the timed region
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    exp_ms = sum(a.elapsed_time(b) for a, b in exp) / args.steps
+    flop = 6.0 * w.d * w.m * rows / args.steps
+    tf = flop / (exp_ms / 1000.0) / 1e12
+    tf_slow = -max_over_ranks(-tf, world)  # the slowest rank's expert GEMMs
+    peaks, peak_src = load_peaks()
+    peak_t = peaks["bf16_tflops_sustained"]
+    torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "MoE-layer tokens/s (expert parallel)",
+        "value": tokens_per_s(w.T, args.steps, world, ms), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(w, C), workload="ep%d_%s" % (world, w.name),
+                       parallelism="ep%d" % world, tokens_per_rank=w.T,
+                       experts_per_rank=El, capacity_scope="global",
+                       global_batch=w.T * world),
+        "roofline": {"kernel": "moe_expert_ffn on the received rows (grouped GEMM 1 + SwiGLU, "
+                               "GEMM 2) of the slowest rank",
+                     "bound": "tensor", "achieved": tf_slow, "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": tf_slow / peak_t, "traffic": None,
+                     "peak_source": "%s bf16_tflops_sustained" % peak_src,
+                     "algorithmic": "6*d*m FLOP per received row"},
+        "kernels": {"expert_ffn_ms": exp_ms, "rows_in_per_step": rows / args.steps},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": launches, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_train(args, w, p, moe, fwd_step, b, x, Wg, Wn, eps, bias, W13_e, W2_e, C, inp, shared,
               rank, world, local):
     """A training step of the layer: the forward (the six step calls) and the backward
@@ -712,6 +836,8 @@ def main():
     torch.cuda.set_device(local)
     if args.cluster:
         return run_cluster(args, rank, world, local)
+    if args.expert_parallel:
+        return run_expert_parallel(args, rank, world, local)
     import top_routing_grouped_noisy_b200 as moe
 
     w = wl.WORKLOADS[args.workload]
