@@ -228,3 +228,33 @@ def test_ep_layer_over_gloo_equals_one_process_layer(tmp_path, world, Ts, E, k, 
         assert res[i]["keep_all"] == res[0]["keep_all"]
     if capacity >= 0:
         assert any(v == -1 for rr in res for row in rr["slot_row"] for v in row)
+
+
+@pytest.mark.parametrize("N,E,k,capacity", [(2, 8, 2, 5), (4, 8, 3, 7), (8, 16, 4, 2), (2, 4, 1, 0)])
+def test_plan_global_drops_equal_oracle_dispatch_of_concatenated_batch(N, E, k, capacity):
+    """The plan's kept prefix of each (rank, expert) block, applied to every rank's
+    dropless dispatch, keeps exactly the assignments the oracle's dispatch keeps on the
+    ranks' batches concatenated in rank order."""
+    import oracle
+    rng = np.random.default_rng(N * 97 + E + k)
+    Ts = [int(t) for t in rng.integers(0, 40, size=N)]
+    idx_all = np.stack([rng.permutation(E)[:k] for _ in range(sum(Ts))]).astype(np.int32) \
+        if sum(Ts) else np.zeros((0, k), np.int32)
+    full = oracle.dispatch(idx_all, E, capacity)
+    counts = []
+    dsp = []
+    a = 0
+    for T in Ts:
+        d = oracle.dispatch(idx_all[a:a + T], E, -1)
+        dsp.append(d)
+        counts.append(d["counts"])
+        a += T
+    pl = moe.moe_ep_plan(torch.from_numpy(np.array(counts, np.int32)), 0, capacity, GLOBAL)
+    keep = pl.keep_all.numpy()
+    a = 0
+    for r, T in enumerate(Ts):
+        sr = dsp[r]["slot_row"]
+        ix = idx_all[a:a + T]
+        mine = (sr >= 0) & (sr - dsp[r]["offsets"][ix] < keep[r][ix])
+        np.testing.assert_array_equal(mine, full["slot_row"][a:a + T] >= 0)
+        a += T
