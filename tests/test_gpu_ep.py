@@ -1,8 +1,8 @@
 """Expert-parallel layer on the GPU through the C ABI ("Llama 3 Meets MoE", section
 "训练框架", Expert Parallelism).
 
-Every gpurun box has one GPU, so the ranks are emulated: the layer objects of N
-ranks run their steps in lockstep in one process on one device, and a copy
+The ranks are emulated on one GPU: the layer objects of N ranks run their steps
+in lockstep in one process on one device, and a copy
 transport (below) stands in for the collectives by matching each rank's send
 runs with the receiving rank's runs of the same expert.  No kernel waits for
 another rank.  The result is checked against the fp64 oracle on the ranks'
