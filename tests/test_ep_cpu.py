@@ -258,3 +258,37 @@ def test_plan_global_drops_equal_oracle_dispatch_of_concatenated_batch(N, E, k, 
         mine = (sr >= 0) & (sr - dsp[r]["offsets"][ix] < keep[r][ix])
         np.testing.assert_array_equal(mine, full["slot_row"][a:a + T] >= 0)
         a += T
+
+
+def _dying_worker(rank, world, port, out_dir):
+    """Rank 1 leaves between the count gather and the row exchange (with nothing in
+    flight); rank 0 must get an error from its exchange, not wait for ever."""
+    import datetime
+    sys.path.insert(0, ROOT)
+    from top_routing_grouped_noisy_b200 import moe_ep_plan
+    from top_routing_grouped_noisy_b200.expert_parallel import DistTransport
+    dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=10))
+    tr = DistTransport()
+    counts_all = tr.all_gather(torch.tensor([3, 2, 1, 4, 0], dtype=torch.int32))
+    if rank == 1:
+        os._exit(0)
+    plan = moe_ep_plan(counts_all[:, :4].contiguous(), rank)
+    src = torch.zeros(10, 8)
+    dst = torch.zeros(max(plan.rows_in, 1), 8)
+    err = None
+    try:
+        tr.exchange(src, plan.send_runs(), dst, plan.recv_runs())
+    except Exception as e:  # the peer is gone: gloo reports it or the group times out
+        err = type(e).__name__
+    with open(os.path.join(out_dir, "dying.json"), "w") as fh:
+        json.dump({"error": err}, fh)
+    os._exit(0)
+
+
+@pytest.mark.timeout(180)
+def test_exchange_reports_a_rank_that_left(tmp_path):
+    port = 30700 + os.getpid() % 900
+    mp.spawn(_dying_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    res = json.load(open(tmp_path / "dying.json"))
+    assert res["error"] is not None
