@@ -158,8 +158,7 @@ def _one_rank_main(out_path):
     import datetime
     import torch.distributed as dist
     torch.cuda.set_device(0)
-    port = 29400 + os.getpid() % 500
-    dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % port, rank=0,
+    dist.init_process_group("nccl", init_method="file://%s.store" % out_path, rank=0,
                             world_size=1, timeout=datetime.timedelta(seconds=60))
     res = {}
     try:
