@@ -227,3 +227,41 @@ def test_expert_parallel_calls_reject_bad_arguments_before_the_device(L):
     assert stats(N=0) == moe.MOE_ERR_SHAPE
     assert stats(N=16) == moe.MOE_ERR_SHAPE
     assert b"N must divide E" in L.moe_last_error_string()
+
+
+def test_plain_c_program_links_and_plans(tmp_path):
+    """The boundary is plain C: a C99 program compiled against include/moe.h and linked
+    with libmoe.so calls the host-only exchange plan (no GPU needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "plan.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "moe.h"
+int main(void)
+{
+    const int32_t counts[2][4] = {{3, 1, 0, 2}, {1, 2, 2, 2}};
+    int32_t keep[2][4], srow[4], scnt[4], rrow[4], rcnt[4], off[3];
+    int rc = moe_ep_plan(&counts[0][0], 2, 4, 1, 3, MOE_EP_CAPACITY_GLOBAL, &keep[0][0], srow,
+                         scnt, rrow, rcnt, off);
+    if (rc != MOE_OK)
+        return 1;
+    for (int p = 0; p < 2; ++p)
+        for (int e = 0; e < 4; ++e)
+            printf("%d ", keep[p][e]);
+    printf("| %d %d %d\n", off[0], off[1], off[2]);
+    return moe_ep_plan(&counts[0][0], 2, 3, 0, -1, 0, &keep[0][0], srow, scnt, rrow, rcnt,
+                       off) == MOE_ERR_SHAPE ? 0 : 2;
+}
+''')
+    exe = tmp_path / "plan"
+    libdir = os.path.dirname(moe.LIB_PATH)
+    inc = os.path.join(os.path.dirname(libdir), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                    moe.LIB_PATH, "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    # expert 0: rank 0 fills the capacity of 3; expert 3: rank 0 holds 2, rank 1 keeps 1
+    assert out.stdout.split() == "3 1 0 2 0 2 2 1 | 0 2 5".split()
