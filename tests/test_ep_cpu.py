@@ -75,6 +75,38 @@ def test_plan_matches_recount_and_pairs_up(N, E, capacity, scope):
             assert sent == got
 
 
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.data())
+def test_plan_property_random_shapes(data):
+    """Random rank counts, expert counts, capacities and scopes: the plan equals the
+    brute-force recount, every receive buffer is tiled exactly, and the kept totals per
+    expert are min(routed, C) under GLOBAL."""
+    N = data.draw(st.sampled_from([1, 2, 4, 8]))
+    E = N * data.draw(st.integers(1, 64 // N))
+    counts = np.array(data.draw(st.lists(st.lists(st.integers(0, 20), min_size=E, max_size=E),
+                                         min_size=N, max_size=N)), np.int32)
+    C = data.draw(st.integers(-1, 50))
+    scope = data.draw(st.sampled_from([GLOBAL, LOCAL]))
+    want = _brute_keep(counts, C, scope)
+    rows_in = 0
+    for r in range(N):
+        pl = moe.moe_ep_plan(torch.from_numpy(counts), r, C, scope)
+        assert np.array_equal(pl.keep_all.numpy(), want)
+        runs = sorted((row, n) for (_, row, n, _) in pl.recv_runs())
+        pos = 0
+        for row, n in runs:
+            assert row == pos
+            pos += n
+        assert pos == pl.rows_in
+        rows_in += pl.rows_in
+    assert rows_in == want.sum()
+    if scope == GLOBAL and C >= 0:
+        assert np.array_equal(want.sum(0), np.minimum(counts.sum(0), C))
+
+
 def test_plan_global_capacity_totals():
     counts = np.array([[5, 0, 2, 9], [4, 3, 0, 1], [6, 6, 6, 6], [0, 1, 2, 3]], np.int32)
     pl = moe.moe_ep_plan(torch.from_numpy(counts), 0, capacity=7, scope=GLOBAL)
