@@ -36,6 +36,8 @@ def lib():
         _lib.oracle_silu.restype = d
         _lib.oracle_silu.argtypes = [d]
         _lib.oracle_capacity.argtypes = [i, i, d]
+        _lib.oracle_set_num_threads.argtypes = [i]
+        _lib.oracle_set_num_threads.restype = None
         _lib.oracle_partition.argtypes = [p, p, p, i, i, i, i, i, p, p, p, p]
         _lib.oracle_topk.argtypes = [i, i, p, p]
         _lib.oracle_router.argtypes = [i, i, i, i, i, p, i, p, p, p, p, p, p, p, p, p, p]
@@ -60,6 +62,11 @@ def lib():
 
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Host threads of the oracle's parallel loops from now on (results do not change)."""
+    lib().oracle_set_num_threads(int(n))
 
 
 def _dt(a: np.ndarray) -> int:

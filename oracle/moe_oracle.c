@@ -87,6 +87,19 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Sets the number of host threads later parallel loops use (n >= 1); the per-row
+ * arithmetic, and so every result, does not depend on it.  Used to time the oracle
+ * on one core. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n < 1 ? 1 : n);
+#else
+    (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------- */
 /* a0. Expert construction [V2 "专家构建方法"; UPCYCLE section 2].
  * DISJOINT: expert e owns intermediate neurons perm[e*m .. (e+1)*m), m = d_ff/E;
