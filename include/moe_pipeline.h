@@ -33,6 +33,8 @@ extern "C" {
 typedef struct moe_pipeline moe_pipeline_t; /* opaque */
 
 #define MOE_PIPELINE_MAX_DEPTH 4
+/* moe_pipeline_wait reports the status of any of the last this many batches. */
+#define MOE_PIPELINE_STATUS_RING 64
 
 /* Creates a pipeline for layer `p` (p->T >= 1) over caller-owned device
  * weights: Wg [d][E] and Wnoise [d][E] (NULL: no noise term) in p->dtype, bias
@@ -57,9 +59,10 @@ int moe_pipeline_submit(moe_pipeline_t *pl, const void *x_host, const float *noi
 
 /* Blocks until the outputs of batch `ticket` (and of every batch submitted
  * before it) are in host memory.  Returns MOE_OK, MOE_ERR_INVALID_ARG for a
- * ticket never issued, MOE_ERR_CUDA, or the device status the layer recorded
- * for this batch (MOE_ERR_DEVICE_*; the status word is sticky, so later
- * batches report it as well). */
+ * ticket never issued or older than the last MOE_PIPELINE_STATUS_RING
+ * submitted, MOE_ERR_CUDA, or the device status that this batch's own kernels
+ * recorded (MOE_ERR_DEVICE_*).  Every batch starts from a clear status word:
+ * an error in one batch is not reported for the batches before or after it. */
 int moe_pipeline_wait(moe_pipeline_t *pl, int64_t ticket);
 
 /* Waits for every submitted batch, then frees the streams, events and device

@@ -71,8 +71,9 @@ def test_pipeline_matches_forward(name):
 
 
 def test_pipeline_reports_bad_index_status():
-    """A NaN routing logit in batch 1 is reported by wait() for that batch and,
-    the status word being sticky, for the batches after it."""
+    """A NaN routing logit in batch 1 is reported by wait() for that batch only:
+    batches 0 and 2, queued around it before any wait, report MOE_OK, and batch 0's
+    status stays its own although batch 1's kernels ran before it was read."""
     w = W("pipe_nan", T=300, d=128, d_ff=512, E=8, k=2, seed=44)
     inp = wl.make_inputs(w)
     p = H.layer_params(w)
@@ -82,12 +83,18 @@ def test_pipeline_reports_bad_index_status():
     x_bad = inp["x"].clone()
     x_bad[17, :] = float("nan")
     x_bad = x_bad.pin_memory()
-    y = [torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
-    loss = [torch.empty(1).pin_memory() for _ in range(3)]
+    y = [torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    loss = [torch.empty(1).pin_memory() for _ in range(4)]
     with moe.Pipeline(p, inp["Wg"].cuda(), W13_e, W2_e, depth=2) as pl:
         t0 = pl.submit(x_ok, y[0], loss[0])
-        pl.wait(t0)
         t1 = pl.submit(x_bad, y[1], loss[1])
+        t2 = pl.submit(x_ok, y[2], loss[2])
+        pl.wait(t2)  # every batch is done; each status was snapshotted on its own
+        pl.wait(t0)
         with pytest.raises(moe.MoeError) as ei:
             pl.wait(t1)
         assert ei.value.code == moe.MOE_ERR_DEVICE_BADINDEX
+        pl.wait(t2)
+        t3 = pl.submit(x_ok, y[3], loss[3])
+        pl.wait(t3)
+    assert torch.equal(y[0].view(torch.int16), y[2].view(torch.int16))

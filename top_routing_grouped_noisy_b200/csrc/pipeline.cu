@@ -7,7 +7,9 @@
 //   compute(i) waits until h2d(i) landed and d2h(i - depth) emptied y of slot s,
 //   d2h(i)     waits until compute(i) finished.
 // The intermediates are shared by all slots because compute runs one batch at a
-// time on its own stream.
+// time on its own stream.  So is the workspace's status word: after each batch
+// the compute stream moves it into the slot's own device word and clears it, so
+// every batch reports only what its own kernels recorded.
 #include <cstring>
 #include <new>
 
@@ -27,7 +29,8 @@ struct moe_pipeline {
     cudaEvent_t out_done[MOE_PIPELINE_MAX_DEPTH] = {};
     int64_t slot_ticket[MOE_PIPELINE_MAX_DEPTH] = {};
     void *arena = nullptr;
-    int32_t *host_status = nullptr;  // pinned, one word per slot
+    int32_t *host_status = nullptr;  // pinned, one word per ticket modulo MOE_PIPELINE_STATUS_RING
+    int32_t *dev_status[MOE_PIPELINE_MAX_DEPTH] = {};  // the slot's batch's status word
     void *x[MOE_PIPELINE_MAX_DEPTH] = {};
     float *noise[MOE_PIPELINE_MAX_DEPTH] = {};
     void *y[MOE_PIPELINE_MAX_DEPTH] = {};
@@ -125,8 +128,8 @@ int moe_pipeline_create(const moe_params_t *p, const void *Wg, const void *Wnois
     PL_TRY(cudaStreamCreateWithFlags(&pl->h2d, cudaStreamNonBlocking));
     PL_TRY(cudaStreamCreateWithFlags(&pl->compute, cudaStreamNonBlocking));
     PL_TRY(cudaStreamCreateWithFlags(&pl->d2h, cudaStreamNonBlocking));
-    PL_TRY(cudaHostAlloc((void **)&pl->host_status, sizeof(int32_t) * MOE_PIPELINE_MAX_DEPTH,
-                         cudaHostAllocDefault));
+    PL_TRY(cudaHostAlloc((void **)&pl->host_status,
+                         sizeof(int32_t) * MOE_PIPELINE_STATUS_RING, cudaHostAllocDefault));
     if (e != cudaSuccess) {
         release(pl);
         return report_cuda(e, fn);
@@ -146,12 +149,13 @@ int moe_pipeline_create(const moe_params_t *p, const void *Wg, const void *Wnois
         return o;
     };
     size_t o_x[MOE_PIPELINE_MAX_DEPTH], o_n[MOE_PIPELINE_MAX_DEPTH], o_y[MOE_PIPELINE_MAX_DEPTH],
-        o_l[MOE_PIPELINE_MAX_DEPTH];
+        o_l[MOE_PIPELINE_MAX_DEPTH], o_st[MOE_PIPELINE_MAX_DEPTH];
     for (int s = 0; s < depth; ++s) {
         o_x[s] = take(pl->x_bytes);
         o_n[s] = take(pl->noise_bytes);
         o_y[s] = take(pl->x_bytes);
         o_l[s] = take(sizeof(float));
+        o_st[s] = take(sizeof(int32_t));
     }
     const size_t o_counts = take(E * 4), o_imp = take(E * 4), o_f = take(E * 4),
                  o_P = take(E * 4), o_idx = take(T * k * 4), o_w = take(T * k * 4),
@@ -170,6 +174,7 @@ int moe_pipeline_create(const moe_params_t *p, const void *Wg, const void *Wnois
         pl->noise[s] = pl->noise_bytes ? (float *)(a + o_n[s]) : nullptr;
         pl->y[s] = a + o_y[s];
         pl->loss[s] = (float *)(a + o_l[s]);
+        pl->dev_status[s] = (int32_t *)(a + o_st[s]);
         pl->slot_ticket[s] = -1;
     }
     moe_buffers_t &b = pl->shared;
@@ -261,7 +266,14 @@ int moe_pipeline_submit(moe_pipeline_t *pl, const void *x_host, const float *noi
         pl->broken = true;
         return rc;
     }
-    e = cudaEventRecord(pl->consumed[s], pl->compute);
+    // this batch's status word into the slot, then cleared for the next batch; both on
+    // the compute stream, so no later batch's kernels can touch it first
+    e = cudaMemcpyAsync(pl->dev_status[s], pl->ws, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                        pl->compute);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(pl->ws, 0, sizeof(int32_t), pl->compute);
+    if (e == cudaSuccess)
+        e = cudaEventRecord(pl->consumed[s], pl->compute);
     // out: y, L_balance and the status word of this batch
     if (e == cudaSuccess)
         e = cudaStreamWaitEvent(pl->d2h, pl->consumed[s], 0);
@@ -271,8 +283,8 @@ int moe_pipeline_submit(moe_pipeline_t *pl, const void *x_host, const float *noi
         e = cudaMemcpyAsync(loss_host, pl->loss[s], sizeof(float), cudaMemcpyDeviceToHost,
                             pl->d2h);
     if (e == cudaSuccess)
-        e = cudaMemcpyAsync(&pl->host_status[s], pl->ws, sizeof(int32_t),
-                            cudaMemcpyDeviceToHost, pl->d2h);
+        e = cudaMemcpyAsync(&pl->host_status[i % MOE_PIPELINE_STATUS_RING], pl->dev_status[s],
+                            sizeof(int32_t), cudaMemcpyDeviceToHost, pl->d2h);
     if (e == cudaSuccess)
         e = cudaEventRecord(pl->out_done[s], pl->d2h);
     if (e != cudaSuccess)
@@ -290,13 +302,17 @@ int moe_pipeline_wait(moe_pipeline_t *pl, int64_t ticket)
         return report_error(MOE_ERR_INVALID_ARG, "moe_pipeline_wait: pipeline is NULL");
     if (ticket < 0 || ticket >= pl->next_ticket)
         return report_error(MOE_ERR_INVALID_ARG, "moe_pipeline_wait: ticket was never issued");
+    if (pl->next_ticket - ticket > MOE_PIPELINE_STATUS_RING)
+        return report_error(MOE_ERR_INVALID_ARG,
+                            "moe_pipeline_wait: ticket older than the last "
+                            "MOE_PIPELINE_STATUS_RING batches (its status is no longer held)");
     const int s = (int)(ticket % pl->depth);
     // the slot's event marks its latest batch; d2h is in order, so that batch
     // finishing implies this one has
     cudaError_t e = cudaEventSynchronize(pl->out_done[s]);
     if (e != cudaSuccess)
         return pl_cuda(pl, e, fn);
-    const int32_t st = pl->host_status[s];
+    const int32_t st = pl->host_status[ticket % MOE_PIPELINE_STATUS_RING];
     if (st != 0)
         return report_error(st, "moe_pipeline_wait: a kernel recorded an error for this batch "
                                 "(status word of the pipeline's workspace)");
