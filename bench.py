@@ -43,8 +43,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes of one a3 launch (expert GEMM 1 + SwiGLU) from an ncu capture, keyed by
 # the source it was taken on; reported as null once the kernel source changes.
+# (default tile band of 2048 rows)
 NCU_TRAFFIC = {
-    "moe_2of8": {"src": "96ed2dffb627d991", "T": 16384, "bytes_per_launch": 589.66e6 + 110.52e6},
+    "moe_2of8": {"src": "2616f859d0f485cf", "T": 16384, "bytes_per_launch": 514.69e6 + 93.67e6},
+    "e8t2_cf4": {"src": "2616f859d0f485cf", "T": 32768,
+                 "bytes_per_launch": 19564.92e6 + 2852.40e6},
 }
 
 
@@ -967,6 +970,9 @@ def forward_line(args, w, rank, world, local):
         out_s = torch.empty(w.T, w.d, dtype=dt, device="cuda")
     b = moe.ForwardBuffers(p)
     x, Wg, Wn, eps, bias = inp["x"], inp["Wg"], inp["Wnoise"], inp["eps"], inp["bias"]
+    # the router weights in the tensor-core router's layout, packed once like W13_e / W2_e
+    Wt = moe.moe_router_pack(p, Wg, Wn) if dt == torch.bfloat16 else None
+    b.router_packed = Wt
     stream = torch.cuda.current_stream()
     # moe_forward's path: the dispatch materialises x_perm (the row-gathering GEMM 1
     # variant, moe_expert_up_gather, is slower on B200)
@@ -986,8 +992,12 @@ def forward_line(args, w, rank, world, local):
                 ev[i].record(stream)
 
         mark()
-        moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b.topk_idx, b.topk_w, b.probs_sum,
-                      b.importance)
+        if Wt is not None:  # router weights packed once per weight set
+            moe.moe_route_packed(p, x, Wg, Wn, Wt, eps, bias, ws, b.topk_idx, b.topk_w,
+                                 b.probs_sum, b.importance)
+        else:
+            moe.moe_route(p, x, Wg, Wn, eps, bias, ws, b.topk_idx, b.topk_w, b.probs_sum,
+                          b.importance)
         mark()
         if gather:
             moe.moe_dispatch_rows(p, b.topk_idx, ws, b.row_token, b.slot_row, b.counts, b.kept,

@@ -159,6 +159,32 @@ int moe_route(const moe_params_t *p, const void *x, const void *Wg, const void *
               const float *noise, const float *bias, int32_t *topk_idx, float *topk_w,
               float *probs_sum, float *importance, void *ws, size_t ws_bytes, void *stream);
 
+/* The router weights W_g (and W_noise) as the tensor-core router reads them: one
+ * K-major row per logit ([rows][d] bf16: row 2e = W_g[:, e], row 2e+1 = W_noise[:, e]
+ * with noise, row e = W_g[:, e] without; rows = 2E or E rounded up to 16, 32, 64 or
+ * 128; the other rows zero).  moe_route rebuilds them in the workspace on every call;
+ * a caller whose router weights do not change between calls (inference, or until the
+ * next optimizer step) packs them once with moe_router_pack and passes them to
+ * moe_route_packed or moe_forward (moe_buffers_t.router_packed), and must pack them
+ * again after changing W_g or W_noise.
+ * moe_router_packed_bytes: bytes of the packed buffer for p (bf16), noisy = whether
+ * W_noise is part of the router; 0 on bad params.  Host-only.
+ * moe_router_pack: writes the packed buffer Wt (device, 16-byte aligned) from Wg and
+ * Wnoise (NULL: none) [d][E] bf16.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_ALIGN,
+ * MOE_ERR_DTYPE (f32), MOE_ERR_CUDA. */
+size_t moe_router_packed_bytes(const moe_params_t *p, int32_t noisy);
+int moe_router_pack(const moe_params_t *p, const void *Wg, const void *Wnoise, void *Wt,
+                    void *stream);
+
+/* a1 with the router weights packed by moe_router_pack (Wt, for the same Wg/Wnoise
+ * and E): the same outputs as moe_route, without the packing pass.  Wg and Wnoise
+ * are still required: batches that do not run on the tensor-core router (f32, up to
+ * 64 tokens) read them directly. */
+int moe_route_packed(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
+                     const void *Wt, const float *noise, const float *bias, int32_t *topk_idx,
+                     float *topk_w, float *probs_sum, float *importance, void *ws,
+                     size_t ws_bytes, void *stream);
+
 /* a2. Dispatch with capacity ["Llama 3 Meets MoE", section 3 "容量因子"].
  * Stable counting sort of the T*k assignments by expert, token-ascending inside
  * an expert; assignment (t,j) is dropped iff its rank inside its expert is
@@ -173,6 +199,21 @@ int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx,
                  void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
                  int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* a2 right after moe_route ["Llama 3 Meets MoE", section 3 "容量因子"]: the same
+ * outputs as moe_dispatch for the indices that the last moe_route call on this
+ * workspace wrote, without counting them again.  moe_route leaves, in the
+ * workspace, how many tokens of each 32-token chunk it sent to each expert (the
+ * tensor-core router counts them in its gate epilogue), scanned into the chunks'
+ * rank bases; this call only ranks, writes the tables and copies x.  Requirements:
+ * the same workspace, the same p (T, E, k), topk_idx as written by that moe_route
+ * call and not changed since, and no other moe_route / moe_dispatch on this
+ * workspace in between; otherwise the results are undefined (use moe_dispatch).
+ * p->capacity may differ from the routing call's (it is applied here). */
+int moe_dispatch_routed(const moe_params_t *p, const void *x, const int32_t *topk_idx,
+                        void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
+                        int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes,
+                        void *stream);
+
 /* a2, tables only: moe_dispatch without the permuted copy of x (x_perm).  Same
  * counts, kept, offsets, row_token and slot_row.  For moe_expert_up_gather, which
  * reads the rows of x through row_token itself. */
@@ -184,8 +225,11 @@ int moe_dispatch_rows(const moe_params_t *p, const int32_t *topk_idx, int32_t *r
  * for callers that cannot allocate device memory or pass a workspace (for
  * example a host engine whose plugin interface hands a layer only its input and
  * output tensors and forbids allocation while work is enqueued).  Same inputs,
- * outputs and results as moe_dispatch; `status` (device int32, may be NULL)
- * receives MOE_ERR_DEVICE_BADINDEX like the workspace status word.
+ * outputs and results as moe_dispatch; `status` (device int32, 4-byte aligned)
+ * receives MOE_ERR_DEVICE_BADINDEX like the workspace status word (set only,
+ * never cleared: the caller zeroes it).  It is required when T > 0, since it is
+ * the only place a bad expert index is reported (MOE_ERR_INVALID_ARG if NULL);
+ * with T = 0 it may be NULL.
  * Scratch: a fixed 256 KiB array inside the library image, reserved on every
  * GPU that loads libmoe.so until the process exits; limit E * ceil(T/32) <=
  * 65536 (T <= 32768 at E = 64), larger sizes return MOE_ERR_SHAPE.  The first
@@ -269,6 +313,8 @@ typedef struct {
     int32_t *offsets;       /* [E+1] */
     void *h;                /* [T*k][m8] */
     void *out;              /* [T*k][d] */
+    /* optional input: Wg / Wnoise packed by moe_router_pack, or NULL (packed per call) */
+    const void *router_packed;
 } moe_buffers_t;
 
 /* a1 -> a2 -> a3 -> a4 -> a5 -> a6 on one stream, no host synchronisation. */
@@ -506,6 +552,15 @@ int moe_get_device_status(void *ws, int32_t *status, int32_t clear, void *stream
  * launch after this call (default 2e9).  0 makes every such wait give up at its
  * first check, which exercises the timeout path; tests use it.  Host-only. */
 void moe_set_wait_limit_ns(uint64_t ns);
+
+/* Tile order of the expert GEMMs on 2-SM pairs (4096 rows or more), a tuning knob
+ * with no effect on results: the CTA pairs that run at the same time take the
+ * output tiles of a band of `rows` rows of an expert (rounded up to 256) across all
+ * output columns before the next band, so the band's activations stay in L2 while
+ * the weight tiles stream past, and each weight tile is read by the band's pairs at
+ * about the same time.  Default 2048; 0 makes the band an expert's whole row range.
+ * Launches after the call use it.  Host-only. */
+void moe_set_gemm_band_rows(int32_t rows);
 
 #ifdef __cplusplus
 }

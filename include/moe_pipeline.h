@@ -13,7 +13,8 @@
  * Unlike the rest of the library the pipeline owns device memory: at create it
  * allocates, on the current device, `depth` input slots (x, noise), `depth`
  * output slots (y, loss, status), one set of intermediates (the layer runs one
- * batch at a time) and a workspace; destroy frees them.
+ * batch at a time), a workspace and, for bf16 layers, the router weights packed
+ * once for the tensor-core router (moe_router_pack); destroy frees them.
  *
  * Host buffers passed to submit should be page-locked (cudaHostAlloc or
  * cudaHostRegister); pageable memory works, but then CUDA copies it

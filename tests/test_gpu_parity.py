@@ -164,6 +164,52 @@ def test_steps_reproduce_forward_bit_exactly(name):
     assert torch.equal(bufs.h[:R, :w.m], b2.h[:R, :w.m])
 
 
+ROUTED_CASES = {
+    # the tensor-core router counts the chunks in its epilogue (vector and scalar B
+    # writer: E % 8 == 0 and E = 5; NOUT 16, 32 and 128; ragged last chunk)
+    "tc_noisy_cap": W("r_tc_noisy_cap", T=1000, d=256, d_ff=8 * 64, E=8, k=2, noisy=True,
+                      cf=1.1, seed=50),
+    "tc_e16_st_bias": W("r_tc_e16_st", T=2100, d=192, d_ff=16 * 48, E=16, k=4, router=wl.ST,
+                        noisy=True, bias=True, cf=0.9, seed=51),
+    "tc_e64_k8": W("r_tc_e64_k8", T=777, d=128, d_ff=64 * 16, E=64, k=8, noisy=True, seed=52),
+    "tc_e5_plain": W("r_tc_e5", T=301, d=136, d_ff=5 * 32, E=5, k=2, cf=0.7, seed=53),
+    # the other router paths end with the count kernel
+    "small_t40": W("r_small_t40", T=40, d=256, d_ff=8 * 32, E=8, k=2, noisy=True, cf=1.0,
+                   seed=54),
+    "f32": W("r_f32", T=300, d=64, d_ff=8 * 24, E=8, k=3, dtype="f32", cf=1.2, seed=55),
+}
+
+
+@pytest.mark.parametrize("name", list(ROUTED_CASES))
+def test_routed_dispatch_equals_dispatch(name):
+    """moe_dispatch_routed (the router's own chunk counts) gives the bytes moe_dispatch
+    gives on the same indices, with the routing call's capacity and with another one,
+    twice in a row; the tables are those of the oracle's dispatch of those indices."""
+    w = ROUTED_CASES[name]
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    x, Wg, Wn, eps, bias = (None if inp.get(n) is None else inp[n].to("cuda")
+                            for n in ("x", "Wg", "Wnoise", "eps", "bias"))
+    for rep, cap in enumerate((p.capacity, max(1, w.T * w.k // (2 * w.E)), p.capacity)):
+        q = H.layer_params(w, capacity=cap)
+        a, b = moe.ForwardBuffers(q), moe.ForwardBuffers(q)
+        moe.moe_route(p, x, Wg, Wn, eps, bias, ws, a.topk_idx, a.topk_w, a.probs_sum,
+                      a.importance)
+        moe.moe_dispatch_routed(q, x, a.topk_idx, ws, a.x_perm, a.row_token, a.slot_row,
+                                a.counts, a.kept, a.offsets)
+        moe.moe_dispatch(q, x, a.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
+                         b.kept, b.offsets)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status(ws) == 0
+        R = int(b.offsets[-1])
+        for n in ("counts", "kept", "offsets", "slot_row"):
+            assert torch.equal(getattr(a, n), getattr(b, n)), (rep, n)
+        assert torch.equal(a.row_token[:R], b.row_token[:R]), rep
+        assert torch.equal(a.x_perm[:R], b.x_perm[:R]), rep
+        H.check_dispatch(w, inp, q, a)
+
+
 @pytest.mark.parametrize("T,d,E,k", [(600, 320, 8, 2), (2500, 320, 8, 2), (2500, 200, 8, 2),
                                      (1100, 136, 16, 4)],
                          ids=["one_sm_kernel", "two_sm_kernel", "two_sm_k_tail",
@@ -287,3 +333,61 @@ def test_full_size_workload(name):
         C = moe.moe_capacity(w.T, w.E, w.cf)
         assert C == oracle.capacity(w.T, w.E, w.cf)
         assert (res["bufs"].kept.cpu() <= C).all()
+
+
+def test_gemm_band_order_changes_no_result():
+    """The 2-SM expert GEMMs give the same bytes whatever band of rows the concurrent
+    clusters sweep N over (whole experts, and bands of one, three and eight m-tiles)."""
+    w = W("band", T=5000, d=256, d_ff=8 * 176, E=8, k=2, noisy=True, cf=1.3, seed=56)
+    inp = wl.make_inputs(w)
+    p = H.layer_params(w)
+    ws = moe.Workspace(p)
+    W13_e, W2_e = H.gpu_weights(w, inp, ws)
+    b = moe.ForwardBuffers(p)
+    x, Wg, Wn, eps = (inp[n].cuda() for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_route(p, x, Wg, Wn, eps, None, ws, b.topk_idx, b.topk_w, b.probs_sum, b.importance)
+    moe.moe_dispatch_routed(p, x, b.topk_idx, ws, b.x_perm, b.row_token, b.slot_row, b.counts,
+                            b.kept, b.offsets)
+    R = int(b.offsets[-1].item())
+    res = []
+    try:
+        for band in (0, 256, 700, 2048):
+            moe.moe_set_gemm_band_rows(band)
+            h = torch.zeros_like(b.h)
+            out = torch.zeros_like(b.out)
+            moe.moe_expert_ffn(p, b.x_perm, b.offsets, W13_e, W2_e, h, out, ws)
+            torch.cuda.synchronize()
+            res.append((h[:R, :w.m].clone(), out[:R].clone()))
+    finally:
+        moe.moe_set_gemm_band_rows(2048)
+    assert moe.moe_get_device_status(ws) == 0
+    for h, out in res[1:]:
+        assert torch.equal(h, res[0][0]) and torch.equal(out, res[0][1])
+
+
+@pytest.mark.parametrize("name", ["mid_mixtral_noisy", "mid_st_bias_cap", "e64_k8", "odd_m_d",
+                                  "pair_e16_odd", "copy_exact"])
+def test_packed_router_weights_give_the_same_layer(name):
+    """moe_route_packed with the weights packed once by moe_router_pack, and moe_forward
+    given them, produce the bytes of moe_route / moe_forward packing per call."""
+    w = SMALL[name]
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, (W13_e, W2_e) = H.run_forward(w, inp)
+    assert status == 0
+    x, Wg, Wn, eps, bias = (None if inp.get(n) is None else inp[n].to("cuda")
+                            for n in ("x", "Wg", "Wnoise", "eps", "bias"))
+    Wt = moe.moe_router_pack(p, Wg, Wn)
+    assert Wt.numel() == moe.moe_router_packed_bytes(p, Wn is not None)
+    a = moe.ForwardBuffers(p)
+    moe.moe_route_packed(p, x, Wg, Wn, Wt, eps, bias, ws, a.topk_idx, a.topk_w, a.probs_sum,
+                         a.importance)
+    c = moe.ForwardBuffers(p)
+    moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, c, Wnoise=Wn, noise=eps, bias=bias,
+                    router_packed=Wt)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    for n in ("topk_idx", "topk_w", "probs_sum", "importance"):
+        assert torch.equal(getattr(a, n), getattr(bufs, n)), n
+    for n in ("y", "topk_idx", "topk_w", "probs_sum", "importance", "counts", "kept", "offsets",
+              "slot_row", "loss"):
+        assert torch.equal(getattr(c, n), getattr(bufs, n)), n

@@ -61,6 +61,10 @@ def test_noalloc_dispatch_rejects_oversize_and_reports_bad_index():
     f = [C.c_void_p(0x100000 + 256 * i) for i in range(10)]
     assert L.moe_dispatch_noalloc(C.byref(big), *f[:8], None, None) == moe.MOE_ERR_SHAPE
     assert b"fixed scratch" in L.moe_last_error_string()
+    small = moe.params(64, 64, 4, 2, 16)
+    # no status word for a non-empty batch: a bad index would go unreported
+    assert L.moe_dispatch_noalloc(C.byref(small), *f[:8], None, None) == moe.MOE_ERR_INVALID_ARG
+    assert b"status is NULL" in L.moe_last_error_string()
     w = wl.Workload("nb", T=64, d=64, d_ff=128, E=4, k=2, seed=92)
     x = wl.make_inputs(w)["x"].cuda()
     p = moe.params(w.T, w.d, w.E, w.k, w.m, torch.bfloat16)

@@ -19,10 +19,11 @@ import torch
 
 __all__ = [
     "MoeError", "Params", "lib", "params", "moe_capacity", "moe_version", "moe_launch_count",
-    "moe_partition_experts", "moe_workspace_size", "Workspace", "moe_route", "moe_dispatch",
-    "moe_dispatch_noalloc", "moe_dispatch_rows", "moe_expert_up_gather",
+    "moe_partition_experts", "moe_workspace_size", "Workspace", "moe_route", "moe_route_packed",
+    "moe_router_pack", "moe_router_packed_bytes", "moe_dispatch", "moe_dispatch_routed", "moe_dispatch_noalloc", "moe_dispatch_rows", "moe_expert_up_gather",
     "moe_expert_up", "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_gate_stats",
     "moe_forward", "ForwardBuffers", "moe_get_device_status", "moe_set_wait_limit_ns",
+    "moe_set_gemm_band_rows",
     "packed_w13_elems", "packed_w2_elems", "h_ld", "Pipeline", "moe_partition_residual",
     "moe_combine_residual", "moe_forward_residual", "moe_cluster_workspace_size",
     "moe_cluster_partition", "moe_cluster_distances", "moe_backward_workspace_size",
@@ -71,7 +72,7 @@ class Params(C.Structure):
 
 _BUF_FIELDS = ["x", "Wg", "Wnoise", "noise", "bias", "W13_e", "W2_e", "y", "loss", "counts",
                "importance", "f", "P", "topk_idx", "topk_w", "probs_sum", "x_perm", "row_token",
-               "slot_row", "kept", "offsets", "h", "out"]
+               "slot_row", "kept", "offsets", "h", "out", "router_packed"]
 
 
 class _Buffers(C.Structure):
@@ -104,6 +105,7 @@ def lib():
             "moe_last_error_string": (C.c_char_p, []),
             "moe_launch_count": (C.c_uint64, []),
             "moe_set_wait_limit_ns": (None, [C.c_uint64]),
+            "moe_set_gemm_band_rows": (None, [C.c_int32]),
             "moe_capacity": (i32, [i32, i32, f64]),
             "moe_packed_w13_elems": (i64, [i32, i32, i32]),
             "moe_packed_w2_elems": (i64, [i32, i32, i32]),
@@ -112,7 +114,11 @@ def lib():
             "moe_workspace_size": (sz, [P]),
             "moe_workspace_init": (C.c_int, [v, sz, v]),
             "moe_route": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v, sz, v]),
+            "moe_route_packed": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v, v, sz, v]),
+            "moe_router_pack": (C.c_int, [P, v, v, v, v]),
+            "moe_router_packed_bytes": (sz, [P, i32]),
             "moe_dispatch": (C.c_int, [P, v, v, v, v, v, v, v, v, v, sz, v]),
+            "moe_dispatch_routed": (C.c_int, [P, v, v, v, v, v, v, v, v, v, sz, v]),
             "moe_dispatch_noalloc": (C.c_int, [P, v, v, v, v, v, v, v, v, v, v]),
             "moe_dispatch_rows": (C.c_int, [P, v, v, v, v, v, v, v, sz, v]),
             "moe_expert_up_gather": (C.c_int, [P, v, v, v, v, v, v, sz, v]),
@@ -201,6 +207,11 @@ def moe_set_wait_limit_ns(ns: int) -> None:
     lib().moe_set_wait_limit_ns(int(ns))
 
 
+def moe_set_gemm_band_rows(rows: int) -> None:
+    """Tuning knob of the 2-SM expert GEMMs' tile order (results do not change)."""
+    lib().moe_set_gemm_band_rows(int(rows))
+
+
 def moe_capacity(T: int, E: int, cf: float) -> int:
     return int(lib().moe_capacity(T, E, float(cf)))
 
@@ -276,11 +287,41 @@ def moe_route(p, x, Wg, Wnoise, noise, bias, ws, topk_idx, topk_w, probs_sum, im
                            ws.nbytes, _stream(stream)))
 
 
+def moe_router_packed_bytes(p, noisy) -> int:
+    return int(lib().moe_router_packed_bytes(C.byref(p), 1 if noisy else 0))
+
+
+def moe_router_pack(p, Wg, Wnoise=None, out=None, stream=None):
+    """The router weights packed once for the tensor-core router (include/moe.h);
+    returns the packed device buffer (uint8)."""
+    n = moe_router_packed_bytes(p, Wnoise is not None)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=Wg.device)
+    _check(lib().moe_router_pack(C.byref(p), _p(Wg), _p(Wnoise), _p(out), _stream(stream)))
+    return out
+
+
+def moe_route_packed(p, x, Wg, Wnoise, Wt, noise, bias, ws, topk_idx, topk_w, probs_sum,
+                     importance, stream=None):
+    _check(lib().moe_route_packed(C.byref(p), _p(x), _p(Wg), _p(Wnoise), _p(Wt), _p(noise),
+                                  _p(bias), _p(topk_idx), _p(topk_w), _p(probs_sum),
+                                  _p(importance), ws.ptr, ws.nbytes, _stream(stream)))
+
+
 def moe_dispatch(p, x, topk_idx, ws, x_perm, row_token, slot_row, counts, kept, offsets,
                  stream=None):
     _check(lib().moe_dispatch(C.byref(p), _p(x), _p(topk_idx), _p(x_perm), _p(row_token),
                               _p(slot_row), _p(counts), _p(kept), _p(offsets), ws.ptr,
                               ws.nbytes, _stream(stream)))
+
+
+def moe_dispatch_routed(p, x, topk_idx, ws, x_perm, row_token, slot_row, counts, kept, offsets,
+                        stream=None):
+    """a2 right after moe_route on the same workspace: reuses the chunk counts the
+    router left there (topk_idx must be that call's output, unchanged)."""
+    _check(lib().moe_dispatch_routed(C.byref(p), _p(x), _p(topk_idx), _p(x_perm),
+                                     _p(row_token), _p(slot_row), _p(counts), _p(kept),
+                                     _p(offsets), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def moe_dispatch_rows(p, topk_idx, ws, row_token, slot_row, counts, kept, offsets, stream=None):
@@ -297,8 +338,10 @@ def moe_expert_up_gather(p, x, row_token, offsets, W13_e, h, ws, stream=None):
 
 
 def moe_dispatch_noalloc(p, x, topk_idx, x_perm, row_token, slot_row, counts, kept, offsets,
-                         status=None, stream=None):
-    """a2 without a workspace (fixed scratch inside the library; see include/moe.h)."""
+                         status, stream=None):
+    """a2 without a workspace (fixed scratch inside the library; see include/moe.h).
+    ``status`` is a device int32 tensor the caller zeroes; it is required for T > 0,
+    being the only place a bad expert index is reported."""
     _check(lib().moe_dispatch_noalloc(C.byref(p), _p(x), _p(topk_idx), _p(x_perm),
                                       _p(row_token), _p(slot_row), _p(counts), _p(kept),
                                       _p(offsets), _p(status), _stream(stream)))
@@ -419,12 +462,15 @@ class ForwardBuffers:
         self.offsets = torch.empty(E + 1, **i32)
         self.h = torch.empty(rows, h_ld(p.m), dtype=dt, device=device)
         self.out = torch.empty(rows, d, dtype=dt, device=device)
+        self.router_packed = None  # optional: moe_router_pack output for moe_forward
 
 
 def moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs: ForwardBuffers, Wnoise=None, noise=None,
-                bias=None, stream=None):
+                bias=None, stream=None, router_packed=None):
     b = _Buffers()
     vals = dict(x=x, Wg=Wg, Wnoise=Wnoise, noise=noise, bias=bias, W13_e=W13_e, W2_e=W2_e)
+    if router_packed is not None:  # else bufs.router_packed (None: packed per call)
+        vals["router_packed"] = router_packed
     for n in _BUF_FIELDS:
         t = vals[n] if n in vals else getattr(bufs, n)
         setattr(b, n, _p(t))

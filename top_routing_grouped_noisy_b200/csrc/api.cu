@@ -15,9 +15,13 @@ namespace moe {
 static thread_local char g_err[512] = "";
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+// 8 pair m-tiles: with the 74 clusters of a B200 at work, about an 8 x 9 block of
+// output tiles at a time, each A band and B tile read about once per block
+static std::atomic<int32_t> g_band_rows{2048};
 
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+int gemm_band_rows() { return g_band_rows.load(std::memory_order_relaxed); }
 
 static int fail(int code, const char *fmt, ...)
 {
@@ -101,15 +105,18 @@ WsLayout ws_layout(const moe_params_t *p)
         off += (bytes + 255) / 256 * 256;
         return o;
     };
+    L.dtick = take((size_t)kDecTickets * sizeof(int32_t));  // first: a fixed offset
     L.wt = take((size_t)kWtRows * p->d * es);
     const size_t blocks = (size_t)ceil_div(p->T > 0 ? p->T : 1, kRouterMinTokens);
     L.rpart = take(blocks * 2 * p->E * sizeof(float));
     const size_t chunks = (size_t)ceil_div(p->T > 0 ? p->T : 1, kDispatchChunk);
     L.hist = take(chunks * p->E * sizeof(int32_t));
+    L.dcounts = take(MOE_MAX_EXPERTS * sizeof(int32_t));
     // Sections for small batches are sized for min(T, 64) tokens even when T is
     // larger, so that a workspace sized for T also serves every smaller batch.
     const int t_small = p->T < kRouterSmallTokens ? (p->T > 0 ? p->T : 1) : kRouterSmallTokens;
     L.rsmall = take((size_t)kRouterSmallSplit * t_small * 2 * p->E * sizeof(float));
+    L.dpre = take(p->dtype == MOE_BF16 ? decode_partial_floats(p) * sizeof(float) : 0);
     L.total = off;
     return L;
 }
@@ -155,6 +162,8 @@ const char *moe_last_error_string(void) { return g_err; }
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+void moe_set_gemm_band_rows(int32_t rows) { g_band_rows.store(rows < 0 ? 0 : rows); }
 
 int32_t moe_capacity(int32_t T, int32_t E, double cf)
 {
@@ -260,11 +269,11 @@ int moe_partition_experts(const void *W1, const void *W3, const void *W2, int32_
     return after_launch(fn, e);
 }
 
-int moe_route(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
-              const float *noise, const float *bias, int32_t *topk_idx, float *topk_w,
-              float *probs_sum, float *importance, void *ws, size_t ws_bytes, void *stream)
+static int route_impl(const char *fn, const moe_params_t *p, const void *x, const void *Wg,
+                      const void *Wnoise, const void *Wt, const float *noise, const float *bias,
+                      int32_t *topk_idx, float *topk_w, float *probs_sum, float *importance,
+                      void *ws, size_t ws_bytes, void *stream)
 {
-    const char *fn = "moe_route";
     int rc = check_params(fn, p);
     if (rc != MOE_OK)
         return rc;
@@ -282,10 +291,52 @@ int moe_route(const moe_params_t *p, const void *x, const void *Wg, const void *
     if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
         return rc;
     char *w = static_cast<char *>(ws);
-    cudaError_t e = launch_route(p, x, Wg, Wnoise, noise, bias, topk_idx, topk_w, probs_sum,
-                                 importance, w, reinterpret_cast<int32_t *>(w),
+    cudaError_t e = launch_route(p, x, Wg, Wnoise, Wt, noise, bias, topk_idx, topk_w,
+                                 probs_sum, importance, w, reinterpret_cast<int32_t *>(w),
                                  (cudaStream_t)stream);
     return after_launch(fn, e);
+}
+
+int moe_route(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
+              const float *noise, const float *bias, int32_t *topk_idx, float *topk_w,
+              float *probs_sum, float *importance, void *ws, size_t ws_bytes, void *stream)
+{
+    return route_impl("moe_route", p, x, Wg, Wnoise, nullptr, noise, bias, topk_idx, topk_w,
+                      probs_sum, importance, ws, ws_bytes, stream);
+}
+
+size_t moe_router_packed_bytes(const moe_params_t *p, int32_t noisy)
+{
+    if (check_params("moe_router_packed_bytes", p) != MOE_OK)
+        return 0;
+    const size_t es = p->dtype == MOE_BF16 ? 2 : 4;
+    return (size_t)router_packed_rows(p->E, noisy != 0) * p->d * es;
+}
+
+int moe_router_pack(const moe_params_t *p, const void *Wg, const void *Wnoise, void *Wt,
+                    void *stream)
+{
+    const char *fn = "moe_router_pack";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    REQUIRE_PTR(Wg);
+    OPTIONAL_PTR(Wnoise);
+    REQUIRE_PTR(Wt);
+    if (p->dtype != MOE_BF16)
+        return fail(MOE_ERR_DTYPE, "%s: only bf16 router weights are packed", fn);
+    return after_launch(fn, launch_router_pack(p, Wg, Wnoise, Wt, (cudaStream_t)stream));
+}
+
+int moe_route_packed(const moe_params_t *p, const void *x, const void *Wg, const void *Wnoise,
+                     const void *Wt, const float *noise, const float *bias, int32_t *topk_idx,
+                     float *topk_w, float *probs_sum, float *importance, void *ws,
+                     size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_route_packed";
+    REQUIRE_PTR(Wt);
+    return route_impl(fn, p, x, Wg, Wnoise, Wt, noise, bias, topk_idx, topk_w, probs_sum,
+                      importance, ws, ws_bytes, stream);
 }
 
 int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx, void *x_perm,
@@ -308,7 +359,32 @@ int moe_dispatch(const moe_params_t *p, const void *x, const int32_t *topk_idx, 
         return rc;
     char *w = static_cast<char *>(ws);
     cudaError_t e = launch_dispatch(p, x, topk_idx, x_perm, row_token, slot_row, counts, kept,
-                                    offsets, w, reinterpret_cast<int32_t *>(w),
+                                    offsets, w, reinterpret_cast<int32_t *>(w), false,
+                                    (cudaStream_t)stream);
+    return after_launch(fn, e);
+}
+
+int moe_dispatch_routed(const moe_params_t *p, const void *x, const int32_t *topk_idx,
+                        void *x_perm, int32_t *row_token, int32_t *slot_row, int32_t *counts,
+                        int32_t *kept, int32_t *offsets, void *ws, size_t ws_bytes, void *stream)
+{
+    const char *fn = "moe_dispatch_routed";
+    int rc = check_params(fn, p);
+    if (rc != MOE_OK)
+        return rc;
+    REQUIRE_TOK(x);
+    REQUIRE_TOK(topk_idx);
+    REQUIRE_TOK(x_perm);
+    REQUIRE_TOK(row_token);
+    REQUIRE_TOK(slot_row);
+    REQUIRE_PTR(counts);
+    REQUIRE_PTR(kept);
+    REQUIRE_PTR(offsets);
+    if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+        return rc;
+    char *w = static_cast<char *>(ws);
+    cudaError_t e = launch_dispatch(p, x, topk_idx, x_perm, row_token, slot_row, counts, kept,
+                                    offsets, w, reinterpret_cast<int32_t *>(w), true,
                                     (cudaStream_t)stream);
     return after_launch(fn, e);
 }
@@ -331,7 +407,7 @@ int moe_dispatch_rows(const moe_params_t *p, const int32_t *topk_idx, int32_t *r
         return rc;
     char *w = static_cast<char *>(ws);
     cudaError_t e = launch_dispatch(p, nullptr, topk_idx, nullptr, row_token, slot_row, counts,
-                                    kept, offsets, w, reinterpret_cast<int32_t *>(w),
+                                    kept, offsets, w, reinterpret_cast<int32_t *>(w), false,
                                     (cudaStream_t)stream);
     return after_launch(fn, e);
 }
@@ -379,8 +455,8 @@ int moe_expert_up(const moe_params_t *p, const void *x_perm, const int32_t *offs
     cudaError_t e;
     if (p->dtype == MOE_F32)
         e = launch_up_simt(p, (const float *)x_perm, offsets, (const float *)W13_e, (float *)h, s);
-    else if (p->T <= kDecodeMaxTokens)
-        e = launch_up_decode(p, x_perm, offsets, W13_e, h, s);
+    else if (decode_fits(p))
+        e = launch_up_decode(p, x_perm, offsets, W13_e, h, static_cast<char *>(ws), s);
     else
         e = launch_up_tc(p, x_perm, offsets, W13_e, h, reinterpret_cast<int32_t *>(ws), s);
     return after_launch(fn, e);
@@ -405,8 +481,8 @@ int moe_expert_down(const moe_params_t *p, const void *h, const int32_t *offsets
     cudaError_t e;
     if (p->dtype == MOE_F32)
         e = launch_down_simt(p, (const float *)h, offsets, (const float *)W2_e, (float *)out, s);
-    else if (p->T <= kDecodeMaxTokens)
-        e = launch_down_decode(p, h, offsets, W2_e, out, s);
+    else if (decode_fits(p))
+        e = launch_down_decode(p, h, offsets, W2_e, out, static_cast<char *>(ws), s);
     else
         e = launch_down_tc(p, h, offsets, W2_e, out, reinterpret_cast<int32_t *>(ws), s);
     return after_launch(fn, e);
@@ -468,9 +544,10 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
     REQUIRE_PTR(b->loss);
     REQUIRE_PTR(b->f);
     REQUIRE_PTR(b->P);
-    if (small_forward_fits(p, b->Wnoise != nullptr)) {
-        // decode-shaped batch: router slices, then router finish + dispatch tables +
-        // gate statistics in one CTA, GEMM 1 gathering rows of x, GEMM 2, combine
+    if (small_forward_fits(p, b->Wnoise != nullptr) && decode_fits(p)) {
+        // decode-shaped batch, three launches: router slices whose last CTA finishes
+        // the router and builds the dispatch tables and gate statistics; GEMM 1
+        // gathering rows of x; GEMM 2 with the combine
         REQUIRE_PTR(b->x);
         REQUIRE_PTR(b->Wg);
         OPTIONAL_PTR(b->Wnoise);
@@ -499,18 +576,19 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
         cudaError_t e = launch_route_dispatch_small(p, b, w, reinterpret_cast<int32_t *>(w), s);
         if (e == cudaSuccess)
             e = launch_up_decode_gather(p, b->x, b->row_token, b->offsets, b->W13_e, b->h,
-                                        b->x_perm, s);
-        if (e == cudaSuccess)
-            e = launch_down_decode(p, b->h, b->offsets, b->W2_e, b->out, s);
-        if (e == cudaSuccess)
-            e = launch_combine(p, b->out, b->slot_row, b->topk_w, b->y, s);
+                                        b->x_perm, w, b->W2_e, s);
+        if (e == cudaSuccess)  // GEMM 2 with the combine of the columns it finishes
+            e = launch_down_decode(p, b->h, b->offsets, b->W2_e, b->out, w, s, b->slot_row,
+                                   b->topk_w, b->y);
         return after_launch(fn, e);
     }
-    if ((rc = moe_route(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx, b->topk_w,
-                        b->probs_sum, b->importance, ws, ws_bytes, stream)) != MOE_OK)
+    if ((rc = route_impl("moe_forward", p, b->x, b->Wg, b->Wnoise, b->router_packed, b->noise,
+                         b->bias, b->topk_idx, b->topk_w, b->probs_sum, b->importance, ws,
+                         ws_bytes, stream)) != MOE_OK)
         return rc;
-    if ((rc = moe_dispatch(p, b->x, b->topk_idx, b->x_perm, b->row_token, b->slot_row,
-                           b->counts, b->kept, b->offsets, ws, ws_bytes, stream)) != MOE_OK)
+    if ((rc = moe_dispatch_routed(p, b->x, b->topk_idx, b->x_perm, b->row_token, b->slot_row,
+                                  b->counts, b->kept, b->offsets, ws, ws_bytes, stream)) !=
+        MOE_OK)
         return rc;
     if ((rc = moe_expert_ffn(p, b->x_perm, b->offsets, b->W13_e, b->W2_e, b->h, b->out, ws,
                              ws_bytes, stream)) != MOE_OK)
@@ -613,8 +691,9 @@ int moe_forward_residual(const moe_params_t *p, const moe_buffers_t *b, const vo
     if ((rc = moe_route(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, b->topk_idx, b->topk_w,
                         b->probs_sum, b->importance, ws, ws_bytes, stream)) != MOE_OK)
         return rc;
-    if ((rc = moe_dispatch(p, b->x, b->topk_idx, b->x_perm, b->row_token, b->slot_row,
-                           b->counts, b->kept, b->offsets, ws, ws_bytes, stream)) != MOE_OK)
+    if ((rc = moe_dispatch_routed(p, b->x, b->topk_idx, b->x_perm, b->row_token, b->slot_row,
+                                  b->counts, b->kept, b->offsets, ws, ws_bytes, stream)) !=
+        MOE_OK)
         return rc;
     if ((rc = moe_expert_ffn(p, b->x_perm, b->offsets, b->W13_e, b->W2_e, b->h, b->out, ws,
                              ws_bytes, stream)) != MOE_OK)

@@ -23,6 +23,8 @@ constexpr size_t kWsHeader = 256;
 constexpr int kWsCounterWord = 1;
 // Word 2: ticket counter of the tensor-core router (zero between calls).
 constexpr int kWsRouterCounterWord = 2;
+// Word 3: ticket counter of the decode-size router + dispatch kernel (zero between calls).
+constexpr int kWsSmallCounterWord = 3;
 // Header bytes that clearing the status resets (status word and counters).
 constexpr size_t kWsResetBytes = 32;
 // Words 8-9: offsets {0, T} of the shared block's one-expert GEMMs (residual MoE).

@@ -568,7 +568,12 @@ struct PairTile {
     int e, row0, row_end, n0;
 };
 
-__device__ __forceinline__ PairTile decode_pair_tile(const Aux *aux, int tile)
+// Tile order inside an expert: bands of `band` m-tiles (0: the whole expert, split
+// into equal bands), m-tiles fastest inside a band, then the band's n-tiles, then the
+// next band.  Clusters working at the same time share one band of A rows (kept in L2
+// while the band sweeps N) and the few B tiles of its current n-tiles.
+__device__ __forceinline__ PairTile decode_pair_tile(const Aux *aux, int tile, int n_tiles,
+                                                     int band)
 {
     PairTile t;
     int e = 0;
@@ -577,7 +582,13 @@ __device__ __forceinline__ PairTile decode_pair_tile(const Aux *aux, int tile)
     const int local = tile - aux->tstart[e];
     const int rows = aux->off[e + 1] - aux->off[e];
     const int mtiles = (rows + 2 * BM - 1) / (2 * BM);
-    const int mt = local % mtiles, nt = local / mtiles;
+    int G = (band > 0 && band < mtiles) ? band : mtiles;
+    const int nbands = (mtiles + G - 1) / G;
+    G = (mtiles + nbands - 1) / nbands;
+    const int bi = local / (G * n_tiles);
+    const int rem = local - bi * G * n_tiles;
+    const int gr = mtiles - bi * G < G ? mtiles - bi * G : G;
+    const int mt = bi * G + rem % gr, nt = rem / gr;
     t.e = e;
     t.row0 = aux->off[e] + mt * 2 * BM;
     t.row_end = aux->off[e + 1];
@@ -592,7 +603,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             const __grid_constant__ CUtensorMap tmO,
                             const int32_t *__restrict__ offsets, int E, int N, int K,
                             bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
-                            uint64_t wait_ns, const int32_t *__restrict__ row_token)
+                            uint64_t wait_ns, const int32_t *__restrict__ row_token, int band)
 {
     pdl_wait();
     pdl_trigger();
@@ -660,7 +671,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int tile = cluster_id; tile < total; tile += nclusters) {
             if (__shfl_sync(0xffffffffu, (int)*abort_flag, 0))
                 break;
-            const PairTile t = decode_pair_tile(aux, tile);
+            const PairTile t = decode_pair_tile(aux, tile, n_tiles, band);
             int src[4] = {0, 0, 0, 0};
             if constexpr (GATHER) {
 #pragma unroll
@@ -768,7 +779,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster_id; tile < total; tile += nclusters) {
-            const PairTile t = decode_pair_tile(aux, tile);
+            const PairTile t = decode_pair_tile(aux, tile, n_tiles, band);
             if (!tc::mbar_wait(tc::smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag,
                                status))
                 break;
@@ -952,12 +963,16 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
+    // band of A rows that concurrent clusters sweep N over, in pair m-tiles (0: the
+    // whole expert)
+    const int band_rows = gemm_band_rows();
+    const int band = band_rows <= 0 ? 0 : (band_rows + 2 * BM - 1) / (2 * BM);
     if (gather)
         return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, true>, ta, tb, to,
                                   offsets, E, N, K, out, ld_out, n_valid, status, wait_ns,
-                                  row_token);
+                                  row_token, band);
     return cudaLaunchKernelEx(&cfg, tc2::grouped_gemm_2sm_kernel<EPI, false>, ta, tb, to, offsets,
-                              E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+                              E, N, K, out, ld_out, n_valid, status, wait_ns, row_token, band);
 }
 
 }  // namespace tc

@@ -31,16 +31,24 @@ __host__ __device__ inline int router_small_kc(int d)
 
 // Byte offsets of the sections of the caller's workspace.
 struct WsLayout {
-    size_t wt;     // router weights transposed to [nout_pad][d] (dtype)
+    size_t wt;     // router weights transposed to [nout_pad][d] (dtype; backward, f32 router)
     size_t rpart;  // router per-CTA partial sums [blocks][2][E] f32
     size_t hist;   // dispatch per-chunk counts, then bases, [E][chunks] int32
+    size_t dcounts;// routed count of every expert [E] int32 (next to the chunk bases)
     size_t rsmall; // small-batch router partial logits [32][T][2E] f32 (T <= 64)
+    size_t dtick;  // decode GEMM block tickets, kDecTickets int32 right after the header
+    size_t dpre;   // decode GEMM partial sums (T <= 16) f32
     size_t total;
 };
+// The decode GEMMs' tickets sit at the same offset, with the same size, in the
+// layout of every parameter set, so calls with other shapes on the same workspace
+// (a shared block, a changing row count) never find stale data there: every
+// ticket is zero between calls.
+constexpr int kDecTickets = 16384;
 WsLayout ws_layout(const moe_params_t *p);
 
-inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
-inline int ceil_div(int v, int m) { return (v + m - 1) / m; }
+__host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+__host__ __device__ inline int ceil_div(int v, int m) { return (v + m - 1) / m; }
 
 // Error reporting of the C ABI, for entry points outside api.cu.
 int validate_params(const char *fn, const moe_params_t *p);
@@ -72,29 +80,51 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 void count_launch(int n = 1);
 // Current time limit of bounded device waits (ns).
 uint64_t wait_limit_ns();
+// Rows of A that the 2-SM grouped GEMM's concurrent clusters sweep N over (0: all
+// of an expert's rows).
+int gemm_band_rows();
 
 // Every launcher returns cudaSuccess or the launch error.
 cudaError_t launch_partition(const void *W1, const void *W3, const void *W2, int d, int d_ff,
                              int E, int m, int mode, const int32_t *perm, int dtype,
                              void *W13_e, void *W2_e, int32_t *status, cudaStream_t s);
 
+// a1; Wt: the router weights packed by launch_router_pack (used by the tensor-core
+// router), or NULL to pack them into the workspace first
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
-                         const void *Wnoise, const float *noise, const float *bias,
-                         int32_t *idx, float *w, float *probs_sum, float *importance,
-                         char *ws, int32_t *status, cudaStream_t s);
+                         const void *Wnoise, const void *Wt, const float *noise,
+                         const float *bias, int32_t *idx, float *w, float *probs_sum,
+                         float *importance, char *ws, int32_t *status, cudaStream_t s);
 
+// Rows of the packed router weights [rows][d]: 2E (noisy) or E, padded to 16..128.
+int router_packed_rows(int E, bool noisy);
+cudaError_t launch_router_pack(const moe_params_t *p, const void *Wg, const void *Wnoise, void *Wt,
+                               cudaStream_t s);
 // a1 on the tcgen05 tensor cores (bf16), token sums included (per-CTA partials in
 // `part`, added by the CTA that finishes last; `counter` is zero between calls).
-cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wg,
-                            const void *Wnoise, const float *noise, const float *bias,
-                            int32_t *idx, float *w, float *probs_sum, float *importance,
-                            float *part, int32_t *counter, __nv_bfloat16 *Wt, int32_t *status,
-                            cudaStream_t s);
+// The gate epilogue also counts the chunks of a2 (hist), which the last CTA scans
+// into chunk bases and routed counts (dcounts).
+cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wt, bool noisy,
+                            const float *noise, const float *bias, int32_t *idx, float *w,
+                            float *probs_sum, float *importance, float *part, int32_t *counter,
+                            int32_t *hist, int32_t *dcounts, int32_t *status, cudaStream_t s);
 
+// a2 count step: chunk histogram of idx, scanned into bases (hist) and routed
+// counts (dcounts) by the CTA that finishes last (`counter` zero between calls).
+cudaError_t launch_count(const moe_params_t *p, const int32_t *idx, int32_t *hist,
+                         int32_t *counter, int32_t *dcounts, int32_t *status, cudaStream_t s);
+// a2 scatter step: kept, offsets, slot_row, row_token and x_perm (NULL: tables only)
+// from the bases and counts of the count step (or of the router).
+cudaError_t launch_scatter(const moe_params_t *p, const void *x, const int32_t *idx,
+                           const int32_t *bases, const int32_t *dcounts, void *x_perm,
+                           int32_t *row_token, int32_t *slot_row, int32_t *counts,
+                           int32_t *kept, int32_t *offsets, cudaStream_t s);
+// count + scatter; routed: skip the count (the router of the same workspace left
+// the bases and counts of these indices)
 cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t *idx,
                             void *x_perm, int32_t *row_token, int32_t *slot_row,
                             int32_t *counts, int32_t *kept, int32_t *offsets, char *ws,
-                            int32_t *status, cudaStream_t s);
+                            int32_t *status, bool routed, cudaStream_t s);
 
 // a3 / a4 for f32 (CUDA-core FMA)
 cudaError_t launch_up_simt(const moe_params_t *p, const float *x_perm, const int32_t *offsets,
@@ -116,14 +146,24 @@ cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *
 // run the tcgen05 grouped GEMMs, which stream the selected experts' weights
 // faster once each expert has a few rows.
 constexpr int kDecodeMaxTokens = 16;
+// workspace need of the decode GEMMs (partial sums; tickets, which must fit kDecTickets)
+size_t decode_partial_floats(const moe_params_t *p);
+size_t decode_ticket_ints(const moe_params_t *p);
+// bf16, 1 <= T <= kDecodeMaxTokens and the tickets fit: the decode GEMMs serve the layer
+bool decode_fits(const moe_params_t *p);
 cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
-                             const void *W13, void *h, cudaStream_t s);
+                             const void *W13, void *h, char *ws, cudaStream_t s);
+// a4; with y (and slot_row, topk_w) also a5 for the columns each block finishes
 cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32_t *offsets,
-                               const void *W2, void *out, cudaStream_t s);
+                               const void *W2, void *out, char *ws, cudaStream_t s,
+                               const int32_t *slot_row = nullptr, const float *topk_w = nullptr,
+                               void *y = nullptr);
 // a3 reading rows of x through row_token, writing x_perm alongside (moe_forward)
+// (W2_prefetch, may be NULL: the GEMM 2 weights the next launch reads, prefetched to L2)
 cudaError_t launch_up_decode_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
                                     const int32_t *offsets, const void *W13, void *h,
-                                    void *x_perm_out, cudaStream_t s);
+                                    void *x_perm_out, char *ws, const void *W2_prefetch,
+                                    cudaStream_t s);
 // a1 finish + a2 + a6 for at most kDecodeMaxTokens tokens in one CTA, after the
 // split-K router slices (moe_forward); false when the batch does not qualify.
 bool small_forward_fits(const moe_params_t *p, bool noisy);

@@ -163,6 +163,10 @@ int moe_pipeline_create(const moe_params_t *p, const void *Wg, const void *Wnois
                  o_sr = take(T * k * 4), o_kept = take(E * 4), o_off = take((E + 1) * 4),
                  o_h = take(rows * m8 * es), o_out = take(rows * d * es),
                  o_ws = take(pl->ws_bytes);
+    // the router weights packed once (they stay unchanged until destroy)
+    const bool pack = p->dtype == MOE_BF16;
+    const size_t o_wt =
+        take(pack ? (size_t)router_packed_rows(p->E, Wnoise != nullptr) * d * es : 0);
     PL_TRY(cudaMalloc(&pl->arena, off));
     if (e != cudaSuccess) {
         release(pl);
@@ -197,8 +201,17 @@ int moe_pipeline_create(const moe_params_t *p, const void *Wg, const void *Wnois
     b.offsets = (int32_t *)(a + o_off);
     b.h = a + o_h;
     b.out = a + o_out;
+    b.router_packed = nullptr;
     pl->ws = a + o_ws;
     rc = moe_workspace_init(pl->ws, pl->ws_bytes, pl->compute);
+    if (rc == MOE_OK && pack) {
+        e = launch_router_pack(p, Wg, Wnoise, a + o_wt, pl->compute);
+        if (e != cudaSuccess) {
+            release(pl);
+            return report_cuda(e, fn);
+        }
+        b.router_packed = a + o_wt;
+    }
     if (rc != MOE_OK) {
         release(pl);
         return rc;

@@ -6,21 +6,26 @@
 // The logits x.[W_g | W_noise] are a T x d x NOUT product (NOUT = E or 2E padded to
 // 16..128) that must run at HBM speed.  A persistent kernel streams 128-token tiles
 // of x through a TMA ring (box 64 K x 128 tokens, 128-byte swizzle) together with
-// the transposed router weights (box 64 K x NOUT), and tcgen05.mma (M = 128, N =
-// NOUT) accumulates the logits in TMEM (two buffers, so one tile's gate overlaps the
-// next tile's loads).  The epilogue gives each thread one token row: it reads the
-// NOUT logits from TMEM and runs the gate in f32: noise, KeepTopK (ties to the lower
-// expert index), Mixtral or ST weights, and the token's contributions to the
-// per-expert sums of softmax(H) and of G, which are reduced over the CTA in a fixed
-// order (warp butterflies, then the four warps in order) and written as one partial
-// per CTA; a finishing kernel adds the CTA partials in a fixed order.
+// the router weights packed K-major (box 64 K x NOUT; packed once per weight set by
+// router_pack_tc_kernel), and tcgen05.mma (M = 128, N = NOUT) accumulates the logits
+// in TMEM (two buffers, so one tile's gate overlaps the next tile's loads).  The
+// epilogue gives each thread one token row: it reads the NOUT logits from TMEM and
+// runs the gate in f32: noise, KeepTopK (ties to the lower expert index), Mixtral or
+// ST weights, and the token's contributions to the per-expert sums of softmax(H) and
+// of G, which are reduced over the CTA in a fixed order (warp butterflies, then the
+// four warps in order) and written as one partial per CTA.  Each gate warp also
+// counts, per expert, the tokens of its 32-token chunk routed there (the count step
+// of a2's counting sort).  The CTA that finishes last adds the CTA partials in CTA
+// order (f64) and scans the chunk counts into rank bases and routed counts, so a
+// dispatch that follows needs no count pass of its own.
 //
 // Warps: 0 TMA producer (one lane), 1 TMEM allocator and MMA issuer (one lane),
 // 2-5 gate (warp w reads TMEM lanes 32*(w%4)..+31 = tokens of the tile).
-// Router weight rows in the workspace: noisy -> row 2e = W_g[:, e], row 2e+1 =
-// W_noise[:, e]; otherwise row e = W_g[:, e]; the other rows are zero.
+// Packed router weight rows: noisy -> row 2e = W_g[:, e], row 2e+1 = W_noise[:, e];
+// otherwise row e = W_g[:, e]; the other rows are zero.
 #include <math.h>
 
+#include "dispatch_scan.cuh"
 #include "tc_common.cuh"
 
 namespace moe {
@@ -84,6 +89,9 @@ __device__ __forceinline__ float warp_sum(float v)
 
 // named barrier over the 4 gate warps (128 threads)
 __device__ __forceinline__ void gate_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+struct GateBar {
+    __device__ void operator()() const { gate_bar(); }
+};
 
 // the same barrier, returning whether v held on every gate thread: the gate warps
 // leave their tile loop together, so their barrier counts never diverge
@@ -103,15 +111,14 @@ __device__ __forceinline__ bool gate_all(bool v)
 
 template <int NOUT, bool NOISY>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     int T, int d, int E, int k, const float *__restrict__ noise,
-                     const float *__restrict__ bias, int router_type, int32_t *__restrict__ idx_out,
-                     float *__restrict__ w_out, float *__restrict__ part, int32_t *counter,
-                     float *__restrict__ probs_sum, float *__restrict__ importance,
-                     int32_t *status, uint64_t wait_ns)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                     const __grid_constant__ CUtensorMap tmW, int T, int d, int E, int k,
+                     const float *__restrict__ noise, const float *__restrict__ bias,
+                     int router_type, int32_t *__restrict__ idx_out, float *__restrict__ w_out,
+                     float *__restrict__ part, int32_t *counter, float *__restrict__ probs_sum,
+                     float *__restrict__ importance, int32_t *__restrict__ hist,
+                     int32_t *__restrict__ dcounts, int32_t *status, uint64_t wait_ns)
 {
-    pdl_wait();
-    pdl_trigger();
     using C = Cfg<NOUT>;
     constexpr int STAGES = C::STAGES;
     constexpr int EMAX = NOISY ? NOUT / 2 : NOUT;
@@ -123,7 +130,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int32_t *abort_flag = &aux->abort_flag;
     const int n_tiles = (T + BM - 1) / BM;
     const int num_kb = (d + BK - 1) / BK;
+    const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
+    // CTA b sweeps K starting at block kstart and wraps around: the CTAs' concurrent
+    // TMA reads (128 rows of 128 bytes, 8 KB apart in x) then differ in their low
+    // address bits instead of all landing on the same few DRAM channels
+    const int kstart = (int)((int64_t)blockIdx.x * num_kb / gridDim.x);
 
+    // set-up that touches no global memory overlaps the previous kernel's tail
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(tc::smem_u32(&aux->full[s]), 1);
@@ -141,6 +154,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = threadIdx.x; i < 2 * MOE_MAX_EXPERTS; i += blockDim.x)
         aux->acc[i] = 0.f;
+    pdl_wait();
+    pdl_trigger();
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          tc::smem_u32(&aux->tmem_base)),
@@ -156,13 +171,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // -------------------------------------------------------------- TMA producer
+            // -------------------------------------------------------------- TMA producer (A)
             int stage = 0;
             uint32_t phase = 0;
             int64_t fills = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int i = 0; i < num_kb; ++i) {
+                    const int kb = kstart + i < num_kb ? kstart + i : kstart + i - num_kb;
                     if (!tc::mbar_wait(tc::smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns,
                                        abort_flag, status)) {
                         ok = false;
@@ -180,6 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             }
+            // every issued copy has landed before the CTA can exit (bounded)
             for (int s = 0; s < STAGES; ++s) {
                 const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
                 if (n > 0)
@@ -200,7 +217,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 tc::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NOUT);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int i = 0; i < num_kb; ++i) {  // the producer's K order
                     if (!tc::mbar_wait(tc::smem_u32(&aux->full[stage]), phase, wait_ns,
                                        abort_flag, status)) {
                         ok = false;
@@ -212,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
                         tc::umma_f16(d_tmem, da + (uint64_t)(2 * kk), db + (uint64_t)(2 * kk),
-                                     C::IDESC, (kb | kk) != 0);
+                                     C::IDESC, (i | kk) != 0);
                     tc::umma_commit(tc::smem_u32(&aux->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -234,9 +251,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------------------ gate
         const int wq = warp & 3;
         const int lane_base = wq * 32;
+        const int gt = threadIdx.x - 64;  // 0..127 over the gate warps
+        float bias_r[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+            bias_r[e] = (bias != nullptr && e < E) ? bias[e] : 0.f;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int64_t t = (int64_t)tile * BM + lane_base + lane;
+            const bool tv = t < T;
+            // the token's noise draws are loaded before the logits are ready
+            float nz[EMAX];
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e)
+                nz[e] = (NOISY && tv && e < E) ? __ldg(noise + t * E + e) : 0.f;
             const bool got = tc::mbar_wait(tc::smem_u32(&aux->tfull[acc]), acc_phase, wait_ns,
                                            abort_flag, status);
             if (!gate_all(got))
@@ -264,8 +293,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 acc_phase ^= 1u;
             }
 
-            const int64_t t = (int64_t)tile * BM + lane_base + lane;
-            const bool tv = t < T;
             float H[EMAX];
             bool bad = false;
 #pragma unroll
@@ -274,9 +301,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (e < E) {
                     h = NOISY ? lg[2 * e] : lg[e];
                     if (bias)
-                        h += bias[e];
+                        h += bias_r[e];
                     if (NOISY && tv)
-                        h += noise[t * E + e] * softplus_f(lg[2 * e + 1]);
+                        h += nz[e] * softplus_f(lg[2 * e + 1]);
                     bad |= !isfinite(h);
                 }
                 H[e] = h;
@@ -339,11 +366,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
             }
             const bool contrib = tv && !bad;
+            // a2's chunk histogram: this warp's 32 tokens are chunk tile*4 + wq
+            const int chunk = tile * (BM / kDispatchChunk) + wq;
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) {
+                if (e < E) {  // E is uniform: every lane takes part in the ballot
+                    bool has = false;
+#pragma unroll
+                    for (int j = 0; j < MOE_MAX_TOPK; ++j)
+                        has |= contrib && j < k && sel[j] == e;
+                    const unsigned b = __ballot_sync(0xffffffffu, has);
+                    if (lane == (e & 31) && chunk < nch)
+                        hist[(int64_t)e * nch + chunk] = __popc(b);
+                }
+            }
             // per-expert sums over the tile's tokens: softmax(H) and gate weights
             gate_bar();  // red[][] of the previous tile has been consumed
 #pragma unroll
             for (int e = 0; e < EMAX; ++e) {
-                if (e < E) {  // E is uniform: every lane takes part in the shuffles
+                if (e < E) {
                     float p = contrib ? expf(H[e] - hmax) * invz : 0.f;
                     float g = 0.f;
 #pragma unroll
@@ -358,15 +399,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             gate_bar();
-            const int gt = threadIdx.x - 64;  // 0..127 over the gate warps
             for (int i = gt; i < 2 * E; i += 128)
                 aux->acc[i] += ((aux->red[0][i] + aux->red[1][i]) + aux->red[2][i]) + aux->red[3][i];
         }
         gate_bar();
-        const int gt = threadIdx.x - 64;
         for (int i = gt; i < 2 * E; i += 128)
             part[(int64_t)blockIdx.x * 2 * E + i] = aux->acc[i];
-        // the CTA that finishes last adds every CTA's partials in CTA order (f64)
+        // the CTA that finishes last adds every CTA's partials in CTA order (f64) and
+        // scans the chunk histogram; its ring is idle by now (every stage it loaded was
+        // consumed before its last tile's logits were ready), so both are staged there
         __threadfence();
         gate_bar();
         if (gt == 0)
@@ -374,15 +415,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         gate_bar();
         if (aux->last) {
             __threadfence();
+            float *s_part = reinterpret_cast<float *>(smem);
+            const int np = (int)gridDim.x * 2 * E;  // <= 148 x 128 floats: fits the ring
+            for (int i = gt; i < np; i += 128)
+                s_part[i] = __ldcg(part + i);
+            gate_bar();
             for (int o = gt; o < 2 * E; o += 128) {
                 double sum = 0.0;
                 for (int b = 0; b < (int)gridDim.x; ++b)
-                    sum += (double)__ldcg(part + (int64_t)b * 2 * E + o);
+                    sum += (double)s_part[b * 2 * E + o];
                 if (o < E)
                     probs_sum[o] = (float)sum;
                 else
                     importance[o - E] = (float)sum;
             }
+            gate_bar();
+            scan_chunk_counts(hist, E, nch, dcounts, reinterpret_cast<int32_t *>(smem),
+                              C::TILE_BYTES / 4, gt, 128, GateBar());
             if (gt == 0)
                 *counter = 0;
         }
@@ -397,7 +446,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
-// Router weights into the layout the kernel reads (see the file comment).
+// Router weights into the packed layout the kernel reads (see the file comment).
 __global__ void router_pack_tc_kernel(const bf16 *__restrict__ Wg, const bf16 *__restrict__ Wn,
                                       int d, int E, int rows, bf16 *__restrict__ Wt)
 {
@@ -418,13 +467,15 @@ __global__ void router_pack_tc_kernel(const bf16 *__restrict__ Wg, const bf16 *_
 }
 
 template <int NOUT, bool NOISY>
-static cudaError_t run(const moe_params_t *p, const void *x, const bf16 *Wt, const float *noise,
-                       const float *bias, int32_t *idx, float *w, float *part, int32_t *counter,
-                       float *probs_sum, float *importance, int32_t *status, cudaStream_t s)
+static cudaError_t run(const moe_params_t *p, const void *x, const bf16 *Wt,
+                       const float *noise, const float *bias, int32_t *idx, float *w,
+                       float *part, int32_t *counter, float *probs_sum, float *importance,
+                       int32_t *hist, int32_t *dcounts, int32_t *status, cudaStream_t s)
 {
     using C = Cfg<NOUT>;
     constexpr int SMEM = 1024 + C::TILE_BYTES + (int)sizeof(Aux);
     static_assert(SMEM <= 227 * 1024, "router shared memory");
+    static_assert(148 * 2 * MOE_MAX_EXPERTS * 4 <= C::TILE_BYTES, "CTA partials fit the ring");
     static bool attr_done[64] = {false};
     static int sms_cached[64] = {0};
     int dev = 0;
@@ -441,6 +492,8 @@ static cudaError_t run(const moe_params_t *p, const void *x, const bf16 *Wt, con
         e = cudaDeviceGetAttribute(&sms_cached[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess)
             return e;
+        if (sms_cached[dev] > 148)  // the staged CTA partials are sized for 148 CTAs
+            sms_cached[dev] = 148;
         attr_done[dev] = true;
     }
     CUtensorMap tx, tw;
@@ -454,36 +507,46 @@ static cudaError_t run(const moe_params_t *p, const void *x, const bf16 *Wt, con
         return e;
     const int n_tiles = ceil_div(p->T, BM);
     const int grid = n_tiles < sms_cached[dev] ? n_tiles : sms_cached[dev];
-    launch_pdl(router_tc_kernel<NOUT, NOISY>, dim3(grid), dim3(NUM_THREADS), SMEM, s, 
-        tx, tw, p->T, p->d, p->E, p->k, noise, bias, p->router_type, idx, w, part, counter,
-        probs_sum, importance, status, wait_limit_ns());
+    launch_pdl(router_tc_kernel<NOUT, NOISY>, dim3(grid), dim3(NUM_THREADS), SMEM, s, tx, tw,
+               p->T, p->d, p->E, p->k, noise, bias, p->router_type, idx, w, part, counter,
+               probs_sum, importance, hist, dcounts, status, wait_limit_ns());
     return cudaGetLastError();
 }
 
 }  // namespace rtc
 
-// Routes a bf16 batch on the tensor cores, token sums included.
-cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wg,
-                            const void *Wnoise, const float *noise, const float *bias,
-                            int32_t *idx, float *w, float *probs_sum, float *importance,
-                            float *part, int32_t *counter, bf16 *Wt, int32_t *status,
-                            cudaStream_t s)
+int router_packed_rows(int E, bool noisy)
 {
-    const bool noisy = Wnoise != nullptr;
-    const int nout = noisy ? 2 * p->E : p->E;
-    const int rows = nout <= 16 ? 16 : nout <= 32 ? 32 : nout <= 64 ? 64 : 128;
+    const int nout = noisy ? 2 * E : E;
+    return nout <= 16 ? 16 : nout <= 32 ? 32 : nout <= 64 ? 64 : 128;
+}
+
+cudaError_t launch_router_pack(const moe_params_t *p, const void *Wg, const void *Wnoise, void *Wt,
+                               cudaStream_t s)
+{
+    const int rows = router_packed_rows(p->E, Wnoise != nullptr);
     const int64_t n = (int64_t)rows * p->d;
-    launch_pdl(rtc::router_pack_tc_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, 
-        (const bf16 *)Wg, (const bf16 *)Wnoise, p->d, p->E, rows, Wt);
+    launch_pdl(rtc::router_pack_tc_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+               (const bf16 *)Wg, (const bf16 *)Wnoise, p->d, p->E, rows, (bf16 *)Wt);
     count_launch();
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return e;
+    return cudaGetLastError();
+}
+
+// Routes a bf16 batch on the tensor cores with packed router weights, token sums and
+// a2's chunk counts included.
+cudaError_t launch_route_tc(const moe_params_t *p, const void *x, const void *Wt, bool noisy,
+                            const float *noise, const float *bias, int32_t *idx, float *w,
+                            float *probs_sum, float *importance, float *part, int32_t *counter,
+                            int32_t *hist, int32_t *dcounts, int32_t *status, cudaStream_t s)
+{
+    const int rows = router_packed_rows(p->E, noisy);
+    const bf16 *t = (const bf16 *)Wt;
+    cudaError_t e;
 #define MOE_RTC(NO)                                                                          \
-    (noisy ? rtc::run<NO, true>(p, x, Wt, noise, bias, idx, w, part, counter, probs_sum,        \
-                                importance, status, s)                                          \
-           : rtc::run<NO, false>(p, x, Wt, noise, bias, idx, w, part, counter, probs_sum,       \
-                                 importance, status, s))
+    (noisy ? rtc::run<NO, true>(p, x, t, noise, bias, idx, w, part, counter, probs_sum,         \
+                                importance, hist, dcounts, status, s)                           \
+           : rtc::run<NO, false>(p, x, t, noise, bias, idx, w, part, counter, probs_sum,        \
+                                 importance, hist, dcounts, status, s))
     if (rows == 16)
         e = MOE_RTC(16);
     else if (rows == 32)

@@ -111,6 +111,18 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes (16-byte aligned, a multiple of
+// 16) from global memory into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 // Four rows r0..r3 of a 2-D tensor (box one row high), 64 columns from `col`,
 // written as four consecutive 128-byte rows at dst (128-byte swizzle as a tile).
 __device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint32_t bar, uint32_t dst,
