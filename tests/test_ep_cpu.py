@@ -1,9 +1,10 @@
 """Expert-parallel layer on the CPU: the exchange plan of libmoe (host code, no GPU)
-against a brute-force recount, and the layer's multi-rank data path (the plan plus
-``expert_parallel.exchange_runs`` over gloo, world size 2 and 4) with the fp64
-oracle doing each rank's arithmetic, against the oracle's one-process layer on the
-ranks' batches concatenated in rank order ("Llama 3 Meets MoE", section "训练框架",
-Expert Parallelism; section 3 "容量因子" for the capacity)."""
+against a brute-force recount, and ``ExpertParallelMoE.forward`` itself in world
+sizes 2 and 4 over gloo (its plan, slot mask, row exchange and gate statistics,
+with the fp64 oracle standing in for the GPU kernels' arithmetic), against the
+oracle's one-process layer on the ranks' batches concatenated in rank order
+("Llama 3 Meets MoE", section "训练框架", Expert Parallelism; section 3 "容量因子"
+for the capacity)."""
 import json
 import os
 import sys
@@ -151,11 +152,101 @@ def _layer_inputs(Ts, d, E, m, seed):
     return dict(x=f(x), Wg=f(Wg), Wn=f(Wn), eps=f(eps), W1=f(W1), W3=f(W3), W2=f(W2))
 
 
+class OracleOps:
+    """ExpertParallelMoE's arithmetic on the host in fp64 (the oracle), for CPU tensors
+    of float64 that hold f32 values exactly: the same calls, arguments and in-place
+    outputs as the library's entry points, which need a GPU.  Everything else of the
+    layer -- the class's steps, the exchange plan (libmoe host code), the collectives
+    and the row exchange over gloo -- is the code under test.  Outputs the library
+    keeps in f32 (gate weights, token sums, statistics) are stored in the f32 tensors
+    the class allocates for them."""
+
+    def __init__(self, W1l, W3l, W2l, lam):
+        self.W1l, self.W3l, self.W2l, self.lam = W1l, W3l, W2l, lam
+
+    @staticmethod
+    def dtype_code(dt):
+        return moe.MOE_F32  # a tag of the call shapes; the tensors are float64
+
+    class _Ws:
+        nbytes = 1 << 62
+
+    def workspace(self, p, device):
+        return self._Ws()
+
+    @staticmethod
+    def workspace_size(p):
+        return 0
+
+    @staticmethod
+    def _f32(t):
+        return np.ascontiguousarray(t.numpy().astype(np.float32))
+
+    def route(self, p, x, Wg, Wn, noise, bias, ws, topk_idx, topk_w, probs_sum, importance):
+        import oracle
+        r = oracle.router(self._f32(x), self._f32(Wg), None if Wn is None else self._f32(Wn),
+                          None if noise is None else self._f32(noise),
+                          None if bias is None else bias.numpy(), p.k, p.router_type)
+        T = p.T
+        topk_idx[:T] = torch.from_numpy(r["idx"])
+        topk_w[:T] = torch.from_numpy(r["G"]).to(topk_w.dtype)
+        probs_sum.copy_(torch.from_numpy(r["probs_sum"]))
+        importance.copy_(torch.from_numpy(r["importance"]))
+
+    def dispatch(self, p, x, topk_idx, ws, x_perm, row_token, slot_row, counts, kept, offsets):
+        import oracle
+        d = oracle.dispatch(topk_idx[:p.T].numpy(), p.E, p.capacity)
+        R = d["R"]
+        rt = torch.from_numpy(d["row_token"]).long()
+        x_perm[:R] = x[rt]
+        row_token[:R] = torch.from_numpy(d["row_token"])
+        slot_row[:p.T] = torch.from_numpy(d["slot_row"])
+        counts.copy_(torch.from_numpy(d["counts"]))
+        kept.copy_(torch.from_numpy(d["kept"]))
+        offsets[:p.E + 1] = torch.from_numpy(d["offsets"])
+
+    @staticmethod
+    def mask_slots(p, topk_idx, offsets, keep, slot_row):
+        # an assignment whose position inside its expert's block is past keep[e] drops
+        for t in range(p.T):
+            for j in range(p.k):
+                r = int(slot_row[t, j])
+                if r >= 0:
+                    e = int(topk_idx[t, j])
+                    if r - int(offsets[e]) >= int(keep[e]):
+                        slot_row[t, j] = -1
+
+    def expert_ffn(self, p, xin, in_offsets, W13, W2, h, out, ws):
+        import oracle
+        R = p.T
+        off = in_offsets.numpy()
+        eor = (np.searchsorted(off, np.arange(R), side="right") - 1).astype(np.int32)
+        out[:R] = torch.from_numpy(oracle.expert_ffn(self.W1l, self.W3l, self.W2l,
+                                                     self._f32(xin[:R]), eor))
+
+    @staticmethod
+    def combine(p, out, slot_row, topk_w, y):
+        import oracle
+        scale = p.E / p.k if p.rescale else 1.0
+        y.copy_(torch.from_numpy(oracle.combine(out.numpy(), slot_row[:p.T].numpy(),
+                                                topk_w[:p.T].numpy().astype(np.float64),
+                                                scale)))
+
+    def gate_stats(self, pg, counts_all, N, probs_sum, counts, f, P, loss):
+        import oracle
+        c = counts_all.numpy().sum(0).astype(np.int32)
+        fe, Pe, L = oracle.gate_stats(pg.T, pg.k, c, probs_sum.numpy().astype(np.float64),
+                                      self.lam)
+        counts.copy_(torch.from_numpy(c))
+        f.copy_(torch.from_numpy(fe))
+        P.copy_(torch.from_numpy(Pe))
+        loss[0] = L
+
+
 def _ep_worker(rank, world, port, out_dir, cfg):
+    """One rank of the layer: ExpertParallelMoE.forward over gloo, oracle arithmetic."""
     sys.path.insert(0, ROOT)
-    import oracle
-    from top_routing_grouped_noisy_b200 import moe_ep_plan
-    from top_routing_grouped_noisy_b200.expert_parallel import DistTransport
+    from top_routing_grouped_noisy_b200.expert_parallel import ExpertParallelMoE
     dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
                             world_size=world)
     try:
@@ -163,55 +254,48 @@ def _ep_worker(rank, world, port, out_dir, cfg):
         inp = _layer_inputs(Ts, d, E, m, cfg["seed"])
         a = sum(Ts[:rank])
         T = Ts[rank]
-        x, eps = inp["x"][a:a + T], inp["eps"][a:a + T]
+        t64 = lambda v: torch.from_numpy(v.astype(np.float64))
         El = E // world
         lo = rank * El
-        tr = DistTransport()
-        # step 1: route and dispatch this rank's tokens, no capacity
-        r = oracle.router(x, inp["Wg"], inp["Wn"], eps, None, k, cfg["router"])
-        dsp = oracle.dispatch(r["idx"], E, -1)
-        counts_T = torch.tensor(list(dsp["counts"]) + [T], dtype=torch.int32)
-        # step 2: collectives
-        counts_all = tr.all_gather(counts_T)
-        sums = torch.from_numpy(np.concatenate([r["probs_sum"], r["importance"]]))
-        tr.all_reduce_sum(sums)
-        # step 3: plan and the drop mask (slot position inside its expert's block >= keep)
-        plan = moe_ep_plan(counts_all[:, :E].contiguous(), rank, cfg["capacity"], cfg["scope"])
-        keep = plan.keep_all[rank].numpy()
-        sr = dsp["slot_row"].copy()
-        for t in range(T):
-            for j in range(k):
-                if sr[t, j] >= 0:
-                    e = r["idx"][t, j]
-                    if sr[t, j] - dsp["offsets"][e] >= keep[e]:
-                        sr[t, j] = -1
-        # step 4: rows to the experts' owners
-        x_perm = torch.from_numpy(np.ascontiguousarray(x[dsp["row_token"]])) if dsp["R"] else \
-            torch.zeros(1, d)
-        xin = torch.zeros(max(plan.rows_in, 1), d)
-        tr.exchange(x_perm, plan.send_runs(), xin, plan.recv_runs())
-        # step 5: the local experts (fp64 oracle)
-        R_in = plan.rows_in
-        off = plan.in_offsets.numpy()
-        eor = (np.searchsorted(off, np.arange(R_in), side="right") - 1).astype(np.int32)
-        if R_in:
-            out_loc = oracle.expert_ffn(inp["W1"][lo:lo + El], inp["W3"][lo:lo + El],
-                                        inp["W2"][lo:lo + El], xin[:R_in].numpy(), eor)
-        else:
-            out_loc = np.zeros((1, d))
-        # step 6: outputs back
-        out = torch.zeros(max(T * k, 1), d, dtype=torch.float64)
-        tr.exchange(torch.from_numpy(np.ascontiguousarray(out_loc)), plan.recv_runs(), out,
-                    plan.send_runs())
-        # step 7: combine
-        scale = E / k if cfg["rescale"] else 1.0
-        y = oracle.combine(out.numpy(), sr, r["G"], scale)
-        np.save(os.path.join(out_dir, "y%d.npy" % rank), y)
+        ops = OracleOps(inp["W1"][lo:lo + El], inp["W3"][lo:lo + El], inp["W2"][lo:lo + El], 0.01)
+        layer = ExpertParallelMoE(d, E, k, m, None, None, t64(inp["Wg"]), t64(inp["Wn"]), None,
+                                  torch.float64, cfg["router"], cfg["capacity"], cfg["scope"],
+                                  cfg["rescale"], 0.01, ops=ops)
+        s = layer.forward(t64(inp["x"][a:a + T]), t64(inp["eps"][a:a + T]))
+        np.save(os.path.join(out_dir, "y%d.npy" % rank), s.y.numpy())
         with open(os.path.join(out_dir, "r%d.json" % rank), "w") as fh:
-            json.dump({"counts_all": counts_all.tolist(), "sums": sums.tolist(),
-                       "keep_all": plan.keep_all.tolist(), "slot_row": sr.tolist()}, fh)
+            json.dump({"counts_all": s.counts_all_dev.tolist(),
+                       "sums": s.sums[:E].tolist() + s.sums[-(s.sums.numel() // 2):][:E].tolist(),
+                       "keep_all": s.ep.keep_all.tolist(),
+                       "slot_row": s.slot_row[:T].tolist(),
+                       "counts": s.counts_global.tolist(), "f": s.f.tolist(), "P": s.P.tolist(),
+                       "loss": float(s.loss[0]), "T_all": s.T_all}, fh)
     finally:
         dist.destroy_process_group()
+
+
+def _one_process_layer(inp, Ts, E, k, capacity, scope, router, rescale):
+    """The oracle's layer on the ranks' batches (concatenated under GLOBAL, each rank's
+    batch alone under LOCAL), with the gate weights rounded to f32 as the layer stores
+    them; y per rank."""
+    import oracle
+    scale = E / k if rescale else 1.0
+    spans = [(sum(Ts[:i]), sum(Ts[:i + 1])) for i in range(len(Ts))]
+    groups = [(0, sum(Ts))] if scope == GLOBAL else spans
+    y = np.zeros((sum(Ts), inp["x"].shape[1]))
+    for a, b in groups:
+        if b == a:
+            continue
+        r = oracle.router(inp["x"][a:b], inp["Wg"], inp["Wn"], inp["eps"][a:b], None, k, router)
+        dsp = oracle.dispatch(r["idx"], E, capacity)
+        R = dsp["R"]
+        eor = (np.searchsorted(dsp["offsets"], np.arange(R), side="right") - 1).astype(np.int32)
+        out = oracle.expert_ffn(inp["W1"], inp["W3"], inp["W2"],
+                                np.ascontiguousarray(inp["x"][a:b][dsp["row_token"]]), eor) \
+            if R else np.zeros((1, inp["x"].shape[1]))
+        G32 = r["G"].astype(np.float32).astype(np.float64)
+        y[a:b] = oracle.combine(out, dsp["slot_row"], G32, scale)
+    return [y[a:b] for a, b in spans]
 
 
 @pytest.mark.parametrize("world,Ts,E,k,capacity,scope,router,rescale", [
@@ -223,6 +307,9 @@ def _ep_worker(rank, world, port, out_dir, cfg):
 ])
 def test_ep_layer_over_gloo_equals_one_process_layer(tmp_path, world, Ts, E, k, capacity, scope,
                                                       router, rescale):
+    """ExpertParallelMoE.forward on every rank (its plan, slot mask, row exchange over
+    gloo and gate statistics; the oracle doing the arithmetic) gives each rank's rows of
+    the one-process layer bit for bit, and the statistics of all ranks' tokens."""
     import oracle
     cfg = dict(Ts=Ts, d=16, E=E, k=k, m=8, capacity=capacity, scope=scope, router=router,
                rescale=rescale, seed=sum(Ts) + E)
@@ -232,29 +319,24 @@ def test_ep_layer_over_gloo_equals_one_process_layer(tmp_path, world, Ts, E, k, 
     res = [json.load(open(tmp_path / ("r%d.json" % i))) for i in range(world)]
     ys = [np.load(tmp_path / ("y%d.npy" % i)) for i in range(world)]
     counts_all = np.array(res[0]["counts_all"])[:, :E]
-    if scope == GLOBAL:
-        full = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k, router,
-                              inp["Wn"], inp["eps"], None, capacity, rescale, 0.01)
-        want = [full["y"][sum(Ts[:i]):sum(Ts[:i + 1])] for i in range(world)]
-        assert np.array_equal(counts_all.sum(0), full["dispatch"]["counts"])
-        assert np.array_equal(np.array(res[0]["keep_all"]).sum(0), full["dispatch"]["kept"])
-        s = np.array(res[0]["sums"])
-        np.testing.assert_allclose(s[:E], full["router"]["probs_sum"], rtol=1e-12)
-        np.testing.assert_allclose(s[E:], full["router"]["importance"], rtol=1e-12)
-        _, _, L = oracle.gate_stats(sum(Ts), k, counts_all.sum(0), s[:E], 0.01)
-        assert L == pytest.approx(full["L"], rel=1e-12)
-    else:
-        want = []
-        for i in range(world):
-            a, b = sum(Ts[:i]), sum(Ts[:i + 1])
-            want.append(oracle.forward(inp["x"][a:b], inp["Wg"], inp["W1"], inp["W3"], inp["W2"],
-                                       k, router, inp["Wn"], inp["eps"][a:b], None, capacity,
-                                       rescale, 0.01)["y"])
+    want = _one_process_layer(inp, Ts, E, k, capacity, scope, router, rescale)
     for i in range(world):
-        # every rank's rows equal those of the one-process layer exactly: the same
-        # per-row fp64 arithmetic, only the rows' places differ
+        # the same per-row fp64 arithmetic; only the rows' places differ
         assert ys[i].shape == want[i].shape
-        assert np.array_equal(ys[i], want[i])
+        assert np.array_equal(ys[i], want[i]), i
+    full = oracle.forward(inp["x"], inp["Wg"], inp["W1"], inp["W3"], inp["W2"], k, router,
+                          inp["Wn"], inp["eps"], None, capacity, rescale, 0.01)
+    # statistics over all ranks' tokens (pre-drop counts, f32 token sums)
+    assert np.array_equal(counts_all.sum(0), full["dispatch"]["counts"])
+    for rr in res:
+        assert rr["counts"] == full["dispatch"]["counts"].tolist()
+        assert rr["T_all"] == sum(Ts)
+        s = np.array(rr["sums"])
+        np.testing.assert_allclose(s[:E], full["router"]["probs_sum"], rtol=1e-6)
+        np.testing.assert_allclose(s[E:], full["router"]["importance"], rtol=1e-6)
+        assert rr["loss"] == pytest.approx(full["L"], rel=1e-5)
+    if scope == GLOBAL:
+        assert np.array_equal(np.array(res[0]["keep_all"]).sum(0), full["dispatch"]["kept"])
     # every rank got the same plan
     for i in range(1, world):
         assert res[i]["keep_all"] == res[0]["keep_all"]
