@@ -85,3 +85,31 @@ def test_backward_wait_timeout_is_reported_and_context_survives(T):
     assert (bufs.topk_idx.cpu().numpy() == ref["fwd"]["router"]["idx"]).all()
     dx = H.f64(g.dx)
     assert np.abs(dx - ref["dx"]).max() <= 2e-2 * np.abs(ref["dx"]).max()
+
+
+def test_decode_forward_wait_timeout_is_reported_and_context_survives():
+    """The one-launch decode layer (bulk-copy ring, grid barrier) gives up at a wait
+    limit of 0, reports MOE_ERR_DEVICE_TIMEOUT and returns; its grid barrier words are
+    back at zero, so the next forward on the same workspace is correct."""
+    w = wl.Workload("to_dec", T=4, d=512, d_ff=8 * 96, E=8, k=2, noisy=True, rescale=True,
+                    seed=83)
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, weights = H.run_forward(w, inp)
+    assert status == 0
+    dev = "cuda"
+    W13_e, W2_e = weights
+    x, Wg, Wn, eps = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_set_wait_limit_ns(0)
+    try:
+        moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs, Wnoise=Wn, noise=eps)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert moe.moe_get_device_status(ws) == 0
+    moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs, Wnoise=Wn, noise=eps)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    r, ties = H.check_routing(w, inp, bufs, 5e-5)
+    dsp = H.check_dispatch(w, inp, p, bufs)
+    H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)

@@ -105,7 +105,6 @@ WsLayout ws_layout(const moe_params_t *p)
         off += (bytes + 255) / 256 * 256;
         return o;
     };
-    L.dtick = take((size_t)kDecTickets * sizeof(int32_t));  // first: a fixed offset
     L.wt = take((size_t)kWtRows * p->d * es);
     const size_t blocks = (size_t)ceil_div(p->T > 0 ? p->T : 1, kRouterMinTokens);
     L.rpart = take(blocks * 2 * p->E * sizeof(float));
@@ -116,7 +115,6 @@ WsLayout ws_layout(const moe_params_t *p)
     // larger, so that a workspace sized for T also serves every smaller batch.
     const int t_small = p->T < kRouterSmallTokens ? (p->T > 0 ? p->T : 1) : kRouterSmallTokens;
     L.rsmall = take((size_t)kRouterSmallSplit * t_small * 2 * p->E * sizeof(float));
-    L.dpre = take(p->dtype == MOE_BF16 ? decode_partial_floats(p) * sizeof(float) : 0);
     L.total = off;
     return L;
 }
@@ -544,10 +542,8 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
     REQUIRE_PTR(b->loss);
     REQUIRE_PTR(b->f);
     REQUIRE_PTR(b->P);
-    if (small_forward_fits(p, b->Wnoise != nullptr) && decode_fits(p)) {
-        // decode-shaped batch, three launches: router slices whose last CTA finishes
-        // the router and builds the dispatch tables and gate statistics; GEMM 1
-        // gathering rows of x; GEMM 2 with the combine
+    if (decode_forward_fits(p, b->Wnoise != nullptr)) {
+        // decode-shaped batch: the whole layer in one cooperative launch
         REQUIRE_PTR(b->x);
         REQUIRE_PTR(b->Wg);
         OPTIONAL_PTR(b->Wnoise);
@@ -573,14 +569,7 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
             return rc;
         char *w = static_cast<char *>(ws);
         cudaStream_t s = (cudaStream_t)stream;
-        cudaError_t e = launch_route_dispatch_small(p, b, w, reinterpret_cast<int32_t *>(w), s);
-        if (e == cudaSuccess)
-            e = launch_up_decode_gather(p, b->x, b->row_token, b->offsets, b->W13_e, b->h,
-                                        b->x_perm, w, b->W2_e, s);
-        if (e == cudaSuccess)  // GEMM 2 with the combine of the columns it finishes
-            e = launch_down_decode(p, b->h, b->offsets, b->W2_e, b->out, w, s, b->slot_row,
-                                   b->topk_w, b->y);
-        return after_launch(fn, e);
+        return after_launch(fn, launch_forward_decode(p, b, w, s));
     }
     if ((rc = route_impl("moe_forward", p, b->x, b->Wg, b->Wnoise, b->router_packed, b->noise,
                          b->bias, b->topk_idx, b->topk_w, b->probs_sum, b->importance, ws,

@@ -25,6 +25,8 @@ constexpr int kWsCounterWord = 1;
 constexpr int kWsRouterCounterWord = 2;
 // Word 3: ticket counter of the decode-size router + dispatch kernel (zero between calls).
 constexpr int kWsSmallCounterWord = 3;
+// Words 4-5: grid barrier of the decode forward kernel (arrive, depart; zero between calls).
+constexpr int kWsDecodeBarrierWord = 4;
 // Header bytes that clearing the status resets (status word and counters).
 constexpr size_t kWsResetBytes = 32;
 // Words 8-9: offsets {0, T} of the shared block's one-expert GEMMs (residual MoE).

@@ -9,6 +9,31 @@
 
 namespace moe {
 
+// Copies n 32-bit words from global memory (written by other CTAs, read at L2) to
+// shared memory, the nthr calling threads striding by nthr: every thread issues
+// kStageBatch loads before it stores any, so the copy takes a few L2 round trips
+// instead of one per word a thread handles.
+constexpr int kStageBatch = 8;
+template <typename W>
+__device__ __forceinline__ void stage_words(W *dst, const W *src, int64_t n, int tid, int nthr)
+{
+    for (int64_t i0 = tid; i0 < n; i0 += (int64_t)nthr * kStageBatch) {
+        W v[kStageBatch];
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+            const int64_t i = i0 + (int64_t)u * nthr;
+            if (i < n)
+                v[u] = __ldcg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < kStageBatch; ++u) {
+            const int64_t i = i0 + (int64_t)u * nthr;
+            if (i < n)
+                dst[i] = v[u];
+        }
+    }
+}
+
 // hist [E][nch]: on entry the number of tokens of chunk c routed to expert e; on
 // exit the exclusive prefix over chunks (the rank inside expert e of the chunk's
 // first such token).  dcounts [E] receives each expert's total (its routed count).
@@ -27,8 +52,7 @@ __device__ __forceinline__ void scan_chunk_counts(int32_t *hist, int E, int nch,
     const int64_t nhist = (int64_t)E * nch;
     const bool staged = nhist <= smem_ints;
     if (staged) {
-        for (int64_t i = tid; i < nhist; i += nthr)
-            s_hist[i] = __ldcg(hist + i);
+        stage_words(s_hist, hist, nhist, tid, nthr);
         bar();
     }
     for (int e = warp; e < E; e += nwarps) {

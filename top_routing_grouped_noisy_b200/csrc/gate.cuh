@@ -223,115 +223,4 @@ __device__ inline void router_small_finish(const float *__restrict__ part, int T
                        importance, status, lg + (size_t)T * nout);
 }
 
-// ------------------------------------------------------------------ one-CTA router
-// Logits of at most 16 tokens and NT * 8 >= nout outputs on the tensor cores, in one
-// CTA of kOneWarps warps: warp w takes K columns [w kw, (w+1) kw) (kw = d / kOneWarps
-// rounded up to 16), staged 64 at a time in its own shared memory (x rows padded by 16
-// bytes, so the 32-bit fragment reads are free of bank conflicts; the router rows
-// copied as they lie in W_g / W_noise, which are contiguous for a run of K), and
-// accumulates mma.sync m16n8k16 fragments (bf16 in, f32); the warps' partial logits are
-// then added in warp order.  Output lg [T][nout] f32 in shared memory.  The result is
-// one fixed function of the inputs, whichever kernel calls it.
-constexpr int kOneWarps = 16;
-constexpr int kOneKC = 64;
-constexpr int kOneXPitch = kOneKC + 8;  // bf16 per staged x row
-__host__ __device__ constexpr size_t one_cta_warp_smem(int nt)
-{
-    // x [16][kOneXPitch] bf16, then the W_g rows [kOneKC][E] and the W_noise rows
-    // [kOneKC][E] (2E <= 8 nt with noise, E <= 8 nt without)
-    return (size_t)16 * kOneXPitch * 2 + (size_t)kOneKC * 8 * nt * 2;
-}
-__host__ __device__ constexpr size_t one_cta_logits_smem(int nt)
-{
-    return kOneWarps * one_cta_warp_smem(nt) + (size_t)kOneWarps * 16 * nt * 8 * 4;
-}
-
-__device__ __forceinline__ uint32_t bf16_pair(const uint16_t *p0, const uint16_t *p1)
-{
-    return (uint32_t)*p0 | ((uint32_t)*p1 << 16);
-}
-
-template <int NT>
-__device__ inline void router_logits_one_cta(const bf16 *__restrict__ x, const bf16 *__restrict__ Wg,
-                                             const bf16 *__restrict__ Wn, int T, int d, int E,
-                                             float *lg, char *smem)
-{
-    const int nout = Wn ? 2 * E : E;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int kw = (d + kOneWarps * 16 - 1) / (kOneWarps * 16) * 16;
-    const int kbeg = warp * kw, kend = min(d, kbeg + kw);
-    char *wb = smem + (size_t)warp * one_cta_warp_smem(NT);
-    uint16_t *xs = reinterpret_cast<uint16_t *>(wb);
-    uint16_t *gs = xs + 16 * kOneXPitch;  // [kOneKC][E]
-    uint16_t *ns = gs + kOneKC * E;        // [kOneKC][E] (noise rows)
-    float *red = reinterpret_cast<float *>(smem + (size_t)kOneWarps * one_cta_warp_smem(NT));
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            acc[nt][c] = 0.f;
-    for (int k0 = kbeg; k0 < kend; k0 += kOneKC) {
-        const int kc = min(kOneKC, kend - k0);  // a multiple of 8
-        __syncwarp();
-        for (int i = lane; i < 16 * (kOneKC / 8); i += 32) {
-            const int t = i / (kOneKC / 8), v = i % (kOneKC / 8);
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (t < T && v * 8 < kc)
-                val = ld_nc(x + (int64_t)t * d + k0 + v * 8);
-            *reinterpret_cast<uint4 *>(xs + t * kOneXPitch + v * 8) = val;
-        }
-        const int wv = kc * E / 8;  // 16-byte vectors of a run of router rows
-        for (int i = lane; i < wv; i += 32) {
-            reinterpret_cast<uint4 *>(gs)[i] = ld_nc(Wg + (int64_t)k0 * E + (int64_t)i * 8);
-            if (Wn != nullptr)
-                reinterpret_cast<uint4 *>(ns)[i] = ld_nc(Wn + (int64_t)k0 * E + (int64_t)i * 8);
-        }
-        __syncwarp();
-        for (int kk = 0; kk < kc; kk += 16) {
-            // rows past kc read as zero (kc is a multiple of 8: the upper half may be out)
-            const bool hi = kk + 8 < kc;
-            const uint16_t *xr0 = xs + g * kOneXPitch + kk + 2 * q;
-            const uint16_t *xr1 = xs + (g + 8) * kOneXPitch + kk + 2 * q;
-            const uint32_t a0 = *reinterpret_cast<const uint32_t *>(xr0);
-            const uint32_t a1 = *reinterpret_cast<const uint32_t *>(xr1);
-            const uint32_t a2 = hi ? *reinterpret_cast<const uint32_t *>(xr0 + 8) : 0u;
-            const uint32_t a3 = hi ? *reinterpret_cast<const uint32_t *>(xr1 + 8) : 0u;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int n = nt * 8 + g;
-                const uint16_t *src = n < E ? gs + n : (n < nout ? ns + (n - E) : nullptr);
-                const int r = kk + 2 * q;
-                uint32_t b0 = 0u, b1 = 0u;
-                if (src != nullptr) {
-                    b0 = bf16_pair(src + r * E, src + (r + 1) * E);
-                    if (hi)
-                        b1 = bf16_pair(src + (r + 8) * E, src + (r + 9) * E);
-                }
-                mma_bf16_16816(acc[nt], a0, a1, a2, a3, b0, b1);
-            }
-        }
-    }
-    // this warp's partial logits, then the sum over warps in warp order
-    constexpr int NP = NT * 8;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        float *rw = red + (size_t)warp * 16 * NP;
-        const int n = nt * 8 + 2 * q;
-        rw[g * NP + n] = acc[nt][0];
-        rw[g * NP + n + 1] = acc[nt][1];
-        rw[(g + 8) * NP + n] = acc[nt][2];
-        rw[(g + 8) * NP + n + 1] = acc[nt][3];
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
-        const int t = i / nout, o = i % nout;
-        float sum = 0.f;
-        for (int w = 0; w < kOneWarps; ++w)
-            sum += red[((size_t)w * 16 + t) * NP + o];
-        lg[i] = sum;
-    }
-    __syncthreads();
-}
-
 }  // namespace moe

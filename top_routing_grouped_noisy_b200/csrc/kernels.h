@@ -36,15 +36,8 @@ struct WsLayout {
     size_t hist;   // dispatch per-chunk counts, then bases, [E][chunks] int32
     size_t dcounts;// routed count of every expert [E] int32 (next to the chunk bases)
     size_t rsmall; // small-batch router partial logits [32][T][2E] f32 (T <= 64)
-    size_t dtick;  // decode GEMM block tickets, kDecTickets int32 right after the header
-    size_t dpre;   // decode GEMM partial sums (T <= 16) f32
     size_t total;
 };
-// The decode GEMMs' tickets sit at the same offset, with the same size, in the
-// layout of every parameter set, so calls with other shapes on the same workspace
-// (a shared block, a changing row count) never find stale data there: every
-// ticket is zero between calls.
-constexpr int kDecTickets = 16384;
 WsLayout ws_layout(const moe_params_t *p);
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
@@ -141,34 +134,25 @@ cudaError_t launch_up_tc_gather(const moe_params_t *p, const void *x, const int3
 cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *offsets,
                            const void *W2, void *out, int32_t *status, cudaStream_t s);
 
-// a3 / a4 for decode-shaped bf16 batches (T <= kDecodeMaxTokens): weight
-// streaming on the CUDA-core/mma.sync path.  Larger batches, from 17 tokens up,
-// run the tcgen05 grouped GEMMs, which stream the selected experts' weights
-// faster once each expert has a few rows.
+// Decode-shaped bf16 batches (1 <= T <= kDecodeMaxTokens): the weight-streaming
+// kernel of decode.cu.  Larger batches run the tcgen05 grouped GEMMs.
 constexpr int kDecodeMaxTokens = 16;
-// workspace need of the decode GEMMs (partial sums; tickets, which must fit kDecTickets)
-size_t decode_partial_floats(const moe_params_t *p);
-size_t decode_ticket_ints(const moe_params_t *p);
-// bf16, 1 <= T <= kDecodeMaxTokens and the tickets fit: the decode GEMMs serve the layer
+// a1 (logits and gate, one CTA) for such a batch: nout <= 32 and the token rows fit
+bool decode_route_fits(const moe_params_t *p, bool noisy);
+cudaError_t launch_route_decode(const moe_params_t *p, const void *x, const void *Wg,
+                                const void *Wn, const float *noise, const float *bias,
+                                int32_t *idx, float *w, float *probs_sum, float *importance,
+                                int32_t *status, cudaStream_t s);
+// a3 / a4 for such a batch (the step calls)
 bool decode_fits(const moe_params_t *p);
 cudaError_t launch_up_decode(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                              const void *W13, void *h, char *ws, cudaStream_t s);
-// a4; with y (and slot_row, topk_w) also a5 for the columns each block finishes
 cudaError_t launch_down_decode(const moe_params_t *p, const void *h, const int32_t *offsets,
-                               const void *W2, void *out, char *ws, cudaStream_t s,
-                               const int32_t *slot_row = nullptr, const float *topk_w = nullptr,
-                               void *y = nullptr);
-// a3 reading rows of x through row_token, writing x_perm alongside (moe_forward)
-// (W2_prefetch, may be NULL: the GEMM 2 weights the next launch reads, prefetched to L2)
-cudaError_t launch_up_decode_gather(const moe_params_t *p, const void *x, const int32_t *row_token,
-                                    const int32_t *offsets, const void *W13, void *h,
-                                    void *x_perm_out, char *ws, const void *W2_prefetch,
-                                    cudaStream_t s);
-// a1 finish + a2 + a6 for at most kDecodeMaxTokens tokens in one CTA, after the
-// split-K router slices (moe_forward); false when the batch does not qualify.
-bool small_forward_fits(const moe_params_t *p, bool noisy);
-cudaError_t launch_route_dispatch_small(const moe_params_t *p, const moe_buffers_t *b, char *ws,
-                                        int32_t *status, cudaStream_t s);
+                               const void *W2, void *out, char *ws, cudaStream_t s);
+// the whole layer (a1..a6) in one cooperative launch
+bool decode_forward_fits(const moe_params_t *p, bool noisy);
+cudaError_t launch_forward_decode(const moe_params_t *p, const moe_buffers_t *b, char *ws,
+                                  cudaStream_t s);
 
 cudaError_t launch_combine(const moe_params_t *p, const void *out, const int32_t *slot_row,
                            const float *w, void *y, cudaStream_t s, const void *resid = nullptr);

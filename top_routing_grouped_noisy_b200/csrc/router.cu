@@ -142,246 +142,6 @@ __global__ void __launch_bounds__(256) router_small_finish_kernel(
                         probs_sum, importance, status, sm);
 }
 
-// ---------------------------------------------------------------- small-batch forward
-// For at most kDecodeMaxTokens tokens moe_forward runs the split-K router slices
-// and then, in the CTA that finishes its slice last, adds the slices, builds the
-// dispatch tables and computes the gate statistics: one launch on a path that is
-// bound by latency.  The arithmetic is that of router_small_finish_kernel,
-// dispatch_count_kernel + dispatch_scatter_kernel ("Llama 3 Meets MoE", section 3
-// "容量因子": stable by token, assignments past the capacity dropped) and
-// gate_stats_kernel ("LLaMA-MoE v2", section "门控机制设计"), so moe_forward gives the
-// same bits as the step calls.  x_perm is written by the GEMM 1 kernel, which reads
-// the rows of x through row_token.
-__device__ void route_dispatch_small_body(
-    float *lg, int T, int E, int k, int C, int noisy,
-    const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
-    float lambda, int32_t *__restrict__ idx, float *__restrict__ w_out,
-    float *__restrict__ probs_sum, float *__restrict__ importance, int32_t *__restrict__ counts,
-    int32_t *__restrict__ kept, int32_t *__restrict__ offsets, int32_t *__restrict__ row_token,
-    int32_t *__restrict__ slot_row, float *__restrict__ f, float *__restrict__ P,
-    float *__restrict__ loss, int32_t *status)
-{
-    __shared__ int32_t s_idx[kDecodeMaxTokens * MOE_MAX_TOPK];
-    __shared__ int32_t s_cnt[MOE_MAX_EXPERTS], s_kept[MOE_MAX_EXPERTS];
-    __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
-    __shared__ double s_fp[MOE_MAX_EXPERTS];
-    const int nout = noisy ? 2 * E : E;
-    router_gate_tokens(lg, T, E, k, noisy, noise, bias, router_type, idx, w_out, probs_sum,
-                       importance, status, lg + (size_t)T * nout);
-    __syncthreads();
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x)
-        s_idx[i] = idx[i];
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int i = 0; i < T * k; ++i)
-            c += s_idx[i] == e;
-        s_cnt[e] = c;
-        s_kept[e] = C < 0 ? c : min(c, C);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int e = 0; e < E; ++e) {
-            s_off[e] = acc;
-            acc += s_kept[e];
-        }
-        s_off[E] = acc;
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        counts[e] = s_cnt[e];
-        kept[e] = s_kept[e];
-    }
-    for (int e = threadIdx.x; e <= E; e += blockDim.x)
-        offsets[e] = s_off[e];
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-        const int t = i / k, e = s_idx[i];
-        int row = -1;
-        if (e < 0 || e >= E) {
-            set_status(status, MOE_ERR_DEVICE_BADINDEX);
-        } else {
-            int rank = 0;  // the expert's assignments of earlier tokens
-            for (int i2 = 0; i2 < t * k; ++i2)
-                rank += s_idx[i2] == e;
-            if (rank < s_kept[e]) {
-                row = s_off[e] + rank;
-                row_token[row] = t;
-            }
-        }
-        slot_row[i] = row;
-    }
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const double fe = (double)s_cnt[e] / ((double)T * k);
-        const double pe = (double)probs_sum[e] / (double)T;
-        f[e] = (float)fe;
-        P[e] = (float)pe;
-        s_fp[e] = fe * pe;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double sfp = 0.0;
-        for (int i = 0; i < E; ++i)
-            sfp += s_fp[i];
-        loss[0] = (float)(lambda * sfp);
-    }
-}
-
-// The slices of the split-K router in kRouterSmallSplit CTAs; the CTA that finishes
-// last (ticket counter, zero between calls, reset by that CTA) runs the body above.
-// No CTA waits for another.
-__global__ void __launch_bounds__(256) route_dispatch_small_kernel(
-    const bf16 *__restrict__ x, const bf16 *__restrict__ Wg, const bf16 *__restrict__ Wn,
-    int d, float *__restrict__ part, int32_t *counter, int T, int E, int k, int C,
-    const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
-    float lambda, int32_t *__restrict__ idx, float *__restrict__ w_out,
-    float *__restrict__ probs_sum, float *__restrict__ importance, int32_t *__restrict__ counts,
-    int32_t *__restrict__ kept, int32_t *__restrict__ offsets, int32_t *__restrict__ row_token,
-    int32_t *__restrict__ slot_row, float *__restrict__ f, float *__restrict__ P,
-    float *__restrict__ loss, int32_t *status)
-{
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ float sm[];
-    __shared__ int s_last;
-    router_small_slice(blockIdx.x, x, Wg, Wn, T, d, E, part, sm);
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0)
-        s_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!s_last)
-        return;
-    __threadfence();
-    const int nout = Wn != nullptr ? 2 * E : E;
-    float *lg = sm;  // the slices added in order
-    for (int i = threadIdx.x; i < T * nout; i += blockDim.x) {
-        float v[kRouterSmallSplit];
-#pragma unroll
-        for (int ks = 0; ks < kRouterSmallSplit; ++ks)
-            v[ks] = __ldcg(part + (int64_t)ks * T * nout + i);
-        float acc = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < kRouterSmallSplit; ++ks)
-            acc += v[ks];
-        lg[i] = acc;
-    }
-    __syncthreads();
-    route_dispatch_small_body(lg, T, E, k, C, Wn != nullptr ? 1 : 0, noise, bias, router_type,
-                              lambda, idx, w_out, probs_sum, importance, counts, kept, offsets,
-                              row_token, slot_row, f, P, loss, status);
-    if (threadIdx.x == 0)
-        *counter = 0;
-}
-
-// ---------------------------------------------------------------- one-CTA router
-// bf16 batches of at most 16 tokens with at most 32 logits: the logits on the tensor
-// cores in one CTA (router_logits_one_cta), then the gate; with `dispatch`, also the
-// dispatch tables and the gate statistics (moe_forward's decode path).  moe_route and
-// moe_forward run the same logit and gate code, so the step calls reproduce the
-// forward bit for bit.
-template <int NT>
-__global__ void __launch_bounds__(kOneWarps * 32) router_one_cta_kernel(
-    const bf16 *__restrict__ x, const bf16 *__restrict__ Wg, const bf16 *__restrict__ Wn, int d,
-    int T, int E, int k, int C, const float *__restrict__ noise, const float *__restrict__ bias,
-    int router_type, float lambda, int dispatch, int32_t *__restrict__ idx,
-    float *__restrict__ w_out, float *__restrict__ probs_sum, float *__restrict__ importance,
-    int32_t *__restrict__ counts, int32_t *__restrict__ kept, int32_t *__restrict__ offsets,
-    int32_t *__restrict__ row_token, int32_t *__restrict__ slot_row, float *__restrict__ f,
-    float *__restrict__ P, float *__restrict__ loss, int32_t *status)
-{
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ __align__(16) char smo[];
-    const int nout = Wn != nullptr ? 2 * E : E;
-    float *lg = reinterpret_cast<float *>(smo + one_cta_logits_smem(NT));
-    router_logits_one_cta<NT>(x, Wg, Wn, T, d, E, lg, smo);
-    if (dispatch)
-        route_dispatch_small_body(lg, T, E, k, C, Wn != nullptr ? 1 : 0, noise, bias,
-                                  router_type, lambda, idx, w_out, probs_sum, importance, counts,
-                                  kept, offsets, row_token, slot_row, f, P, loss, status);
-    else
-        router_gate_tokens(lg, T, E, k, Wn != nullptr ? 1 : 0, noise, bias, router_type, idx,
-                           w_out, probs_sum, importance, status, lg + (size_t)T * nout);
-}
-
-static int one_cta_nt(const moe_params_t *p, bool noisy)
-{
-    const int nout = noisy ? 2 * p->E : p->E;
-    if (p->dtype != MOE_BF16 || p->T < 1 || p->T > 16 || nout > 32)
-        return 0;
-    return (nout + 7) / 8;
-}
-
-static cudaError_t launch_one_cta(const moe_params_t *p, const void *x, const void *Wg,
-                                  const void *Wn, const float *noise, const float *bias,
-                                  int dispatch, int32_t *idx, float *w, float *probs_sum,
-                                  float *importance, const moe_buffers_t *b, int32_t *status,
-                                  cudaStream_t s)
-{
-    const int nt = one_cta_nt(p, Wn != nullptr);
-    const size_t smem = one_cta_logits_smem(nt) + sizeof(float) * 16 * (32 + 2 * 32);
-    static bool attr_done[64][5] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 0 || dev >= 64)
-        return cudaErrorInvalidDevice;
-#define MOE_ONE(NT)                                                                                do {                                                                                               if (!attr_done[dev][NT]) {                                                                         e = cudaFuncSetAttribute(router_one_cta_kernel<NT>,                                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,                                                  (int)(one_cta_logits_smem(NT) + sizeof(float) * 16 * 96));             if (e != cudaSuccess)                                                                              return e;                                                                                  attr_done[dev][NT] = true;                                                                 }                                                                                              e = launch_pdl(router_one_cta_kernel<NT>, dim3(1), dim3(kOneWarps * 32), smem, s,                             (const bf16 *)x, (const bf16 *)Wg, (const bf16 *)Wn, p->d, p->T, p->E,                         p->k, p->capacity, noise, bias, p->router_type, p->balance_lambda,                            dispatch, idx, w, probs_sum, importance, b ? b->counts : nullptr,                             b ? b->kept : nullptr, b ? b->offsets : nullptr,                                             b ? b->row_token : nullptr, b ? b->slot_row : nullptr,                                       b ? b->f : nullptr, b ? b->P : nullptr, b ? b->loss : nullptr, status);     } while (0)
-    if (nt == 1)
-        MOE_ONE(1);
-    else if (nt == 2)
-        MOE_ONE(2);
-    else if (nt == 3)
-        MOE_ONE(3);
-    else
-        MOE_ONE(4);
-#undef MOE_ONE
-    count_launch();
-    return e == cudaSuccess ? cudaGetLastError() : e;
-}
-
-static void small_router_smem(const moe_params_t *p, bool noisy, size_t *sm1, size_t *sm2)
-{
-    const int nout = noisy ? 2 * p->E : p->E;
-    const int kc = router_small_kc(p->d);
-    *sm1 = sizeof(float) * ((size_t)p->T * kc + (size_t)kc * nout);
-    *sm2 = sizeof(float) * ((size_t)p->T * nout + 2 * (size_t)p->T * p->E);
-}
-
-bool small_forward_fits(const moe_params_t *p, bool noisy)
-{
-    if (p->dtype != MOE_BF16 || p->T < 1 || p->T > kDecodeMaxTokens)
-        return false;
-    size_t sm1, sm2;
-    small_router_smem(p, noisy, &sm1, &sm2);
-    return sm1 <= 48 * 1024 && sm2 <= 48 * 1024;
-}
-
-cudaError_t launch_route_dispatch_small(const moe_params_t *p, const moe_buffers_t *b, char *ws,
-                                        int32_t *status, cudaStream_t s)
-{
-    const WsLayout L = ws_layout(p);
-    float *sp = reinterpret_cast<float *>(ws + L.rsmall);
-    const bool noisy = b->Wnoise != nullptr;
-    if (one_cta_nt(p, noisy) > 0)
-        return launch_one_cta(p, b->x, b->Wg, b->Wnoise, b->noise, b->bias, 1, b->topk_idx,
-                              b->topk_w, b->probs_sum, b->importance, b, status, s);
-    size_t sm1, sm2;
-    small_router_smem(p, noisy, &sm1, &sm2);
-    int32_t *counter = reinterpret_cast<int32_t *>(ws) + kWsSmallCounterWord;
-    cudaError_t e = launch_pdl(route_dispatch_small_kernel, dim3(kRouterSmallSplit), dim3(256),
-                               sm1 > sm2 ? sm1 : sm2, s, (const bf16 *)b->x, (const bf16 *)b->Wg,
-                               (const bf16 *)b->Wnoise, p->d, sp, counter, p->T, p->E, p->k,
-                               p->capacity, b->noise, b->bias, p->router_type,
-                               p->balance_lambda, b->topk_idx, b->topk_w, b->probs_sum,
-                               b->importance, b->counts, b->kept, b->offsets, b->row_token,
-                               b->slot_row, b->f, b->P, b->loss, status);
-    count_launch();
-    return e;
-}
-
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
                          const void *Wnoise, const void *Wt, const float *noise,
                          const float *bias, int32_t *idx, float *w, float *probs_sum,
@@ -403,9 +163,9 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
     const size_t sm1 = sizeof(float) * ((size_t)p->T * small_kc + (size_t)small_kc * small_nout);
     const size_t sm2 =
         sizeof(float) * ((size_t)p->T * small_nout + 2 * (size_t)p->T * p->E);
-    if (one_cta_nt(p, Wnoise != nullptr) > 0) {
-        if ((e = launch_one_cta(p, x, Wg, Wnoise, noise, bias, 0, idx, w, probs_sum, importance,
-                                nullptr, status, s)) != cudaSuccess)
+    if (decode_route_fits(p, Wnoise != nullptr)) {  // the decode forward's router, one CTA
+        if ((e = launch_route_decode(p, x, Wg, Wnoise, noise, bias, idx, w, probs_sum,
+                                     importance, status, s)) != cudaSuccess)
             return e;
         return launch_count(p, idx, hist, dcounter, dcounts, status, s);
     }

@@ -417,8 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __threadfence();
             float *s_part = reinterpret_cast<float *>(smem);
             const int np = (int)gridDim.x * 2 * E;  // <= 148 x 128 floats: fits the ring
-            for (int i = gt; i < np; i += 128)
-                s_part[i] = __ldcg(part + i);
+            stage_words(s_part, part, np, gt, 128);
             gate_bar();
             for (int o = gt; o < 2 * E; o += 128) {
                 double sum = 0.0;
