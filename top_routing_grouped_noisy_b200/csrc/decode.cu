@@ -71,7 +71,8 @@ constexpr int kDsRows = 8;                   // neurons (GEMM 1) or output colum
 constexpr int kDsMaxStages = 16;
 constexpr int kDsMinStages = 2;
 constexpr int kDsBarBytes = 512;                     // full[16], empty[16], x, W
-constexpr int kDsRedBytes = 2 * kDsCw * 32 * 8 * 4;  // two buffers of the warps' sums
+// two buffers of the warps' sums, 4 NB floats per lane
+__host__ __device__ constexpr int ds_red_bytes(int nb) { return 2 * kDsCw * 32 * 4 * nb * 4; }
 constexpr int kDsRouterRed = kDsCw * 16 * 32 * 4;    // the warps' partial logits
 constexpr int kDsRouterLg = 16 * 32 * 4;             // logits [T][nout]
 constexpr int kDsRouterGate = 2 * 16 * 32 * 4;       // gate scratch [T][E] x 2
@@ -568,7 +569,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm);
     float *red = reinterpret_cast<float *>(sm + kDsBarBytes);
-    char *breg = sm + kDsBarBytes + kDsRedBytes;
+    char *breg = sm + kDsBarBytes + ds_red_bytes(NB);
     float *outs = reinterpret_cast<float *>(breg + a.bbytes);  // forward: rounded out values
     DsRing ring{breg + a.bbytes + a.obytes, bars, bars + kDsMaxStages, a.stages, a.stage_bytes,
                 0, 0};
@@ -756,16 +757,17 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
         // The warps' sums of an item: v[0..nv) into red, then epi(sum) with sum(L, q)
         // = value q of lane L added over the warps in warp order.
         auto reduce = [&](const float *v, int nv, auto epi) {
-            float *rw = red + (size_t)rb * kDsCw * 32 * 8 + ((size_t)cw * 32 + lane) * 8;
+            constexpr int RS = 4 * NB;  // floats per lane
+            float *rw = red + (size_t)rb * kDsCw * 32 * RS + ((size_t)cw * 32 + lane) * RS;
             for (int q = 0; q < nv; ++q)
                 rw[q] = v[q];
             cw_sync();
-            const float *rr = red + (size_t)rb * kDsCw * 32 * 8;
+            const float *rr = red + (size_t)rb * kDsCw * 32 * RS;
             epi([&](int L, int q) {
                 float sum = 0.f;
 #pragma unroll
                 for (int w = 0; w < kDsCw; ++w)
-                    sum += rr[((size_t)w * 32 + L) * 8 + q];
+                    sum += rr[((size_t)w * 32 + L) * RS + q];
                 return sum;
             });
             rb ^= 1;
@@ -834,9 +836,9 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
                 const int G = (int)gridDim.x;
                 __threadfence();  // this CTA's h, ordered before by the barrier above
                 if (atomicAdd(a.gbar, 1) == G - 1) {  // the last to arrive releases the others
-                    atomicExch(a.gbar, 0);
                     __threadfence();
                     atomicAdd(a.gbar + 1, 1);
+                    asm volatile("red.relaxed.gpu.global.and.b32 [%0], 0;" ::"l"(a.gbar) : "memory");
                 } else {
                     const uint64_t t0 = globaltimer_ns();
                     while (!*abort_flag && ld_acquire_gpu(a.gbar + 1) == gen) {
@@ -848,7 +850,6 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
                         __nanosleep(32);
                     }
                 }
-                __threadfence();
             } else {
                 const int nt = kDsCw * 32 - 1, t1 = ct - 1;
                 for (int r = blockIdx.x; r < R; r += gridDim.x)
@@ -1009,7 +1010,7 @@ static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
     const int ncol = (p->d + ds_grid() - 1) / ds_grid() + 1;
     g->obytes = (mode & kDsForward) ? round_up(p->T * p->k * ncol * 4, 128) : 0;
     g->stage_bytes = round_up(kDsRows * sp, 128);
-    const size_t fixed = (size_t)kDsBarBytes + kDsRedBytes + g->bbytes + g->obytes;
+    const size_t fixed = (size_t)kDsBarBytes + ds_red_bytes(g->nb) + g->bbytes + g->obytes;
     if (fixed + (size_t)kDsMinStages * g->stage_bytes > kDsSmemCap)
         return false;
     const int st = (int)((kDsSmemCap - fixed) / g->stage_bytes);
