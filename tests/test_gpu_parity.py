@@ -48,6 +48,9 @@ SMALL = {
                          seed=29),
     "decode_t16_st_cap": W("decode_t16_st_cap", T=16, d=264, d_ff=8 * 120, E=8, k=3,
                            router=wl.ST, noisy=True, bias=True, cf=1.0, rescale=True, seed=31),
+    # wide rows and 12 tokens: the decode kernel's 1024-column GEMM 1 stages
+    "decode_t12_wide": W("decode_t12_wide", T=12, d=4096, d_ff=8 * 64, E=8, k=2, noisy=True,
+                         rescale=True, seed=32),
     "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
                           router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
     "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",
@@ -129,6 +132,7 @@ STEP_CASES = {
     "decode_ragged_d": SMALL["decode_ragged_d"],
     "decode_t16_st_cap": SMALL["decode_t16_st_cap"],
     "one_token": SMALL["one_token"],
+    "decode_t12_wide": SMALL["decode_t12_wide"],
     "decode_st_bias_cap": W("decode_st_bias_cap", T=48, d=192, d_ff=16 * 40, E=16, k=4,
                             router=wl.ST, noisy=True, bias=True, cf=1.0, rescale=True,
                             lam=0.01, seed=30),

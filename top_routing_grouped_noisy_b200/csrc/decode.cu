@@ -65,7 +65,9 @@ enum : int { kDsRoute = 1, kDsUp = 2, kDsDown = 4, kDsForward = 8 };
 
 constexpr int kDsCw = 8;                     // multiplying warps (1..8); warp 0 loads
 constexpr int kDsThreads = 32 * (kDsCw + 1);
-constexpr int kDsKc1 = 2048;                 // GEMM 1: K columns per stage (16 rows)
+// GEMM 1: K columns per stage (16 rows): 2048 (4 KB copies) where two such stages fit
+// beside the rest, else 1024
+constexpr int kDsKc1 = 2048, kDsKc1Small = 1024;
 constexpr int kDsKc2 = 2048;                 // GEMM 2: K columns per stage (8 rows)
 constexpr int kDsRows = 8;                   // neurons (GEMM 1) or output columns (GEMM 2) per item
 constexpr int kDsMaxStages = 16;
@@ -109,7 +111,7 @@ struct DsArgs {
     uint64_t wait_ns;
     float lambda, scale;
     int T, d, m, E, k, C, router_type;
-    int stages, stage_bytes, bpitch, hpitch, bbytes, obytes;
+    int stages, stage_bytes, bpitch, hpitch, bbytes, obytes, kc1;
 };
 
 __device__ __forceinline__ uint4 lds128(const char *p) { return *reinterpret_cast<const uint4 *>(p); }
@@ -690,7 +692,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
         __syncthreads();
     }
     const int nsel = s_nsel;
-    const int pitch1 = ds_pitch(d, kDsKc1), pitch2 = ds_pitch(m8, kDsKc2);
+    const int kc1 = a.kc1, pitch1 = ds_pitch(d, kc1), pitch2 = ds_pitch(m8, kDsKc2);
 
     if (warp == 0) {
         // ---------------------------------------------------------------- loader
@@ -699,9 +701,9 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
             if constexpr (kUp) {
                 ds_walk_up(nsel, s_sel, s_off, m, RG, [&](int e, int j0, int nv, int, int) {
                     const bf16 *base = a.W13 + (size_t)e * 2 * m16 * d;
-                    for (int k0 = 0; k0 < d; k0 += kDsKc1)  // W1 rows to 0.., W3 rows to 8..
+                    for (int k0 = 0; k0 < d; k0 += kc1)  // W1 rows to 0.., W3 rows to 8..
                         ds_issue(
-                            ring, 2 * nv, min(kDsKc1, d - k0), d, pitch1,
+                            ring, 2 * nv, min(kc1, d - k0), d, pitch1,
                             [&](int i) {
                                 const int n = j0 + (i < nv ? i : i - nv);
                                 const int row = (n >> 4) * 32 + (n & 15) + (i < nv ? 0 : 16);
@@ -731,7 +733,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
         int ss = 0;          // the ring stage taken next
         uint32_t phase = 0;  // its phase parity
         // Takes the next stage of the ring: acc += its rows * B (GEMM 1: 16 rows and
-        // kDsKc1 columns per stage, GEMM 2: 8 rows and kDsKc2 columns).
+        // kc1 columns per stage, GEMM 2: 8 rows and kDsKc2 columns).
         auto take_stage = [&](auto gemm1, float (&acc)[NB][4], int pitch, int len, int k0,
                               const uint32_t (&bpt)[NB]) {
             const int s = ss;
@@ -743,10 +745,14 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
             }
             const uint32_t st = ring_s + (uint32_t)(s * ring.stage_bytes);
             if (ok) {
-                if constexpr (decltype(gemm1)::value)
-                    ds_stage_mma<NB, kDsKc1 / (32 * kDsCw), true>(acc, st, pitch, len, k0, bpt, cw,
-                                                                  g, c);
-                else
+                if constexpr (decltype(gemm1)::value) {
+                    if (kc1 == kDsKc1)
+                        ds_stage_mma<NB, kDsKc1 / (32 * kDsCw), true>(acc, st, pitch, len, k0, bpt,
+                                                                      cw, g, c);
+                    else
+                        ds_stage_mma<NB, kDsKc1Small / (32 * kDsCw), true>(acc, st, pitch, len,
+                                                                           k0, bpt, cw, g, c);
+                } else
                     ds_stage_mma<NB, kDsKc2 / (32 * kDsCw), false>(acc, st, pitch, len, k0, bpt,
                                                                    cw, g, c);
             }
@@ -803,8 +809,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         acc[nb][q] = 0.f;
-                for (int k0 = 0; k0 < d; k0 += kDsKc1)
-                    take_stage(std::true_type(), acc, pitch1, min(kDsKc1, d - k0), k0, bpt);
+                for (int k0 = 0; k0 < d; k0 += kc1)
+                    take_stage(std::true_type(), acc, pitch1, min(kc1, d - k0), k0, bpt);
                 float v[8];
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb)
@@ -963,7 +969,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
 
 // --------------------------------------------------------------------- host side
 struct DsGeom {
-    int nb, bpitch, hpitch, bbytes, obytes, stage_bytes, stages;
+    int nb, bpitch, hpitch, bbytes, obytes, stage_bytes, stages, kc1;
     size_t smem;
 };
 
@@ -981,11 +987,10 @@ static int ds_grid()
     return cached[dev];
 }
 
-static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
+static bool ds_geom_kc(const moe_params_t *p, int mode, bool noisy, int kc1, DsGeom *g)
 {
-    if (p->dtype != MOE_BF16 || p->T < 1 || p->T > kDecodeMaxTokens)
-        return false;
     g->nb = p->T <= 8 ? 1 : 2;
+    g->kc1 = kc1;
     const int m8 = round_up(p->m, 8);
     const int xp = round_up(p->d * 2, 128) + 16;
     const int hp = round_up(m8 * 2, 128) + 16;
@@ -997,7 +1002,7 @@ static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
     g->bpitch = g->hpitch = 0;
     if (mode & (kDsRoute | kDsUp | kDsForward)) {
         g->bpitch = xp;
-        sp = 2 * ds_pitch(p->d, kDsKc1);  // 16 rows
+        sp = 2 * ds_pitch(p->d, kc1);  // 16 rows
         xbytes = ((mode & kDsUp) ? group : p->T) * xp;
     }
     if (mode & (kDsDown | kDsForward)) {
@@ -1025,6 +1030,13 @@ static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
             return false;
     }
     return true;
+}
+
+static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
+{
+    if (p->dtype != MOE_BF16 || p->T < 1 || p->T > kDecodeMaxTokens)
+        return false;
+    return ds_geom_kc(p, mode, noisy, kDsKc1, g) || ds_geom_kc(p, mode, noisy, kDsKc1Small, g);
 }
 
 template <int NB, int MODE>
@@ -1073,6 +1085,7 @@ static cudaError_t ds_dispatch(const DsGeom &g, int grid, DsArgs &a, cudaStream_
     a.hpitch = g.hpitch;
     a.bbytes = g.bbytes;
     a.obytes = g.obytes;
+    a.kc1 = g.kc1;
     a.wait_ns = wait_limit_ns();
     return g.nb == 1 ? ds_launch<1, MODE>(g, grid, a, s) : ds_launch<2, MODE>(g, grid, a, s);
 }
