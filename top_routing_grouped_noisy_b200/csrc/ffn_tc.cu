@@ -102,7 +102,8 @@ __device__ __forceinline__ void stage_box(EpiStore &st, const uint32_t (&pk)[16]
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-        tma_store_2d(st.map, st.slots + (uint32_t)(st.slot * kStageSlotBytes), col, row0);
+        tma_store_2d_evict_first(st.map, st.slots + (uint32_t)(st.slot * kStageSlotBytes), col,
+                                 row0);
         bulk_commit();
     }
     st.slot ^= 1;
