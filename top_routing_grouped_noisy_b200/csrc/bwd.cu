@@ -21,20 +21,19 @@
 namespace moe {
 
 cudaError_t launch_bwd_dh(const moe_params_t *p, const void *d_out, const int32_t *offsets,
-                          const void *W2T, void *dh, int32_t *status, cudaStream_t s);
+                          const void *W2_e, void *dh, int32_t *status, cudaStream_t s);
 cudaError_t launch_bwd_dgu(const moe_params_t *p, const void *x_perm, const int32_t *offsets,
                            const void *W13, const void *dh, void *dgu, int32_t *status,
                            cudaStream_t s);
 cudaError_t launch_bwd_dx(const moe_params_t *p, const void *dgu, const int32_t *offsets,
-                          const void *W13T, void *dx_perm, int32_t *status, cudaStream_t s);
+                          const void *W13_e, void *dx_perm, int32_t *status, cudaStream_t s);
 cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *AT, int M, const void *BT,
                              int b_rows, uint64_t kmax, const int32_t *offsets, void *dW,
                              int ld_dw, int n_valid, int32_t *status, cudaStream_t s);
 cudaError_t launch_transpose_rows(const void *src, int ld_src, const int32_t *offsets, int E,
                                   int c_valid, int c_pad, void *dst, int ld_dst, int64_t kmax,
                                   cudaStream_t s);
-cudaError_t launch_transpose_weights(const void *src, int a, int ld_src, int b_valid, int b_pad,
-                                     int E, void *dst, cudaStream_t s);
+
 
 namespace {
 
@@ -42,7 +41,7 @@ constexpr int kPartChunks = 64;  // token chunks of the router weight-gradient p
 
 // Sections of the backward workspace (after the 256-byte header).
 struct BwdLayout {
-    size_t w2t, w13t, dgu, doutT, hT, dguT, xT, dln, wt, part, total;
+    size_t dgu, doutT, hT, dguT, xT, dln, wt, part, total;
     int64_t kmax;
 };
 
@@ -56,10 +55,6 @@ BwdLayout bwd_layout(const moe_params_t *p)
     const int64_t rows = T * k;
     L.kmax = (rows + 63) / 64 * 64 + 64 * E;
     size_t o = kWsHeader;
-    L.w2t = o;
-    o = al256(o + (size_t)(E * m16 * d) * 2);
-    L.w13t = o;
-    o = al256(o + (size_t)(E * d * 2 * m16) * 2);
     L.dgu = o;
     o = al256(o + (size_t)(rows * 2 * m16) * 2);
     L.doutT = o;
@@ -687,9 +682,7 @@ extern "C" int moe_expert_down_backward(const moe_params_t *p, const void *d_out
     int32_t *status = reinterpret_cast<int32_t *>(ws);
     cudaStream_t s = (cudaStream_t)stream;
     const int d = p->d, m = p->m, m8 = round_up(m, 8), m16 = round_up(m, 16);
-    cudaError_t e = launch_transpose_weights(W2_e, d, m8, m, m16, p->E, w + L.w2t, s);
-    if (e == cudaSuccess)
-        e = launch_bwd_dh(p, d_out, offsets, w + L.w2t, dh, status, s);
+    cudaError_t e = launch_bwd_dh(p, d_out, offsets, W2_e, dh, status, s);
     if (e == cudaSuccess)
         e = launch_transpose_rows(d_out, d, offsets, p->E, d, d, w + L.doutT, (int)L.kmax, L.kmax,
                                   s);
@@ -722,9 +715,7 @@ extern "C" int moe_expert_up_backward(const moe_params_t *p, const void *x_perm,
     const int d = p->d, m16 = round_up(p->m, 16);
     cudaError_t e = launch_bwd_dgu(p, x_perm, offsets, W13_e, dh, w + L.dgu, status, s);
     if (e == cudaSuccess)
-        e = launch_transpose_weights(W13_e, 2 * m16, d, d, d, p->E, w + L.w13t, s);
-    if (e == cudaSuccess)
-        e = launch_bwd_dx(p, w + L.dgu, offsets, w + L.w13t, dx_perm, status, s);
+        e = launch_bwd_dx(p, w + L.dgu, offsets, W13_e, dx_perm, status, s);
     if (e == cudaSuccess)
         e = launch_transpose_rows(w + L.dgu, 2 * m16, offsets, p->E, 2 * m16, 2 * m16, w + L.dguT,
                                   (int)L.kmax, L.kmax, s);

@@ -93,6 +93,13 @@ constexpr int SMEM_BYTES = 1024 + TILE_BYTES + kEpiStageBytes + (int)sizeof(Aux)
 // kind::f16: D f32, A and B bf16, both K-major, N = BN, M = BM.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
+// the same with B MN-major (bit 16): the dgrad GEMMs read the expert weights as they
+// are packed, N contiguous, instead of a transposed copy
+constexpr uint32_t kIdescBt = kIdesc | (1u << 16);
+// MN-major B in shared memory: 64-wide N chunks of BK K rows (128 bytes each)
+constexpr uint32_t kMnChunkBytes = BK * 128;
+// descriptor advance for 16 more K rows of an MN-major tile (2048 bytes, 16-byte units)
+constexpr int kMnKStep = 2048 >> 4;
 
 // Output staging as in the forward kernel: two 2 KB slots per epilogue warp, each a
 // [32 rows][64 bytes] box in the 64-byte swizzle the output map expects.
@@ -246,7 +253,7 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     return t;
 }
 
-template <int EPI, bool KG>
+template <int EPI, bool KG, bool BT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO, const int32_t *__restrict__ offsets,
@@ -334,10 +341,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     mbar_expect_tx(fb, STAGE_BYTES);
                     const int kc = t.k0 + kb * BK;
                     tma_load_2d(&tmA, fb, sa, kc, t.a_row);
-                    if constexpr (KG)
+                    if constexpr (BT) {  // MN-major B: 64-wide N chunks of BK K rows
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_3d(&tmB, fb, sa + A_BYTES + j * kMnChunkBytes, t.n0 + 64 * j,
+                                        kc, t.e);
+                    } else if constexpr (KG) {
                         tma_load_2d(&tmB, fb, sa + A_BYTES, kc, t.n0);
-                    else
+                    } else {
                         tma_load_3d(&tmB, fb, sa + A_BYTES, kc, t.n0, t.e);
+                    }
                     ++fills;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -376,11 +389,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    const uint64_t da = sdesc(sa), db = sdesc(sa + A_BYTES);
+                    const uint64_t da = sdesc(sa);
+                    const uint64_t db = BT ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
+                                           : sdesc(sa + A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_f16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), kIdesc,
-                                 (kb | k) != 0);
+                        umma_f16(d_tmem, da + (uint64_t)(2 * k),
+                                 db + (uint64_t)(BT ? kMnKStep * k : 2 * k),
+                                 BT ? kIdescBt : kIdesc, (kb | k) != 0);
                     umma_commit(smem_u32(&aux->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -519,13 +535,14 @@ __device__ __forceinline__ void tma_load_3d_pair(const CUtensorMap *map, uint32_
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
-__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t acc)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(kIdesc2), "r"(acc)
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
 __device__ __forceinline__ void umma_commit_both(uint32_t bar)
@@ -578,7 +595,7 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     return t;
 }
 
-template <int EPI, bool KG>
+template <int EPI, bool KG, bool BT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -672,11 +689,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
                     const int kc = t.k0 + kb * BK;
                     tma_load_2d_pair(&tmA, fb0, sa, kc, t.a_row + (int)rank * BM);
-                    if constexpr (KG)
+                    if constexpr (BT) {  // MN-major B: this CTA's 64-wide N chunks
+#pragma unroll
+                        for (int j = 0; j < BNH / 64; ++j)
+                            tma_load_3d_pair(&tmB, fb0, sa + A_BYTES + j * kMnChunkBytes,
+                                             t.n0 + (int)rank * BNH + 64 * j, kc, t.e);
+                    } else if constexpr (KG) {
                         tma_load_2d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH);
-                    else
+                    } else {
                         tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH,
                                          t.e);
+                    }
                     ++fills;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -717,11 +740,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    const uint64_t da = sdesc(sa), db = sdesc(sa + A_BYTES);
+                    const uint64_t da = sdesc(sa);
+                    const uint64_t db = BT ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
+                                           : sdesc(sa + A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_pair(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
-                                  (kb | k) != 0);
+                        umma_pair(d_tmem, da + (uint64_t)(2 * k),
+                                  db + (uint64_t)(BT ? kMnKStep * k : 2 * k),
+                                  BT ? kIdesc2 | (1u << 16) : kIdesc2, (kb | k) != 0);
                     umma_commit_both(smem_u32(&aux->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -880,47 +906,12 @@ __global__ void __launch_bounds__(256) transpose_rows_kernel(
             *reinterpret_cast<uint4 *>(dst + (int64_t)(col + i) * ld_dst + kc0 + 8 * rg) = out[i];
 }
 
-// Batched weight transpose: src [E][a][ld_src] (columns [0, b_valid) meaningful) ->
-// dst [E][b_pad][a], zero rows for b in [b_valid, b_pad).  a % 8 == 0.  CTA = 64
-// src rows x 256 src columns of one expert.
-__global__ void __launch_bounds__(256) transpose_weights_kernel(const bf16 *__restrict__ src,
-                                                                int a, int ld_src, int b_valid,
-                                                                int b_pad, bf16 *__restrict__ dst)
-{
-    pdl_wait();
-    pdl_trigger();
-    const int e = blockIdx.z;
-    const int a0 = blockIdx.x * 64, b0 = blockIdx.y * 256;
-    const bf16 *S = src + (int64_t)e * a * ld_src;
-    bf16 *Dd = dst + (int64_t)e * b_pad * a;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int rg = lane & 7, cq = (lane >> 3) + 4 * warp;
-    const int col = b0 + 8 * cq;
-    const int row0 = a0 + 8 * rg;
-    if (col >= b_pad || row0 >= a)
-        return;
-    uint4 in[8], out[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        in[i] = make_uint4(0, 0, 0, 0);
-        if (row0 + i < a && col + 8 <= ld_src && col < b_valid)
-            in[i] = mask_cols(*reinterpret_cast<const uint4 *>(S + (int64_t)(row0 + i) * ld_src +
-                                                               col),
-                              col, b_valid);
-    }
-    transpose8x8(in, out);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (col + i < b_pad)
-            *reinterpret_cast<uint4 *>(Dd + (int64_t)(col + i) * a + row0) = out[i];
-}
-
 // ------------------------------------------------------------------------ host side
 
 struct DevInfo {
     int sms = 0;
     int pair_clusters = 0;
-    bool attr[6] = {false, false, false, false, false, false};
+    bool attr[8] = {false, false, false, false, false, false, false, false};
 };
 static std::mutex g_mu;
 static DevInfo g_dev[64];
@@ -950,14 +941,15 @@ static cudaError_t prepare(DevInfo **out)
     if (di.sms == 0 &&
         (e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    if ((e = set_attr(bwd_gemm_kernel<EPI_STORE, false>, di.attr[0])) != cudaSuccess ||
-        (e = set_attr(bwd_gemm_kernel<EPI_SWIGLU_BWD, false>, di.attr[1])) != cudaSuccess ||
-        (e = set_attr(bwd_gemm_kernel<EPI_STORE, true>, di.attr[2])) != cudaSuccess ||
-        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, false>, di.attr[3],
+    if ((e = set_attr(bwd_gemm_kernel<EPI_STORE, false, true>, di.attr[0])) != cudaSuccess ||
+        (e = set_attr(bwd_gemm_kernel<EPI_SWIGLU_BWD, false, false>, di.attr[1])) !=
+            cudaSuccess ||
+        (e = set_attr(bwd_gemm_kernel<EPI_STORE, true, false>, di.attr[2])) != cudaSuccess ||
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, false, true>, di.attr[3],
                       pair::SMEM_BYTES)) != cudaSuccess ||
-        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_SWIGLU_BWD, false>, di.attr[4],
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_SWIGLU_BWD, false, false>, di.attr[4],
                       pair::SMEM_BYTES)) != cudaSuccess ||
-        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, true>, di.attr[5],
+        (e = set_attr(pair::bwd_gemm_2sm_kernel<EPI_STORE, true, false>, di.attr[5],
                       pair::SMEM_BYTES)) != cudaSuccess)
         return e;
     if (di.pair_clusters == 0) {
@@ -973,7 +965,8 @@ static cudaError_t prepare(DevInfo **out)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, pair::bwd_gemm_2sm_kernel<EPI_STORE, false>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, pair::bwd_gemm_2sm_kernel<EPI_STORE, false, true>,
+                                           &cfg);
         if (e != cudaSuccess)
             return e;
         di.pair_clusters = n > 0 ? n : 1;
@@ -986,8 +979,9 @@ static cudaError_t prepare(DevInfo **out)
 constexpr int64_t kPairMinRows = 4096;
 
 // One backward GEMM.  A [a_rows][a_ld] (K extent a_k); B: row-grouped [E][b_rows][b_ld],
-// K-grouped [b_rows][b_ld] (K extent b_k); out [out_rows][ld_out], n_valid columns.
-template <int EPI, bool KG>
+// K-grouped [b_rows][b_ld] (K extent b_k); with BT (MN-major B) [E][b_k][b_ld] with N
+// extent b_rows; out [out_rows][ld_out], n_valid columns.
+template <int EPI, bool KG, bool BT>
 static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a_rows,
                           const void *B, uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
                           const int32_t *offsets, int E, int M, bf16 *out, int ld_out,
@@ -1004,7 +998,14 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     const uint32_t b_box = use_pair ? (uint32_t)pair::BNH : (uint32_t)BN;
     if ((e = tc::make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
         return e;
-    if constexpr (KG) {
+    if constexpr (BT) {
+        // N innermost: boxes of 64 N x BK K rows, N and K past their extents read as zero
+        const uint64_t db[3] = {b_rows, b_k, (uint64_t)E};
+        const uint64_t sb[2] = {b_ld * 2, b_k * b_ld * 2};
+        const uint32_t bb[3] = {64, BK, 1};
+        if ((e = tc::make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
+            return e;
+    } else if constexpr (KG) {
         const uint64_t db[2] = {b_k, b_rows}, sb[1] = {b_ld * 2};
         const uint32_t bb[2] = {BK, b_box};
         if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
@@ -1023,7 +1024,7 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
         return e;
     count_launch();
     if (!use_pair)
-        return launch_pdl(bwd_gemm_kernel<EPI, KG>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES,
+        return launch_pdl(bwd_gemm_kernel<EPI, KG, BT>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES,
                           s, ta, tb, to, offsets, E, (int)b_rows, (int)a_k, M, out, ld_out,
                           n_valid, dh, ld_dh, status, wait_limit_ns());
     cudaLaunchConfig_t cfg = {};
@@ -1040,7 +1041,7 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, pair::bwd_gemm_2sm_kernel<EPI, KG>, ta, tb, to, offsets, E,
+    return cudaLaunchKernelEx(&cfg, pair::bwd_gemm_2sm_kernel<EPI, KG, BT>, ta, tb, to, offsets, E,
                               (int)b_rows, (int)a_k, M, out, ld_out, n_valid, dh, ld_dh, status,
                               wait_limit_ns());
 }
@@ -1049,15 +1050,15 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
 
 using namespace bwd;
 
-// dh [rows][m8] = d_out [rows][d] x W2T_e [m16][d]^T
+// dh [rows][m8] = d_out [rows][d] x W2_e [d][m8] (B MN-major: the packed W2 as it is)
 cudaError_t launch_bwd_dh(const moe_params_t *p, const void *d_out, const int32_t *offsets,
-                          const void *W2T, void *dh, int32_t *status, cudaStream_t s)
+                          const void *W2_e, void *dh, int32_t *status, cudaStream_t s)
 {
-    const uint64_t d = p->d, m8 = round_up(p->m, 8), m16 = round_up(p->m, 16);
+    const uint64_t d = p->d, m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    return launch<EPI_STORE, false>(d_out, d, d, rows, W2T, d, d, m16, offsets, p->E, 0,
-                                    (bf16 *)dh, (int)m8, rows, (int)m8, nullptr, 0, status, s,
-                                    (int64_t)rows >= kPairMinRows);
+    return launch<EPI_STORE, false, true>(d_out, d, d, rows, W2_e, d, m8, m8, offsets, p->E, 0,
+                                          (bf16 *)dh, (int)m8, rows, (int)m8, nullptr, 0, status,
+                                          s, (int64_t)rows >= kPairMinRows);
 }
 
 // dGU [rows][2 m16] = SwiGLU backward of (x_perm x W13_e^T) with dh [rows][m8]
@@ -1067,21 +1068,21 @@ cudaError_t launch_bwd_dgu(const moe_params_t *p, const void *x_perm, const int3
 {
     const uint64_t d = p->d, m8 = round_up(p->m, 8), m16 = round_up(p->m, 16);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    return launch<EPI_SWIGLU_BWD, false>(x_perm, d, d, rows, W13, d, d, 2 * m16, offsets, p->E,
+    return launch<EPI_SWIGLU_BWD, false, false>(x_perm, d, d, rows, W13, d, d, 2 * m16, offsets, p->E,
                                          0, (bf16 *)dgu, (int)(2 * m16), rows, (int)(2 * m16),
                                          (const bf16 *)dh, (int)m8, status, s,
                                          (int64_t)rows >= kPairMinRows);
 }
 
-// dx_perm [rows][d] = dGU [rows][2 m16] x W13T_e [d][2 m16]^T
+// dx_perm [rows][d] = dGU [rows][2 m16] x W13_e [2 m16][d] (B MN-major: the packed W13)
 cudaError_t launch_bwd_dx(const moe_params_t *p, const void *dgu, const int32_t *offsets,
-                          const void *W13T, void *dx_perm, int32_t *status, cudaStream_t s)
+                          const void *W13_e, void *dx_perm, int32_t *status, cudaStream_t s)
 {
     const uint64_t d = p->d, m16 = round_up(p->m, 16);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    return launch<EPI_STORE, false>(dgu, 2 * m16, 2 * m16, rows, W13T, 2 * m16, 2 * m16, d,
-                                    offsets, p->E, 0, (bf16 *)dx_perm, (int)d, rows, (int)d,
-                                    nullptr, 0, status, s, (int64_t)rows >= kPairMinRows);
+    return launch<EPI_STORE, false, true>(dgu, 2 * m16, 2 * m16, rows, W13_e, 2 * m16, d, d,
+                                          offsets, p->E, 0, (bf16 *)dx_perm, (int)d, rows, (int)d,
+                                          nullptr, 0, status, s, (int64_t)rows >= kPairMinRows);
 }
 
 // dW [E][M][n_valid]: A^T [M][kmax] and B^T [b_rows][kmax] in the padded K order
@@ -1089,7 +1090,7 @@ cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *AT, int M, const
                              int b_rows, uint64_t kmax, const int32_t *offsets, void *dW,
                              int ld_dw, int n_valid, int32_t *status, cudaStream_t s)
 {
-    return launch<EPI_STORE, true>(AT, kmax, kmax, (uint64_t)M, BT, kmax, kmax, (uint64_t)b_rows,
+    return launch<EPI_STORE, true, false>(AT, kmax, kmax, (uint64_t)M, BT, kmax, kmax, (uint64_t)b_rows,
                                    offsets, p->E, M, (bf16 *)dW, ld_dw, (uint64_t)p->E * M,
                                    n_valid, nullptr, 0, status, s,
                                    (int64_t)p->T * p->k >= kPairMinRows);
@@ -1105,12 +1106,5 @@ cudaError_t launch_transpose_rows(const void *src, int ld_src, const int32_t *of
                       (bf16 *)dst, ld_dst);
 }
 
-cudaError_t launch_transpose_weights(const void *src, int a, int ld_src, int b_valid, int b_pad,
-                                     int E, void *dst, cudaStream_t s)
-{
-    count_launch();
-    return launch_pdl(transpose_weights_kernel, dim3((a + 63) / 64, (b_pad + 255) / 256, E),
-                      dim3(256), 0, s, (const bf16 *)src, a, ld_src, b_valid, b_pad, (bf16 *)dst);
-}
 
 }  // namespace moe

@@ -33,6 +33,20 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr)
     return d;
 }
 
+// Descriptor of an MN-major, 128B-swizzled tile: chunks of 64 MN elements (128-byte
+// rows, one per K index; 8-row K groups 1024 bytes apart) lbo bytes apart; tile base
+// 1024-aligned.  Advancing K by 16 adds 2048 bytes (two 8-row groups).
+__device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr, uint32_t lbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);      // start address, 16-byte units
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;   // leading byte offset: next 64-wide MN chunk
+    d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: next 8-row K group
+    d |= (uint64_t)1 << 46;                        // descriptor version
+    d |= (uint64_t)2 << 61;                        // 128-byte swizzle
+    return d;
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
