@@ -112,6 +112,7 @@ struct DsArgs {
     float lambda, scale;
     int T, d, m, E, k, C, router_type;
     int stages, stage_bytes, bpitch, hpitch, bbytes, obytes, kc1;
+    int split13;  // GEMM 1 stages of 8 rows (W1 rows, then W3 rows) instead of 16
 };
 
 __device__ __forceinline__ uint4 lds128(const char *p) { return *reinterpret_cast<const uint4 *>(p); }
@@ -256,18 +257,21 @@ __device__ __forceinline__ uint4 lds128_s(uint32_t addr)
     return v;
 }
 
-// acc[nb] += A (the stage's rows at `pitch`: rows 0..7, and with ROWS16 rows 8..15
-// too; `len` columns) * B (shared addresses bp[nb] of this lane's B row, 0 for
-// none; columns k0 + ...), over this warp's 32-column steps of the stage.  Every
-// fragment load of the stage is issued before the first mma: the loop is bound by
-// shared-memory latency otherwise.
+// acc[.][nb] += A * B over this warp's 32-column steps of a stage: A rows 0..7 are
+// the stage's rows at `pitch` from st, and with ROWS16 rows 8..15 those from st8 (the
+// next 8 rows of the same stage, or the rows of a second stage); `len` columns; B at
+// the shared addresses bp[nb] of this lane's B row (0 for none), columns k0 + ....
+// Even steps add into acc[0], odd ones into acc[1] (two independent mma chains; the
+// split depends only on the column index).  Every fragment load of the stage is
+// issued before the first mma: the loop is bound by shared-memory latency otherwise.
 template <int NB, int KS, bool ROWS16>
-__device__ __forceinline__ void ds_stage_mma(float (&acc)[NB][4], uint32_t st, int pitch, int len,
-                                             int k0, const uint32_t (&bp)[NB], int cw, int g, int c)
+__device__ __forceinline__ void ds_stage_mma(float (&acc)[2][NB][4], uint32_t st, uint32_t st8,
+                                             int pitch, int len, int k0,
+                                             const uint32_t (&bp)[NB], int cw, int g, int c)
 {
     const uint4 zero = make_uint4(0, 0, 0, 0);
     const uint32_t arow = st + (uint32_t)(g * pitch + 16 * c);
-    const uint32_t arow8 = arow + (uint32_t)(8 * pitch);
+    const uint32_t arow8 = st8 + (uint32_t)(g * pitch + 16 * c);
     uint4 A[KS], A8[KS], B[KS][NB];
 #pragma unroll
     for (int j = 0; j < KS; ++j) {
@@ -283,8 +287,10 @@ __device__ __forceinline__ void ds_stage_mma(float (&acc)[NB][4], uint32_t st, i
     for (int j = 0; j < KS; ++j)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-            mma_bf16_16816(acc[nb], A[j].x, A8[j].x, A[j].y, A8[j].y, B[j][nb].x, B[j][nb].y);
-            mma_bf16_16816(acc[nb], A[j].z, A8[j].z, A[j].w, A8[j].w, B[j][nb].z, B[j][nb].w);
+            mma_bf16_16816(acc[j & 1][nb], A[j].x, A8[j].x, A[j].y, A8[j].y, B[j][nb].x,
+                           B[j][nb].y);
+            mma_bf16_16816(acc[j & 1][nb], A[j].z, A8[j].z, A[j].w, A8[j].w, B[j][nb].z,
+                           B[j][nb].w);
         }
 }
 
@@ -701,15 +707,28 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
             if constexpr (kUp) {
                 ds_walk_up(nsel, s_sel, s_off, m, RG, [&](int e, int j0, int nv, int, int) {
                     const bf16 *base = a.W13 + (size_t)e * 2 * m16 * d;
-                    for (int k0 = 0; k0 < d; k0 += kc1)  // W1 rows to 0.., W3 rows to 8..
-                        ds_issue(
-                            ring, 2 * nv, min(kc1, d - k0), d, pitch1,
-                            [&](int i) {
-                                const int n = j0 + (i < nv ? i : i - nv);
-                                const int row = (n >> 4) * 32 + (n & 15) + (i < nv ? 0 : 16);
-                                return base + (size_t)row * d + k0;
-                            },
-                            [&](int i) { return i < nv ? i : 8 + i - nv; }, a, abort_flag);
+                    for (int k0 = 0; k0 < d; k0 += kc1) {
+                        if (a.split13) {  // a stage of W1 rows, then one of W3 rows
+                            for (int half = 0; half < 2; ++half)
+                                ds_issue(
+                                    ring, nv, min(kc1, d - k0), d, pitch1,
+                                    [&](int i) {
+                                        const int n = j0 + i;
+                                        const int row = (n >> 4) * 32 + (n & 15) + 16 * half;
+                                        return base + (size_t)row * d + k0;
+                                    },
+                                    [&](int i) { return i; }, a, abort_flag);
+                        } else {  // W1 rows to stage rows 0.., W3 rows to 8..
+                            ds_issue(
+                                ring, 2 * nv, min(kc1, d - k0), d, pitch1,
+                                [&](int i) {
+                                    const int n = j0 + (i < nv ? i : i - nv);
+                                    const int row = (n >> 4) * 32 + (n & 15) + (i < nv ? 0 : 16);
+                                    return base + (size_t)row * d + k0;
+                                },
+                                [&](int i) { return i < nv ? i : 8 + i - nv; }, a, abort_flag);
+                        }
+                    }
                 });
             }
             if constexpr (kDown) {
@@ -732,33 +751,46 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
         const uint32_t ring_s = smem_u32(ring.base), breg_s = smem_u32(breg);
         int ss = 0;          // the ring stage taken next
         uint32_t phase = 0;  // its phase parity
-        // Takes the next stage of the ring: acc += its rows * B (GEMM 1: 16 rows and
-        // kc1 columns per stage, GEMM 2: 8 rows and kDsKc2 columns).
-        auto take_stage = [&](auto gemm1, float (&acc)[NB][4], int pitch, int len, int k0,
+        // Takes the next stage of the ring (GEMM 1 with paired 8-row stages: the next two,
+        // W1 rows then W3 rows) and adds its rows * B into acc.  kind: 2 = GEMM 1 with
+        // 16-row stages of kc1 columns, 1 = GEMM 1 with paired 8-row stages, 0 = GEMM 2
+        // (8 rows, kDsKc2 columns).
+        auto take_stage = [&](auto kind, float (&acc)[2][NB][4], int pitch, int len, int k0,
                               const uint32_t (&bpt)[NB]) {
-            const int s = ss;
-            const bool ok = mbar_wait(smem_u32(&ring.full[s]), phase, a.wait_ns, abort_flag,
-                                      a.status);
-            if (++ss == ring.stages) {
-                ss = 0;
-                phase ^= 1u;
+            constexpr int KIND = decltype(kind)::value;
+            constexpr int NS = KIND == 1 ? 2 : 1;
+            int sl[NS];
+            bool ok = true;
+#pragma unroll
+            for (int i = 0; i < NS; ++i) {
+                sl[i] = ss;
+                ok = ok && mbar_wait(smem_u32(&ring.full[ss]), phase, a.wait_ns, abort_flag,
+                                     a.status);
+                if (++ss == ring.stages) {
+                    ss = 0;
+                    phase ^= 1u;
+                }
             }
-            const uint32_t st = ring_s + (uint32_t)(s * ring.stage_bytes);
+            const uint32_t st = ring_s + (uint32_t)(sl[0] * ring.stage_bytes);
+            const uint32_t st8 = KIND == 1 ? ring_s + (uint32_t)(sl[NS - 1] * ring.stage_bytes)
+                                           : st + (uint32_t)(8 * pitch);
             if (ok) {
-                if constexpr (decltype(gemm1)::value) {
+                if constexpr (KIND > 0) {
                     if (kc1 == kDsKc1)
-                        ds_stage_mma<NB, kDsKc1 / (32 * kDsCw), true>(acc, st, pitch, len, k0, bpt,
-                                                                      cw, g, c);
+                        ds_stage_mma<NB, kDsKc1 / (32 * kDsCw), true>(acc, st, st8, pitch, len, k0,
+                                                                      bpt, cw, g, c);
                     else
-                        ds_stage_mma<NB, kDsKc1Small / (32 * kDsCw), true>(acc, st, pitch, len,
-                                                                           k0, bpt, cw, g, c);
+                        ds_stage_mma<NB, kDsKc1Small / (32 * kDsCw), true>(acc, st, st8, pitch,
+                                                                           len, k0, bpt, cw, g, c);
                 } else
-                    ds_stage_mma<NB, kDsKc2 / (32 * kDsCw), false>(acc, st, pitch, len, k0, bpt,
-                                                                   cw, g, c);
+                    ds_stage_mma<NB, kDsKc2 / (32 * kDsCw), false>(acc, st, st8, pitch, len, k0,
+                                                                   bpt, cw, g, c);
             }
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(smem_u32(&ring.empty[s]));
+#pragma unroll
+                for (int i = 0; i < NS; ++i)
+                    mbar_arrive(smem_u32(&ring.empty[sl[i]]));
         };
         // The warps' sums of an item: v[0..nv) into red, then epi(sum) with sum(L, q)
         // = value q of lane L added over the warps in warp order.
@@ -802,21 +834,29 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
                         bpt[nb] = j < nr ? breg_s + (uint32_t)(s_rtok[r0 + j] * bp + 16 * c) : 0u;
                     }
                 }
-                // row g: W1 of neuron g (acc 0, 1), row g + 8: its W3 row (acc 2, 3)
-                float acc[NB][4];
+                // A row g is the W1 row of neuron g (acc 0, 1), row g + 8 its W3 row (acc 2, 3)
+                float acc[2][NB][4];
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        acc[nb][q] = 0.f;
-                for (int k0 = 0; k0 < d; k0 += kc1)
-                    take_stage(std::true_type(), acc, pitch1, min(kc1, d - k0), k0, bpt);
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            acc[h][nb][q] = 0.f;
+                for (int k0 = 0; k0 < d; k0 += kc1) {
+                    if (a.split13)
+                        take_stage(std::integral_constant<int, 1>(), acc, pitch1, min(kc1, d - k0),
+                                   k0, bpt);
+                    else
+                        take_stage(std::integral_constant<int, 2>(), acc, pitch1, min(kc1, d - k0),
+                                   k0, bpt);
+                }
                 float v[8];
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        v[nb * 4 + q] = acc[nb][q];
+                        v[nb * 4 + q] = acc[0][nb][q] + acc[1][nb][q];
                 reduce(v, 4 * NB, [&](auto sum) {
                     for (int i = ct; i < 32 * 2 * NB; i += kDsCw * 32) {
                         const int L = i & 31, q = i >> 5, nb = q >> 1, jj = q & 1;
@@ -918,19 +958,22 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
                     const int j = nb * 8 + g;
                     bpt[nb] = j < nr ? breg_s + (uint32_t)((rb0 + j) * a.hpitch + 16 * c) : 0u;
                 }
-                float acc[NB][4];
+                float acc[2][NB][4];
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        acc[nb][q] = 0.f;
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            acc[h][nb][q] = 0.f;
                 for (int k0 = 0; k0 < m8; k0 += kDsKc2)
-                    take_stage(std::false_type(), acc, pitch2, min(kDsKc2, m8 - k0), k0, bpt);
+                    take_stage(std::integral_constant<int, 0>(), acc, pitch2, min(kDsKc2, m8 - k0),
+                               k0, bpt);
                 float v[8];
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
-                    v[nb * 2 + 0] = acc[nb][0];
-                    v[nb * 2 + 1] = acc[nb][1];
+                    v[nb * 2 + 0] = acc[0][nb][0] + acc[1][nb][0];
+                    v[nb * 2 + 1] = acc[0][nb][1] + acc[1][nb][1];
                 }
                 reduce(v, 2 * NB, [&](auto sum) {
                     for (int i = ct; i < 32 * 2 * NB; i += kDsCw * 32) {
@@ -969,7 +1012,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
 
 // --------------------------------------------------------------------- host side
 struct DsGeom {
-    int nb, bpitch, hpitch, bbytes, obytes, stage_bytes, stages, kc1;
+    int nb, bpitch, hpitch, bbytes, obytes, stage_bytes, stages, kc1, split13;
     size_t smem;
 };
 
@@ -987,10 +1030,12 @@ static int ds_grid()
     return cached[dev];
 }
 
-static bool ds_geom_kc(const moe_params_t *p, int mode, bool noisy, int kc1, DsGeom *g)
+static bool ds_geom_kc(const moe_params_t *p, int mode, bool noisy, int kc1, int split13,
+                       DsGeom *g)
 {
     g->nb = p->T <= 8 ? 1 : 2;
     g->kc1 = kc1;
+    g->split13 = split13;
     const int m8 = round_up(p->m, 8);
     const int xp = round_up(p->d * 2, 128) + 16;
     const int hp = round_up(m8 * 2, 128) + 16;
@@ -1002,7 +1047,7 @@ static bool ds_geom_kc(const moe_params_t *p, int mode, bool noisy, int kc1, DsG
     g->bpitch = g->hpitch = 0;
     if (mode & (kDsRoute | kDsUp | kDsForward)) {
         g->bpitch = xp;
-        sp = 2 * ds_pitch(p->d, kc1);  // 16 rows
+        sp = (split13 ? 1 : 2) * ds_pitch(p->d, kc1);  // 8 or 16 rows
         xbytes = ((mode & kDsUp) ? group : p->T) * xp;
     }
     if (mode & (kDsDown | kDsForward)) {
@@ -1036,7 +1081,17 @@ static bool ds_geom(const moe_params_t *p, int mode, bool noisy, DsGeom *g)
 {
     if (p->dtype != MOE_BF16 || p->T < 1 || p->T > kDecodeMaxTokens)
         return false;
-    return ds_geom_kc(p, mode, noisy, kDsKc1, g) || ds_geom_kc(p, mode, noisy, kDsKc1Small, g);
+    // GEMM 1 stages: 16 rows x 2048 columns while the forward layout fits 3 of them, else
+    // 8 rows (W1 and W3 rows in alternate stages) x 2048, else 8 rows x 1024 -- decided on
+    // the forward layout for every mode, so the step calls stream like the forward
+    DsGeom f;
+    int split = 0, kc = kDsKc1;
+    if (!(ds_geom_kc(p, kDsForward, false, kDsKc1, 0, &f) && f.stages >= 3)) {
+        split = 1;
+        if (!ds_geom_kc(p, kDsForward, false, kDsKc1, 1, &f))
+            kc = kDsKc1Small;
+    }
+    return ds_geom_kc(p, mode, noisy, kc, split, g);
 }
 
 template <int NB, int MODE>
@@ -1086,6 +1141,7 @@ static cudaError_t ds_dispatch(const DsGeom &g, int grid, DsArgs &a, cudaStream_
     a.bbytes = g.bbytes;
     a.obytes = g.obytes;
     a.kc1 = g.kc1;
+    a.split13 = g.split13;
     a.wait_ns = wait_limit_ns();
     return g.nb == 1 ? ds_launch<1, MODE>(g, grid, a, s) : ds_launch<2, MODE>(g, grid, a, s);
 }
