@@ -420,8 +420,9 @@ int moe_cluster_distances(const void *F, int32_t d, int32_t d_ff, int32_t E, int
  * are rounded once from f32 sums; router weight gradients are f32.  g and u are
  * recomputed (x_perm W13_e^T), not stored by the forward.
  * The workspace (moe_backward_workspace_size bytes, zeroed once with
- * moe_workspace_init) holds the transposed weights and activations the
- * weight-gradient GEMMs read (1.29 GB at T=16384, d=4096, 8 x 1376, k=2). */
+ * moe_workspace_init) holds dGU [T*k][2 m16] (the gate and up gradients of every
+ * row) and the router-gradient partials (0.20 GB at T=16384, d=4096, 8 x 1376,
+ * k=2); the weight-gradient GEMMs read the activations in place. */
 typedef struct {
     const void *dy;    /* [T][d] dl/dy */
     void *dx;          /* [T][d] out: dl/dx (complete: experts and router) */

@@ -27,12 +27,9 @@ cudaError_t launch_bwd_dgu(const moe_params_t *p, const void *x_perm, const int3
                            cudaStream_t s);
 cudaError_t launch_bwd_dx(const moe_params_t *p, const void *dgu, const int32_t *offsets,
                           const void *W13_e, void *dx_perm, int32_t *status, cudaStream_t s);
-cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *AT, int M, const void *BT,
-                             int b_rows, uint64_t kmax, const int32_t *offsets, void *dW,
-                             int ld_dw, int n_valid, int32_t *status, cudaStream_t s);
-cudaError_t launch_transpose_rows(const void *src, int ld_src, const int32_t *offsets, int E,
-                                  int c_valid, int c_pad, void *dst, int ld_dst, int64_t kmax,
-                                  cudaStream_t s);
+cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *A, int M, int a_ld, const void *B,
+                             int n_cols, int b_ld, const int32_t *offsets, void *dW, int ld_dw,
+                             int n_valid, int32_t *status, cudaStream_t s);
 
 
 namespace {
@@ -41,8 +38,7 @@ constexpr int kPartChunks = 64;  // token chunks of the router weight-gradient p
 
 // Sections of the backward workspace (after the 256-byte header).
 struct BwdLayout {
-    size_t dgu, doutT, hT, dguT, xT, dln, wt, part, total;
-    int64_t kmax;
+    size_t dgu, dln, wt, part, total;
 };
 
 size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -53,18 +49,9 @@ BwdLayout bwd_layout(const moe_params_t *p)
     const int64_t T = p->T, d = p->d, E = p->E, k = p->k;
     const int64_t m16 = round_up(p->m, 16);
     const int64_t rows = T * k;
-    L.kmax = (rows + 63) / 64 * 64 + 64 * E;
     size_t o = kWsHeader;
     L.dgu = o;
     o = al256(o + (size_t)(rows * 2 * m16) * 2);
-    L.doutT = o;
-    o = al256(o + (size_t)(d * L.kmax) * 2);
-    L.hT = o;
-    o = al256(o + (size_t)(m16 * L.kmax) * 2);
-    L.dguT = o;
-    o = al256(o + (size_t)(2 * m16 * L.kmax) * 2);
-    L.xT = o;
-    o = al256(o + (size_t)(d * L.kmax) * 2);
     L.dln = o;
     o = al256(o + (size_t)(T * 2 * E) * 4);
     L.wt = o;  // router weights transposed, [NE2 <= 128][d] bf16
@@ -677,20 +664,12 @@ extern "C" int moe_expert_down_backward(const moe_params_t *p, const void *d_out
     NEED(W2_e);
     NEED(dh);
     NEED(dW2_e);
-    const BwdLayout L = bwd_layout(p);
-    char *w = static_cast<char *>(ws);
-    int32_t *status = reinterpret_cast<int32_t *>(ws);
+    int32_t *status = reinterpret_cast<int32_t *>(ws);  // the workspace holds the status only
     cudaStream_t s = (cudaStream_t)stream;
-    const int d = p->d, m = p->m, m8 = round_up(m, 8), m16 = round_up(m, 16);
+    const int d = p->d, m = p->m, m8 = round_up(m, 8);
     cudaError_t e = launch_bwd_dh(p, d_out, offsets, W2_e, dh, status, s);
-    if (e == cudaSuccess)
-        e = launch_transpose_rows(d_out, d, offsets, p->E, d, d, w + L.doutT, (int)L.kmax, L.kmax,
-                                  s);
-    if (e == cudaSuccess)
-        e = launch_transpose_rows(h, m8, offsets, p->E, m, m16, w + L.hT, (int)L.kmax, L.kmax, s);
-    if (e == cudaSuccess)
-        e = launch_bwd_wgrad(p, w + L.doutT, d, w + L.hT, m16, (uint64_t)L.kmax, offsets, dW2_e,
-                             m8, m8, status, s);
+    if (e == cudaSuccess)  // dW2_e = d_out_e^T h_e (h columns past m read as zero)
+        e = launch_bwd_wgrad(p, d_out, d, d, h, m, m8, offsets, dW2_e, m8, m8, status, s);
     return finish(fn, e);
 }
 
@@ -716,15 +695,9 @@ extern "C" int moe_expert_up_backward(const moe_params_t *p, const void *x_perm,
     cudaError_t e = launch_bwd_dgu(p, x_perm, offsets, W13_e, dh, w + L.dgu, status, s);
     if (e == cudaSuccess)
         e = launch_bwd_dx(p, w + L.dgu, offsets, W13_e, dx_perm, status, s);
-    if (e == cudaSuccess)
-        e = launch_transpose_rows(w + L.dgu, 2 * m16, offsets, p->E, 2 * m16, 2 * m16, w + L.dguT,
-                                  (int)L.kmax, L.kmax, s);
-    if (e == cudaSuccess)
-        e = launch_transpose_rows(x_perm, d, offsets, p->E, d, d, w + L.xT, (int)L.kmax, L.kmax,
-                                  s);
-    if (e == cudaSuccess)
-        e = launch_bwd_wgrad(p, w + L.dguT, 2 * m16, w + L.xT, d, (uint64_t)L.kmax, offsets,
-                             dW13_e, d, d, status, s);
+    if (e == cudaSuccess)  // dW13_e = dGU_e^T x_e
+        e = launch_bwd_wgrad(p, w + L.dgu, 2 * m16, 2 * m16, x_perm, d, d, offsets, dW13_e, d, d,
+                             status, s);
     return finish(fn, e);
 }
 

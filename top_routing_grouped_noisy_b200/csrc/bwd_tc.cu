@@ -3,22 +3,22 @@
 // backwards: the gradients of out = W2 (silu(W1 x) * W3 x)).
 //
 // One persistent kernel, two tile orders:
-//   row-grouped (dgrad): C[rows of expert e][N] = A[rows][K] B_e[N][K]^T, the rows
-//     of expert e being [offsets[e], offsets[e+1]) -- the forward's tile order:
-//       dh      = d_out  W2_e        (A = d_out,  B = W2_e^T  [m16][d])
-//       dGU     = SwiGLU backward of x_perm W13_e^T   (fused epilogue, below)
-//       dx_perm = dGU    W13_e       (A = dGU,    B = W13_e^T [d][2 m16])
-//   K-grouped (wgrad): C_e[M][N] = A[M][K_e] B[N][K_e]^T, the reduction running over
-//     the rows of expert e, which the transposes below lay out as the column range
-//     [koff[e], koff[e+1]) of A and B, koff[e] = sum over e' < e of the rows of e'
-//     rounded up to 64 (zero columns pad each range):
-//       dW2_e  = d_out_e^T h_e       (A = d_out^T [d][K], B = h^T [m16][K])
-//       dW13_e = dGU_e^T x_e         (A = dGU^T [2 m16][K], B = x_perm^T [d][K])
-//     An expert with no rows gets a zero gradient.
-// Both operands are K-major bf16 loaded by TMA (128-byte swizzle, 128x64 and
-// 256x64 boxes, 4-stage ring); every K coordinate is a multiple of 64, so every
-// TMA x coordinate is 128-byte aligned.  f32 accumulators in TMEM, double
-// buffered; outputs rounded to bf16 once.
+//   row-grouped (dgrad): C[rows of expert e][N] = A[rows][K] B_e, the rows of expert
+//     e being [offsets[e], offsets[e+1]) -- the forward's tile order:
+//       dh      = d_out  W2_e        (B = the packed W2_e [d][m8], read MN-major)
+//       dGU     = SwiGLU backward of x_perm W13_e^T   (B K-major; fused epilogue, below)
+//       dx_perm = dGU    W13_e       (B = the packed W13_e [2 m16][d], read MN-major)
+//   K-grouped (wgrad): C_e[M][N] = A_e^T B_e, the reduction running over the rows
+//     [offsets[e], offsets[e+1]) of expert e of two row-major activations, both read
+//     MN-major (64-wide column chunks of 64 rows):
+//       dW2_e  = d_out_e^T h_e       (A = d_out [rows][d], B = h [rows][m8])
+//       dW13_e = dGU_e^T x_e         (A = dGU [rows][2 m16], B = x_perm [rows][d])
+//     The last K block of an expert also holds the first rows of the next expert:
+//     the MMA warp zeroes those K rows of both operands in shared memory before its
+//     MMAs.  An expert with no rows gets a zero gradient.
+// Operands bf16, loaded by TMA (128-byte swizzle, 4-stage ring); every TMA x
+// coordinate is a multiple of 64 elements (128-byte aligned).  f32 accumulators in
+// TMEM, double buffered; outputs rounded to bf16 once.
 //
 // SwiGLU backward epilogue: the accumulator tile is [g | u] of the packed W13
 // layout (per 32 columns: the gate values of 16 neurons, then their up values);
@@ -80,6 +80,8 @@ enum { EPI_STORE = 0, EPI_SWIGLU_BWD = 1 };
 struct Aux {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
+    uint64_t tbar[STAGES];  // K-grouped: the copies of an expert's last K block landed
+    uint64_t zbar[STAGES];  // K-grouped: the K rows past the expert zeroed
     uint64_t tfull[ACC];
     uint64_t tempty[ACC];
     uint64_t drain;
@@ -96,7 +98,9 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN 
 // the same with B MN-major (bit 16): the dgrad GEMMs read the expert weights as they
 // are packed, N contiguous, instead of a transposed copy
 constexpr uint32_t kIdescBt = kIdesc | (1u << 16);
-// MN-major B in shared memory: 64-wide N chunks of BK K rows (128 bytes each)
+// both operands MN-major (bits 15 and 16): the K-grouped wgrad
+constexpr uint32_t kIdescMn = kIdesc | (1u << 15) | (1u << 16);
+// MN-major operand in shared memory: 64-wide M or N chunks of BK K rows (128 bytes each)
 constexpr uint32_t kMnChunkBytes = BK * 128;
 // descriptor advance for 16 more K rows of an MN-major tile (2048 bytes, 16-byte units)
 constexpr int kMnKStep = 2048 >> 4;
@@ -216,10 +220,22 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
 
 struct Tile {
     int e, a_row, row0, row_end, n0, k0, nkb;
+    int kv;  // K-grouped: rows of the expert in its last K block (1..BK)
 };
 
-// KG = false: tiles of expert e are its row tiles x N tiles (forward order).
-// KG = true:  every expert has ceil(M / BM) x N tiles; K range from aux->off.
+// Zeroes K rows [r0, BK) of n MN-major chunks from chunk address base (each K row
+// 128 bytes, so the swizzle does not matter); lanes 1..31 of the calling warp.
+__device__ __forceinline__ void zero_k_rows(uint32_t base, int n, int r0)
+{
+    const int lane = threadIdx.x & 31;
+    const int per = (BK - r0) * 8;  // 16-byte units per chunk
+    for (int i = lane - 1; i < n * per; i += 31) {
+        const int c = i / per, rem = i - c * per;
+        st_shared_v4(base + (uint32_t)(c * kMnChunkBytes + (r0 + (rem >> 3)) * 128 + (rem & 7) * 16),
+                     0u, 0u, 0u, 0u);
+    }
+}
+
 template <bool KG>
 __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tiles, int M,
                                             int num_kb)
@@ -238,7 +254,9 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
         t.row_end = e * M + M;
         t.n0 = nt * BN;
         t.k0 = aux->off[e];
-        t.nkb = (aux->off[e + 1] - aux->off[e]) / BK;
+        const int rows = aux->off[e + 1] - aux->off[e];
+        t.nkb = (rows + BK - 1) / BK;
+        t.kv = rows - (t.nkb - 1) * BK;
     } else {
         const int rows = aux->off[e + 1] - aux->off[e];
         const int mtiles = (rows + BM - 1) / BM;
@@ -249,6 +267,7 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
         t.n0 = nt * BN;
         t.k0 = 0;
         t.nkb = num_kb;
+        t.kv = BK;
     }
     return t;
 }
@@ -273,6 +292,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&aux->full[s]), 1);
             mbar_init(smem_u32(&aux->empty[s]), 1);
+            mbar_init(smem_u32(&aux->tbar[s]), 1);
+            mbar_init(smem_u32(&aux->zbar[s]), 1);
         }
         for (int a = 0; a < ACC; ++a) {
             mbar_init(smem_u32(&aux->tfull[a]), 1);
@@ -287,21 +308,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     const int n_tiles = (N + BN - 1) / BN;
     if (warp == 2 && lane == 0) {
-        // row offsets; in the K-grouped order their rounded-up prefix sums
-        int acc = 0, kacc = 0;
+        // row offsets: the row tiles of the dgrad order, the K ranges of the wgrad order
+        int acc = 0;
         for (int e = 0; e < E; ++e) {
             const int rows = offsets[e + 1] - offsets[e];
             aux->tstart[e] = acc;
-            if constexpr (KG) {
-                aux->off[e] = kacc;
-                kacc += (rows + BK - 1) / BK * BK;
-                acc += (M + BM - 1) / BM * n_tiles;
-            } else {
-                aux->off[e] = offsets[e];
-                acc += (rows + BM - 1) / BM * n_tiles;
-            }
+            aux->off[e] = offsets[e];
+            acc += KG ? (M + BM - 1) / BM * n_tiles : (rows + BM - 1) / BM * n_tiles;
         }
-        aux->off[E] = KG ? kacc : offsets[E];
+        aux->off[E] = offsets[E];
         aux->tstart[E] = acc;
     }
     if (warp == 1) {
@@ -325,6 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int64_t fills = 0;
+            int tfills[STAGES] = {};
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 if (*abort_flag)
@@ -336,19 +352,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = smem_u32(&aux->full[stage]);
+                    uint32_t fb = smem_u32(&aux->full[stage]);
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    mbar_expect_tx(fb, STAGE_BYTES);
                     const int kc = t.k0 + kb * BK;
-                    tma_load_2d(&tmA, fb, sa, kc, t.a_row);
-                    if constexpr (BT) {  // MN-major B: 64-wide N chunks of BK K rows
+                    if constexpr (KG) {  // both MN-major: 64-wide chunks of BK rows from row kc
+                        if (kb == t.nkb - 1 && t.kv < BK) {
+                            // an expert's last block: its copies complete on tbar, for lanes
+                            // 1-31 to zero the rows past the expert; full completes now
+                            mbar_arrive(fb);
+                            fb = smem_u32(&aux->tbar[stage]);
+                            ++tfills[stage];
+                        }
+                        mbar_expect_tx(fb, STAGE_BYTES);
+#pragma unroll
+                        for (int j = 0; j < BM / 64; ++j)
+                            tma_load_2d(&tmA, fb, sa + j * kMnChunkBytes, t.a_row + 64 * j, kc);
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(&tmB, fb, sa + A_BYTES + j * kMnChunkBytes, t.n0 + 64 * j,
+                                        kc);
+                    } else if constexpr (BT) {  // MN-major B: 64-wide N chunks of BK K rows
+                        mbar_expect_tx(fb, STAGE_BYTES);
+                        tma_load_2d(&tmA, fb, sa, kc, t.a_row);
 #pragma unroll
                         for (int j = 0; j < BN / 64; ++j)
                             tma_load_3d(&tmB, fb, sa + A_BYTES + j * kMnChunkBytes, t.n0 + 64 * j,
                                         kc, t.e);
-                    } else if constexpr (KG) {
-                        tma_load_2d(&tmB, fb, sa + A_BYTES, kc, t.n0);
                     } else {
+                        mbar_expect_tx(fb, STAGE_BYTES);
+                        tma_load_2d(&tmA, fb, sa, kc, t.a_row);
                         tma_load_3d(&tmB, fb, sa + A_BYTES, kc, t.n0, t.e);
                     }
                     ++fills;
@@ -362,6 +394,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
                 if (n > 0)
                     mbar_drain(smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
+                if (tfills[s] > 0)
+                    mbar_drain(smem_u32(&aux->tbar[s]), (uint32_t)((tfills[s] - 1) & 1));
+            }
+        } else if constexpr (KG) {
+            // ------------------------------------------- lanes 1-31: tail zeroing
+            // Once an expert's last K block has landed, zero its K rows past the
+            // expert in both operands (they hold the next expert's rows) and arrive
+            // on zbar, which the MMA issuer waits for.  Lane 1 waits; the other lanes
+            // follow its verdict, so the 31 lanes stay converged.
+            int stage = 0;
+            uint32_t tpar = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb);
+                if (t.nkb > 0 && t.kv < BK) {
+                    const int ts = (stage + t.nkb - 1) % STAGES;
+                    bool ok = true;
+                    if (lane == 1)
+                        ok = mbar_wait(smem_u32(&aux->tbar[ts]), (tpar >> ts) & 1u, wait_ns,
+                                       abort_flag, status);
+                    if (!__shfl_sync(0xfffffffeu, ok ? 1 : 0, 1))
+                        break;
+                    tpar ^= 1u << ts;
+                    const uint32_t sa = smem_base + ts * STAGE_BYTES;
+                    zero_k_rows(sa, BM / 64, t.kv);
+                    zero_k_rows(sa + A_BYTES, BN / 64, t.kv);
+                    fence_proxy_async_smem();
+                    __syncwarp(0xfffffffeu);
+                    if (lane == 1)
+                        mbar_arrive(smem_u32(&aux->zbar[ts]));
+                }
+                stage = (stage + t.nkb) % STAGES;
             }
         }
     } else if (warp == 1) {
@@ -369,6 +432,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // ---------------------------------------------------------- MMA issuer
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t tpar = 0;  // K-grouped: phase parity of each stage's zbar
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
@@ -387,16 +451,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if (KG && kb == t.nkb - 1 && t.kv < BK) {  // the K rows past the expert zeroed
+                        if (!mbar_wait(smem_u32(&aux->zbar[stage]), (tpar >> stage) & 1u, wait_ns,
+                                       abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tpar ^= 1u << stage;
+                    }
                     tc_fence_after();
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    const uint64_t da = sdesc(sa);
-                    const uint64_t db = BT ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
-                                           : sdesc(sa + A_BYTES);
+                    const uint64_t da = KG ? tc::sdesc_mn(sa, kMnChunkBytes) : sdesc(sa);
+                    const uint64_t db = (KG || BT) ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
+                                                   : sdesc(sa + A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_f16(d_tmem, da + (uint64_t)(2 * k),
-                                 db + (uint64_t)(BT ? kMnKStep * k : 2 * k),
-                                 BT ? kIdescBt : kIdesc, (kb | k) != 0);
+                        umma_f16(d_tmem, da + (uint64_t)(KG ? kMnKStep * k : 2 * k),
+                                 db + (uint64_t)((KG || BT) ? kMnKStep * k : 2 * k),
+                                 KG ? kIdescMn : (BT ? kIdescBt : kIdesc), (kb | k) != 0);
                     umma_commit(smem_u32(&aux->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -475,6 +547,8 @@ constexpr uint64_t kAbortSettleNs = 200000ull;
 struct Aux {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
+    uint64_t tbar[STAGES];  // K-grouped: the copies of an expert's last K block landed
+    uint64_t zbar[STAGES];  // K-grouped: the K rows past the expert zeroed
     uint64_t tfull[ACC];
     uint64_t tempty[ACC];
     uint64_t drain;
@@ -580,7 +654,9 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
         t.row_end = e * M + M;
         t.n0 = nt * BN;
         t.k0 = aux->off[e];
-        t.nkb = (aux->off[e + 1] - aux->off[e]) / BK;
+        const int rows = aux->off[e + 1] - aux->off[e];
+        t.nkb = (rows + BK - 1) / BK;
+        t.kv = rows - (t.nkb - 1) * BK;
     } else {
         const int rows = aux->off[e + 1] - aux->off[e];
         const int mtiles = (rows + 2 * BM - 1) / (2 * BM);
@@ -591,6 +667,7 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
         t.n0 = nt * BN;
         t.k0 = 0;
         t.nkb = num_kb;
+        t.kv = BK;
     }
     return t;
 }
@@ -620,6 +697,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&aux->full[s]), 1);
             mbar_init(smem_u32(&aux->empty[s]), 1);
+            mbar_init(smem_u32(&aux->tbar[s]), 1);
+            mbar_init(smem_u32(&aux->zbar[s]), 2);  // one arrival from each CTA
         }
         for (int a = 0; a < ACC; ++a) {
             mbar_init(smem_u32(&aux->tfull[a]), 1);
@@ -634,20 +713,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     const int n_tiles = (N + BN - 1) / BN;
     if (warp == 2 && lane == 0) {
-        int acc = 0, kacc = 0;
+        int acc = 0;
         for (int e = 0; e < E; ++e) {
             const int rows = offsets[e + 1] - offsets[e];
             aux->tstart[e] = acc;
-            if constexpr (KG) {
-                aux->off[e] = kacc;
-                kacc += (rows + BK - 1) / BK * BK;
-                acc += (M + 2 * BM - 1) / (2 * BM) * n_tiles;
-            } else {
-                aux->off[e] = offsets[e];
-                acc += (rows + 2 * BM - 1) / (2 * BM) * n_tiles;
-            }
+            aux->off[e] = offsets[e];
+            acc += KG ? (M + 2 * BM - 1) / (2 * BM) * n_tiles
+                      : (rows + 2 * BM - 1) / (2 * BM) * n_tiles;
         }
-        aux->off[E] = KG ? kacc : offsets[E];
+        aux->off[E] = offsets[E];
         aux->tstart[E] = acc;
     }
     if (warp == 1) {
@@ -671,6 +745,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int64_t fills = 0;
+            int tfills[STAGES] = {};
             bool ok = true;
             for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
                 if (*abort_flag)
@@ -683,20 +758,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     const uint32_t fb = smem_u32(&aux->full[stage]);
-                    if (leader)
-                        mbar_expect_tx(fb, 2 * STAGE_BYTES);
                     const uint32_t fb0 = map_rank(fb, 0);
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
                     const int kc = t.k0 + kb * BK;
-                    tma_load_2d_pair(&tmA, fb0, sa, kc, t.a_row + (int)rank * BM);
-                    if constexpr (BT) {  // MN-major B: this CTA's 64-wide N chunks
+                    if (KG && kb == t.nkb - 1 && t.kv < BK) {
+                        // an expert's last block: each CTA's copies complete on its own
+                        // tbar, for its lanes 1-31 to zero the rows past the expert; the
+                        // leader's full completes now
+                        if (leader)
+                            mbar_arrive(fb);
+                        const uint32_t tb = smem_u32(&aux->tbar[stage]);
+                        ++tfills[stage];
+                        mbar_expect_tx(tb, STAGE_BYTES);
+#pragma unroll
+                        for (int j = 0; j < BM / 64; ++j)
+                            tma_load_2d(&tmA, tb, sa + j * kMnChunkBytes,
+                                        t.a_row + (int)rank * BM + 64 * j, kc);
+#pragma unroll
+                        for (int j = 0; j < BNH / 64; ++j)
+                            tma_load_2d(&tmB, tb, sa + A_BYTES + j * kMnChunkBytes,
+                                        t.n0 + (int)rank * BNH + 64 * j, kc);
+                    } else if constexpr (KG) {  // both MN-major: this CTA's 64-wide chunks
+                        if (leader)
+                            mbar_expect_tx(fb, 2 * STAGE_BYTES);
+#pragma unroll
+                        for (int j = 0; j < BM / 64; ++j)
+                            tma_load_2d_pair(&tmA, fb0, sa + j * kMnChunkBytes,
+                                             t.a_row + (int)rank * BM + 64 * j, kc);
+#pragma unroll
+                        for (int j = 0; j < BNH / 64; ++j)
+                            tma_load_2d_pair(&tmB, fb0, sa + A_BYTES + j * kMnChunkBytes,
+                                             t.n0 + (int)rank * BNH + 64 * j, kc);
+                    } else if constexpr (BT) {
+                        if (leader)
+                            mbar_expect_tx(fb, 2 * STAGE_BYTES);  // MN-major B: this CTA's 64-wide N chunks
+                        tma_load_2d_pair(&tmA, fb0, sa, kc, t.a_row + (int)rank * BM);
 #pragma unroll
                         for (int j = 0; j < BNH / 64; ++j)
                             tma_load_3d_pair(&tmB, fb0, sa + A_BYTES + j * kMnChunkBytes,
                                              t.n0 + (int)rank * BNH + 64 * j, kc, t.e);
-                    } else if constexpr (KG) {
-                        tma_load_2d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH);
                     } else {
+                        if (leader)
+                            mbar_expect_tx(fb, 2 * STAGE_BYTES);
+                        tma_load_2d_pair(&tmA, fb0, sa, kc, t.a_row + (int)rank * BM);
                         tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, kc, t.n0 + (int)rank * BNH,
                                          t.e);
                     }
@@ -714,12 +818,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         mbar_drain(smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
                 }
             }
+            for (int s = 0; s < STAGES; ++s)
+                if (tfills[s] > 0)
+                    mbar_drain(smem_u32(&aux->tbar[s]), (uint32_t)((tfills[s] - 1) & 1));
+        } else if constexpr (KG) {
+            // ------------------------------------------- lanes 1-31: tail zeroing
+            // As in the 1-SM kernel, in this CTA's tiles; the arrival goes to the
+            // leader's zbar (count 2, one per CTA).
+            int stage = 0;
+            uint32_t tpar = 0;
+            for (int tile = cluster_id; tile < total; tile += nclusters) {
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb);
+                if (t.nkb > 0 && t.kv < BK) {
+                    const int ts = (stage + t.nkb - 1) % STAGES;
+                    bool ok = true;
+                    if (lane == 1)
+                        ok = mbar_wait(smem_u32(&aux->tbar[ts]), (tpar >> ts) & 1u, wait_ns,
+                                       abort_flag, status);
+                    if (!__shfl_sync(0xfffffffeu, ok ? 1 : 0, 1))
+                        break;
+                    tpar ^= 1u << ts;
+                    const uint32_t sa = smem_base + ts * STAGE_BYTES;
+                    zero_k_rows(sa, BM / 64, t.kv);
+                    zero_k_rows(sa + A_BYTES, BNH / 64, t.kv);
+                    fence_proxy_async_smem();
+                    __syncwarp(0xfffffffeu);
+                    if (lane == 1)
+                        mbar_arrive_cluster(map_rank(smem_u32(&aux->zbar[ts]), 0));
+                }
+                stage = (stage + t.nkb) % STAGES;
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ------------------------------------------------------- MMA issuer (leader)
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t tpar = 0;  // K-grouped: phase parity of each stage's zbar
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
@@ -738,16 +873,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
+                    if (KG && kb == t.nkb - 1 && t.kv < BK) {  // both CTAs' tails zeroed
+                        if (!mbar_wait(smem_u32(&aux->zbar[stage]), (tpar >> stage) & 1u, wait_ns,
+                                       abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tpar ^= 1u << stage;
+                    }
                     tc_fence_after();
                     const uint32_t sa = smem_base + stage * STAGE_BYTES;
-                    const uint64_t da = sdesc(sa);
-                    const uint64_t db = BT ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
-                                           : sdesc(sa + A_BYTES);
+                    const uint64_t da = KG ? tc::sdesc_mn(sa, kMnChunkBytes) : sdesc(sa);
+                    const uint64_t db = (KG || BT) ? tc::sdesc_mn(sa + A_BYTES, kMnChunkBytes)
+                                                   : sdesc(sa + A_BYTES);
+                    const uint32_t idesc = KG ? kIdesc2 | (1u << 15) | (1u << 16)
+                                              : (BT ? kIdesc2 | (1u << 16) : kIdesc2);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_pair(d_tmem, da + (uint64_t)(2 * k),
-                                  db + (uint64_t)(BT ? kMnKStep * k : 2 * k),
-                                  BT ? kIdesc2 | (1u << 16) : kIdesc2, (kb | k) != 0);
+                        umma_pair(d_tmem, da + (uint64_t)(KG ? kMnKStep * k : 2 * k),
+                                  db + (uint64_t)((KG || BT) ? kMnKStep * k : 2 * k), idesc,
+                                  (kb | k) != 0);
                     umma_commit_both(smem_u32(&aux->empty[stage]));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -815,96 +960,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 }  // namespace pair
-
-// ------------------------------------------------------------------------ transposes
-// Both transposes move 8 x 8 bf16 blocks through registers: a thread loads 8 rows
-// of 8 columns (8 x 16 bytes), transposes them with byte permutes and stores 8
-// rows of 8 columns.  Lane l of a warp takes row group l % 8 and column group
-// l / 8 (+ 4 per warp), so a warp reads 8 rows x 64 bytes and writes 4 rows x
-// 128 bytes per instruction; a CTA (8 warps) covers 64 rows x 256 columns.
-
-// out[c] = column c of the 8 x 8 block whose rows are in[0..7].
-__device__ __forceinline__ void transpose8x8(const uint4 (&in)[8], uint4 (&out)[8])
-{
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t *a = reinterpret_cast<const uint32_t *>(&in[2 * q]);
-            const uint32_t *b = reinterpret_cast<const uint32_t *>(&in[2 * q + 1]);
-            w[q] = __byte_perm(a[c >> 1], b[c >> 1], sel);
-        }
-        out[c] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-// Zeroes the elements of v at columns >= limit, v holding columns col .. col+7.
-__device__ __forceinline__ uint4 mask_cols(uint4 v, int col, int limit)
-{
-    if (col + 8 <= limit)
-        return v;
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (col + i >= limit)
-            w[i >> 1] &= (i & 1) ? 0x0000ffffu : 0xffff0000u;
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Row-segment transpose for the K-grouped GEMMs: src [rows][ld_src] (columns
-// [0, c_valid) meaningful, ld_src >= c_valid rounded up to 8), rows grouped by
-// expert through offsets; dst [c_pad][ld_dst] with dst[c][koff[e] + j] =
-// src[offsets[e] + j][c] for j < rows_e, zero for j in [rows_e, round_up(rows_e, 64))
-// and for c in [c_valid, c_pad).  CTA = 64 padded columns of dst (64 consecutive
-// rows of one expert) x 256 rows of dst.
-__global__ void __launch_bounds__(256) transpose_rows_kernel(
-    const bf16 *__restrict__ src, int ld_src, const int32_t *__restrict__ offsets, int E,
-    int c_valid, int c_pad, bf16 *__restrict__ dst, int ld_dst)
-{
-    pdl_wait();
-    pdl_trigger();
-    __shared__ int32_t s_koff[MOE_MAX_EXPERTS + 1];
-    if (threadIdx.x == 0) {
-        int k = 0;
-        for (int e = 0; e < E; ++e) {
-            s_koff[e] = k;
-            k += (offsets[e + 1] - offsets[e] + 63) / 64 * 64;
-        }
-        s_koff[E] = k;
-    }
-    __syncthreads();
-    const int kc0 = blockIdx.x * 64;   // padded column of dst
-    const int c0 = blockIdx.y * 256;   // first dst row (src column)
-    if (kc0 >= s_koff[E])
-        return;
-    int e = 0;
-    while (kc0 >= s_koff[e + 1])
-        ++e;
-    const int rows = offsets[e + 1] - offsets[e];
-    const int j0 = kc0 - s_koff[e];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int rg = lane & 7, cq = (lane >> 3) + 4 * warp;
-    const int col = c0 + 8 * cq;
-    if (col >= c_pad)
-        return;
-    uint4 in[8], out[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int j = j0 + 8 * rg + i;
-        in[i] = make_uint4(0, 0, 0, 0);
-        if (j < rows && col < c_valid)
-            in[i] = mask_cols(*reinterpret_cast<const uint4 *>(
-                                  src + (int64_t)(offsets[e] + j) * ld_src + col),
-                              col, c_valid);
-    }
-    transpose8x8(in, out);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (col + i < c_pad)
-            *reinterpret_cast<uint4 *>(dst + (int64_t)(col + i) * ld_dst + kc0 + 8 * rg) = out[i];
-}
 
 // ------------------------------------------------------------------------ host side
 
@@ -978,9 +1033,11 @@ static cudaError_t prepare(DevInfo **out)
 // Rows (T*k) from which the 2-SM kernels are used, as in the forward.
 constexpr int64_t kPairMinRows = 4096;
 
-// One backward GEMM.  A [a_rows][a_ld] (K extent a_k); B: row-grouped [E][b_rows][b_ld],
-// K-grouped [b_rows][b_ld] (K extent b_k); with BT (MN-major B) [E][b_k][b_ld] with N
-// extent b_rows; out [out_rows][ld_out], n_valid columns.
+// One backward GEMM; out [out_rows][ld_out], n_valid columns.
+//   row-grouped: A [a_rows][a_ld] (K extent a_k); B [E][b_rows][b_ld] (K extent b_k),
+//     with BT (MN-major B) [E][b_k][b_ld] with N extent b_rows.
+//   K-grouped: A [a_rows][a_ld] with M extent a_k, B [a_rows][b_ld] with N extent
+//     b_rows (rows = the experts' rows, the K of the reduction; b_k unused).
 template <int EPI, bool KG, bool BT>
 static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a_rows,
                           const void *B, uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
@@ -994,21 +1051,23 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
         return e;
     CUtensorMap ta, tb, to;
     const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
-    const uint32_t ba[2] = {BK, BM};
+    const uint32_t ba[2] = {KG ? 64u : (uint32_t)BK, KG ? (uint32_t)BK : (uint32_t)BM};
     const uint32_t b_box = use_pair ? (uint32_t)pair::BNH : (uint32_t)BN;
     if ((e = tc::make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
         return e;
-    if constexpr (BT) {
+    if constexpr (KG) {
+        // MN-major boxes of 64 columns x BK rows; columns and rows past the extents
+        // read as zero
+        const uint64_t db[2] = {b_rows, a_rows}, sb[1] = {b_ld * 2};
+        const uint32_t bb[2] = {64, BK};
+        if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
+            return e;
+    } else if constexpr (BT) {
         // N innermost: boxes of 64 N x BK K rows, N and K past their extents read as zero
         const uint64_t db[3] = {b_rows, b_k, (uint64_t)E};
         const uint64_t sb[2] = {b_ld * 2, b_k * b_ld * 2};
         const uint32_t bb[3] = {64, BK, 1};
         if ((e = tc::make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
-            return e;
-    } else if constexpr (KG) {
-        const uint64_t db[2] = {b_k, b_rows}, sb[1] = {b_ld * 2};
-        const uint32_t bb[2] = {BK, b_box};
-        if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
             return e;
     } else {
         const uint64_t db[3] = {b_k, b_rows, (uint64_t)E};
@@ -1085,26 +1144,18 @@ cudaError_t launch_bwd_dx(const moe_params_t *p, const void *dgu, const int32_t 
                                           nullptr, 0, status, s, (int64_t)rows >= kPairMinRows);
 }
 
-// dW [E][M][n_valid]: A^T [M][kmax] and B^T [b_rows][kmax] in the padded K order
-cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *AT, int M, const void *BT,
-                             int b_rows, uint64_t kmax, const int32_t *offsets, void *dW,
-                             int ld_dw, int n_valid, int32_t *status, cudaStream_t s)
+// dW [E][M][n_valid] (ld_dw): dW_e = A_e^T B_e over the rows of expert e, A [rows][a_ld]
+// with M columns, B [rows][b_ld] with n_cols columns (N extent; columns up to the next
+// multiple of 256 read as zero)
+cudaError_t launch_bwd_wgrad(const moe_params_t *p, const void *A, int M, int a_ld, const void *B,
+                             int n_cols, int b_ld, const int32_t *offsets, void *dW, int ld_dw,
+                             int n_valid, int32_t *status, cudaStream_t s)
 {
-    return launch<EPI_STORE, true, false>(AT, kmax, kmax, (uint64_t)M, BT, kmax, kmax, (uint64_t)b_rows,
-                                   offsets, p->E, M, (bf16 *)dW, ld_dw, (uint64_t)p->E * M,
-                                   n_valid, nullptr, 0, status, s,
-                                   (int64_t)p->T * p->k >= kPairMinRows);
+    const uint64_t rows = (uint64_t)p->T * p->k;
+    return launch<EPI_STORE, true, false>(A, (uint64_t)M, (uint64_t)a_ld, rows, B, 0,
+                                          (uint64_t)b_ld, (uint64_t)n_cols, offsets, p->E, M,
+                                          (bf16 *)dW, ld_dw, (uint64_t)p->E * M, n_valid, nullptr,
+                                          0, status, s, (int64_t)rows >= kPairMinRows);
 }
-
-cudaError_t launch_transpose_rows(const void *src, int ld_src, const int32_t *offsets, int E,
-                                  int c_valid, int c_pad, void *dst, int ld_dst, int64_t kmax,
-                                  cudaStream_t s)
-{
-    count_launch();
-    return launch_pdl(transpose_rows_kernel, dim3((unsigned)(kmax / 64), (c_pad + 255) / 256),
-                      dim3(256), 0, s, (const bf16 *)src, ld_src, offsets, E, c_valid, c_pad,
-                      (bf16 *)dst, ld_dst);
-}
-
 
 }  // namespace moe
