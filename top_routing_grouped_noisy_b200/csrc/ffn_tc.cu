@@ -40,6 +40,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle-128B row
 constexpr int STAGES = 4;
+constexpr int kMaxStages = 5;  // the 160-wide tiles leave room for a fifth stage
 constexpr int ACC = 2;
 constexpr int TMEM_COLS = ACC * BN;  // 512
 constexpr int A_BYTES = BM * BK * 2;
@@ -52,8 +53,8 @@ constexpr int EPI_WARPS = 8;
 enum { EPI_SWIGLU = 0, EPI_STORE = 1 };
 
 struct Aux {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[ACC];
     uint64_t tempty[ACC];
     uint64_t drain;
@@ -64,14 +65,26 @@ struct Aux {
 };
 constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux);
 
-// kind::f16 instruction descriptor: D f32, A and B bf16, both K-major, N = BN, M = BM.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// kind::f16 instruction descriptors (D f32, A and B bf16, both K-major, M = BM) are
+// per tile width: Geo<BNT>::IDESC.
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc)
-{
-    umma_f16(d_tmem, a, b, kIdesc, acc);
-}
+// Geometry of a 1-SM kernel instance with tiles BNT columns wide: 256, or 160 when
+// the narrower tile puts every tile of a small batch on an SM of its own (a batch of
+// at most 128 rows per expert has one row tile per expert, E x ceil(N / BNT) tiles).
+// The accumulators keep the 256-column TMEM stride.
+template <int BNT>
+struct Geo {
+    static constexpr int B_BYTES = BNT * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int NSTAGES = BNT == BN ? STAGES : kMaxStages;
+    static constexpr int TILE_BYTES = NSTAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux);
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                      ((uint32_t)(BNT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static_assert(BNT % 32 == 0 && BNT <= BN && STAGE_BYTES % 1024 == 0, "tile width");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+constexpr int kNarrowBN = 160;
 
 // Output staging: each epilogue warp owns two 2 KB shared-memory slots, each one
 // [32 rows][64 bytes] box laid out with the 64-byte swizzle (16-byte chunk j of row
@@ -129,6 +142,47 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
 #pragma unroll 1
     for (int c = c_first; c < c_first + n_chunks; c += 2) {
         uint32_t v[2][32];
+        if (c + 1 == c_first + n_chunks) {
+            // an odd last chunk (160-column tiles): 32 columns, stored per lane
+            tmem_ld32_async(taddr + (uint32_t)(c * 32), v[0]);
+            tmem_wait_ld();
+            if constexpr (EPI == EPI_SWIGLU) {
+                const int nb = n0 / 2 + c * 16;  // 16 neurons
+                float hv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float g = __uint_as_float(v[0][i]);
+                    const float u = __uint_as_float(v[0][16 + i]);
+                    hv[i] = g / (1.0f + __expf(-g)) * u;
+                }
+                if (rv && nb < n_valid) {
+                    bf16 *dst = out + (int64_t)row * ld_out + nb;
+                    if (nb + 16 <= n_valid) {
+                        st_v4(dst, f32x8_to_bf16(hv));
+                        st_v4(dst + 8, f32x8_to_bf16(hv + 8));
+                    } else {
+                        for (int i = 0; i < 16 && nb + i < n_valid; ++i)
+                            dst[i] = __float2bfloat16_rn(hv[i]);
+                    }
+                }
+            } else {
+                const int col = n0 + c * 32;
+                if (rv) {
+                    bf16 *dst = out + (int64_t)row * ld_out + col;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        if (col + q * 8 < n_valid) {
+                            float f[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                f[i] = __uint_as_float(v[0][q * 8 + i]);
+                            st_v4(dst + q * 8, f32x8_to_bf16(f));
+                        }
+                    }
+                }
+            }
+            break;
+        }
         tmem_ld32_async(taddr + (uint32_t)(c * 32), v[0]);
         tmem_ld32_async(taddr + (uint32_t)((c + 1) * 32), v[1]);
         tmem_wait_ld();
@@ -193,6 +247,7 @@ struct Tile {
     int e, row0, row_end, n0;
 };
 
+template <int BNT>
 __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tiles)
 {
     Tile t;
@@ -207,14 +262,14 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     t.e = e;
     t.row0 = aux->off[e] + mt * BM;
     t.row_end = aux->off[e + 1];
-    t.n0 = nt * BN;
+    t.n0 = nt * BNT;
     return t;
 }
 
 // GATHER: tmA covers the unpermuted activations x [T][K] with a box one row high;
 // the A rows of a tile are gathered through row_token (4 rows per TMA, one TMA
 // per producer lane) instead of being read from a permuted copy.
-template <int EPI, bool GATHER>
+template <int EPI, bool GATHER, int BNT = BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -228,12 +283,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Aux *aux = reinterpret_cast<Aux *>(smem + TILE_BYTES + kEpiStageBytes);
+    Aux *aux = reinterpret_cast<Aux *>(smem + Geo<BNT>::TILE_BYTES + kEpiStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int32_t *abort_flag = &aux->abort_flag;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < Geo<BNT>::NSTAGES; ++s) {
             mbar_init(smem_u32(&aux->full[s]), 1);
             mbar_init(smem_u32(&aux->empty[s]), 1);
         }
@@ -248,7 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
     }
-    const int n_tiles = (N + BN - 1) / BN;
+    const int n_tiles = (N + BNT - 1) / BNT;
     if (warp == 2) {
         for (int i = lane; i <= E; i += 32)
             aux->off[i] = offsets[i];
@@ -288,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             if (__shfl_sync(0xffffffffu, (int)*abort_flag, 0))
                 break;
-            const Tile t = decode_tile(aux, tile, n_tiles);
+            const Tile t = decode_tile<BNT>(aux, tile, n_tiles);
             int src[4] = {0, 0, 0, 0};
             if constexpr (GATHER) {
 #pragma unroll
@@ -308,9 +363,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 const uint32_t fb = smem_u32(&aux->full[stage]);
-                const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                const uint32_t sa = smem_base + stage * Geo<BNT>::STAGE_BYTES;
                 if (lane == 0)
-                    mbar_expect_tx(fb, STAGE_BYTES);
+                    mbar_expect_tx(fb, Geo<BNT>::STAGE_BYTES);
                 __syncwarp();
                 if constexpr (GATHER)
                     tma_gather4(&tmA, fb, sa + lane * 4 * 128, kb * BK, src[0], src[1], src[2],
@@ -320,7 +375,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (lane == 0)
                     tma_load_3d(&tmB, fb, sa + A_BYTES, kb * BK, t.n0, t.e);
                 ++fills;
-                if (++stage == STAGES) {
+                if (++stage == Geo<BNT>::NSTAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -330,8 +385,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // drain: the last fill of every stage has landed before the CTA may exit
         if (lane == 0) {
-            for (int s = 0; s < STAGES; ++s) {
-                const int64_t n = fills / STAGES + (s < fills % STAGES ? 1 : 0);
+            for (int s = 0; s < Geo<BNT>::NSTAGES; ++s) {
+                const int64_t n = fills / Geo<BNT>::NSTAGES + (s < fills % Geo<BNT>::NSTAGES ? 1 : 0);
                 if (n > 0)
                     mbar_drain(smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
             }
@@ -359,14 +414,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_base + stage * STAGE_BYTES;
+                    const uint32_t sa = smem_base + stage * Geo<BNT>::STAGE_BYTES;
                     const uint64_t da = sdesc(sa), db = sdesc(sa + A_BYTES);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)  // +32 bytes (16 bf16) per step
-                        umma_bf16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
-                                  (kb | k) != 0);
+                        umma_f16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
+                                 Geo<BNT>::IDESC, (kb | k) != 0);
                     umma_commit(smem_u32(&aux->empty[stage]));
-                    if (++stage == STAGES) {
+                    if (++stage == Geo<BNT>::NSTAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -385,21 +440,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue
-        // warp w reads TMEM lanes 32*(w%4)..+31 (tile rows); warps 2-5 take columns
-        // 0..127 of the accumulator, warps 6-9 columns 128..255
+        // warp w reads TMEM lanes 32*(w%4)..+31 (tile rows); warps 2-5 take the first
+        // half of the accumulator's 32-column chunks (the larger half of an odd
+        // count), warps 6-9 the rest
         const int wq = warp & 3;
         const int lane_base = wq * 32;
-        const int c_first = ((warp - 2) / 4) * (BN / 64);
-        EpiStore st{&tmO, smem_base + TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
+        constexpr int kChunks = BNT / 32, kHalf0 = (kChunks + 1) / 2;
+        const bool upper = (warp - 2) / 4 != 0;
+        const int c_first = upper ? kHalf0 : 0, n_chunks = upper ? kChunks - kHalf0 : kHalf0;
+        EpiStore st{&tmO, smem_base + Geo<BNT>::TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile(aux, tile, n_tiles);
+            const Tile t = decode_tile<BNT>(aux, tile, n_tiles);
             if (!mbar_wait(smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag, status))
                 break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-            epilogue_slab<EPI>(taddr, c_first, BN / 64, t.row0 + lane_base, t.row_end, t.n0, out,
+            epilogue_slab<EPI>(taddr, c_first, n_chunks, t.row0 + lane_base, t.row_end, t.n0, out,
                                ld_out, n_valid, st);
             tc_fence_before();
             __syncwarp();
@@ -829,7 +887,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 struct DevInfo {
     int sms = 0;
     int pair_clusters = 0;
-    bool attr[8] = {false, false, false, false, false, false, false, false};
+    bool attr[10] = {false, false, false, false, false, false, false, false, false, false};
 };
 static std::mutex g_dev_mu;
 static DevInfo g_dev[64];
@@ -877,7 +935,11 @@ static cudaError_t prepare_device(DevInfo **out)
         (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_SWIGLU, true>, tc2::SMEM_BYTES,
                            di.attr[6])) != cudaSuccess ||
         (e = set_smem_attr(tc2::grouped_gemm_2sm_kernel<EPI_STORE, true>, tc2::SMEM_BYTES,
-                           di.attr[7])) != cudaSuccess)
+                           di.attr[7])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, false, kNarrowBN>,
+                           Geo<kNarrowBN>::SMEM_BYTES, di.attr[8])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, false, kNarrowBN>,
+                           Geo<kNarrowBN>::SMEM_BYTES, di.attr[9])) != cudaSuccess)
         return e;
     if (di.pair_clusters == 0) {
         cudaLaunchConfig_t cfg = {};
@@ -909,10 +971,11 @@ constexpr int64_t kPairMinRows = 4096;
 // One grouped GEMM launch.  A: [a_rows][a_ld] activations (K extent a_k), read in
 // expert-grouped row order, or -- when row_token is given -- gathered: tile row r is
 // row row_token[r] of A; B: [E][b_rows][b_ld] expert weights (K extent b_k, N =
-// b_rows); out: [rows][ld_out], first n_valid columns written; rows = T*k.
+// b_rows); out: [rows][ld_out], first n_valid columns written; rows = T*k, k_rows = k
+// (an expert has at most rows / k_rows rows).
 template <int EPI>
 static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a_rows,
-                               const int32_t *row_token, uint64_t rows, const void *B,
+                               const int32_t *row_token, uint64_t rows, int k_rows, const void *B,
                                uint64_t b_k, uint64_t b_ld, uint64_t b_rows,
                                const int32_t *offsets, int E, bf16 *out, int ld_out, int n_valid,
                                int32_t *status, cudaStream_t s)
@@ -925,10 +988,17 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     const bool gather = row_token != nullptr;
     CUtensorMap ta, tb;
     const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
-    const uint32_t ba[2] = {BK, gather ? 1u : (uint32_t)BM};  // gather4 boxes are one row high
     const uint64_t db[3] = {b_k, b_rows, (uint64_t)E};
     const uint64_t sb[2] = {b_ld * 2, b_rows * b_ld * 2};
-    const uint32_t bb[3] = {BK, pair ? (uint32_t)tc2::BNH : (uint32_t)BN, 1};
+    // 1-SM tiles 160 wide instead of 256 when every expert has at most 128 rows (T <=
+    // 128, one row tile each) and the narrower tiles still fit one wave of the SMs
+    const int64_t T = (int64_t)rows / (k_rows > 0 ? k_rows : 1);
+    const int64_t n_wide = (int64_t)E * (((int64_t)b_rows + BN - 1) / BN);
+    const int64_t n_narrow = (int64_t)E * (((int64_t)b_rows + kNarrowBN - 1) / kNarrowBN);
+    const bool narrow = !pair && !gather && T <= BM && n_wide < di->sms && n_narrow <= di->sms;
+    const uint32_t ba[2] = {BK, gather ? 1u : (uint32_t)BM};  // gather4 boxes are one row high
+    const uint32_t bb[3] = {BK, pair ? (uint32_t)tc2::BNH : (uint32_t)(narrow ? kNarrowBN : BN),
+                            1};
     if ((e = make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
         return e;
     if ((e = make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
@@ -941,6 +1011,12 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
         return e;
     const uint64_t wait_ns = wait_limit_ns();
     const int N = (int)b_rows, K = (int)a_k;
+    if (narrow) {
+        launch_pdl(grouped_gemm_kernel<EPI, false, kNarrowBN>, dim3(di->sms), dim3(NUM_THREADS),
+                   Geo<kNarrowBN>::SMEM_BYTES, s, ta, tb, to, offsets, E, N, K, out, ld_out,
+                   n_valid, status, wait_ns, row_token);
+        return cudaGetLastError();
+    }
     if (!pair) {
         if (gather)
             launch_pdl(grouped_gemm_kernel<EPI, true>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s, 
@@ -985,7 +1061,7 @@ cudaError_t launch_up_tc(const moe_params_t *p, const void *x_perm, const int32_
 {
     const uint64_t d = p->d, m = p->m, m16 = round_up(p->m, 16), m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    cudaError_t e = launch_gemm<EPI_SWIGLU>(x_perm, d, d, rows, nullptr, rows, W13, d, d, 2 * m16,
+    cudaError_t e = launch_gemm<EPI_SWIGLU>(x_perm, d, d, rows, nullptr, rows, p->k, W13, d, d, 2 * m16,
                                             offsets, p->E, (bf16 *)h, (int)m8, (int)m, status, s);
     count_launch();
     return e;
@@ -997,7 +1073,7 @@ cudaError_t launch_up_tc_gather(const moe_params_t *p, const void *x, const int3
 {
     const uint64_t d = p->d, m = p->m, m16 = round_up(p->m, 16), m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    cudaError_t e = launch_gemm<EPI_SWIGLU>(x, d, d, (uint64_t)p->T, row_token, rows, W13, d, d,
+    cudaError_t e = launch_gemm<EPI_SWIGLU>(x, d, d, (uint64_t)p->T, row_token, rows, p->k, W13, d, d,
                                             2 * m16, offsets, p->E, (bf16 *)h, (int)m8, (int)m,
                                             status, s);
     count_launch();
@@ -1009,7 +1085,7 @@ cudaError_t launch_down_tc(const moe_params_t *p, const void *h, const int32_t *
 {
     const uint64_t d = p->d, m = p->m, m8 = round_up(p->m, 8);
     const uint64_t rows = (uint64_t)p->T * p->k;
-    cudaError_t e = launch_gemm<EPI_STORE>(h, m, m8, rows, nullptr, rows, W2, m, m8, d, offsets,
+    cudaError_t e = launch_gemm<EPI_STORE>(h, m, m8, rows, nullptr, rows, p->k, W2, m, m8, d, offsets,
                                            p->E, (bf16 *)out, (int)d, (int)d, status, s);
     count_launch();
     return e;
