@@ -491,13 +491,17 @@ __device__ void ds_gate(const float *lg, const DsArgs &a, int32_t *idx_out, floa
             }
             continue;
         }
+        // (the loops over the k picks leave at k: a round of shuffles per pick is the
+        // gate's longest chain)
         int sel[MOE_MAX_TOPK];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_TOPK; ++j)
+            sel[j] = 0;
         bool taken = false;
 #pragma unroll
         for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-            sel[j] = 0;
             if (j >= k)
-                continue;
+                break;
             float v = (on && !taken) ? h : -INFINITY;
             int vi = (on && !taken) ? lane : 0x7fffffff;
 #pragma unroll
@@ -523,9 +527,11 @@ __device__ void ds_gate(const float *lg, const DsArgs &a, int32_t *idx_out, floa
         if (a.router_type == MOE_ROUTER_MIXTRAL) {
             float zs = 0.f;
 #pragma unroll
-            for (int j = 0; j < MOE_MAX_TOPK; ++j)
-                if (j < k)
-                    zs += __shfl_sync(0xffffffffu, ex, sel[j]);
+            for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+                if (j >= k)
+                    break;
+                zs += __shfl_sync(0xffffffffu, ex, sel[j]);
+            }
             const float is = 1.f / zs;
             wsel = ex * is;
         } else {
@@ -538,7 +544,7 @@ __device__ void ds_gate(const float *lg, const DsArgs &a, int32_t *idx_out, floa
 #pragma unroll
         for (int j = 0; j < MOE_MAX_TOPK; ++j) {
             if (j >= k)
-                continue;
+                break;
             const float wj = __shfl_sync(0xffffffffu, wsel, sel[j]);
             if (lane == j) {
                 idx_out[t * k + j] = sel[j];
