@@ -238,7 +238,7 @@ __device__ __forceinline__ void zero_k_rows(uint32_t base, int n, int r0)
 
 template <bool KG>
 __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tiles, int M,
-                                            int num_kb, int nfast)
+                                            int num_kb, int order)
 {
     Tile t;
     int e = 0;
@@ -248,11 +248,11 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     t.e = e;
     if constexpr (KG) {
         const int mtiles = (M + BM - 1) / BM;
-        // m-tiles fastest (concurrent tiles share a B chunk, A_e is reused across n)
-        // or, with nfast, n-tiles fastest (B_e reused across m): the smaller operand
+        // order 0: m-tiles fastest (concurrent tiles share a B chunk, A_e is reused
+        // across n); 1: n-tiles fastest (B_e reused across m): the smaller operand
         // stays in L2
-        const int mt = nfast ? local / n_tiles : local % mtiles;
-        const int nt = nfast ? local % n_tiles : local / mtiles;
+        const int mt = order ? local / n_tiles : local % mtiles;
+        const int nt = order ? local % n_tiles : local / mtiles;
         t.a_row = mt * BM;
         t.row0 = e * M + mt * BM;
         t.row_end = e * M + M;
@@ -262,9 +262,14 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
         t.nkb = (rows + BK - 1) / BK;
         t.kv = rows - (t.nkb - 1) * BK;
     } else {
+        // bands of `order` m-tiles (0: the whole expert), m-tiles fastest inside a band:
+        // concurrent tiles share the band's A rows while it sweeps N
         const int rows = aux->off[e + 1] - aux->off[e];
         const int mtiles = (rows + BM - 1) / BM;
-        const int mt = local % mtiles, nt = local / mtiles;
+        const int G = (order > 0 && order < mtiles) ? order : mtiles;
+        const int bi = local / (G * n_tiles), rem = local - bi * G * n_tiles;
+        const int gr = min(G, mtiles - bi * G);
+        const int mt = bi * G + rem % gr, nt = rem / gr;
         t.a_row = aux->off[e] + mt * BM;
         t.row0 = t.a_row;
         t.row_end = aux->off[e + 1];
@@ -282,7 +287,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmO, const int32_t *__restrict__ offsets,
                     int E, int N, int K, int M, bf16 *__restrict__ out, int ld_out, int n_valid,
                     const bf16 *__restrict__ dh, int ld_dh, int32_t *status, uint64_t wait_ns,
-                    int nfast)
+                    int order)
 {
     pdl_wait();
     pdl_trigger();
@@ -350,7 +355,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
                 if (*abort_flag)
                     break;
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 for (int kb = 0; kb < t.nkb; ++kb) {
                     if (!mbar_wait(smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns, abort_flag,
                                    status)) {
@@ -411,7 +416,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t tpar = 0;
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 if (t.nkb > 0 && t.kv < BK) {
                     const int ts = (stage + t.nkb - 1) % STAGES;
                     bool ok = true;
@@ -442,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 if (!mbar_wait(smem_u32(&aux->tempty[acc]), acc_phase ^ 1u, wait_ns, abort_flag,
                                status)) {
                     ok = false;
@@ -500,7 +505,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-            const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+            const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
             if (!mbar_wait(smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag, status))
                 break;
             tc_fence_after();
@@ -643,7 +648,7 @@ __device__ __forceinline__ void umma_commit_own(uint32_t bar)
 // rows of every expert per tile.  row0 / a_row: the pair's first row (rank 0).
 template <bool KG>
 __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tiles, int M,
-                                            int num_kb, int nfast)
+                                            int num_kb, int order)
 {
     Tile t;
     int e = 0;
@@ -653,8 +658,8 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     t.e = e;
     if constexpr (KG) {
         const int mtiles = (M + 2 * BM - 1) / (2 * BM);
-        const int mt = nfast ? local / n_tiles : local % mtiles;
-        const int nt = nfast ? local % n_tiles : local / mtiles;
+        const int mt = order ? local / n_tiles : local % mtiles;
+        const int nt = order ? local % n_tiles : local / mtiles;
         t.a_row = mt * 2 * BM;
         t.row0 = e * M + mt * 2 * BM;
         t.row_end = e * M + M;
@@ -666,7 +671,10 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     } else {
         const int rows = aux->off[e + 1] - aux->off[e];
         const int mtiles = (rows + 2 * BM - 1) / (2 * BM);
-        const int mt = local % mtiles, nt = local / mtiles;
+        const int G = (order > 0 && order < mtiles) ? order : mtiles;
+        const int bi = local / (G * n_tiles), rem = local - bi * G * n_tiles;
+        const int gr = min(G, mtiles - bi * G);
+        const int mt = bi * G + rem % gr, nt = rem / gr;
         t.a_row = aux->off[e] + mt * 2 * BM;
         t.row0 = t.a_row;
         t.row_end = aux->off[e + 1];
@@ -686,7 +694,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const int32_t *__restrict__ offsets, int E, int N, int K, int M,
                         bf16 *__restrict__ out, int ld_out, int n_valid,
                         const bf16 *__restrict__ dh, int ld_dh, int32_t *status, uint64_t wait_ns,
-                    int nfast)
+                    int order)
 {
     pdl_wait();
     pdl_trigger();
@@ -757,7 +765,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
                 if (*abort_flag)
                     break;
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 for (int kb = 0; kb < t.nkb; ++kb) {
                     if (!mbar_wait(smem_u32(&aux->empty[stage]), phase ^ 1u, wait_ns, abort_flag,
                                    status)) {
@@ -835,7 +843,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t tpar = 0;
             for (int tile = cluster_id; tile < total; tile += nclusters) {
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 if (t.nkb > 0 && t.kv < BK) {
                     const int ts = (stage + t.nkb - 1) % STAGES;
                     bool ok = true;
@@ -866,7 +874,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
-                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+                const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
                 if (!mbar_wait(smem_u32(&aux->tempty[acc]), acc_phase ^ 1u, wait_ns, abort_flag,
                                status)) {
                     ok = false;
@@ -928,7 +936,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = cluster_id; tile < total; tile += nclusters) {
-            const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, nfast);
+            const Tile t = decode_tile<KG>(aux, tile, n_tiles, M, num_kb, order);
             if (!mbar_wait(smem_u32(&aux->tfull[acc]), acc_phase, wait_ns, abort_flag, status))
                 break;
             tc_fence_after();
@@ -1088,13 +1096,21 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     if ((e = tc::make_map(&to, out, 2, dout, sout, bout, CU_TENSOR_MAP_SWIZZLE_64B)) !=
         cudaSuccess)
         return e;
-    // K-grouped: n-tiles fastest when B_e (N columns) is the smaller operand
-    const int nfast = (KG && b_rows < (uint64_t)M) ? 1 : 0;
+    // tile order: K-grouped, n-tiles fastest when B_e (N columns) is the smaller
+    // operand; row-grouped, bands of m-tiles whose A rows take ~16 MB
+    int order = 0;
+    if constexpr (KG) {
+        order = b_rows < (uint64_t)M ? 1 : 0;
+    } else {
+        const uint64_t tile_a = (use_pair ? 2ull : 1ull) * BM * a_k * 2;
+        const uint64_t g = (16ull << 20) / (tile_a > 0 ? tile_a : 1);
+        order = g < 1 ? 1 : (int)(g > 1024 ? 1024 : g);
+    }
     count_launch();
     if (!use_pair)
         return launch_pdl(bwd_gemm_kernel<EPI, KG, BT>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES,
                           s, ta, tb, to, offsets, E, (int)b_rows, (int)a_k, M, out, ld_out,
-                          n_valid, dh, ld_dh, status, wait_limit_ns(), nfast);
+                          n_valid, dh, ld_dh, status, wait_limit_ns(), order);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1111,7 +1127,7 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, pair::bwd_gemm_2sm_kernel<EPI, KG, BT>, ta, tb, to, offsets, E,
                               (int)b_rows, (int)a_k, M, out, ld_out, n_valid, dh, ld_dh, status,
-                              wait_limit_ns(), nfast);
+                              wait_limit_ns(), order);
 }
 
 }  // namespace bwd
