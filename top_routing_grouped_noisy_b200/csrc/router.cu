@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "dispatch_scan.cuh"
 #include "gate.cuh"
 #include "kernels.h"
 
@@ -129,17 +130,55 @@ __global__ void __launch_bounds__(256) router_small_partial_kernel(
     router_small_slice(blockIdx.x, x, Wg, Wn, T, d, E, part, sm);
 }
 
+struct SmallFinishBar {
+    __device__ void operator()() const { __syncthreads(); }
+};
+
+// ... then, for a2, the count step of the counting sort on the indices just written
+// (dispatch_count_kernel's arithmetic: one ballot per expert and 32-token chunk, then
+// the exclusive scan over chunks per expert into rank bases and routed counts), so no
+// count launch follows the small router.
 __global__ void __launch_bounds__(256) router_small_finish_kernel(
     const float *__restrict__ part, int T, int E, int k, int noisy,
     const float *__restrict__ noise, const float *__restrict__ bias, int router_type,
     int32_t *__restrict__ idx_out, float *__restrict__ w_out, float *__restrict__ probs_sum,
-    float *__restrict__ importance, int32_t *status)
+    float *__restrict__ importance, int32_t *status, int32_t *__restrict__ hist,
+    int32_t *__restrict__ dcounts)
 {
     pdl_wait();
     pdl_trigger();
     extern __shared__ float sm[];
     router_small_finish(part, T, E, k, noisy, noise, bias, router_type, idx_out, w_out,
                         probs_sum, importance, status, sm);
+    __syncthreads();  // this CTA's indices are visible to all its threads
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nch = (T + kDispatchChunk - 1) / kDispatchChunk;
+    for (int c = warp; c < nch; c += (int)(blockDim.x >> 5)) {
+        const int t = c * kDispatchChunk + lane;
+        int ej[MOE_MAX_TOPK];
+        for (int j = 0; j < k; ++j) {
+            int e = -1;
+            if (t < T) {
+                e = idx_out[t * k + j];
+                if (e < 0 || e >= E) {
+                    set_status(status, MOE_ERR_DEVICE_BADINDEX);
+                    e = -1;
+                }
+            }
+            ej[j] = e;
+        }
+        for (int e = 0; e < E; ++e) {
+            bool has = false;
+            for (int j = 0; j < k; ++j)
+                has |= ej[j] == e;
+            const unsigned b = __ballot_sync(0xffffffffu, has);
+            if (lane == (e & 31))
+                hist[e * nch + c] = __popc(b);
+        }
+    }
+    __syncthreads();
+    scan_chunk_counts(hist, E, nch, dcounts, nullptr, 0, (int)threadIdx.x, (int)blockDim.x,
+                      SmallFinishBar());
 }
 
 cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
@@ -183,11 +222,9 @@ cudaError_t launch_route(const moe_params_t *p, const void *x, const void *Wg,
             return e;
         launch_pdl(router_small_finish_kernel, dim3(1), dim3(256), sm2, s, sp, p->T, p->E, p->k, noisy, noise, bias,
                                                        p->router_type, idx, w, probs_sum,
-                                                       importance, status);
+                                                       importance, status, hist, dcounts);
         count_launch();
-        if ((e = cudaGetLastError()) != cudaSuccess)
-            return e;
-        return launch_count(p, idx, hist, dcounter, dcounts, status, s);
+        return cudaGetLastError();  // the finishing CTA also did a2's count step
     }
     if (p->T > 0 && p->dtype == MOE_BF16) {
         int32_t *counter = reinterpret_cast<int32_t *>(ws) + kWsRouterCounterWord;
