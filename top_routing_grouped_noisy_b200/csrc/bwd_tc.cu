@@ -248,11 +248,11 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     t.e = e;
     if constexpr (KG) {
         const int mtiles = (M + BM - 1) / BM;
-        // order 0: m-tiles fastest (concurrent tiles share a B chunk, A_e is reused
-        // across n); 1: n-tiles fastest (B_e reused across m): the smaller operand
-        // stays in L2
-        const int mt = order ? local / n_tiles : local % mtiles;
-        const int nt = order ? local % n_tiles : local / mtiles;
+        // order bit 0 clear: m-tiles fastest (concurrent tiles share a B chunk, A_e is
+        // reused across n); set: n-tiles fastest (B_e reused across m): the smaller
+        // operand stays in L2.  Bits 1 and 2: A and B come as one 3-D box per stage.
+        const int mt = (order & 1) ? local / n_tiles : local % mtiles;
+        const int nt = (order & 1) ? local % n_tiles : local / mtiles;
         t.a_row = mt * BM;
         t.row0 = e * M + mt * BM;
         t.row_end = e * M + M;
@@ -374,13 +374,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ++tfills[stage];
                         }
                         mbar_expect_tx(fb, STAGE_BYTES);
+                        if (order & 2)  // one 3-D box: the tile's 64-wide chunks of BK rows
+                            tma_load_3d(&tmA, fb, sa, 0, kc, t.a_row / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            tma_load_2d(&tmA, fb, sa + j * kMnChunkBytes, t.a_row + 64 * j, kc);
+                            for (int j = 0; j < BM / 64; ++j)
+                                tma_load_2d(&tmA, fb, sa + j * kMnChunkBytes, t.a_row + 64 * j,
+                                            kc);
+                        if (order & 4)
+                            tma_load_3d(&tmB, fb, sa + A_BYTES, 0, kc, t.n0 / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(&tmB, fb, sa + A_BYTES + j * kMnChunkBytes, t.n0 + 64 * j,
-                                        kc);
+                            for (int j = 0; j < BN / 64; ++j)
+                                tma_load_2d(&tmB, fb, sa + A_BYTES + j * kMnChunkBytes,
+                                            t.n0 + 64 * j, kc);
                     } else if constexpr (BT) {  // MN-major B: 64-wide N chunks of BK K rows
                         mbar_expect_tx(fb, STAGE_BYTES);
                         tma_load_2d(&tmA, fb, sa, kc, t.a_row);
@@ -658,8 +665,8 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     t.e = e;
     if constexpr (KG) {
         const int mtiles = (M + 2 * BM - 1) / (2 * BM);
-        const int mt = order ? local / n_tiles : local % mtiles;
-        const int nt = order ? local % n_tiles : local / mtiles;
+        const int mt = (order & 1) ? local / n_tiles : local % mtiles;
+        const int nt = (order & 1) ? local % n_tiles : local / mtiles;
         t.a_row = mt * 2 * BM;
         t.row0 = e * M + mt * 2 * BM;
         t.row_end = e * M + M;
@@ -785,25 +792,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const uint32_t tb = smem_u32(&aux->tbar[stage]);
                         ++tfills[stage];
                         mbar_expect_tx(tb, STAGE_BYTES);
+                        if (order & 2)
+                            tma_load_3d(&tmA, tb, sa, 0, kc, (t.a_row + (int)rank * BM) / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            tma_load_2d(&tmA, tb, sa + j * kMnChunkBytes,
-                                        t.a_row + (int)rank * BM + 64 * j, kc);
+                            for (int j = 0; j < BM / 64; ++j)
+                                tma_load_2d(&tmA, tb, sa + j * kMnChunkBytes,
+                                            t.a_row + (int)rank * BM + 64 * j, kc);
+                        if (order & 4)
+                            tma_load_3d(&tmB, tb, sa + A_BYTES, 0, kc,
+                                        (t.n0 + (int)rank * BNH) / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BNH / 64; ++j)
-                            tma_load_2d(&tmB, tb, sa + A_BYTES + j * kMnChunkBytes,
-                                        t.n0 + (int)rank * BNH + 64 * j, kc);
+                            for (int j = 0; j < BNH / 64; ++j)
+                                tma_load_2d(&tmB, tb, sa + A_BYTES + j * kMnChunkBytes,
+                                            t.n0 + (int)rank * BNH + 64 * j, kc);
                     } else if constexpr (KG) {  // both MN-major: this CTA's 64-wide chunks
                         if (leader)
                             mbar_expect_tx(fb, 2 * STAGE_BYTES);
+                        if (order & 2)  // one 3-D box: this CTA's chunks of BK rows
+                            tma_load_3d_pair(&tmA, fb0, sa, 0, kc, (t.a_row + (int)rank * BM) / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BM / 64; ++j)
-                            tma_load_2d_pair(&tmA, fb0, sa + j * kMnChunkBytes,
-                                             t.a_row + (int)rank * BM + 64 * j, kc);
+                            for (int j = 0; j < BM / 64; ++j)
+                                tma_load_2d_pair(&tmA, fb0, sa + j * kMnChunkBytes,
+                                                 t.a_row + (int)rank * BM + 64 * j, kc);
+                        if (order & 4)
+                            tma_load_3d_pair(&tmB, fb0, sa + A_BYTES, 0, kc,
+                                             (t.n0 + (int)rank * BNH) / 64);
+                        else
 #pragma unroll
-                        for (int j = 0; j < BNH / 64; ++j)
-                            tma_load_2d_pair(&tmB, fb0, sa + A_BYTES + j * kMnChunkBytes,
-                                             t.n0 + (int)rank * BNH + 64 * j, kc);
+                            for (int j = 0; j < BNH / 64; ++j)
+                                tma_load_2d_pair(&tmB, fb0, sa + A_BYTES + j * kMnChunkBytes,
+                                                 t.n0 + (int)rank * BNH + 64 * j, kc);
                     } else if constexpr (BT) {
                         if (leader)
                             mbar_expect_tx(fb, 2 * STAGE_BYTES);  // MN-major B: this CTA's 64-wide N chunks
@@ -1065,18 +1086,35 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     if (e != cudaSuccess)
         return e;
     CUtensorMap ta, tb, to;
-    const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
-    const uint32_t ba[2] = {KG ? 64u : (uint32_t)BK, KG ? (uint32_t)BK : (uint32_t)BM};
     const uint32_t b_box = use_pair ? (uint32_t)pair::BNH : (uint32_t)BN;
-    if ((e = tc::make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
-        return e;
+    // K-grouped operands whose column count is a multiple of 64 load a stage's 64-wide
+    // chunks with one 3-D box (columns within a chunk, rows, chunks)
+    const bool a3d = KG && a_k % 64 == 0, b3d = KG && b_rows % 64 == 0;
+    if (a3d) {
+        const uint64_t da[3] = {64, a_rows, a_k / 64}, sa[2] = {a_ld * 2, 128};
+        const uint32_t ba[3] = {64, BK, BM / 64};
+        if ((e = tc::make_map(&ta, A, 3, da, sa, ba)) != cudaSuccess)
+            return e;
+    } else {
+        const uint64_t da[2] = {a_k, a_rows}, sa[1] = {a_ld * 2};
+        const uint32_t ba[2] = {KG ? 64u : (uint32_t)BK, KG ? (uint32_t)BK : (uint32_t)BM};
+        if ((e = tc::make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
+            return e;
+    }
     if constexpr (KG) {
         // MN-major boxes of 64 columns x BK rows; columns and rows past the extents
         // read as zero
-        const uint64_t db[2] = {b_rows, a_rows}, sb[1] = {b_ld * 2};
-        const uint32_t bb[2] = {64, BK};
-        if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
-            return e;
+        if (b3d) {
+            const uint64_t db[3] = {64, a_rows, b_rows / 64}, sb[2] = {b_ld * 2, 128};
+            const uint32_t bb[3] = {64, BK, b_box / 64};
+            if ((e = tc::make_map(&tb, B, 3, db, sb, bb)) != cudaSuccess)
+                return e;
+        } else {
+            const uint64_t db[2] = {b_rows, a_rows}, sb[1] = {b_ld * 2};
+            const uint32_t bb[2] = {64, BK};
+            if ((e = tc::make_map(&tb, B, 2, db, sb, bb)) != cudaSuccess)
+                return e;
+        }
     } else if constexpr (BT) {
         // N innermost: boxes of 64 N x BK K rows, N and K past their extents read as zero
         const uint64_t db[3] = {b_rows, b_k, (uint64_t)E};
@@ -1100,7 +1138,7 @@ static cudaError_t launch(const void *A, uint64_t a_k, uint64_t a_ld, uint64_t a
     // operand; row-grouped, bands of m-tiles whose A rows take ~16 MB
     int order = 0;
     if constexpr (KG) {
-        order = b_rows < (uint64_t)M ? 1 : 0;
+        order = (b_rows < (uint64_t)M ? 1 : 0) | (a3d ? 2 : 0) | (b3d ? 4 : 0);
     } else {
         const uint64_t tile_a = (use_pair ? 2ull : 1ull) * BM * a_k * 2;
         const uint64_t g = (16ull << 20) / (tile_a > 0 ? tile_a : 1);
