@@ -113,3 +113,33 @@ def test_decode_forward_wait_timeout_is_reported_and_context_survives():
     r, ties = H.check_routing(w, inp, bufs, 5e-5)
     dsp = H.check_dispatch(w, inp, p, bufs)
     H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)
+
+
+def test_front_small_wait_timeout_is_reported_and_context_survives():
+    """The small-batch front of moe_forward (routing, dispatch and gate statistics in
+    one cooperative launch with two grid barriers) gives up at a wait limit of 0,
+    reports MOE_ERR_DEVICE_TIMEOUT and returns with its barrier words back at zero, so
+    the next forward on the same workspace is correct without a status clear."""
+    w = wl.Workload("to_front", T=40, d=256, d_ff=8 * 64, E=8, k=2, noisy=True, seed=84)
+    inp = wl.make_inputs(w)
+    p, bufs, ws, status, weights = H.run_forward(w, inp)
+    assert status == 0
+    dev = "cuda"
+    W13_e, W2_e = weights
+    x, Wg, Wn, eps = (inp[n].to(dev) for n in ("x", "Wg", "Wnoise", "eps"))
+    moe.moe_set_wait_limit_ns(0)
+    try:
+        moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs, Wnoise=Wn, noise=eps)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    assert moe.moe_get_device_status(ws, clear=False) == moe.MOE_ERR_DEVICE_TIMEOUT
+    hdr = ws.buf[:32].view(torch.int32).cpu()
+    assert int(hdr[6]) == 0 and int(hdr[7]) == 0  # the front barrier words
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_DEVICE_TIMEOUT  # read and clear
+    moe.moe_forward(p, x, Wg, W13_e, W2_e, ws, bufs, Wnoise=Wn, noise=eps)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    r, ties = H.check_routing(w, inp, bufs, 5e-5)
+    dsp = H.check_dispatch(w, inp, p, bufs)
+    H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)

@@ -51,6 +51,10 @@ SMALL = {
     # wide rows and 12 tokens: the decode kernel's 1024-column GEMM 1 stages
     "decode_t12_wide": W("decode_t12_wide", T=12, d=4096, d_ff=8 * 64, E=8, k=2, noisy=True,
                          rescale=True, seed=32),
+    # 17..64 tokens: one cooperative launch routes, dispatches and takes the gate
+    # statistics in moe_forward (f32 here, capacity drops, ST, noise and bias)
+    "front_f32_st_cap": W("front_f32_st_cap", T=33, d=72, d_ff=8 * 40, E=8, k=3, dtype="f32",
+                          router=wl.ST, noisy=True, bias=True, cf=0.5, seed=35),
     "f32_noisy_st_cap": W("f32_noisy_st_cap", T=257, d=64, d_ff=160, E=8, k=2, dtype="f32",
                           router=wl.ST, noisy=True, bias=True, cf=1.5, seed=22),
     "f32_e16_k4": W("f32_e16_k4", T=190, d=96, d_ff=16 * 24, E=16, k=4, dtype="f32",
@@ -136,6 +140,16 @@ STEP_CASES = {
     "decode_st_bias_cap": W("decode_st_bias_cap", T=48, d=192, d_ff=16 * 40, E=16, k=4,
                             router=wl.ST, noisy=True, bias=True, cf=1.0, rescale=True,
                             lam=0.01, seed=30),
+    "front_f32_st_cap": SMALL["front_f32_st_cap"],
+    "front_e32_k8": W("front_e32_k8", T=64, d=128, d_ff=32 * 16, E=32, k=8, noisy=True,
+                      cf=0.8, seed=36),
+    # E = 64 without noise: the front's gate runs one thread per token (E > 32)
+    "front_e64_plain": W("front_e64_plain", T=64, d=128, d_ff=64 * 16, E=64, k=8, cf=1.0,
+                         seed=38),
+    # E = 64 with noise: too many logits for the split-K router, so both sides route
+    # on the tensor cores
+    "e64_k8_t64": W("e64_k8_t64", T=64, d=128, d_ff=64 * 16, E=64, k=8, noisy=True,
+                    cf=0.8, seed=37),
 }
 
 

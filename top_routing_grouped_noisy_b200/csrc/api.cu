@@ -115,6 +115,7 @@ WsLayout ws_layout(const moe_params_t *p)
     // larger, so that a workspace sized for T also serves every smaller batch.
     const int t_small = p->T < kRouterSmallTokens ? (p->T > 0 ? p->T : 1) : kRouterSmallTokens;
     L.rsmall = take((size_t)kRouterSmallSplit * t_small * 2 * p->E * sizeof(float));
+    L.gsmall = take((size_t)2 * t_small * p->E * sizeof(float));
     L.total = off;
     return L;
 }
@@ -570,6 +571,35 @@ int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t 
         char *w = static_cast<char *>(ws);
         cudaStream_t s = (cudaStream_t)stream;
         return after_launch(fn, launch_forward_decode(p, b, w, s));
+    }
+    if (front_small_fits(p, b->Wnoise != nullptr)) {
+        // at most 64 tokens: routing, dispatch and the gate statistics in one launch
+        REQUIRE_PTR(b->x);
+        REQUIRE_PTR(b->Wg);
+        OPTIONAL_PTR(b->Wnoise);
+        OPTIONAL_PTR(b->noise);
+        OPTIONAL_PTR(b->bias);
+        REQUIRE_PTR(b->topk_idx);
+        REQUIRE_PTR(b->topk_w);
+        REQUIRE_PTR(b->probs_sum);
+        REQUIRE_PTR(b->importance);
+        REQUIRE_PTR(b->x_perm);
+        REQUIRE_PTR(b->row_token);
+        REQUIRE_PTR(b->slot_row);
+        REQUIRE_PTR(b->counts);
+        REQUIRE_PTR(b->kept);
+        REQUIRE_PTR(b->offsets);
+        if (b->Wnoise != nullptr && b->noise == nullptr)
+            return fail(MOE_ERR_INVALID_ARG, "%s: Wnoise given without the noise draws", fn);
+        if ((rc = check_ws(fn, p, ws, ws_bytes)) != MOE_OK)
+            return rc;
+        if ((rc = after_launch(fn, launch_front_small(p, b, static_cast<char *>(ws),
+                                                      (cudaStream_t)stream))) != MOE_OK)
+            return rc;
+        if ((rc = moe_expert_ffn(p, b->x_perm, b->offsets, b->W13_e, b->W2_e, b->h, b->out, ws,
+                                 ws_bytes, stream)) != MOE_OK)
+            return rc;
+        return moe_combine(p, b->out, b->slot_row, b->topk_w, b->y, stream);
     }
     if ((rc = route_impl("moe_forward", p, b->x, b->Wg, b->Wnoise, b->router_packed, b->noise,
                          b->bias, b->topk_idx, b->topk_w, b->probs_sum, b->importance, ws,

@@ -198,7 +198,7 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
                 for (int i = 0; i < 16; ++i) {
                     const float g = __uint_as_float(v[q2][i]);
                     const float u = __uint_as_float(v[q2][16 + i]);
-                    const float s = 1.0f / (1.0f + __expf(-g));
+                    const float s = __fdividef(1.0f, 1.0f + __expf(-g));  // as the forward
                     const float dhi = dhv[q2 * 16 + i];
                     o[i] = dhi * u * s * (1.0f + g * (1.0f - s));  // dg
                     o[16 + i] = dhi * g * s;                       // du = dh * silu(g)

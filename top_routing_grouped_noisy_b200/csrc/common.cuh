@@ -23,10 +23,12 @@ constexpr size_t kWsHeader = 256;
 constexpr int kWsCounterWord = 1;
 // Word 2: ticket counter of the tensor-core router (zero between calls).
 constexpr int kWsRouterCounterWord = 2;
-// Word 3: ticket counter of the decode-size router + dispatch kernel (zero between calls).
-constexpr int kWsSmallCounterWord = 3;
-// Words 4-5: grid barrier of the decode forward kernel (arrive, depart; zero between calls).
+// Words 4-5: grid barrier of the decode forward kernel (arrival count, zero between
+// calls; generation, counting up).
 constexpr int kWsDecodeBarrierWord = 4;
+// Words 6-7: grid barriers of the small-batch front kernel (arrivals over both
+// barriers; CTAs past both; zero between calls).
+constexpr int kWsFrontBarrierWord = 6;
 // Header bytes that clearing the status resets (status word and counters).
 constexpr size_t kWsResetBytes = 32;
 // Words 8-9: offsets {0, T} of the shared block's one-expert GEMMs (residual MoE).
@@ -37,7 +39,10 @@ constexpr int kWsTokenRangeWord = 8;
 // while the previous kernel on the stream is still running, so it calls
 // pdl_wait() before it touches global memory (the wait returns once the
 // previous grid has completed and its writes are visible), and pdl_trigger() to
-// let the next kernel be scheduled early in turn.
+// let the next kernel be scheduled early in turn.  A kernel that triggers before
+// its own wait lets the next one start while the previous grid still runs; that
+// one still sees every earlier grid complete at its wait, since this grid cannot
+// complete before its own wait has returned.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger()
 {
@@ -48,6 +53,13 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code)
 {
     if (status != nullptr)
         atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p)
+{
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns()
@@ -119,6 +131,25 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float *f)
 
 // D += A * B on the tensor cores, m16n8k16, bf16 inputs, f32 accumulators
 // (A row-major 16x16 in a0..a3, B column-major 16x8 in b0..b1).
+// B fragment of mma m16n8k16 from a row-major [k][8] bf16 tile: lanes 0..15 give the
+// addresses of rows 0..15 (16-byte aligned)
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &b0, uint32_t &b1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(b0), "=r"(b1)
+                 : "r"(addr));
+}
+
+// A fragment of mma m16n8k16 from a row-major [16][16] bf16 tile: lane l gives the
+// address of row l % 16 at column 8 * (l / 16) (16-byte aligned)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &a0, uint32_t &a1, uint32_t &a2,
+                                        uint32_t &a3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                 : "r"(addr));
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float *c, uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1)
 {

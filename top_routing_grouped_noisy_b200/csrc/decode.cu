@@ -120,27 +120,11 @@ __device__ __forceinline__ uint4 lds128(const char *p) { return *reinterpret_cas
 // barrier of the multiplying warps (named barrier 1, warps 1..8)
 __device__ __forceinline__ void cw_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kDsCw * 32) : "memory"); }
 
-__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p)
-{
-    int32_t v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ uint32_t lds32_s(uint32_t addr)
 {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
-}
-
-// B fragment of mma m16n8k16 from a row-major [k][8] bf16 tile: lanes 0..15 give the
-// addresses of rows 0..15 (16-byte aligned)
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &b0, uint32_t &b1)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
-                 : "=r"(b0), "=r"(b1)
-                 : "r"(addr));
 }
 
 __device__ __forceinline__ uint32_t bf16_pair_s(const bf16 *lo, const bf16 *hi)
@@ -453,11 +437,9 @@ __device__ void ds_router_logits(const char *breg, int bp, const DsArgs &a, char
     __syncthreads();
 }
 
-// The gate of every token (one warp per token, lane e holding expert e; E <= 32),
-// with the arithmetic of finish_token: the same routing logits, the first maximum
-// on ties, the softmax and the Mixtral renormalisation summed in expert / slot
-// order.  Then the token sums probs_sum, importance in token order.  gsm: [T][E]
-// probabilities, then [T][E] gate weights.  Called by every thread of the CTA.
+// The gate of every token (gate_token_warp, one warp per token; E <= 32), then the
+// token sums probs_sum, importance in token order.  gsm: [T][E] probabilities, then
+// [T][E] gate weights.  Called by every thread of the CTA.
 __device__ void ds_gate(const float *lg, const DsArgs &a, int32_t *idx_out, float *w_out,
                         float *probs_sum, float *importance, float *gsm)
 {
@@ -870,7 +852,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) decode_stream_kernel(const __gr
                         if (neuron < nv && tok < nr) {
                             const float gv = sum(L, nb * 4 + jj), uv = sum(L, nb * 4 + 2 + jj);
                             a.h[(size_t)(r0 + tok) * m8 + j0 + neuron] =
-                                __float2bfloat16_rn(gv / (1.0f + __expf(-gv)) * uv);
+                                __float2bfloat16_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
                         }
                     }
                 });

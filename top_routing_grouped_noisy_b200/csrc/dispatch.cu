@@ -115,8 +115,8 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(
     int32_t *__restrict__ row_token, int32_t *__restrict__ slot_row, int32_t *__restrict__ counts,
     int32_t *__restrict__ kept, int32_t *__restrict__ offsets, int tpc)
 {
+    pdl_trigger();  // early: the GEMM after it may prefetch its weights meanwhile
     pdl_wait();
-    pdl_trigger();
     __shared__ int32_t s_cnt[MOE_MAX_EXPERTS];
     __shared__ int32_t s_kept[MOE_MAX_EXPERTS];
     __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];

@@ -153,7 +153,7 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
                 for (int i = 0; i < 16; ++i) {
                     const float g = __uint_as_float(v[0][i]);
                     const float u = __uint_as_float(v[0][16 + i]);
-                    hv[i] = g / (1.0f + __expf(-g)) * u;
+                    hv[i] = __fdividef(g, 1.0f + __expf(-g)) * u;  // see below
                 }
                 if (rv && nb < n_valid) {
                     bf16 *dst = out + (int64_t)row * ld_out + nb;
@@ -161,8 +161,10 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
                         st_v4(dst, f32x8_to_bf16(hv));
                         st_v4(dst + 8, f32x8_to_bf16(hv + 8));
                     } else {
-                        for (int i = 0; i < 16 && nb + i < n_valid; ++i)
-                            dst[i] = __float2bfloat16_rn(hv[i]);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)  // unrolled: hv stays in registers
+                            if (nb + i < n_valid)
+                                dst[i] = __float2bfloat16_rn(hv[i]);
                     }
                 }
             } else {
@@ -195,7 +197,10 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
                 for (int i = 0; i < 16; ++i) {
                     const float g = __uint_as_float(v[q2][i]);
                     const float u = __uint_as_float(v[q2][16 + i]);
-                    hv[q2 * 16 + i] = g / (1.0f + __expf(-g)) * u;
+                    // approximate division (2 ulp, 0 once 1 + e^-g > 2^126, silu's limit):
+                    // the IEEE quotient's longer code took the small-batch epilogue
+                    // from about 1 to 9 us; h is rounded to bf16 either way
+                    hv[q2 * 16 + i] = __fdividef(g, 1.0f + __expf(-g)) * u;
                 }
             if (full_rows && nb + 32 <= n_valid) {
                 uint32_t pk[16];
@@ -210,8 +215,10 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
                     for (int q = 0; q < 4; ++q)
                         st_v4(dst + 8 * q, f32x8_to_bf16(hv + 8 * q));
                 } else {
-                    for (int i = 0; i < 32 && nb + i < n_valid; ++i)
-                        dst[i] = __float2bfloat16_rn(hv[i]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (nb + i < n_valid)
+                            dst[i] = __float2bfloat16_rn(hv[i]);
                 }
             }
         } else {
@@ -276,8 +283,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap tmO,
                         const int32_t *__restrict__ offsets, int E, int N, int K,
                         bf16 *__restrict__ out, int ld_out, int n_valid, int32_t *status,
-                        uint64_t wait_ns, const int32_t *__restrict__ row_token)
+                        uint64_t wait_ns, const int32_t *__restrict__ row_token, int pf_kb)
 {
+    // The expert weights are inputs no earlier kernel writes, so they may be read
+    // before the wait on the previous grid.  With at most one row tile per expert (the
+    // host passes pf_kb > 0 only then) tile b is column tile b % n_tiles of expert
+    // b / n_tiles whenever every expert has rows: the first pf_kb K blocks of that
+    // weight tile go to L2 while the routing kernels still run (an expert without rows
+    // only wastes its prefetch).
+    if (pf_kb > 0 && threadIdx.x == 0) {
+        const int nt = (N + BNT - 1) / BNT;
+        if ((int)blockIdx.x < E * nt) {
+            const int e = (int)blockIdx.x / nt, n0 = ((int)blockIdx.x % nt) * BNT;
+            const int kbs = min(pf_kb, (K + BK - 1) / BK);
+            for (int kb = 0; kb < kbs; ++kb)
+                tma_prefetch_l2_3d(&tmB, kb * BK, n0, e);
+        }
+    }
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
@@ -968,6 +990,13 @@ static cudaError_t prepare_device(DevInfo **out)
 // the few tiles over more SMs.
 constexpr int64_t kPairMinRows = 4096;
 
+// Bytes of its first weight tile (KiB) that each CTA of a small-batch GEMM (at most one
+// row tile per expert) brings into L2 before it waits for the routing kernels.
+#ifndef MOE_L2_PREFETCH_KIB
+#define MOE_L2_PREFETCH_KIB 640
+#endif
+constexpr int kL2PrefetchKiB = MOE_L2_PREFETCH_KIB;
+
 // One grouped GEMM launch.  A: [a_rows][a_ld] activations (K extent a_k), read in
 // expert-grouped row order, or -- when row_token is given -- gathered: tile row r is
 // row row_token[r] of A; B: [E][b_rows][b_ld] expert weights (K extent b_k, N =
@@ -1011,19 +1040,25 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
         return e;
     const uint64_t wait_ns = wait_limit_ns();
     const int N = (int)b_rows, K = (int)a_k;
+    // L2 prefetch depth of the first weight tile (K blocks), for one row tile per expert
+    const int bnt = narrow ? kNarrowBN : BN;
+    const int pf_kb = !pair && !gather && T <= BM
+                          ? (int)((int64_t)kL2PrefetchKiB * 1024 / ((int64_t)bnt * BK * 2))
+                          : 0;
     if (narrow) {
         launch_pdl(grouped_gemm_kernel<EPI, false, kNarrowBN>, dim3(di->sms), dim3(NUM_THREADS),
                    Geo<kNarrowBN>::SMEM_BYTES, s, ta, tb, to, offsets, E, N, K, out, ld_out,
-                   n_valid, status, wait_ns, row_token);
+                   n_valid, status, wait_ns, row_token, pf_kb);
         return cudaGetLastError();
     }
     if (!pair) {
         if (gather)
             launch_pdl(grouped_gemm_kernel<EPI, true>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s, 
-                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token, 0);
         else
             launch_pdl(grouped_gemm_kernel<EPI, false>, dim3(di->sms), dim3(NUM_THREADS), SMEM_BYTES, s, 
-                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token);
+                ta, tb, to, offsets, E, N, K, out, ld_out, n_valid, status, wait_ns, row_token,
+                pf_kb);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};

@@ -29,6 +29,19 @@ __host__ __device__ inline int router_small_kc(int d)
     return ((d + kRouterSmallSplit - 1) / kRouterSmallSplit + 7) / 8 * 8;
 }
 
+// Shared memory of one split-K router slice (bytes): bf16 stages the slice's x rows
+// [round16(T)][round16(kc) + 8] and weight columns [round16(kc)][round8(nout) + 8] as bf16
+// tiles for mma.sync; f32 stages x [T][kc] and the columns [kc][nout] as f32.
+__host__ __device__ inline size_t router_small_slice_smem(int T, int d, int nout, int dtype)
+{
+    const int kc = router_small_kc(d);
+    if (dtype == MOE_BF16) {
+        const int kp = (kc + 15) / 16 * 16, np = (nout + 7) / 8 * 8;
+        return 2 * ((size_t)(T + 15) / 16 * 16 * (kp + 8) + (size_t)kp * (np + 8));
+    }
+    return sizeof(float) * ((size_t)T * kc + (size_t)kc * nout);
+}
+
 // Byte offsets of the sections of the caller's workspace.
 struct WsLayout {
     size_t wt;     // router weights transposed to [nout_pad][d] (dtype; backward, f32 router)
@@ -36,6 +49,7 @@ struct WsLayout {
     size_t hist;   // dispatch per-chunk counts, then bases, [E][chunks] int32
     size_t dcounts;// routed count of every expert [E] int32 (next to the chunk bases)
     size_t rsmall; // small-batch router partial logits [32][T][2E] f32 (T <= 64)
+    size_t gsmall; // small-batch forward: softmax and gate weight rows [2][T][E] f32
     size_t total;
 };
 WsLayout ws_layout(const moe_params_t *p);
@@ -118,6 +132,12 @@ cudaError_t launch_dispatch(const moe_params_t *p, const void *x, const int32_t 
                             void *x_perm, int32_t *row_token, int32_t *slot_row,
                             int32_t *counts, int32_t *kept, int32_t *offsets, char *ws,
                             int32_t *status, bool routed, cudaStream_t s);
+
+// moe_forward's a1 + a2 + a6 for 1 <= T <= 64 (cooperative, 32 CTAs): the indices,
+// weights, token sums, tables, x_perm, counts / kept / offsets and f, P, L_balance
+cudaError_t launch_front_small(const moe_params_t *p, const moe_buffers_t *b, char *ws,
+                               cudaStream_t s);
+bool front_small_fits(const moe_params_t *p, bool noisy);
 
 // a3 / a4 for f32 (CUDA-core FMA)
 cudaError_t launch_up_simt(const moe_params_t *p, const float *x_perm, const int32_t *offsets,

@@ -115,6 +115,16 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint32_t bar
         : "memory");
 }
 
+// Bring one box of a 3-D tensor into L2 (no shared memory, no barrier; the copy has
+// no effect a program can observe except on timing).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint32_t bar, uint32_t dst,
                                             int c0, int c1, int c2)
 {
