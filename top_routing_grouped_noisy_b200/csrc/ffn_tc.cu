@@ -39,8 +39,9 @@ namespace tc {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle-128B row
+constexpr int kABoxRows = 64;  // rows of one A box (two per 128-row tile)
 constexpr int STAGES = 4;
-constexpr int kMaxStages = 5;  // the 160-wide tiles leave room for a fifth stage
+constexpr int kMaxStages = 8;  // stages of the small-batch 160-wide tiles
 constexpr int ACC = 2;
 constexpr int TMEM_COLS = ACC * BN;  // 512
 constexpr int A_BYTES = BM * BK * 2;
@@ -68,30 +69,41 @@ constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux
 // kind::f16 instruction descriptors (D f32, A and B bf16, both K-major, M = BM) are
 // per tile width: Geo<BNT>::IDESC.
 
-// Geometry of a 1-SM kernel instance with tiles BNT columns wide: 256, or 160 when
-// the narrower tile puts every tile of a small batch on an SM of its own (a batch of
-// at most 128 rows per expert has one row tile per expert, E x ceil(N / BNT) tiles).
-// The accumulators keep the 256-column TMEM stride.
-template <int BNT>
-struct Geo {
-    static constexpr int B_BYTES = BNT * BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int NSTAGES = BNT == BN ? STAGES : kMaxStages;
-    static constexpr int TILE_BYTES = NSTAGES * STAGE_BYTES;
-    static constexpr int SMEM_BYTES = 1024 + TILE_BYTES + 8 * 2 * 32 * 64 + (int)sizeof(Aux);
-    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                      ((uint32_t)(BNT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-    static_assert(BNT % 32 == 0 && BNT <= BN && STAGE_BYTES % 1024 == 0, "tile width");
-    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-};
-constexpr int kNarrowBN = 160;
-
 // Output staging: each epilogue warp owns two 2 KB shared-memory slots, each one
 // [32 rows][64 bytes] box laid out with the 64-byte swizzle (16-byte chunk j of row
 // r at r*64 + ((j ^ ((r >> 1) & 3)) * 16)), the layout the output tensor map's
 // SWIZZLE_64B expects; the 32 lanes write their rows without bank conflicts.
 constexpr int kStageSlotBytes = 32 * 64;
 constexpr int kEpiStageBytes = 8 /* warps */ * 2 * kStageSlotBytes;
+
+// Geometry of a 1-SM kernel instance with tiles BNT columns wide: 256, or 160 when
+// the narrower tile puts every tile of a small batch on an SM of its own (a batch of
+// at most 128 rows per expert has one row tile per expert, E x ceil(N / BNT) tiles).
+// The accumulators keep the 256-column TMEM stride.  SMALL (every tile at most 64
+// rows): a stage holds one 64-row A box and the B box -- the MMA's other 64 A rows are
+// the first bytes of the B box, and only make accumulator rows nobody stores -- and
+// the epilogue writes per lane without staging, so the ring gets the space: 8 stages
+// of 160-wide tiles, 5 of 256-wide ones.
+template <int BNT, bool SMALL = false>
+struct Geo {
+    static constexpr int A_REGION = SMALL ? kABoxRows * BK * 2 : A_BYTES;
+    static constexpr int B_BYTES = BNT * BK * 2;
+    static constexpr int STAGE_BYTES = A_REGION + B_BYTES;
+    static constexpr int EPI_BYTES = SMALL ? 0 : kEpiStageBytes;
+    static constexpr int FIXED_BYTES = 1024 + EPI_BYTES + (int)sizeof(Aux);
+    static constexpr int FIT = (227 * 1024 - FIXED_BYTES) / STAGE_BYTES;
+    static constexpr int NSTAGES =
+        SMALL ? (FIT < kMaxStages ? FIT : kMaxStages) : (BNT == BN ? STAGES : 5);
+    static constexpr int TILE_BYTES = NSTAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = FIXED_BYTES + TILE_BYTES;
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                      ((uint32_t)(BNT >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static_assert(BNT % 32 == 0 && BNT <= BN && STAGE_BYTES % 1024 == 0, "tile width");
+    static_assert(A_BYTES <= STAGE_BYTES, "the MMA's 128 A rows lie inside the stage");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+constexpr int kNarrowBN = 160;
+
 
 struct EpiStore {
     const CUtensorMap *map;  // output [rows][cols], box {32 cols, 32 rows}, SWIZZLE_64B
@@ -129,7 +141,7 @@ __device__ __forceinline__ void stage_box(EpiStore &st, const uint32_t (&pk)[16]
 //   Store:  the 32 columns rounded to bf16.
 // Boxes wholly inside the expert's rows and the valid columns go out through the
 // staging slots as bulk tensor stores; the others are written per lane, masked.
-template <int EPI>
+template <int EPI, bool NOSTAGE = false>
 __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n_chunks,
                                               int row0, int row_end, int n0,
                                               bf16 *__restrict__ out, int ld_out, int n_valid,
@@ -138,7 +150,7 @@ __device__ __forceinline__ void epilogue_slab(uint32_t taddr, int c_first, int n
     const int lane = threadIdx.x & 31;
     const int row = row0 + lane;
     const bool rv = row < row_end;
-    const bool full_rows = row0 + 32 <= row_end;
+    const bool full_rows = !NOSTAGE && row0 + 32 <= row_end;  // NOSTAGE: no staging slots
 #pragma unroll 1
     for (int c = c_first; c < c_first + n_chunks; c += 2) {
         uint32_t v[2][32];
@@ -273,10 +285,14 @@ __device__ __forceinline__ Tile decode_tile(const Aux *aux, int tile, int n_tile
     return t;
 }
 
+// Without GATHER, tmA's box is 64 rows high: a tile with at most 64 rows (every tile of
+// a batch of at most 64 tokens) loads one box per stage, others two.  The MMA always
+// reads 128 rows; rows a tile does not load keep whatever the stage held and only make
+// accumulator rows past the tile's last row, which the epilogue never stores.
 // GATHER: tmA covers the unpermuted activations x [T][K] with a box one row high;
 // the A rows of a tile are gathered through row_token (4 rows per TMA, one TMA
 // per producer lane) instead of being read from a permuted copy.
-template <int EPI, bool GATHER, int BNT = BN>
+template <int EPI, bool GATHER, int BNT = BN, bool SMALL = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -305,12 +321,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Aux *aux = reinterpret_cast<Aux *>(smem + Geo<BNT>::TILE_BYTES + kEpiStageBytes);
+    using G = Geo<BNT, SMALL>;
+    Aux *aux = reinterpret_cast<Aux *>(smem + G::TILE_BYTES + G::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int32_t *abort_flag = &aux->abort_flag;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Geo<BNT>::NSTAGES; ++s) {
+        for (int s = 0; s < G::NSTAGES; ++s) {
             mbar_init(smem_u32(&aux->full[s]), 1);
             mbar_init(smem_u32(&aux->empty[s]), 1);
         }
@@ -366,6 +383,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (__shfl_sync(0xffffffffu, (int)*abort_flag, 0))
                 break;
             const Tile t = decode_tile<BNT>(aux, tile, n_tiles);
+            // A rows landing per stage: gather4 fills all BM rows; a SMALL stage has room
+            // for one box (more rows than that: offsets no dispatch can give, reported)
+            const bool big = t.row_end - t.row0 > kABoxRows;
+            if (SMALL && big && lane == 0)
+                set_status(status, MOE_ERR_DEVICE_BADINDEX);
+            const int a_boxes = GATHER ? BM / kABoxRows : (big && !SMALL ? 2 : 1);
             int src[4] = {0, 0, 0, 0};
             if constexpr (GATHER) {
 #pragma unroll
@@ -385,19 +408,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
                 }
                 const uint32_t fb = smem_u32(&aux->full[stage]);
-                const uint32_t sa = smem_base + stage * Geo<BNT>::STAGE_BYTES;
+                const uint32_t sa = smem_base + stage * G::STAGE_BYTES;
                 if (lane == 0)
-                    mbar_expect_tx(fb, Geo<BNT>::STAGE_BYTES);
+                    mbar_expect_tx(fb, (uint32_t)(a_boxes * kABoxRows * BK * 2 +
+                                                  G::B_BYTES));
                 __syncwarp();
                 if constexpr (GATHER)
                     tma_gather4(&tmA, fb, sa + lane * 4 * 128, kb * BK, src[0], src[1], src[2],
                                 src[3]);
-                else if (lane == 0)
+                else if (lane == 0) {
                     tma_load_2d(&tmA, fb, sa, kb * BK, t.row0);
+                    if (a_boxes == 2)
+                        tma_load_2d(&tmA, fb, sa + kABoxRows * BK * 2, kb * BK,
+                                    t.row0 + kABoxRows);
+                }
                 if (lane == 0)
-                    tma_load_3d(&tmB, fb, sa + A_BYTES, kb * BK, t.n0, t.e);
+                    tma_load_3d(&tmB, fb, sa + G::A_REGION, kb * BK, t.n0, t.e);
                 ++fills;
-                if (++stage == Geo<BNT>::NSTAGES) {
+                if (++stage == G::NSTAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -407,8 +435,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // drain: the last fill of every stage has landed before the CTA may exit
         if (lane == 0) {
-            for (int s = 0; s < Geo<BNT>::NSTAGES; ++s) {
-                const int64_t n = fills / Geo<BNT>::NSTAGES + (s < fills % Geo<BNT>::NSTAGES ? 1 : 0);
+            for (int s = 0; s < G::NSTAGES; ++s) {
+                const int64_t n = fills / G::NSTAGES + (s < fills % G::NSTAGES ? 1 : 0);
                 if (n > 0)
                     mbar_drain(smem_u32(&aux->full[s]), (uint32_t)((n - 1) & 1));
             }
@@ -436,14 +464,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_base + stage * Geo<BNT>::STAGE_BYTES;
-                    const uint64_t da = sdesc(sa), db = sdesc(sa + A_BYTES);
+                    const uint32_t sa = smem_base + stage * G::STAGE_BYTES;
+                    const uint64_t da = sdesc(sa), db = sdesc(sa + G::A_REGION);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)  // +32 bytes (16 bf16) per step
                         umma_f16(d_tmem, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k),
-                                 Geo<BNT>::IDESC, (kb | k) != 0);
+                                 G::IDESC, (kb | k) != 0);
                     umma_commit(smem_u32(&aux->empty[stage]));
-                    if (++stage == Geo<BNT>::NSTAGES) {
+                    if (++stage == G::NSTAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -470,7 +498,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         constexpr int kChunks = BNT / 32, kHalf0 = (kChunks + 1) / 2;
         const bool upper = (warp - 2) / 4 != 0;
         const int c_first = upper ? kHalf0 : 0, n_chunks = upper ? kChunks - kHalf0 : kHalf0;
-        EpiStore st{&tmO, smem_base + Geo<BNT>::TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
+        EpiStore st{&tmO, smem_base + G::TILE_BYTES + (uint32_t)((warp - 2) * 2 * kStageSlotBytes), 0};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -479,8 +507,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + (uint32_t)(acc * BN);
-            epilogue_slab<EPI>(taddr, c_first, n_chunks, t.row0 + lane_base, t.row_end, t.n0, out,
-                               ld_out, n_valid, st);
+            if (!SMALL || t.row0 + lane_base < t.row_end)  // SMALL: warps past the rows idle
+                epilogue_slab<EPI, SMALL>(taddr, c_first, n_chunks, t.row0 + lane_base,
+                                          t.row_end, t.n0, out, ld_out, n_valid, st);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -909,7 +938,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 struct DevInfo {
     int sms = 0;
     int pair_clusters = 0;
-    bool attr[10] = {false, false, false, false, false, false, false, false, false, false};
+    bool attr[14] = {};
 };
 static std::mutex g_dev_mu;
 static DevInfo g_dev[64];
@@ -925,7 +954,7 @@ static cudaError_t set_smem_attr(Kern kern, int bytes, bool &done)
     return e;
 }
 
-// SM count, dynamic shared memory opt-in of the four GEMM kernels, and how many
+// SM count, dynamic shared memory opt-in of the GEMM kernels, and how many
 // 2-CTA clusters of the pair kernel fit at once (per device, cached).
 static cudaError_t prepare_device(DevInfo **out)
 {
@@ -961,7 +990,15 @@ static cudaError_t prepare_device(DevInfo **out)
         (e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, false, kNarrowBN>,
                            Geo<kNarrowBN>::SMEM_BYTES, di.attr[8])) != cudaSuccess ||
         (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, false, kNarrowBN>,
-                           Geo<kNarrowBN>::SMEM_BYTES, di.attr[9])) != cudaSuccess)
+                           Geo<kNarrowBN>::SMEM_BYTES, di.attr[9])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, false, kNarrowBN, true>,
+                           Geo<kNarrowBN, true>::SMEM_BYTES, di.attr[10])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, false, kNarrowBN, true>,
+                           Geo<kNarrowBN, true>::SMEM_BYTES, di.attr[11])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_SWIGLU, false, BN, true>,
+                           Geo<BN, true>::SMEM_BYTES, di.attr[12])) != cudaSuccess ||
+        (e = set_smem_attr(grouped_gemm_kernel<EPI_STORE, false, BN, true>,
+                           Geo<BN, true>::SMEM_BYTES, di.attr[13])) != cudaSuccess)
         return e;
     if (di.pair_clusters == 0) {
         cudaLaunchConfig_t cfg = {};
@@ -1025,7 +1062,8 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     const int64_t n_wide = (int64_t)E * (((int64_t)b_rows + BN - 1) / BN);
     const int64_t n_narrow = (int64_t)E * (((int64_t)b_rows + kNarrowBN - 1) / kNarrowBN);
     const bool narrow = !pair && !gather && T <= BM && n_wide < di->sms && n_narrow <= di->sms;
-    const uint32_t ba[2] = {BK, gather ? 1u : (uint32_t)BM};  // gather4 boxes are one row high
+    // A boxes: one row high for gather4, 64 rows for the 1-SM kernel, BM for the pair
+    const uint32_t ba[2] = {BK, gather ? 1u : (pair ? (uint32_t)BM : (uint32_t)kABoxRows)};
     const uint32_t bb[3] = {BK, pair ? (uint32_t)tc2::BNH : (uint32_t)(narrow ? kNarrowBN : BN),
                             1};
     if ((e = make_map(&ta, A, 2, da, sa, ba)) != cudaSuccess)
@@ -1045,6 +1083,21 @@ static cudaError_t launch_gemm(const void *A, uint64_t a_k, uint64_t a_ld, uint6
     const int pf_kb = !pair && !gather && T <= BM
                           ? (int)((int64_t)kL2PrefetchKiB * 1024 / ((int64_t)bnt * BK * 2))
                           : 0;
+    // at most 64 tokens: no expert has more than 64 rows (a token adds at most one row
+    // per expert), so the small-batch stages apply
+    const bool small = !pair && !gather && T <= kABoxRows;
+    if (narrow && small) {
+        launch_pdl(grouped_gemm_kernel<EPI, false, kNarrowBN, true>, dim3(di->sms),
+                   dim3(NUM_THREADS), Geo<kNarrowBN, true>::SMEM_BYTES, s, ta, tb, to, offsets, E,
+                   N, K, out, ld_out, n_valid, status, wait_ns, row_token, pf_kb);
+        return cudaGetLastError();
+    }
+    if (small) {
+        launch_pdl(grouped_gemm_kernel<EPI, false, BN, true>, dim3(di->sms), dim3(NUM_THREADS),
+                   Geo<BN, true>::SMEM_BYTES, s, ta, tb, to, offsets, E, N, K, out, ld_out,
+                   n_valid, status, wait_ns, row_token, pf_kb);
+        return cudaGetLastError();
+    }
     if (narrow) {
         launch_pdl(grouped_gemm_kernel<EPI, false, kNarrowBN>, dim3(di->sms), dim3(NUM_THREADS),
                    Geo<kNarrowBN>::SMEM_BYTES, s, ta, tb, to, offsets, E, N, K, out, ld_out,
