@@ -1030,7 +1030,7 @@ constexpr int64_t kPairMinRows = 4096;
 // Bytes of its first weight tile (KiB) that each CTA of a small-batch GEMM (at most one
 // row tile per expert) brings into L2 before it waits for the routing kernels.
 #ifndef MOE_L2_PREFETCH_KIB
-#define MOE_L2_PREFETCH_KIB 640
+#define MOE_L2_PREFETCH_KIB 400
 #endif
 constexpr int kL2PrefetchKiB = MOE_L2_PREFETCH_KIB;
 
