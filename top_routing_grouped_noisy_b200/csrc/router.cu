@@ -253,6 +253,8 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
     __shared__ int32_t s_cnt[MOE_MAX_EXPERTS], s_kept[MOE_MAX_EXPERTS];
     __shared__ int32_t s_off[MOE_MAX_EXPERTS + 1];
     __shared__ float s_lg[8][2 * MOE_MAX_EXPERTS];
+    constexpr int kChunks = kRouterSmallTokens * MOE_MAX_TOPK / 32;
+    __shared__ int32_t s_ccnt[kChunks][MOE_MAX_EXPERTS], s_cbase[kChunks][MOE_MAX_EXPERTS];
     __shared__ double s_fp[MOE_MAX_EXPERTS];
     constexpr int kTokPerCta = kRouterSmallTokens / kRouterSmallSplit;
     static_assert(kRouterSmallTokens % kRouterSmallSplit == 0, "tokens per CTA");
@@ -306,16 +308,32 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
     front_grid_sync(a, 2, &s_abort);
     if (threadIdx.x == 0)
         front_small_done(a);
-    // a2: every CTA counts all T*k assignments; it writes the tables of its own tokens
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x)
+    // a2: every CTA counts all T*k assignments and writes the tables of its own tokens.
+    // The entries are token-major and a token's k experts differ, so an entry's rank
+    // (its expert's entries of earlier tokens) is the count of equal entries before it:
+    // per 32-entry chunk one ballot per expert, a scan over chunks, then match_any.
+    const int n = T * k, nch = (n + 31) / 32, nwarps = (int)(blockDim.x >> 5);
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
         s_idx[i] = __ldcg(a.idx + i);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int cnt = 0;
-        for (int i = 0; i < T * k; ++i)
-            cnt += s_idx[i] == e;
-        s_cnt[e] = cnt;
-        s_kept[e] = a.C < 0 ? cnt : min(cnt, a.C);
+    for (int c = warp; c < nch; c += nwarps) {
+        const int i = c * 32 + lane;
+        const int e = i < n ? s_idx[i] : -1;
+        for (int x = 0; x < E; ++x) {
+            const unsigned b = __ballot_sync(0xffffffffu, e == x);
+            if (lane == 0)
+                s_ccnt[c][x] = __popc(b);
+        }
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < E; x += blockDim.x) {
+        int run = 0;
+        for (int c = 0; c < nch; ++c) {
+            s_cbase[c][x] = run;
+            run += s_ccnt[c][x];
+        }
+        s_cnt[x] = run;
+        s_kept[x] = a.C < 0 ? run : min(run, a.C);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -327,24 +345,25 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
         s_off[E] = acc;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-        const int t = i / k, e = s_idx[i];
-        if (t % G != (int)blockIdx.x)
-            continue;
-        int row = -1;
-        if (e < 0 || e >= E) {
-            set_status(a.status, MOE_ERR_DEVICE_BADINDEX);
-        } else {
-            int rank = 0;  // the expert's assignments of earlier tokens
-            for (int i2 = 0; i2 < t * k; ++i2)
-                rank += s_idx[i2] == e;
-            if (rank < s_kept[e]) {
-                row = s_off[e] + rank;
-                a.row_token[row] = t;
+    for (int c = warp; c < nch; c += nwarps) {
+        const int i = c * 32 + lane;
+        const int e = i < n ? s_idx[i] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int t = i / k;
+        if (i < n && t % G == (int)blockIdx.x) {
+            int row = -1;
+            if (e < 0 || e >= E) {
+                set_status(a.status, MOE_ERR_DEVICE_BADINDEX);
+            } else {
+                const int rank = s_cbase[c][e] + __popc(same & ((1u << lane) - 1u));
+                if (rank < s_kept[e]) {
+                    row = s_off[e] + rank;
+                    a.row_token[row] = t;
+                }
             }
+            s_row[i] = row;
+            a.slot_row[i] = row;
         }
-        s_row[i] = row;
-        a.slot_row[i] = row;
     }
     __syncthreads();
     const int nv = a.d * (int)sizeof(E_T) / 16;
@@ -376,6 +395,7 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         float sp = 0.f, sg = 0.f;
+#pragma unroll 16
         for (int t = 0; t < T; ++t) {
             sp += pg[t * E + e];
             sg += pg[(T + t) * E + e];
