@@ -45,9 +45,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the source it was taken on; reported as null once the kernel source changes.
 # (default tile band of 2048 rows)
 NCU_TRAFFIC = {
-    "moe_2of8": {"src": "57db11ab329b9b6b", "T": 16384, "bytes_per_launch": 505.54e6 + 100.86e6},
-    "e8t2_cf4": {"src": "57db11ab329b9b6b", "T": 32768,
-                 "bytes_per_launch": 22603.57e6 + 2893.92e6},
+    "moe_2of8": {"src": "6205a369f7ffb96e", "T": 16384, "bytes_per_launch": 468.02e6 + 81.73e6},
+    "e8t2_cf4": {"src": "6205a369f7ffb96e", "T": 32768,
+                 "bytes_per_launch": 16910.92e6 + 1872.96e6},
 }
 
 
