@@ -308,8 +308,9 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
     front_grid_sync(a, 2, &s_abort);
     if (threadIdx.x == 0)
         front_small_done(a);
-    // a2: every CTA counts all T*k assignments and writes the tables of its own tokens.
-    // The entries are token-major and a token's k experts differ, so an entry's rank
+    // a2: every CTA counts all T*k assignments; CTAs 1..G-1 write the tables and x_perm
+    // rows of tokens 1 + t mod (G - 1), so that CTA 0 goes straight on to the token sums
+    // and a6.  The entries are token-major and a token's k experts differ, so an entry's rank
     // (its expert's entries of earlier tokens) is the count of equal entries before it:
     // per 32-entry chunk one ballot per expert, a scan over chunks, then match_any.
     const int n = T * k, nch = (n + 31) / 32, nwarps = (int)(blockDim.x >> 5);
@@ -350,7 +351,7 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
         const int e = i < n ? s_idx[i] : -1;
         const unsigned same = __match_any_sync(0xffffffffu, e);
         const int t = i / k;
-        if (i < n && t % G == (int)blockIdx.x) {
+        if (i < n && 1 + t % (G - 1) == (int)blockIdx.x) {
             int row = -1;
             if (e < 0 || e >= E) {
                 set_status(a.status, MOE_ERR_DEVICE_BADINDEX);
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(256) front_small_kernel(const __grid_constant_
     __syncthreads();
     const int nv = a.d * (int)sizeof(E_T) / 16;
     const char *xb = static_cast<const char *>(a.x);
-    for (int t = blockIdx.x; t < T; t += G) {
+    for (int t = (int)blockIdx.x - 1; blockIdx.x > 0 && t < T; t += G - 1) {
         const char *src = xb + (int64_t)t * nv * 16;
         for (int v = threadIdx.x; v < nv; v += blockDim.x) {
             const uint4 val = ld_nc(src + (int64_t)v * 16);
