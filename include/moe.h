@@ -317,7 +317,15 @@ typedef struct {
     const void *router_packed;
 } moe_buffers_t;
 
-/* a1 -> a2 -> a3 -> a4 -> a5 -> a6 on one stream, no host synchronisation. */
+/* a1 -> a2 -> a3 -> a4 -> a5 -> a6 on one stream, no host synchronisation.
+ * Every output equals what the step calls (moe_route, moe_dispatch, moe_expert_up,
+ * moe_expert_down, moe_combine, moe_gate_stats) give on the same inputs, bit for bit.
+ * How it launches depends on the batch: bf16 batches of at most 16 tokens run the
+ * whole layer as one cooperative launch; batches of at most 64 tokens whose router is
+ * the split-K one run a1, a2 and a6 as one cooperative launch of 32 CTAs before the
+ * expert GEMMs and a5; larger batches run the steps' kernels.  A device wait past the
+ * limit (moe_set_wait_limit_ns) is reported as MOE_ERR_DEVICE_TIMEOUT in the status
+ * word, as in every call. */
 int moe_forward(const moe_params_t *p, const moe_buffers_t *b, void *ws, size_t ws_bytes,
                 void *stream);
 
