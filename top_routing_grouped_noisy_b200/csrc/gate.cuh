@@ -208,40 +208,31 @@ __device__ inline void router_small_slice_mma(int ks, const bf16 *__restrict__ x
     const int T16 = round_up(T, 16);
     bf16 *xs = static_cast<bf16 *>(sm);  // [T16][xp]
     bf16 *wsm = xs + (size_t)T16 * xp;  // [kp][wp]
-    // x: 16-byte vectors, four in flight per thread before any is stored
-    const int vx = kp / 8, nvx = T16 * vx;
-    for (int i0 = threadIdx.x; i0 < nvx; i0 += 4 * blockDim.x) {
+    // x (16-byte vectors) and the weight rows k0 + r (W_g's E columns, then W_noise's;
+    // zero padding written with them): each round has four x vectors and four weight
+    // elements per thread in flight before any is stored
+    const int vx = kp / 8, nvx = T16 * vx, nw = kp * np;
+    for (int i0 = threadIdx.x; i0 < nvx || i0 < nw; i0 += 4 * blockDim.x) {
         uint4 u[4];
+        bf16 wv[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int i = i0 + j * blockDim.x, t = i / vx, v = i % vx;
             u[j] = make_uint4(0, 0, 0, 0);
             if (i < nvx && t < T && v * 8 < kn)
                 u[j] = ld_nc(x + (int64_t)t * d + k0 + v * 8);
+            const int r = i / np, o = i % np;
+            wv[j] = __float2bfloat16_rn(0.f);
+            if (i < nw && r < kn && o < nout)
+                wv[j] = o < E ? Wg[(int64_t)(k0 + r) * E + o] : Wn[(int64_t)(k0 + r) * E + o - E];
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int i = i0 + j * blockDim.x;
             if (i < nvx)
                 *reinterpret_cast<uint4 *>(xs + (size_t)(i / vx) * xp + (i % vx) * 8) = u[j];
-        }
-    }
-    // weight rows k0 + r: W_g's E columns, then W_noise's
-    const int nw = kp * np;
-    for (int i0 = threadIdx.x; i0 < nw; i0 += 4 * blockDim.x) {
-        bf16 u[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j * blockDim.x, r = i / np, o = i % np;
-            u[j] = __float2bfloat16_rn(0.f);
-            if (i < nw && r < kn && o < nout)
-                u[j] = o < E ? Wg[(int64_t)(k0 + r) * E + o] : Wn[(int64_t)(k0 + r) * E + o - E];
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j * blockDim.x;
             if (i < nw)
-                wsm[(size_t)(i / np) * wp + i % np] = u[j];
+                wsm[(size_t)(i / np) * wp + i % np] = wv[j];
         }
     }
     __syncthreads();
