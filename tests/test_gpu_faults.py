@@ -143,3 +143,33 @@ def test_front_small_wait_timeout_is_reported_and_context_survives():
     r, ties = H.check_routing(w, inp, bufs, 5e-5)
     dsp = H.check_dispatch(w, inp, p, bufs)
     H.check_y(w, bufs, r, dsp, H.oracle_weights(w, inp), np.nonzero(~ties)[0], inp=inp)
+
+
+def test_small_batch_gemm_reports_an_expert_with_more_rows_than_tokens():
+    """At most 64 tokens give each expert at most 64 rows, which the small-batch GEMM
+    ring is sized for; offsets that give an expert more (no dispatch can) are reported
+    as MOE_ERR_DEVICE_BADINDEX, every access stays inside the buffers (the rows past 64
+    are computed from whatever the stage held), and the next call is unaffected."""
+    T, d, E, k, m = 64, 256, 4, 2, 64
+    p = moe.params(T, d, E, k, m)
+    ws = moe.Workspace(p)
+    gen = torch.Generator().manual_seed(85)
+    rows = T * k
+    x_perm = (torch.randn(rows, d, generator=gen) * 0.5).to(torch.bfloat16).cuda()
+    W13 = (torch.randn(E, 2 * m, d, generator=gen) * 0.05).to(torch.bfloat16).cuda()
+    h = torch.zeros(rows, m, dtype=torch.bfloat16, device="cuda")
+    bad = torch.tensor([0, 100, 110, 120, rows], dtype=torch.int32, device="cuda")
+    moe.moe_expert_up(p, x_perm, bad, W13, h, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_DEVICE_BADINDEX
+    good = torch.tensor([0, 40, 70, 100, rows], dtype=torch.int32, device="cuda")
+    moe.moe_expert_up(p, x_perm, good, W13, h, ws)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    # expert 1's rows against a plain f32 product: h = silu(g) * u over 32-row groups
+    xe = x_perm[40:70].float()
+    W = W13[1].float()  # rows: per 32-row group 16 W1 rows, then the 16 W3 rows
+    g = torch.cat([W[32 * i:32 * i + 16] for i in range(m // 16)]) @ xe.T
+    u = torch.cat([W[32 * i + 16:32 * i + 32] for i in range(m // 16)]) @ xe.T
+    ref = (torch.nn.functional.silu(g) * u).T
+    assert torch.allclose(h[40:70].float(), ref, atol=2e-2, rtol=2e-2)
