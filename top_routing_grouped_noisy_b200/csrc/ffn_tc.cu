@@ -101,6 +101,8 @@ struct Geo {
     static_assert(BNT % 32 == 0 && BNT <= BN && STAGE_BYTES % 1024 == 0, "tile width");
     static_assert(A_BYTES <= STAGE_BYTES, "the MMA's 128 A rows lie inside the stage");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static_assert(SMEM_BYTES > 114 * 1024,
+                  "one CTA per SM: the kernel allocates TMEM before its wait on the previous grid");
 };
 constexpr int kNarrowBN = 160;
 
@@ -316,8 +318,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tma_prefetch_l2_3d(&tmB, kb * BK, n0, e);
         }
     }
-    pdl_wait();
-    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -342,6 +342,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmO)) : "memory");
     }
+    // The barriers and TMEM are set up before the wait on the previous grid: no kernel of
+    // the library that holds TMEM can share an SM with this one (each takes more than half
+    // of the shared memory), so the allocation cannot wait on a CTA that waits on us.
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&aux->tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    pdl_wait();
+    pdl_trigger();
     const int n_tiles = (N + BNT - 1) / BNT;
     if (warp == 2) {
         for (int i = lane; i <= E; i += 32)
@@ -356,13 +368,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             aux->tstart[E] = acc;
         }
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(&aux->tmem_base)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
