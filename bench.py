@@ -45,9 +45,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the source it was taken on; reported as null once the kernel source changes.
 # (default tile band of 2048 rows)
 NCU_TRAFFIC = {
-    "moe_2of8": {"src": "6205a369f7ffb96e", "T": 16384, "bytes_per_launch": 468.02e6 + 81.73e6},
-    "e8t2_cf4": {"src": "6205a369f7ffb96e", "T": 32768,
-                 "bytes_per_launch": 16910.92e6 + 1872.96e6},
+    "moe_2of8": {"src": "ed7e29b9fa5e804b", "T": 16384, "bytes_per_launch": 471.48e6 + 82.46e6},
+    "e8t2_cf4": {"src": "ed7e29b9fa5e804b", "T": 32768,
+                 "bytes_per_launch": 23875.10e6 + 1875.45e6},
 }
 
 
